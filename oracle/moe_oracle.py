@@ -1,0 +1,275 @@
+"""fp64 CPU oracle of the MoE layer with zero-computation experts.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, the package smoke check and
+the benchmark's CPU-baseline leg may import this module.  The product path
+(the CUDA library and its Python binding) never imports, calls or falls back
+to it, and it imports nothing from the product path.
+
+It follows "LongCat-Flash Technical Report" (Chinese translation):
+  * §2.1 Zero-computation experts, Eq. (1): the layer output
+        MoE(x_t) = sum_{i=1}^{N+Z} g_i E_i(x_t),
+        g_i = R(x_t)_i  if R(x_t)_i + b_i is among the K largest of
+                        {R(x_t)_j + b_j : 1 <= j <= N+Z}, else 0,
+        E_i(x_t) = FFN_i(x_t) for i <= N, and x_t for N < i <= N+Z,
+    with R the softmax router and b_i the expert bias.
+  * §2.1.1 Computation-budget control, Eq. (2): the per-step bias increment
+        Delta b_i = mu (K_e/K * 1/N - T_i/(K T_all))  for i <= N, 0 otherwise.
+  * §2.3.2 Eq. (8): the optional output scale gamma on the whole sum.
+
+Readings taken where the pages are silent (each is also listed in the design
+notes): the router has no bias term and no temperature, and its softmax covers
+all N+Z experts; the gate is the unbiased probability with no renormalisation;
+ties in the biased score go to the lower expert index; the FFN activation is
+SwiGLU, FFN(x) = W2 (SiLU(W1 x) * (W3 x)) with SiLU(a) = a / (1 + e^-a);
+routed rows are laid out expert by expert, ascending token inside an expert,
+and zero experts get no rows.
+
+Everything is computed in float64 with no intermediate rounding.  numpy's
+matmul, exp, sort and bincount are the only library steps.
+
+Parity status: every function here is pinned by the CPU tests
+(brute-force top-K, the Z=0 dense top-K MoE reduction, the all-zero-expert
+and K=E fixed points, closed forms of softmax, SwiGLU and Eq. (2), and the
+hand-derived worked examples under tests/golden/).
+"""
+import numpy as np
+
+
+# ---------------------------------------------------------------------------
+# Input decoding
+# ---------------------------------------------------------------------------
+
+def bf16_bits_to_f64(bits):
+    """Exact value of bf16 numbers given as their uint16 bit patterns.
+
+    A bf16 number is the upper half of an IEEE binary32 number, so placing its
+    16 bits in the high half of a 32-bit word gives that binary32 number, which
+    float64 represents exactly.
+    """
+    bits = np.asarray(bits, dtype=np.uint16)
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def as_f64(a):
+    """float32 / float64 arrays to float64 (exact)."""
+    return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Router: §2.1, Eq. (1) -- R is the softmax router
+# ---------------------------------------------------------------------------
+
+def router_logits(x, w_router, logit_offset=None):
+    """logits[t, i] = sum_j x[t, j] * w_router[i, j] (+ offset[t, i])."""
+    logits = as_f64(x) @ as_f64(w_router).T
+    if logit_offset is not None:
+        logits = logits + as_f64(logit_offset)
+    return logits
+
+
+def softmax_rows(logits):
+    """R(x_t) = softmax over all N+Z experts, max-subtracted for range."""
+    m = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - m)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def biased_topk(probs, bias, K):
+    """Eq. (1) selection: the K experts with the largest R_i + b_i.
+
+    Returns (idx [T, K] int32 ordered by biased score descending, ties to the
+    lower index; margin [T] = K-th minus (K+1)-th biased score, +inf if K = E).
+    """
+    T, E = probs.shape
+    s = probs + as_f64(bias)[None, :]
+    # A stable ascending sort of -s orders by s descending and keeps equal
+    # scores in ascending index order.
+    order = np.argsort(-s, axis=1, kind="stable")
+    idx = order[:, :K].astype(np.int32)
+    if K < E:
+        rows = np.arange(T)
+        margin = s[rows, order[:, K - 1]] - s[rows, order[:, K]]
+    else:
+        margin = np.full(T, np.inf)
+    return idx, margin
+
+
+def gates(probs, idx):
+    """g for each selected slot: the unbiased router probability (Eq. (1))."""
+    return np.take_along_axis(probs, idx.astype(np.int64), axis=1)
+
+
+def expert_counts(idx, E):
+    """T_i of Eq. (2): number of (token, slot) pairs routed to expert i."""
+    return np.bincount(idx.reshape(-1), minlength=E).astype(np.int64)
+
+
+def ffn_experts_per_token(idx, N):
+    """Number of FFN experts (index < N) among each token's K choices."""
+    return (idx < N).sum(axis=1)
+
+
+# ---------------------------------------------------------------------------
+# Dispatch to FFN experts only (zero experts get no rows)
+# ---------------------------------------------------------------------------
+
+def canonical_permutation(idx, N):
+    """Row layout of the routed FFN slots.
+
+    Rows are grouped by FFN expert 0..N-1; inside an expert the rows follow
+    ascending token index (a token picks an expert at most once).  Returns
+    offsets [N+1], row_token [R], slot_pos [T, K] (-1 for zero-expert slots).
+    """
+    T, K = idx.shape
+    ffn = idx[idx < N]
+    counts = np.bincount(ffn, minlength=N)
+    offsets = np.zeros(N + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(counts)
+    row_token = np.zeros(int(offsets[N]), dtype=np.int64)
+    slot_pos = np.full((T, K), -1, dtype=np.int64)
+    nxt = offsets[:N].copy()
+    for t in range(T):
+        for k in range(K):
+            e = int(idx[t, k])
+            if e < N:
+                r = nxt[e]
+                nxt[e] += 1
+                row_token[r] = t
+                slot_pos[t, k] = r
+    return offsets, row_token, slot_pos
+
+
+# ---------------------------------------------------------------------------
+# FFN experts: SwiGLU
+# ---------------------------------------------------------------------------
+
+def silu(a):
+    """SiLU(a) = a * sigmoid(a) = a / (1 + exp(-a))."""
+    with np.errstate(over="ignore"):
+        return a / (1.0 + np.exp(-a))
+
+
+def expert_ffn(x_rows, w1, w3, w2):
+    """FFN_e(x) = W2 (SiLU(W1 x) * (W3 x)) for each row of x_rows.
+
+    w1, w3: [I, d] (gate, up); w2: [d, I] (down); x_rows: [m, d].
+    """
+    a = x_rows @ as_f64(w1).T
+    u = x_rows @ as_f64(w3).T
+    return (silu(a) * u) @ as_f64(w2).T
+
+
+def expert_hidden(x_rows, w1, w3):
+    """The SwiGLU hidden activation SiLU(W1 x) * (W3 x), [m, I]."""
+    return silu(x_rows @ as_f64(w1).T) * (x_rows @ as_f64(w3).T)
+
+
+def grouped_ffn(x_perm, offsets, w1, w3, w2, experts=None, decode=as_f64):
+    """Run every FFN expert on its segment of routed rows.
+
+    ``decode`` maps one expert's stored weight array to float64, so the caller
+    may keep weights as bf16 bit patterns and decode one expert at a time.
+    ``experts`` restricts the work to a subset (other rows stay NaN).
+    """
+    R = int(offsets[-1])
+    d = x_perm.shape[1]
+    y = np.full((R, d), np.nan)
+    N = len(offsets) - 1
+    for e in (range(N) if experts is None else experts):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi > lo:
+            y[lo:hi] = expert_ffn(x_perm[lo:hi], decode(w1[e]), decode(w3[e]), decode(w2[e]))
+    return y
+
+
+# ---------------------------------------------------------------------------
+# Combine: Eq. (1) weighted sum, zero experts as identity, Eq. (8) scale
+# ---------------------------------------------------------------------------
+
+def combine(x, y_perm, idx, g, slot_pos, N, gamma=1.0):
+    """out_t = gamma * (sum_{FFN slots} g * FFN_e(x_t) + (sum_{zero slots} g) * x_t)."""
+    x = as_f64(x)
+    T, K = idx.shape
+    out = np.zeros_like(x)
+    for k in range(K):
+        ffn = idx[:, k] < N
+        if ffn.any():
+            out[ffn] += g[ffn, k][:, None] * y_perm[slot_pos[ffn, k]]
+    zero_mass = np.where(idx >= N, g, 0.0).sum(axis=1)
+    out += zero_mass[:, None] * x
+    return gamma * out
+
+
+def zero_mass(idx, g, N):
+    """sum of the gates of the zero-expert slots of each token."""
+    return np.where(idx >= N, g, 0.0).sum(axis=1)
+
+
+# ---------------------------------------------------------------------------
+# Computation-budget control: §2.1.1, Eq. (2)
+# ---------------------------------------------------------------------------
+
+def bias_update(bias, counts, N, K, K_e, mu, T_all):
+    """b_i + Delta b_i with Delta b_i = mu (K_e/K * 1/N - T_i/(K T_all)), i <= N.
+
+    Zero-computation experts (i > N) are left unchanged.
+    """
+    b = as_f64(bias).copy()
+    Ti = as_f64(counts[:N])
+    target = float(K_e) / (float(K) * float(N))
+    share = Ti / (float(K) * float(T_all))
+    b[:N] = b[:N] + float(mu) * (target - share)
+    return b
+
+
+# ---------------------------------------------------------------------------
+# The whole layer
+# ---------------------------------------------------------------------------
+
+def moe_layer(x, w_router, w1, w3, w2, bias, N, K, gamma=1.0, logit_offset=None,
+              decode=as_f64):
+    """Every intermediate of one forward pass of the layer, in float64.
+
+    ``x`` and ``w_router`` are float64-convertible arrays (decode bf16 first);
+    ``w1/w3/w2`` are per-expert arrays passed through ``decode``.
+    """
+    x = as_f64(x)
+    logits = router_logits(x, w_router, logit_offset)
+    probs = softmax_rows(logits)
+    idx, margin = biased_topk(probs, bias, K)
+    g = gates(probs, idx)
+    E = probs.shape[1]
+    counts = expert_counts(idx, E)
+    offsets, row_token, slot_pos = canonical_permutation(idx, N)
+    x_perm = x[row_token]
+    y_perm = grouped_ffn(x_perm, offsets, w1, w3, w2, decode=decode)
+    out = combine(x, y_perm, idx, g, slot_pos, N, gamma)
+    return dict(logits=logits, probs=probs, idx=idx, margin=margin, gate=g,
+                counts=counts, n_ffn=ffn_experts_per_token(idx, N), offsets=offsets,
+                row_token=row_token, slot_pos=slot_pos, x_perm=x_perm, y_perm=y_perm,
+                out=out)
+
+
+def bias_control_trajectory(steps, route_inputs, w_router, bias0, N, K, K_e, mu):
+    """Closed loop of Eq. (2): route with b_s, count, update to b_{s+1}.
+
+    ``route_inputs(s)`` returns (x_s, logit_offset_s).  Returns per-step
+    dictionaries with the mean / std of FFN experts per token, the max/mean
+    FFN expert load, the counts and the bias used by that step.
+    """
+    b = as_f64(bias0).copy()
+    hist = []
+    for s in range(steps):
+        x, off = route_inputs(s)
+        probs = softmax_rows(router_logits(x, w_router, off))
+        idx, margin = biased_topk(probs, b, K)
+        E = probs.shape[1]
+        counts = expert_counts(idx, E)
+        nf = ffn_experts_per_token(idx, N)
+        load = counts[:N].astype(np.float64)
+        hist.append(dict(bias=b.copy(), counts=counts, n_ffn_mean=float(nf.mean()),
+                         n_ffn_std=float(nf.std()),
+                         max_over_mean_load=float(load.max() / load.mean()),
+                         min_margin=float(margin.min())))
+        b = bias_update(b, counts, N, K, K_e, mu, x.shape[0])
+    return hist, b

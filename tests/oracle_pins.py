@@ -1,0 +1,298 @@
+"""Checks that pin the fp64 oracle to facts that do not come from the oracle.
+
+Each ``check_*`` takes the oracle module and raises AssertionError on a
+mismatch, so the same checks run against the real oracle (test_oracle_pins)
+and against copies with a planted mistake (test_oracle_mutations).
+
+Sources of truth used here, none of them the oracle's own code:
+  * hand derivations of tiny layers stored under tests/golden/ (closed forms);
+  * brute-force enumeration of expert subsets with exact rational sums;
+  * the Z = 0 reduction to a textbook dense top-K MoE, written with torch's
+    float64 CPU linear layer and SiLU;
+  * closed forms of softmax (E = 2 is a logistic sigmoid) and of Eq. (2);
+  * permutation invariants (bijection, sortedness, segment sizes).
+"""
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def load_golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------
+# worked examples (hand derivations)
+# ---------------------------------------------------------------------------
+
+def check_worked_tiny_layer(orc):
+    g = load_golden("worked_example_tiny_layer.json")
+    sh, ex = g["shape"], g["expected"]
+    r = orc.moe_layer(np.array(g["x"]), np.array(g["w_router"]), np.array(g["w1"]),
+                      np.array(g["w3"]), np.array(g["w2"]), np.array(g["bias"]),
+                      N=sh["N"], K=sh["K"])
+    np.testing.assert_allclose(r["probs"], ex["probs"], rtol=0, atol=1e-15)
+    np.testing.assert_array_equal(r["idx"], ex["topk_idx"])
+    np.testing.assert_allclose(r["gate"], ex["gate"], rtol=0, atol=1e-15)
+    np.testing.assert_array_equal(r["counts"], ex["counts"])
+    np.testing.assert_array_equal(r["n_ffn"], ex["n_ffn"])
+    np.testing.assert_allclose(r["y_perm"][0, 0], ex["y_expert0"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(r["out"], ex["out"], rtol=0, atol=1e-15)
+
+
+def check_worked_swiglu(orc):
+    g = load_golden("worked_example_swiglu.json")
+    ex = g["expected"]
+    y = orc.expert_ffn(np.array([[g["x"]]]), np.array([[g["w1"]]]), np.array([[g["w3"]]]),
+                       np.array([[g["w2"]]]))
+    h = orc.expert_hidden(np.array([[g["x"]]]), np.array([[g["w1"]]]), np.array([[g["w3"]]]))
+    np.testing.assert_allclose(orc.silu(np.array([1.0]))[0], ex["silu_a"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(h[0, 0], ex["h"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(y[0, 0], ex["y"], rtol=0, atol=1e-14)
+
+
+def check_worked_bias_update(orc):
+    g = load_golden("worked_example_bias_update.json")
+    b = orc.bias_update(np.array(g["bias"]), np.array(g["counts"]), g["N"], g["K"],
+                        g["K_e"], g["mu"], g["T_all"])
+    np.testing.assert_allclose(b, g["expected_bias"], rtol=0, atol=1e-16)
+    # zero experts unchanged bit for bit
+    assert b[g["N"]:].tobytes() == np.array(g["bias"][g["N"]:]).tobytes()
+
+
+def check_worked_zero_experts(orc):
+    g = load_golden("worked_example_zero_experts.json")
+    sh, ex = g["shape"], g["expected"]
+    probs = orc.softmax_rows(np.array(g["router_logits"]))
+    np.testing.assert_allclose(probs, ex["probs"], rtol=0, atol=1e-15)
+    idx, _ = orc.biased_topk(probs, np.array(g["bias"]), sh["K"])
+    np.testing.assert_array_equal(idx, ex["topk_idx"])
+    gate = orc.gates(probs, idx)
+    _, _, slot_pos = orc.canonical_permutation(idx, sh["N"])
+    out = orc.combine(np.array(g["x"]), np.zeros((0, sh["d"])), idx, gate, slot_pos, sh["N"])
+    np.testing.assert_allclose(orc.zero_mass(idx, gate, sh["N"]), [ex["zero_mass"]],
+                               rtol=0, atol=1e-15)
+    np.testing.assert_allclose(out, ex["out"], rtol=0, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# softmax closed forms
+# ---------------------------------------------------------------------------
+
+def check_softmax_closed_forms(orc, seed=0):
+    rng = np.random.default_rng(seed)
+    lg = rng.normal(size=(64, 2)) * 3
+    p = orc.softmax_rows(lg)
+    sig = np.array([1.0 / (1.0 + math.exp(-(a - b))) for a, b in lg])
+    np.testing.assert_allclose(p[:, 0], sig, rtol=0, atol=1e-15)
+    lg = rng.normal(size=(32, 17))
+    p = orc.softmax_rows(lg)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=0, atol=1e-15)
+    p2 = orc.softmax_rows(lg + rng.normal(size=(32, 1)) * 50)
+    np.testing.assert_allclose(p2, p, rtol=1e-12, atol=0)
+    # ratio of two entries is exp of the logit gap
+    np.testing.assert_allclose(p[:, 3] / p[:, 5], np.exp(lg[:, 3] - lg[:, 5]), rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# top-K against brute force with exact sums
+# ---------------------------------------------------------------------------
+
+def brute_force_topk(s_row, K):
+    """The K-subset with the largest exact sum, ties to the smallest sorted index tuple;
+    returned in (score desc, index asc) order."""
+    E = len(s_row)
+    fr = [Fraction(v) for v in s_row]
+    best, best_sum = None, None
+    for sub in itertools.combinations(range(E), K):
+        sm = sum(fr[i] for i in sub)
+        if best is None or sm > best_sum or (sm == best_sum and sub < best):
+            best, best_sum = sub, sm
+    return sorted(best, key=lambda i: (-fr[i], i))
+
+
+def check_topk_brute_force(orc, cases=300, seed=1):
+    rng = np.random.default_rng(seed)
+    for c in range(cases):
+        E = int(rng.integers(2, 11))
+        K = int(rng.integers(1, min(4, E) + 1))
+        if c % 3 == 0:
+            # forced ties: few distinct dyadic values so sums are exact and equal
+            probs = rng.integers(0, 4, size=(1, E)) / 8.0
+            bias = rng.integers(-1, 2, size=E) / 16.0
+        else:
+            probs = orc.softmax_rows(rng.normal(size=(1, E)))
+            bias = rng.uniform(-0.1, 0.1, size=E)
+        idx, margin = orc.biased_topk(probs, bias, K)
+        s = probs[0] + bias
+        want = brute_force_topk(s, K)
+        assert list(idx[0]) == want, (probs, bias, K, idx, want)
+        srt = sorted(s, reverse=True)
+        m_want = srt[K - 1] - srt[K] if K < E else math.inf
+        assert margin[0] == m_want
+
+
+# ---------------------------------------------------------------------------
+# Z = 0: textbook dense top-K MoE; general Z: dense masked formulation
+# ---------------------------------------------------------------------------
+
+def dense_moe_torch(x, w_router, w1, w3, w2, bias, N, K, gamma=1.0):
+    """Run every expert on every token (zero experts as identity) and mask by
+    the top-K of (p + b); torch float64 CPU ops only."""
+    F = torch.nn.functional
+    x = torch.as_tensor(x, dtype=torch.float64)
+    p = torch.softmax(F.linear(x, torch.as_tensor(w_router, dtype=torch.float64)), dim=1)
+    T, E = p.shape
+    s = p + torch.as_tensor(bias, dtype=torch.float64)[None, :]
+    out = torch.zeros_like(x)
+    for t in range(T):
+        chosen = sorted(range(E), key=lambda i: (-float(s[t, i]), i))[:K]
+        for i in chosen:
+            if i < N:
+                w1e = torch.as_tensor(w1[i], dtype=torch.float64)
+                w3e = torch.as_tensor(w3[i], dtype=torch.float64)
+                w2e = torch.as_tensor(w2[i], dtype=torch.float64)
+                y = F.linear(F.silu(F.linear(x[t], w1e)) * F.linear(x[t], w3e), w2e)
+            else:
+                y = x[t]
+            out[t] += p[t, i] * y
+    return (gamma * out).numpy()
+
+
+def _rand_layer(rng, T, d, N, Z, I, bias_amp):
+    E = N + Z
+    return dict(x=rng.normal(size=(T, d)), w_router=rng.normal(size=(E, d)) * 0.5,
+                w1=rng.normal(size=(N, I, d)) * 0.3, w3=rng.normal(size=(N, I, d)) * 0.3,
+                w2=rng.normal(size=(N, d, I)) * 0.3, bias=rng.uniform(-bias_amp, bias_amp, E))
+
+
+def check_dense_reduction(orc, seed=2):
+    rng = np.random.default_rng(seed)
+    for (T, d, N, Z, K, I, amp, gamma) in ((9, 5, 6, 0, 2, 3, 0.0, 1.0),
+                                           (9, 5, 6, 0, 3, 3, 0.2, 1.0),
+                                           (11, 4, 5, 3, 3, 7, 0.1, 1.0),
+                                           (7, 6, 4, 4, 8, 2, 0.3, 2.5)):
+        L = _rand_layer(rng, T, d, N, Z, I, amp)
+        r = orc.moe_layer(L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"],
+                          N=N, K=K, gamma=gamma)
+        want = dense_moe_torch(L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"],
+                               N, K, gamma)
+        np.testing.assert_allclose(r["out"], want, rtol=1e-12, atol=1e-12)
+
+
+def check_all_zero_experts_fixed_point(orc, seed=3):
+    """b_zero = +10 routes every slot to zero experts: out = (sum g) x exactly."""
+    rng = np.random.default_rng(seed)
+    T, d, N, Z, K, I = 13, 6, 5, 4, 3, 4
+    L = _rand_layer(rng, T, d, N, Z, I, 0.0)
+    L["bias"][N:] = 10.0
+    r = orc.moe_layer(L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"], N=N, K=K)
+    assert (r["idx"] >= N).all()
+    assert r["offsets"][-1] == 0 and (r["slot_pos"] == -1).all()
+    g_sum = r["gate"].sum(axis=1)
+    assert (r["out"] == g_sum[:, None] * L["x"]).all()
+
+
+def check_k_equals_e_fixed_point(orc, seed=4):
+    """K = E selects every expert: the gates sum to 1 and out = sum_i R_i E_i(x)."""
+    rng = np.random.default_rng(seed)
+    T, d, N, Z, I = 6, 4, 3, 2, 5
+    E = N + Z
+    L = _rand_layer(rng, T, d, N, Z, I, 0.1)
+    r = orc.moe_layer(L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"], N=N, K=E)
+    np.testing.assert_allclose(r["gate"].sum(axis=1), 1.0, rtol=0, atol=1e-15)
+    want = dense_moe_torch(L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"], N, E)
+    np.testing.assert_allclose(r["out"], want, rtol=1e-12, atol=1e-12)
+    # for K < E the selected gates sum to at most 1
+    r2 = orc.moe_layer(L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"], N=N, K=2)
+    assert (r2["gate"].sum(axis=1) <= 1.0 + 1e-15).all() and (r2["gate"] > 0).all()
+
+
+# ---------------------------------------------------------------------------
+# permutation invariants
+# ---------------------------------------------------------------------------
+
+def check_permutation_invariants(orc, seed=5):
+    rng = np.random.default_rng(seed)
+    for _ in range(20):
+        T, N, Z = int(rng.integers(1, 60)), int(rng.integers(1, 12)), int(rng.integers(0, 6))
+        E = N + Z
+        K = int(rng.integers(1, E + 1))
+        idx = np.stack([rng.permutation(E)[:K] for _ in range(T)]).astype(np.int32)
+        counts = orc.expert_counts(idx, E)
+        assert counts.sum() == K * T
+        off, row_token, slot_pos = orc.canonical_permutation(idx, N)
+        R = int((idx < N).sum())
+        assert off[0] == 0 and off[N] == R and len(row_token) == R
+        np.testing.assert_array_equal(np.diff(off), counts[:N])
+        seen = np.zeros(R, dtype=bool)
+        for t in range(T):
+            for k in range(K):
+                e, p = idx[t, k], slot_pos[t, k]
+                if e < N:
+                    assert off[e] <= p < off[e + 1] and row_token[p] == t and not seen[p]
+                    seen[p] = True
+                else:
+                    assert p == -1
+        assert seen.all()
+        for e in range(N):
+            seg = row_token[off[e]:off[e + 1]]
+            assert (np.diff(seg) > 0).all()
+
+
+# ---------------------------------------------------------------------------
+# Eq. (2) closed forms
+# ---------------------------------------------------------------------------
+
+def check_bias_update_closed_form(orc, seed=6):
+    rng = np.random.default_rng(seed)
+    for _ in range(50):
+        N, Z = int(rng.integers(1, 40)), int(rng.integers(0, 20))
+        E = N + Z
+        K = int(rng.integers(1, E + 1))
+        T = int(rng.integers(1, 500))
+        K_e = float(rng.uniform(0.5, K))
+        mu = float(rng.uniform(0.001, 1.0))
+        idx = np.stack([rng.permutation(E)[:K] for _ in range(T)])
+        counts = np.bincount(idx.reshape(-1), minlength=E)
+        b0 = rng.normal(size=E)
+        b1 = orc.bias_update(b0, counts, N, K, K_e, mu, T)
+        F = counts[:N].sum()
+        # sum of increments over FFN experts: mu (K_e - F/T) / K
+        np.testing.assert_allclose((b1 - b0)[:N].sum(), mu * (K_e - F / T) / K,
+                                   rtol=1e-9, atol=1e-12)
+        assert b1[N:].tobytes() == b0[N:].tobytes()
+        # experts above their share move down, below it move up
+        share = counts[:N] / (K * T)
+        tgt = K_e / (K * N)
+        assert ((b1 - b0)[:N][share > tgt + 1e-12] < 0).all()
+        assert ((b1 - b0)[:N][share < tgt - 1e-12] > 0).all()
+    # at rest exactly when every FFN expert sits at its target share
+    N, K, T, K_e = 4, 2, 8, 1.0
+    counts = np.array([2, 2, 2, 2, 5, 3])
+    b1 = orc.bias_update(np.zeros(6), counts, N, K, K_e, 0.3, T)
+    assert (b1 == 0).all()
+
+
+def check_bf16_decode(orc):
+    bits = np.array([0x3F80, 0xC000, 0x3F81, 0x7F7F, 0x0001, 0x8000, 0x4049], dtype=np.uint16)
+    want = [1.0, -2.0, 1.0 + 2.0 ** -7, (2 - 2.0 ** -7) * 2.0 ** 127, 2.0 ** -133, -0.0,
+            3.140625]
+    got = orc.bf16_bits_to_f64(bits)
+    assert list(got) == want
+    assert math.copysign(1.0, got[5]) == -1.0
+
+
+ALL_CHECKS = [check_worked_tiny_layer, check_worked_swiglu, check_worked_bias_update,
+              check_worked_zero_experts, check_softmax_closed_forms, check_topk_brute_force,
+              check_dense_reduction, check_all_zero_experts_fixed_point,
+              check_k_equals_e_fixed_point, check_permutation_invariants,
+              check_bias_update_closed_form, check_bf16_decode]

@@ -1,0 +1,133 @@
+"""Plant plausible mistakes in the CPU oracle and check that the pins catch each one.
+
+Every mutation patches one function of the oracle module (on the CPU only)
+and the test passes when at least one pin of ``oracle_pins`` fails.
+"""
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as orc
+from tests import oracle_pins
+
+
+def _mut_gate_renormalised(mp):
+    real = orc.gates
+
+    def gates(probs, idx):
+        g = real(probs, idx)
+        return g / g.sum(axis=1, keepdims=True)
+    mp.setattr(orc, "gates", gates)
+
+
+def _mut_combine_drops_zero_term(mp):
+    real = orc.combine
+
+    def combine(x, y_perm, idx, g, slot_pos, N, gamma=1.0):
+        g2 = np.where(idx >= N, 0.0, g)
+        return real(x, y_perm, idx, g2, slot_pos, N, gamma)
+    mp.setattr(orc, "combine", combine)
+
+
+def _mut_bias_sign(mp):
+    real = orc.bias_update
+
+    def bias_update(bias, counts, N, K, K_e, mu, T_all):
+        return real(bias, counts, N, K, K_e, -mu, T_all)
+    mp.setattr(orc, "bias_update", bias_update)
+
+
+def _mut_bias_updates_zero_experts(mp):
+    def bias_update(bias, counts, N, K, K_e, mu, T_all):
+        b = np.asarray(bias, dtype=np.float64).copy()
+        E = len(b)
+        b += mu * (K_e / (K * N) - np.asarray(counts[:E], dtype=np.float64) / (K * T_all))
+        return b
+    mp.setattr(orc, "bias_update", bias_update)
+
+
+def _mut_tie_to_high_index(mp):
+    def biased_topk(probs, bias, K):
+        T, E = probs.shape
+        s = probs + np.asarray(bias)[None, :]
+        order = np.argsort(-s[:, ::-1], axis=1, kind="stable")
+        order = E - 1 - order
+        idx = order[:, :K].astype(np.int32)
+        rows = np.arange(T)
+        margin = (s[rows, order[:, K - 1]] - s[rows, order[:, K]]) if K < E else np.full(T, np.inf)
+        return idx, margin
+    mp.setattr(orc, "biased_topk", biased_topk)
+
+
+def _mut_select_by_unbiased(mp):
+    real = orc.biased_topk
+
+    def biased_topk(probs, bias, K):
+        return real(probs, np.zeros_like(np.asarray(bias, dtype=np.float64)), K)
+    mp.setattr(orc, "biased_topk", biased_topk)
+
+
+def _mut_no_silu(mp):
+    mp.setattr(orc, "silu", lambda a: a)
+
+
+def _mut_swapped_gate_up(mp):
+    def expert_ffn(x_rows, w1, w3, w2):
+        a = x_rows @ np.asarray(w3, dtype=np.float64).T
+        u = x_rows @ np.asarray(w1, dtype=np.float64).T
+        return (orc.silu(a) * u) @ np.asarray(w2, dtype=np.float64).T
+
+    def expert_hidden(x_rows, w1, w3):
+        return orc.silu(x_rows @ np.asarray(w3).T) * (x_rows @ np.asarray(w1).T)
+    mp.setattr(orc, "expert_ffn", expert_ffn)
+    mp.setattr(orc, "expert_hidden", expert_hidden)
+
+
+def _mut_descending_tokens(mp):
+    real = orc.canonical_permutation
+
+    def canonical_permutation(idx, N):
+        off, row_token, slot_pos = real(idx, N)
+        rt = row_token.copy()
+        sp = slot_pos.copy()
+        for e in range(N):
+            lo, hi = off[e], off[e + 1]
+            rt[lo:hi] = row_token[lo:hi][::-1]
+            mask = (idx == e)
+            sp[mask] = lo + hi - 1 - slot_pos[mask]
+        return off, rt, sp
+    mp.setattr(orc, "canonical_permutation", canonical_permutation)
+
+
+def _mut_softmax_no_max_shift_wrong_axis(mp):
+    def softmax_rows(logits):
+        e = np.exp(logits)
+        return e / e.sum(axis=0, keepdims=True)
+    mp.setattr(orc, "softmax_rows", softmax_rows)
+
+
+def _mut_gamma_only_ffn(mp):
+    real = orc.combine
+
+    def combine(x, y_perm, idx, g, slot_pos, N, gamma=1.0):
+        full = real(x, y_perm, idx, g, slot_pos, N, gamma)
+        zm = np.where(idx >= N, g, 0.0).sum(axis=1)
+        return full - (gamma - 1.0) * zm[:, None] * np.asarray(x, dtype=np.float64)
+    mp.setattr(orc, "combine", combine)
+
+
+MUTATIONS = [_mut_gate_renormalised, _mut_combine_drops_zero_term, _mut_bias_sign,
+             _mut_bias_updates_zero_experts, _mut_tie_to_high_index, _mut_select_by_unbiased,
+             _mut_no_silu, _mut_swapped_gate_up, _mut_descending_tokens,
+             _mut_softmax_no_max_shift_wrong_axis, _mut_gamma_only_ffn]
+
+
+@pytest.mark.parametrize("mutate", MUTATIONS, ids=lambda m: m.__name__)
+def test_pins_catch_planted_mistake(mutate, monkeypatch):
+    mutate(monkeypatch)
+    failed = []
+    for check in oracle_pins.ALL_CHECKS:
+        try:
+            check(orc)
+        except Exception:  # an assertion or a shape error both expose the mistake
+            failed.append(check.__name__)
+    assert failed, f"no pin caught {mutate.__name__}"
