@@ -1,0 +1,166 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE layer with zero-computation experts.
+ *
+ * The layer is the one of "LongCat-Flash Technical Report", §2.1
+ * (zero-computation experts), Eq. (1):
+ *
+ *     MoE(x_t) = gamma * sum_{i=1}^{N+Z} g_i E_i(x_t)
+ *     g_i      = R(x_t)_i  if R(x_t)_i + b_i is among the K largest of
+ *                {R(x_t)_j + b_j}, else 0              (R: softmax router)
+ *     E_i(x_t) = FFN_i(x_t) for i <= N;  x_t for N < i <= N+Z
+ *
+ * with the expert-bias budget control of §2.1.1, Eq. (2), and the optional
+ * output scale gamma of §2.3.2, Eq. (8) (1 unless the caller sets it).
+ * FFN_i is a SwiGLU expert: FFN(x) = W2 (SiLU(W1 x) * (W3 x)).
+ *
+ * The forward pass is four calls on one stream:
+ *     moe_route -> moe_permute -> moe_expert_ffn -> moe_combine
+ * and moe_bias_update runs beside it once per step.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Every pointer argument except the moe_shape pointer is a DEVICE pointer
+ *    owned by the caller.  The library allocates no device memory and keeps no
+ *    device state between calls; scratch space is the caller's workspace.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *    is the legacy default stream).  No call synchronises the host except
+ *    moe_get_device_status.
+ *  - Row-major layouts throughout.  Weights use the out-features x in-features
+ *    layout of a linear layer: w_router [E, d], w1/w3 [N, I, d], w2 [N, d, I].
+ *  - dtype MOE_F32: x, weights, x_perm, y_perm, out are float32.
+ *    dtype MOE_BF16: they are bfloat16; accumulation is always float32,
+ *    softmax and gates are float32, intermediates h and y_perm are rounded to
+ *    bf16 with round-to-nearest-even.
+ *  - Host-side validation returns an error code and never aborts; the message
+ *    is available from moe_last_error() on the calling thread.
+ *  - Errors found on the device (an expert index out of range, inconsistent
+ *    counts, a pipeline wait that ran out of iterations) set bits in the
+ *    workspace status word and never trap; moe_get_device_status reads them.
+ *  - Buffers whose size depends on routing (x_perm, y_perm, h) are sized for
+ *    the worst case R <= T*K rows, so no call needs a device-to-host sync.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* T tokens, d hidden size, N FFN experts, Z zero-computation experts,
+ * K experts per token (1 <= K <= N+Z <= 1024), I expert intermediate size. */
+typedef struct {
+  int32_t T, d, N, Z, K, I;
+  int32_t dtype; /* moe_dtype */
+} moe_shape;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid but not supported (e.g. bf16 d % 64 != 0) */
+  MOE_ERR_WORKSPACE = 3,     /* workspace too small */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime call failed */
+  MOE_ERR_DEVICE_STATUS = 5  /* moe_get_device_status found device-side errors */
+} moe_status;
+
+/* Bits of the device status word. */
+#define MOE_DEV_BAD_EXPERT_INDEX 0x1u  /* topk_idx entry outside [0, N+Z) (ignored) */
+#define MOE_DEV_COUNT_MISMATCH 0x2u    /* counts[] disagrees with topk_idx */
+#define MOE_DEV_BAD_OFFSETS 0x4u       /* offsets not monotone or beyond T*K */
+#define MOE_DEV_PIPELINE_TIMEOUT 0x8u  /* a bounded wait inside a GEMM gave up */
+
+/* Bytes of device workspace the calls below need for this shape.  One
+ * workspace may serve every call of a layer instance, used in stream order.
+ * Returns 0 for an invalid shape. */
+size_t moe_workspace_bytes(const moe_shape* shape);
+
+/* Clears the workspace status word.  Call once after allocating it. */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Router and selection: §2.1, Eq. (1).
+ *   logits[t, i] = sum_j x[t, j] w_router[i, j] (+ logit_offset[t, i])   (fp32)
+ *   R[t, :]      = softmax(logits[t, :]) over all E = N+Z experts          (fp32)
+ *   topk_idx[t, 0..K) = the K experts with the largest R + bias, in order of
+ *                       that score descending, ties to the lower index
+ *   topk_gate[t, k]   = R[t, topk_idx[t, k]]   (unbiased, not renormalised)
+ *   counts[i]         = number of (t, k) with topk_idx[t, k] == i   (T_i of Eq. (2))
+ *   n_ffn[t]          = number of k with topk_idx[t, k] < N
+ * x [T, d] (dtype), w_router [E, d] (dtype), bias [E] fp32,
+ * logit_offset [T, E] fp32 or NULL (an additive input, used by tests and
+ * skewed-routing workloads), topk_idx [T, K] int32, topk_gate [T, K] fp32,
+ * counts [E] int32, n_ffn [T] uint8, probs_out [T, E] fp32 or NULL.
+ * bias entries must be finite. */
+moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router,
+                     const float* bias, const float* logit_offset, int32_t* topk_idx,
+                     float* topk_gate, int32_t* counts, uint8_t* n_ffn, float* probs_out,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Dispatch to the FFN experts only (zero-computation experts get no rows).
+ *   offsets[e] = sum_{e' < e} counts[e'] over FFN experts, e in [0, N];
+ *                offsets[N] = R, the number of routed FFN rows.
+ *   Rows of expert e are offsets[e] .. offsets[e+1]-1, in ascending token order.
+ *   row_token[r] = token of row r (r < R);  slot_pos[t, k] = row of slot (t, k),
+ *   or -1 when topk_idx[t, k] >= N;  x_perm[r, :] = x[row_token[r], :].
+ * topk_idx [T, K] int32, counts [E] int32 (checked against topk_idx; a mismatch
+ * sets MOE_DEV_COUNT_MISMATCH and topk_idx wins), offsets [N+1] int32,
+ * row_token [T*K] int32, slot_pos [T, K] int32, x_perm [T*K, d] (dtype). */
+moe_status moe_permute(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                       const int32_t* counts, int32_t* offsets, int32_t* row_token,
+                       int32_t* slot_pos, void* x_perm, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* First half of the SwiGLU experts on the routed rows:
+ *   h[r, :] = SiLU(x_perm[r, :] W1_e^T) * (x_perm[r, :] W3_e^T)   for rows r of expert e.
+ * x_perm [T*K, d], w1/w3 [N, I, d], offsets [N+1] (from moe_permute),
+ * h [T*K, I] (dtype).  Rows >= offsets[N] are not written. */
+moe_status moe_expert_gate_up(const moe_shape* shape, const void* x_perm, const void* w1,
+                              const void* w3, const int32_t* offsets, void* h, void* ws,
+                              size_t ws_bytes, void* stream);
+
+/* Second half: y_perm[r, :] = h[r, :] W2_e^T.  h [T*K, I], w2 [N, d, I],
+ * y_perm [T*K, d] (dtype). */
+moe_status moe_expert_down(const moe_shape* shape, const void* h, const void* w2,
+                           const int32_t* offsets, void* y_perm, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Both halves with h kept in the workspace:
+ *   y_perm[r, :] = FFN_e(x_perm[r, :]) for each routed row r of expert e. */
+moe_status moe_expert_ffn(const moe_shape* shape, const void* x_perm, const void* w1,
+                          const void* w3, const void* w2, const int32_t* offsets,
+                          void* y_perm, void* ws, size_t ws_bytes, void* stream);
+
+/* Weighted sum of Eq. (1) with the zero-computation experts folded in:
+ *   out[t, :] = gamma * ( sum_{k: idx < N} gate[t,k] * y_perm[slot_pos[t,k], :]
+ *                         + (sum_{k: idx >= N} gate[t,k]) * x[t, :] )
+ * accumulated in fp32 in this fixed order (FFN slots in k order, then the
+ * identity term).  x [T, d], y_perm [T*K, d], out [T, d] (dtype). */
+moe_status moe_combine(const moe_shape* shape, const void* x, const void* y_perm,
+                       const int32_t* topk_idx, const float* topk_gate,
+                       const int32_t* slot_pos, float gamma, void* out, void* stream);
+
+/* Computation-budget control: §2.1.1, Eq. (2), in place on bias [N+Z] fp32:
+ *   bias[i] += mu * (K_e/K * 1/N - counts[i]/(K * T_all))   for i < N,
+ *   bias[i] unchanged for the Z zero-computation experts (i >= N).
+ * counts [N+Z] int32 are the global-batch counts T_i, T_all the global-batch
+ * token count.  The increment is formed in fp64 and the sum rounded once to
+ * fp32. */
+moe_status moe_bias_update(int32_t N, int32_t Z, const int32_t* counts, int64_t T_all,
+                           int32_t K, float K_e, float mu, float* bias, void* stream);
+
+/* Synchronises `stream`, reads the workspace status word into *status_out
+ * (may be NULL) and clears it.  Returns MOE_ERR_DEVICE_STATUS when it was
+ * non-zero. */
+moe_status moe_get_device_status(void* ws, void* stream, uint32_t* status_out);
+
+/* Message of the last error on the calling thread ("" if none). */
+const char* moe_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

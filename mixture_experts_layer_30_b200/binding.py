@@ -1,0 +1,232 @@
+"""ctypes binding of libmoe_b200.so: argument marshalling only.
+
+Every step of the layer runs in the CUDA library; this module checks tensor
+placement/dtype/contiguity, passes raw device pointers and the current torch
+stream, and turns status codes into exceptions.  There is no CPU fallback: if
+the library is missing, every call raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+STATUS_NAMES = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+                3: "MOE_ERR_WORKSPACE", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_STATUS"}
+DEV_BAD_EXPERT_INDEX, DEV_COUNT_MISMATCH, DEV_BAD_OFFSETS, DEV_PIPELINE_TIMEOUT = 1, 2, 4, 8
+
+# Every symbol of include/moe.h, with its ctypes signature.
+_vp, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, \
+    ctypes.c_size_t
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("Z", ctypes.c_int32), ("K", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("dtype", ctypes.c_int32)]
+
+
+_SP = ctypes.POINTER(Shape)
+SIGNATURES = {
+    "moe_workspace_bytes": (_sz, [_SP]),
+    "moe_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
+    "moe_route": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_gate_up": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_down": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_ffn": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_combine": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp]),
+    "moe_bias_update": (ctypes.c_int, [_i32, _i32, _vp, _i64, _i32, _f32, _f32, _vp, _vp]),
+    "moe_get_device_status": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "moe_last_error": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+class MoEError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+def lib():
+    """The loaded CUDA library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library {LIB_PATH} is missing; build it with "
+                               "`python -m mixture_experts_layer_30_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _check(code):
+    if code != 0:
+        raise MoEError(code, lib().moe_last_error().decode())
+
+
+def make_shape(T, d, N, Z, K, I, dtype) -> Shape:
+    code = {"f32": MOE_F32, "bf16": MOE_BF16, torch.float32: MOE_F32,
+            torch.bfloat16: MOE_BF16}[dtype]
+    return Shape(T, d, N, Z, K, I, code)
+
+
+def shape_of(cfg, T=None) -> Shape:
+    return make_shape(cfg.T if T is None else T, cfg.d, cfg.N, cfg.Z, cfg.K, cfg.I, cfg.dtype)
+
+
+def torch_dtype(shape: Shape):
+    return torch.bfloat16 if shape.dtype == MOE_BF16 else torch.float32
+
+
+def _p(t, dtype=None, name="tensor"):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_bytes(shape: Shape) -> int:
+    n = lib().moe_workspace_bytes(ctypes.byref(shape))
+    if n == 0:
+        raise MoEError(1, "invalid shape")
+    return n
+
+
+def new_workspace(shape: Shape, device="cuda", stream=None) -> torch.Tensor:
+    ws = torch.empty(workspace_bytes(shape), dtype=torch.uint8, device=device)
+    _check(lib().moe_workspace_init(_p(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def route(shape, x, w_router, bias, ws, topk_idx, topk_gate, counts, n_ffn,
+          logit_offset=None, probs_out=None, stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_route(ctypes.byref(shape), _p(x, dt, "x"), _p(w_router, dt, "w_router"),
+                           _p(bias, torch.float32, "bias"),
+                           _p(logit_offset, torch.float32, "logit_offset"),
+                           _p(topk_idx, torch.int32, "topk_idx"),
+                           _p(topk_gate, torch.float32, "topk_gate"),
+                           _p(counts, torch.int32, "counts"), _p(n_ffn, torch.uint8, "n_ffn"),
+                           _p(probs_out, torch.float32, "probs_out"), _p(ws), ws.numel(),
+                           _stream(stream)))
+
+
+def permute(shape, x, topk_idx, counts, offsets, row_token, slot_pos, x_perm, ws, stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_permute(ctypes.byref(shape), _p(x, dt, "x"),
+                             _p(topk_idx, torch.int32, "topk_idx"),
+                             _p(counts, torch.int32, "counts"),
+                             _p(offsets, torch.int32, "offsets"),
+                             _p(row_token, torch.int32, "row_token"),
+                             _p(slot_pos, torch.int32, "slot_pos"), _p(x_perm, dt, "x_perm"),
+                             _p(ws), ws.numel(), _stream(stream)))
+
+
+def expert_gate_up(shape, x_perm, w1, w3, offsets, h, ws, stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_expert_gate_up(ctypes.byref(shape), _p(x_perm, dt, "x_perm"),
+                                    _p(w1, dt, "w1"), _p(w3, dt, "w3"),
+                                    _p(offsets, torch.int32, "offsets"), _p(h, dt, "h"),
+                                    _p(ws), ws.numel(), _stream(stream)))
+
+
+def expert_down(shape, h, w2, offsets, y_perm, ws, stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_expert_down(ctypes.byref(shape), _p(h, dt, "h"), _p(w2, dt, "w2"),
+                                 _p(offsets, torch.int32, "offsets"),
+                                 _p(y_perm, dt, "y_perm"), _p(ws), ws.numel(),
+                                 _stream(stream)))
+
+
+def expert_ffn(shape, x_perm, w1, w3, w2, offsets, y_perm, ws, stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_expert_ffn(ctypes.byref(shape), _p(x_perm, dt, "x_perm"), _p(w1, dt, "w1"),
+                                _p(w3, dt, "w3"), _p(w2, dt, "w2"),
+                                _p(offsets, torch.int32, "offsets"), _p(y_perm, dt, "y_perm"),
+                                _p(ws), ws.numel(), _stream(stream)))
+
+
+def combine(shape, x, y_perm, topk_idx, topk_gate, slot_pos, gamma, out, stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_combine(ctypes.byref(shape), _p(x, dt, "x"), _p(y_perm, dt, "y_perm"),
+                             _p(topk_idx, torch.int32, "topk_idx"),
+                             _p(topk_gate, torch.float32, "topk_gate"),
+                             _p(slot_pos, torch.int32, "slot_pos"), float(gamma),
+                             _p(out, dt, "out"), _stream(stream)))
+
+
+def bias_update(N, Z, counts, T_all, K, K_e, mu, bias, stream=None):
+    _check(lib().moe_bias_update(N, Z, _p(counts, torch.int32, "counts"), int(T_all), K,
+                                 float(K_e), float(mu), _p(bias, torch.float32, "bias"),
+                                 _stream(stream)))
+
+
+def device_status(ws, stream=None) -> int:
+    """Synchronises, returns the workspace status bits and clears them."""
+    v = ctypes.c_uint32(0)
+    code = lib().moe_get_device_status(_p(ws), _stream(stream), ctypes.byref(v))
+    if code not in (0, 5):
+        _check(code)
+    return int(v.value)
+
+
+class LayerBuffers:
+    """Every buffer one forward pass of a shape needs, allocated once by torch."""
+
+    def __init__(self, shape: Shape, device="cuda", with_probs=False):
+        T, K, d, I, E = shape.T, shape.K, shape.d, shape.I, shape.N + shape.Z
+        dt = torch_dtype(shape)
+        R = max(T * K, 1)
+        kw = dict(device=device)
+        self.shape = shape
+        self.ws = new_workspace(shape, device)
+        self.topk_idx = torch.empty((T, K), dtype=torch.int32, **kw)
+        self.topk_gate = torch.empty((T, K), dtype=torch.float32, **kw)
+        self.counts = torch.empty(E, dtype=torch.int32, **kw)
+        self.n_ffn = torch.empty(T, dtype=torch.uint8, **kw)
+        self.probs = torch.empty((T, E), dtype=torch.float32, **kw) if with_probs else None
+        self.offsets = torch.empty(shape.N + 1, dtype=torch.int32, **kw)
+        self.row_token = torch.empty(R, dtype=torch.int32, **kw)
+        self.slot_pos = torch.empty((T, K), dtype=torch.int32, **kw)
+        self.x_perm = torch.empty((R, d), dtype=dt, **kw)
+        self.h = torch.empty((R, I), dtype=dt, **kw)
+        self.y_perm = torch.empty((R, d), dtype=dt, **kw)
+        self.out = torch.empty((T, d), dtype=dt, **kw)
+
+
+def forward(buf: LayerBuffers, x, w_router, w1, w3, w2, bias, gamma=1.0, logit_offset=None,
+            stream=None, split_ffn=False):
+    """route -> permute -> expert FFN -> combine; returns buf.out."""
+    s = buf.shape
+    route(s, x, w_router, bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts, buf.n_ffn,
+          logit_offset=logit_offset, probs_out=buf.probs, stream=stream)
+    permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
+            buf.x_perm, buf.ws, stream=stream)
+    if split_ffn:
+        expert_gate_up(s, buf.x_perm, w1, w3, buf.offsets, buf.h, buf.ws, stream=stream)
+        expert_down(s, buf.h, w2, buf.offsets, buf.y_perm, buf.ws, stream=stream)
+    else:
+        expert_ffn(s, buf.x_perm, w1, w3, w2, buf.offsets, buf.y_perm, buf.ws, stream=stream)
+    combine(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, gamma, buf.out,
+            stream=stream)
+    return buf.out

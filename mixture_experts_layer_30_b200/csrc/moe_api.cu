@@ -1,0 +1,425 @@
+// C ABI of the MoE layer with zero-computation experts (declared in moe.h):
+// argument validation, workspace layout and kernel launches.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "moe.h"
+#include "common.cuh"
+#include "route.cuh"
+#include "permute.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+#include "combine.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+moe_status fail(moe_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+moe_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return MOE_OK;
+}
+
+#define MOE_TRY(expr)                 \
+  do {                                \
+    moe_status _s = (expr);           \
+    if (_s != MOE_OK) return _s;      \
+  } while (0)
+
+size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+struct WsLayout {
+  size_t status, logits, route_hist, perm_hist, perm_base, h, total;
+};
+
+int elem_bytes(const moe_shape& s) { return s.dtype == MOE_BF16 ? 2 : 4; }
+int route_ctas(const moe_shape& s) { return (s.T + moe::kRouteTokensPerCta - 1) / moe::kRouteTokensPerCta; }
+int perm_chunks(const moe_shape& s) { return (s.T + moe::kPermChunk - 1) / moe::kPermChunk; }
+
+moe_status validate_shape(const moe_shape* sp) {
+  if (!sp) return fail(MOE_ERR_INVALID_ARG, "shape is NULL");
+  const moe_shape& s = *sp;
+  if (s.dtype != MOE_F32 && s.dtype != MOE_BF16)
+    return fail(MOE_ERR_INVALID_ARG, "dtype %d is neither MOE_F32 nor MOE_BF16", s.dtype);
+  if (s.T < 0 || s.d < 1 || s.N < 1 || s.Z < 0 || s.I < 1)
+    return fail(MOE_ERR_INVALID_ARG, "bad shape T=%d d=%d N=%d Z=%d I=%d", s.T, s.d, s.N, s.Z,
+                s.I);
+  const int E = s.N + s.Z;
+  if (E > moe::kMaxExperts)
+    return fail(MOE_ERR_UNSUPPORTED, "N+Z=%d exceeds %d experts", E, moe::kMaxExperts);
+  if (s.K < 1 || s.K > E) return fail(MOE_ERR_INVALID_ARG, "K=%d outside [1, N+Z=%d]", s.K, E);
+  if ((long long)s.T * s.K > 0x7fffffffLL)
+    return fail(MOE_ERR_UNSUPPORTED, "T*K=%lld routed rows exceed int32", (long long)s.T * s.K);
+  const int vec = 16 / elem_bytes(s);
+  if (s.d % vec)
+    return fail(MOE_ERR_UNSUPPORTED, "d=%d must be a multiple of %d for 16-byte rows", s.d, vec);
+  return MOE_OK;
+}
+
+WsLayout layout_of(const moe_shape& s) {
+  WsLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  const size_t E = (size_t)s.N + s.Z;
+  L.status = take(256);
+  L.logits = take((size_t)s.T * E * 4);
+  L.route_hist = take((size_t)route_ctas(s) * E * 4);
+  L.perm_hist = take((size_t)perm_chunks(s) * s.N * 4);
+  L.perm_base = take((size_t)perm_chunks(s) * s.N * 4);
+  L.h = take((size_t)s.T * s.K * s.I * elem_bytes(s));
+  L.total = off;
+  return L;
+}
+
+moe_status check_ws(const moe_shape& s, void* ws, size_t ws_bytes, WsLayout* L) {
+  *L = layout_of(s);
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % 256)
+    return fail(MOE_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (ws_bytes < L->total)
+    return fail(MOE_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, L->total);
+  return MOE_OK;
+}
+
+moe_status need(const void* p, const char* name, size_t align = 1) {
+  if (!p) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", name);
+  if (reinterpret_cast<uintptr_t>(p) % align)
+    return fail(MOE_ERR_INVALID_ARG, "%s must be %zu-byte aligned", name, align);
+  return MOE_OK;
+}
+
+template <typename T> T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// --- launches ---------------------------------------------------------------
+
+template <int VPL>
+void launch_topk(dim3 grid, cudaStream_t st, const float* logits, const float* bias, int T,
+                 int E, int N, int K, int32_t* idx, float* gate, uint8_t* nffn, float* probs,
+                 int32_t* hist) {
+  moe::softmax_topk_kernel<VPL><<<grid, 256, 0, st>>>(logits, bias, T, E, N, K, idx, gate,
+                                                      nffn, probs, hist);
+}
+
+template <typename T>
+moe_status route_impl(const moe_shape& s, const void* x, const void* w, const float* bias,
+                      const float* off, int32_t* idx, float* gate, int32_t* counts,
+                      uint8_t* nffn, float* probs, void* ws, const WsLayout& L,
+                      cudaStream_t st) {
+  const int E = s.N + s.Z;
+  float* logits = at<float>(ws, L.logits);
+  int32_t* hist = at<int32_t>(ws, L.route_hist);
+  if (s.T > 0) {
+    if (s.dtype == MOE_BF16 && moe::tc::router_supported(s)) {
+      MOE_TRY(moe::tc::launch_router_gemm(s, x, w, off, logits, sm_count(), st, g_err,
+                                          sizeof(g_err)));
+    } else {
+      dim3 g((E + moe::kRgBN - 1) / moe::kRgBN, (s.T + moe::kRgBM - 1) / moe::kRgBM);
+      moe::router_gemm_simt_kernel<T><<<g, 256, 0, st>>>(
+          static_cast<const T*>(x), static_cast<const T*>(w), off, logits, s.T, E, s.d);
+    }
+    MOE_TRY(check_launch("router gemm"));
+    const int vpl = (E + 31) / 32;
+    dim3 g(route_ctas(s));
+    if (vpl <= 1) launch_topk<1>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
+    else if (vpl <= 2) launch_topk<2>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
+    else if (vpl <= 3) launch_topk<3>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
+    else if (vpl <= 4) launch_topk<4>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
+    else if (vpl <= 8) launch_topk<8>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
+    else if (vpl <= 16) launch_topk<16>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
+    else if (vpl <= 24) launch_topk<24>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
+    else launch_topk<32>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
+    MOE_TRY(check_launch("softmax/top-K"));
+  }
+  moe::reduce_hist_kernel<<<(E + 255) / 256, 256, 0, st>>>(hist, route_ctas(s), E, counts);
+  return check_launch("count reduce");
+}
+
+bool g_rank_attr_set[64] = {};
+
+template <typename T>
+moe_status permute_impl(const moe_shape& s, const void* x, const int32_t* idx,
+                        const int32_t* counts, int32_t* offsets, int32_t* row_token,
+                        int32_t* slot_pos, void* x_perm, void* ws, const WsLayout& L,
+                        cudaStream_t st) {
+  const int E = s.N + s.Z, nch = perm_chunks(s);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  int32_t* chist = at<int32_t>(ws, L.perm_hist);
+  int32_t* cbase = at<int32_t>(ws, L.perm_base);
+  if (nch > 0) {
+    moe::chunk_hist_kernel<<<nch, 256, s.N * sizeof(int), st>>>(idx, s.T, s.K, s.N, E, chist,
+                                                                 status);
+    MOE_TRY(check_launch("dispatch histogram"));
+  }
+  moe::perm_scan_kernel<<<1, 1024, 0, st>>>(chist, nch, s.N, counts, offsets, cbase, status);
+  MOE_TRY(check_launch("dispatch scan"));
+  if (nch > 0) {
+    const size_t smem = (size_t)16 * s.N * sizeof(uint32_t);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (smem > 48 * 1024 && dev < 64 && !g_rank_attr_set[dev]) {
+      cudaFuncSetAttribute(moe::perm_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+      g_rank_attr_set[dev] = true;
+    }
+    moe::perm_rank_kernel<<<nch, 256, smem, st>>>(idx, s.T, s.K, s.N, E, cbase, row_token,
+                                                   slot_pos);
+    MOE_TRY(check_launch("dispatch rank"));
+    moe::gather_kernel<T><<<(s.T + 7) / 8, 256, 0, st>>>(
+        static_cast<const T*>(x), slot_pos, s.T, s.K, s.d, static_cast<T*>(x_perm));
+    MOE_TRY(check_launch("dispatch gather"));
+  }
+  return MOE_OK;
+}
+
+template <typename T, bool kGated>
+moe_status grouped_simt(const moe_shape& s, const void* A, const void* B0, const void* B1,
+                        const int32_t* offsets, int n_out, int k_dim, void* C,
+                        uint32_t* status, cudaStream_t st) {
+  const long long max_rows = (long long)s.T * s.K;
+  const long long ncol = (n_out + moe::kSgBN - 1) / moe::kSgBN;
+  const long long max_chunks = s.N + (max_rows + moe::kSgBM - 1) / moe::kSgBM;
+  long long grid = max_chunks * ncol;
+  const long long cap = (long long)sm_count() * 8;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  moe::grouped_gemm_simt_kernel<T, kGated><<<(int)grid, 256, 0, st>>>(
+      static_cast<const T*>(A), static_cast<const T*>(B0), static_cast<const T*>(B1), offsets,
+      s.N, (int)max_rows, n_out, k_dim, static_cast<T*>(C), status);
+  return check_launch(kGated ? "gate/up grouped gemm" : "down grouped gemm");
+}
+
+moe_status gate_up_impl(const moe_shape& s, const void* x_perm, const void* w1, const void* w3,
+                        const int32_t* offsets, void* h, uint32_t* status, cudaStream_t st) {
+  if (s.T == 0) return MOE_OK;
+  if (s.dtype == MOE_BF16) {
+    if (moe::tc::ffn_supported(s))
+      return moe::tc::launch_gate_up(s, x_perm, w1, w3, offsets, h, status, sm_count(), st,
+                                     g_err, sizeof(g_err));
+    return grouped_simt<__nv_bfloat16, true>(s, x_perm, w1, w3, offsets, s.I, s.d, h, status, st);
+  }
+  return grouped_simt<float, true>(s, x_perm, w1, w3, offsets, s.I, s.d, h, status, st);
+}
+
+moe_status down_impl(const moe_shape& s, const void* h, const void* w2, const int32_t* offsets,
+                     void* y_perm, uint32_t* status, cudaStream_t st) {
+  if (s.T == 0) return MOE_OK;
+  if (s.dtype == MOE_BF16) {
+    if (moe::tc::ffn_supported(s))
+      return moe::tc::launch_down(s, h, w2, offsets, y_perm, status, sm_count(), st, g_err,
+                                  sizeof(g_err));
+    return grouped_simt<__nv_bfloat16, false>(s, h, w2, nullptr, offsets, s.d, s.I, y_perm,
+                                              status, st);
+  }
+  return grouped_simt<float, false>(s, h, w2, nullptr, offsets, s.d, s.I, y_perm, status, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_shape* shape) {
+  if (validate_shape(shape) != MOE_OK) return 0;
+  return layout_of(*shape).total;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  if (!ws || ws_bytes < 256) return fail(MOE_ERR_INVALID_ARG, "workspace NULL or < 256 bytes");
+  cudaError_t e = cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router,
+                     const float* bias, const float* logit_offset, int32_t* topk_idx,
+                     float* topk_gate, int32_t* counts, uint8_t* n_ffn, float* probs_out,
+                     void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  WsLayout L;
+  MOE_TRY(check_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(counts, "counts", 4));
+  MOE_TRY(need(bias, "bias", 4));
+  MOE_TRY(need(w_router, "w_router", 16));
+  if (s.T > 0) {
+    MOE_TRY(need(x, "x", 16));
+    MOE_TRY(need(topk_idx, "topk_idx", 4));
+    MOE_TRY(need(topk_gate, "topk_gate", 4));
+    MOE_TRY(need(n_ffn, "n_ffn"));
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.dtype == MOE_BF16)
+    return route_impl<__nv_bfloat16>(s, x, w_router, bias, logit_offset, topk_idx, topk_gate,
+                                     counts, n_ffn, probs_out, ws, L, st);
+  return route_impl<float>(s, x, w_router, bias, logit_offset, topk_idx, topk_gate, counts,
+                           n_ffn, probs_out, ws, L, st);
+}
+
+moe_status moe_permute(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                       const int32_t* counts, int32_t* offsets, int32_t* row_token,
+                       int32_t* slot_pos, void* x_perm, void* ws, size_t ws_bytes,
+                       void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  WsLayout L;
+  MOE_TRY(check_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(offsets, "offsets", 4));
+  if (s.T > 0) {
+    MOE_TRY(need(x, "x", 16));
+    MOE_TRY(need(topk_idx, "topk_idx", 4));
+    MOE_TRY(need(row_token, "row_token", 4));
+    MOE_TRY(need(slot_pos, "slot_pos", 4));
+    MOE_TRY(need(x_perm, "x_perm", 16));
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.dtype == MOE_BF16)
+    return permute_impl<__nv_bfloat16>(s, x, topk_idx, counts, offsets, row_token, slot_pos,
+                                       x_perm, ws, L, st);
+  return permute_impl<float>(s, x, topk_idx, counts, offsets, row_token, slot_pos, x_perm, ws,
+                             L, st);
+}
+
+moe_status moe_expert_gate_up(const moe_shape* shape, const void* x_perm, const void* w1,
+                              const void* w3, const int32_t* offsets, void* h, void* ws,
+                              size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  WsLayout L;
+  MOE_TRY(check_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(x_perm, "x_perm", 16));
+  MOE_TRY(need(w1, "w1", 16));
+  MOE_TRY(need(w3, "w3", 16));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(h, "h", 16));
+  return gate_up_impl(s, x_perm, w1, w3, offsets, h, at<uint32_t>(ws, L.status),
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_down(const moe_shape* shape, const void* h, const void* w2,
+                           const int32_t* offsets, void* y_perm, void* ws, size_t ws_bytes,
+                           void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  WsLayout L;
+  MOE_TRY(check_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(h, "h", 16));
+  MOE_TRY(need(w2, "w2", 16));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(y_perm, "y_perm", 16));
+  return down_impl(s, h, w2, offsets, y_perm, at<uint32_t>(ws, L.status),
+                   static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_ffn(const moe_shape* shape, const void* x_perm, const void* w1,
+                          const void* w3, const void* w2, const int32_t* offsets,
+                          void* y_perm, void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  WsLayout L;
+  MOE_TRY(check_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(x_perm, "x_perm", 16));
+  MOE_TRY(need(w1, "w1", 16));
+  MOE_TRY(need(w3, "w3", 16));
+  MOE_TRY(need(w2, "w2", 16));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(y_perm, "y_perm", 16));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* h = at<char>(ws, L.h);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  MOE_TRY(gate_up_impl(s, x_perm, w1, w3, offsets, h, status, st));
+  return down_impl(s, h, w2, offsets, y_perm, status, st);
+}
+
+moe_status moe_combine(const moe_shape* shape, const void* x, const void* y_perm,
+                       const int32_t* topk_idx, const float* topk_gate,
+                       const int32_t* slot_pos, float gamma, void* out, void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  if (s.T == 0) return MOE_OK;
+  MOE_TRY(need(x, "x", 16));
+  MOE_TRY(need(y_perm, "y_perm", 16));
+  MOE_TRY(need(topk_idx, "topk_idx", 4));
+  MOE_TRY(need(topk_gate, "topk_gate", 4));
+  MOE_TRY(need(slot_pos, "slot_pos", 4));
+  MOE_TRY(need(out, "out", 16));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int E = s.N + s.Z;
+  const int nvec = s.d * elem_bytes(s) / 16;
+  int threads = ((nvec + 31) / 32) * 32;
+  if (threads > 256) threads = 256;
+  const int max_rows = s.T * s.K;
+  if (s.dtype == MOE_BF16)
+    moe::combine_kernel<__nv_bfloat16><<<s.T, threads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y_perm),
+        topk_idx, topk_gate, slot_pos, s.K, s.N, E, s.d, max_rows, gamma,
+        static_cast<__nv_bfloat16*>(out), nullptr);
+  else
+    moe::combine_kernel<float><<<s.T, threads, 0, st>>>(
+        static_cast<const float*>(x), static_cast<const float*>(y_perm), topk_idx, topk_gate,
+        slot_pos, s.K, s.N, E, s.d, max_rows, gamma, static_cast<float*>(out), nullptr);
+  return check_launch("combine");
+}
+
+moe_status moe_bias_update(int32_t N, int32_t Z, const int32_t* counts, int64_t T_all,
+                           int32_t K, float K_e, float mu, float* bias, void* stream) {
+  g_err[0] = 0;
+  if (N < 1 || Z < 0 || N + Z > moe::kMaxExperts)
+    return fail(MOE_ERR_INVALID_ARG, "bad expert counts N=%d Z=%d", N, Z);
+  if (K < 1 || K > N + Z) return fail(MOE_ERR_INVALID_ARG, "K=%d outside [1, N+Z]", K);
+  if (T_all < 1) return fail(MOE_ERR_INVALID_ARG, "T_all=%lld must be >= 1", (long long)T_all);
+  MOE_TRY(need(counts, "counts", 4));
+  MOE_TRY(need(bias, "bias", 4));
+  moe::bias_update_kernel<<<(N + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      N, counts, (long long)T_all, K, K_e, mu, bias);
+  return check_launch("bias update");
+}
+
+moe_status moe_get_device_status(void* ws, void* stream, uint32_t* status_out) {
+  g_err[0] = 0;
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, sizeof(v), st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+  if (status_out) *status_out = v;
+  if (v) return fail(MOE_ERR_DEVICE_STATUS, "device status 0x%x", v);
+  return MOE_OK;
+}
+
+const char* moe_last_error(void) { return g_err; }
+
+}  // extern "C"

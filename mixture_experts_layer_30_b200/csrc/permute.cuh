@@ -1,0 +1,139 @@
+// Dispatch of routed slots to the N FFN experts (zero-computation experts get
+// no rows): LongCat-Flash Technical Report, §2.1 -- an identity expert needs
+// neither compute nor a copy of its token.
+//
+// Row layout: experts 0..N-1 in order, tokens ascending inside an expert.
+// Built without global atomics and without inter-CTA waits:
+//   1. chunk_hist_kernel  per 256-token chunk c: H[c][e] = #tokens of c routed to e
+//   2. scan_kernel        one CTA: offsets = exclusive scan of sum_c H[c][e];
+//                         base[c][e] = offsets[e] + sum_{c' < c} H[c'][e]
+//   3. rank_kernel        per chunk: row of (t, k) = base[c][e] + #earlier tokens of
+//                         the chunk routed to e (warp bitmaps + popcount)
+//   4. gather_kernel      one warp per token: x row copied to each of its rows.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+__global__ void __launch_bounds__(256)
+chunk_hist_kernel(const int32_t* __restrict__ topk_idx, int T, int K, int N, int E,
+                  int32_t* __restrict__ chunk_hist, uint32_t* status) {
+  extern __shared__ int sh_hist[];  // [N]
+  for (int e = threadIdx.x; e < N; e += blockDim.x) sh_hist[e] = 0;
+  __syncthreads();
+  const int t = blockIdx.x * kPermChunk + threadIdx.x;
+  if (t < T) {
+    for (int k = 0; k < K; ++k) {
+      int e = topk_idx[(size_t)t * K + k];
+      if (e < 0 || e >= E) { set_status(status, MOE_DEV_BAD_EXPERT_INDEX); continue; }
+      if (e < N) atomicAdd(&sh_hist[e], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x)
+    chunk_hist[(size_t)blockIdx.x * N + e] = sh_hist[e];
+}
+
+// One CTA of 1024 threads.
+__global__ void __launch_bounds__(1024)
+perm_scan_kernel(const int32_t* __restrict__ chunk_hist, int nchunks, int N,
+                 const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                 int32_t* __restrict__ chunk_base, uint32_t* status) {
+  __shared__ int scan_tmp[33];
+  __shared__ int tot_sh[kMaxExperts];
+  // per-expert totals (thread per expert, chunks in order)
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    int s = 0;
+    for (int c = 0; c < nchunks; ++c) s += chunk_hist[(size_t)c * N + e];
+    tot_sh[e] = s;
+    if (counts && counts[e] != s) set_status(status, MOE_DEV_COUNT_MISMATCH);
+  }
+  __syncthreads();
+  // exclusive scan over experts: each thread owns a run of consecutive experts
+  const int per = (N + blockDim.x - 1) / blockDim.x;
+  const int lo = min(N, (int)threadIdx.x * per), hi = min(N, lo + per);
+  int local = 0;
+  for (int e = lo; e < hi; ++e) local += tot_sh[e];
+  int run = block_exclusive_scan(local, scan_tmp, &scan_tmp[32]);
+  for (int e = lo; e < hi; ++e) {
+    offsets[e] = run;
+    int b = run;
+    for (int c = 0; c < nchunks; ++c) {
+      chunk_base[(size_t)c * N + e] = b;
+      b += chunk_hist[(size_t)c * N + e];
+    }
+    run += tot_sh[e];
+  }
+  if (threadIdx.x == 0) offsets[N] = scan_tmp[32];
+}
+
+// One CTA per 256-token chunk, one thread per token, 8 warps.
+// Shared: bits[8][N] (which lanes of warp w route to e), wbase[8][N].
+__global__ void __launch_bounds__(256)
+perm_rank_kernel(const int32_t* __restrict__ topk_idx, int T, int K, int N, int E,
+                 const int32_t* __restrict__ chunk_base, int32_t* __restrict__ row_token,
+                 int32_t* __restrict__ slot_pos) {
+  extern __shared__ uint32_t sh_rank[];
+  uint32_t* bits = sh_rank;                                   // [8][N]
+  int* wbase = reinterpret_cast<int*>(sh_rank + 8 * N);       // [8][N]
+  for (int i = threadIdx.x; i < 8 * N; i += blockDim.x) bits[i] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = blockIdx.x;
+  const int t = c * kPermChunk + threadIdx.x;
+  if (t < T) {
+    for (int k = 0; k < K; ++k) {
+      int e = topk_idx[(size_t)t * K + k];
+      if (e >= 0 && e < N) atomicOr(&bits[warp * N + e], 1u << lane);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    int b = chunk_base[(size_t)c * N + e];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      wbase[w * N + e] = b;
+      b += __popc(bits[w * N + e]);
+    }
+  }
+  __syncthreads();
+  if (t < T) {
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int k = 0; k < K; ++k) {
+      int e = topk_idx[(size_t)t * K + k];
+      int row = -1;
+      if (e >= 0 && e < N) {
+        row = wbase[warp * N + e] + __popc(bits[warp * N + e] & lt);
+        row_token[row] = t;
+      }
+      slot_pos[(size_t)t * K + k] = row;
+    }
+  }
+}
+
+// One warp per token; copies x[t] (16-byte vectors) to every row of the token.
+template <typename T>
+__global__ void __launch_bounds__(256)
+gather_kernel(const T* __restrict__ x, const int32_t* __restrict__ slot_pos, int ntok, int K,
+              int d, T* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= ntok) return;
+  const int nvec = d * (int)sizeof(T) / 16;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+  for (int kb = 0; kb < K; kb += 32) {
+    // rows of slots kb..kb+31 of this token (lane j holds slot kb+j's row)
+    int my_row = kb + lane < K ? slot_pos[(size_t)t * K + kb + lane] : -1;
+    uint32_t has = __ballot_sync(0xffffffffu, my_row >= 0);
+    while (has) {
+      int j = __ffs(has) - 1;
+      has &= has - 1;
+      int row = __shfl_sync(0xffffffffu, my_row, j);
+      uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * d);
+      for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    }
+  }
+}
+
+}  // namespace moe

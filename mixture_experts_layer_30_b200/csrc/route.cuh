@@ -1,0 +1,160 @@
+// Router and biased top-K selection: LongCat-Flash Technical Report, §2.1, Eq. (1).
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// --- router GEMM on CUDA cores ----------------------------------------------
+// logits[t, e] = sum_j x[t, j] * w[e, j] (+ offset[t, e]), fp32 accumulation.
+// 64x64 output tile per CTA, 256 threads, 4x4 outputs per thread.
+constexpr int kRgBM = 64, kRgBN = 64, kRgBK = 16;
+
+template <typename TIn>
+__global__ void __launch_bounds__(256)
+router_gemm_simt_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
+                        const float* __restrict__ offset, float* __restrict__ logits, int T,
+                        int E, int d) {
+  __shared__ float As[kRgBK][kRgBM + 4];
+  __shared__ float Bs[kRgBK][kRgBN + 4];
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int m0 = blockIdx.y * kRgBM, n0 = blockIdx.x * kRgBN;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < d; k0 += kRgBK) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int idx = tid + i * 256;       // 0..1023 over a 64 x 16 tile
+      int r = idx >> 4, c = idx & 15;
+      int gk = k0 + c;
+      int gm = m0 + r, gn = n0 + r;
+      As[c][r] = (gm < T && gk < d) ? Cvt<TIn>::to_f(x[(size_t)gm * d + gk]) : 0.f;
+      Bs[c][r] = (gn < E && gk < d) ? Cvt<TIn>::to_f(w[(size_t)gn * d + gk]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kRgBK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = As[kk][ty * 4 + i]; b[i] = Bs[kk][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int gm = m0 + ty * 4 + i;
+    if (gm >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      int gn = n0 + tx * 4 + j;
+      if (gn >= E) continue;
+      float v = acc[i][j];
+      if (offset) v += offset[(size_t)gm * E + gn];
+      logits[(size_t)gm * E + gn] = v;
+    }
+  }
+}
+
+// --- softmax + biased top-K + per-CTA histogram -----------------------------
+// One warp per token.  Lane l holds experts e = l + 32*j, j < VPL.
+// Selection key: (R_e + b_e) descending, then e ascending (lower index wins ties).
+template <int VPL>
+__global__ void __launch_bounds__(256)
+softmax_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
+                    int E, int N, int K, int32_t* __restrict__ topk_idx,
+                    float* __restrict__ topk_gate, uint8_t* __restrict__ n_ffn,
+                    float* __restrict__ probs_out, int32_t* __restrict__ partial_hist) {
+  __shared__ int hist[kMaxExperts];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int t_begin = blockIdx.x * kRouteTokensPerCta;
+  const int t_end = min(T, t_begin + kRouteTokensPerCta);
+  for (int t = t_begin + warp; t < t_end; t += nwarps) {
+    const float* lrow = logits + (size_t)t * E;
+    float p[VPL], s[VPL];
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      int e = lane + 32 * j;
+      p[j] = e < E ? lrow[e] : -INFINITY;
+      m = fmaxf(m, p[j]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      int e = lane + 32 * j;
+      p[j] = e < E ? expf(p[j] - m) : 0.f;
+      sum += p[j];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    uint32_t taken = 0;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      int e = lane + 32 * j;
+      p[j] = p[j] / sum;                       // R_e
+      if (e < E) {
+        s[j] = p[j] + bias[e];                 // biased score, selection only
+        if (probs_out) probs_out[(size_t)t * E + e] = p[j];
+      } else {
+        taken |= 1u << j;                      // padding never selected
+        s[j] = -INFINITY;
+      }
+    }
+    int nf = 0;
+    for (int k = 0; k < K; ++k) {
+      // lane-local best among untaken: larger s, then smaller e (= smaller j)
+      float bs = -INFINITY;
+      int bj = -1;
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) {
+        if (!(taken >> j & 1u) && (bj < 0 || s[j] > bs)) { bs = s[j]; bj = j; }
+      }
+      int be = bj >= 0 ? lane + 32 * bj : 0x7fffffff;
+      // warp arg-max on (s desc, e asc)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        float os = __shfl_xor_sync(0xffffffffu, bs, o);
+        int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (oe != 0x7fffffff && (be == 0x7fffffff || os > bs || (os == bs && oe < be))) {
+          bs = os; be = oe;
+        }
+      }
+      const int owner = be & 31, oj = be >> 5;
+      float gate = 0.f;
+#pragma unroll
+      for (int j = 0; j < VPL; ++j)
+        if (j == oj) gate = p[j];
+      gate = __shfl_sync(0xffffffffu, gate, owner);
+      if (lane == owner) taken |= 1u << oj;
+      if (lane == 0) {
+        topk_idx[(size_t)t * K + k] = be;
+        topk_gate[(size_t)t * K + k] = gate;
+        atomicAdd(&hist[be], 1);
+      }
+      nf += be < N;
+    }
+    if (lane == 0) n_ffn[t] = (uint8_t)nf;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    partial_hist[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+// counts[e] = sum over route CTAs of their partial histograms (fixed order).
+__global__ void reduce_hist_kernel(const int32_t* __restrict__ partial, int nparts, int E,
+                                   int32_t* __restrict__ counts) {
+  int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  int c = 0;
+  for (int p = 0; p < nparts; ++p) c += partial[(size_t)p * E + e];
+  counts[e] = c;
+}
+
+}  // namespace moe

@@ -1,0 +1,196 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, stage by stage."""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_layer_30_b200 import binding as B
+from mixture_experts_layer_30_b200 import configs as C
+from mixture_experts_layer_30_b200 import inputs as IN
+from oracle import moe_oracle as orc
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_and_check(shape, dtype, L, N, K, gamma=1.0, logit_offset=None, split_ffn=False,
+                   experts=None):
+    run = P.GpuRun(shape, L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"],
+                   gamma=gamma, logit_offset=logit_offset, split_ffn=split_ffn)
+    assert run.status == 0, hex(run.status)
+    g = run.host()
+    x64 = P.to_f64(L["x"])
+    wr64 = P.to_f64(L["w_router"])
+    idx_ref, probs, nties = P.check_routing_and_dispatch(g, x64, wr64, L["bias"], N, K,
+                                                         logit_offset)
+    gate = orc.gates(probs, idx_ref)
+    off, rt, sp = orc.canonical_permutation(idx_ref, N)
+    y_o = orc.grouped_ffn(x64[rt], off, L["w1"], L["w3"], L["w2"], experts=experts,
+                          decode=P.to_f64)
+    rows = ~np.isnan(y_o[:, 0]) if len(y_o) else np.zeros(0, bool)
+    P.assert_close(g["y_perm"][rows], y_o[rows], dtype, "y_perm")
+    zm = orc.zero_mass(idx_ref, gate, N)
+    if experts is None:
+        out_o = orc.combine(x64, y_o, idx_ref, gate, sp, N, gamma)
+        P.assert_close(g["out"], out_o, dtype, "out")
+        # FFN part alone (the identity term would hide FFN errors)
+        P.assert_close(g["out"] - gamma * zm[:, None] * x64, out_o - gamma * zm[:, None] * x64,
+                       dtype, "out minus identity term")
+    # combine stage on the GPU's own expert outputs
+    out_stage = orc.combine(x64, g["y_perm"], idx_ref, gate, sp, N, gamma)
+    P.assert_close(g["out"], out_stage, dtype, "combine stage")
+    return run, g, nties
+
+
+def _cfg_inputs(cfg, device="cuda", **over):
+    L = IN.make_layer_inputs(cfg, device=device)
+    L.update(over)
+    return L
+
+
+def test_tiny_f32_layer():
+    cfg = C.TINY_F32
+    L = _cfg_inputs(cfg)
+    _run_and_check(B.shape_of(cfg), "f32", L, cfg.N, cfg.K)
+
+
+def test_tiny_f32_layer_split_ffn_and_gamma():
+    cfg = C.TINY_F32
+    L = _cfg_inputs(cfg)
+    _run_and_check(B.shape_of(cfg), "f32", L, cfg.N, cfg.K, gamma=2.5, split_ffn=True)
+
+
+def test_mid_bf16_layer():
+    cfg = C.MID_BF16
+    L = _cfg_inputs(cfg)
+    _, g, nties = _run_and_check(B.shape_of(cfg), "bf16", L, cfg.N, cfg.K, split_ffn=True)
+    # the U(-0.05, 0.05) bias sends roughly a third of the slots to zero experts
+    frac_zero = 1.0 - g["n_ffn"].mean() / cfg.K
+    assert 0.15 < frac_zero < 0.6
+
+
+@pytest.mark.parametrize("cfg", [C.DECODE_T16, C.DECODE_T64, C.DECODE_T256],
+                         ids=lambda c: c.name)
+def test_decode_bf16(cfg):
+    L = _cfg_inputs(cfg)
+    _run_and_check(B.shape_of(cfg), "bf16", L, cfg.N, cfg.K, split_ffn=True)
+
+
+def _small(T, d, N, Z, K, I, dtype, seed=0, bias=None, w_std=0.05):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    E = N + Z
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+
+    def rn(*shape, std=1.0):
+        return (torch.randn(shape, generator=g) * std).to(dt).cuda()
+    L = dict(x=rn(T, d), w_router=rn(E, d, std=0.1), w1=rn(N, I, d, std=w_std),
+             w3=rn(N, I, d, std=w_std), w2=rn(N, d, I, std=w_std),
+             bias=(torch.zeros(E) if bias is None else torch.as_tensor(bias, dtype=torch.float32)).cuda())
+    return B.make_shape(T, d, N, Z, K, I, dtype), L
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [1, 7, 300, 513])
+def test_ragged_token_counts(dtype, T):
+    shape, L = _small(T, 128, 12, 4, 3, 64, dtype, seed=T)
+    _run_and_check(shape, dtype, L, 12, 3)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_k_equals_e(dtype):
+    N, Z = 5, 3
+    shape, L = _small(40, 64, N, Z, N + Z, 64, dtype, seed=11)
+    _, g, _ = _run_and_check(shape, dtype, L, N, N + Z)
+    np.testing.assert_allclose(g["gate"].sum(axis=1), 1.0, atol=1e-5)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_all_slots_to_zero_experts(dtype):
+    N, Z, K = 6, 4, 3
+    bias = [0.0] * N + [10.0] * Z
+    shape, L = _small(70, 64, N, Z, K, 64, dtype, seed=5, bias=bias)
+    run, g, _ = _run_and_check(shape, dtype, L, N, K)
+    assert g["R"] == 0 and (g["slot_pos"] == -1).all()
+    # bit-exact fixed point: out = fl32(sum of the GPU's gates) * x, rounded to dtype
+    zs = torch.zeros(70, dtype=torch.float32)
+    gate = run.buf.topk_gate.cpu()
+    for k in range(K):
+        zs = zs + gate[:, k]
+    want = (zs[:, None] * L["x"].float().cpu()).to(L["x"].dtype)
+    assert torch.equal(run.buf.out.cpu(), want)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_one_hot_expert_long_segment(dtype):
+    N, Z, K = 8, 4, 2
+    bias = [0.0] * (N + Z)
+    bias[3] = 10.0
+    shape, L = _small(700, 128, N, Z, K, 64, dtype, seed=7, bias=bias)
+    _, g, _ = _run_and_check(shape, dtype, L, N, K)
+    assert g["offsets"][4] - g["offsets"][3] == 700
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_no_zero_experts(dtype):
+    shape, L = _small(200, 64, 10, 0, 3, 64, dtype, seed=3)
+    _run_and_check(shape, dtype, L, 10, 3)
+
+
+def test_empty_batch():
+    shape, L = _small(0, 64, 6, 2, 2, 64, "f32", seed=1)
+    L["x"] = torch.empty((0, 64), device="cuda")
+    buf = B.LayerBuffers(shape, with_probs=True)
+    buf.counts.fill_(-1)
+    buf.offsets.fill_(-1)
+    B.forward(buf, L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"])
+    torch.cuda.synchronize()
+    assert (buf.counts == 0).all() and (buf.offsets == 0).all()
+    assert B.device_status(buf.ws) == 0
+
+
+def test_deterministic_bitwise():
+    cfg = C.MID_BF16
+    L = _cfg_inputs(cfg)
+    s = B.shape_of(cfg)
+    outs = []
+    for _ in range(2):
+        buf = B.LayerBuffers(s)
+        B.forward(buf, L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"],
+                  split_ffn=True)
+        outs.append((buf.out.clone(), buf.y_perm.clone(), buf.topk_idx.clone(),
+                     buf.slot_pos.clone()))
+    torch.cuda.synchronize()
+    R = int(buf.offsets[-1])
+    assert torch.equal(outs[0][0], outs[1][0])
+    assert torch.equal(outs[0][1][:R], outs[1][1][:R])
+    assert torch.equal(outs[0][2], outs[1][2]) and torch.equal(outs[0][3], outs[1][3])
+
+
+def test_bad_expert_index_sets_status_without_fault():
+    shape, L = _small(64, 64, 6, 2, 2, 64, "f32", seed=2)
+    buf = B.LayerBuffers(shape)
+    B.route(shape, L["x"], L["w_router"], L["bias"], buf.ws, buf.topk_idx, buf.topk_gate,
+            buf.counts, buf.n_ffn)
+    bad = buf.topk_idx.clone()
+    bad[5, 1] = 99
+    B.permute(shape, L["x"], bad, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
+              buf.x_perm, buf.ws)
+    st = B.device_status(buf.ws)
+    assert st & B.DEV_BAD_EXPERT_INDEX and st & B.DEV_COUNT_MISMATCH
+    assert B.device_status(buf.ws) == 0  # cleared by the read
+
+
+def test_bias_update_open_loop_bit_exact():
+    rng = np.random.default_rng(0)
+    for (N, Z, K, T) in ((16, 8, 4, 16384), (512, 256, 12, 8192), (64, 32, 6, 4096)):
+        E = N + Z
+        counts = rng.multinomial(K * T, np.ones(E) / E).astype(np.int32)
+        b0 = rng.normal(scale=0.05, size=E).astype(np.float32)
+        K_e = np.float32(K * N / E)
+        mu = np.float32(0.1)
+        bias = torch.from_numpy(b0).cuda()
+        B.bias_update(N, Z, torch.from_numpy(counts).cuda(), T, K, float(K_e), float(mu), bias)
+        got = bias.cpu().numpy()
+        want = orc.bias_update(b0.astype(np.float64), counts, N, K, float(K_e), float(mu),
+                               T).astype(np.float32)
+        assert got.tobytes() == want.tobytes()
+        assert got[N:].tobytes() == b0[N:].tobytes()

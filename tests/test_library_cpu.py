@@ -1,0 +1,88 @@
+"""The C-ABI library builds, loads and exports every declared symbol; host-side
+validation returns error codes (no GPU needed: none of these calls launches)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mixture_experts_layer_30_b200 import binding as B
+from mixture_experts_layer_30_b200 import build as BUILD
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    BUILD.build()
+    return B.lib()
+
+
+def declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for fn in sorted(os.listdir(inc)):
+        if fn.endswith(".h"):
+            src = open(os.path.join(inc, fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w \*]*?\b(moe_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 11, names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(B.SIGNATURES), set(names) - set(B.SIGNATURES)
+
+
+def test_workspace_bytes_and_validation(lib):
+    s = B.make_shape(8192, 6144, 512, 256, 12, 2048, "bf16")
+    n = B.workspace_bytes(s)
+    # logits + h dominate: T*E*4 + T*K*I*2
+    assert n >= 8192 * 768 * 4 + 8192 * 12 * 2048 * 2
+    for bad in (B.make_shape(8, 64, 0, 2, 1, 8, "f32"),      # N < 1
+                B.make_shape(8, 64, 4, 2, 7, 8, "f32"),      # K > N+Z
+                B.make_shape(8, 64, 4, 2, 0, 8, "f32"),      # K < 1
+                B.make_shape(8, 62, 4, 2, 2, 8, "f32"),      # rows not 16-byte multiples
+                B.make_shape(8, 64, 1000, 100, 2, 8, "f32"),  # E > 1024
+                B.make_shape(-1, 64, 4, 2, 2, 8, "f32")):
+        assert lib.moe_workspace_bytes(ctypes.byref(bad)) == 0
+
+
+def test_invalid_arguments_return_codes(lib):
+    s = B.make_shape(16, 64, 4, 2, 2, 32, "f32")
+    nb = B.workspace_bytes(s)
+    fake = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
+    # NULL shape
+    assert lib.moe_route(None, fake, fake, fake, None, fake, fake, fake, fake, None, fake, nb,
+                         None) == 1
+    # NULL workspace
+    assert lib.moe_route(ctypes.byref(s), fake, fake, fake, None, fake, fake, fake, fake, None,
+                         None, nb, None) == 1
+    assert b"workspace" in lib.moe_last_error()
+    # workspace too small
+    assert lib.moe_permute(ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake, fake,
+                           nb - 256, None) == 3
+    # misaligned workspace
+    assert lib.moe_expert_ffn(ctypes.byref(s), fake, fake, fake, fake, fake, fake,
+                              ctypes.c_void_p(0x10008), nb, None) == 1
+    # NULL operand
+    assert lib.moe_expert_gate_up(ctypes.byref(s), None, fake, fake, fake, fake, fake, nb,
+                                  None) == 1
+    assert b"x_perm" in lib.moe_last_error()
+    # bias update argument checks
+    assert lib.moe_bias_update(0, 2, fake, 16, 2, 1.0, 0.1, fake, None) == 1
+    assert lib.moe_bias_update(4, 2, fake, 0, 2, 1.0, 0.1, fake, None) == 1
+    assert lib.moe_bias_update(4, 2, fake, 16, 9, 1.0, 0.1, fake, None) == 1
+    # bad dtype code
+    bad = B.Shape(16, 64, 4, 2, 2, 32, 7)
+    assert lib.moe_combine(ctypes.byref(bad), fake, fake, fake, fake, fake, 1.0, fake, None) == 1
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    monkeypatch.setattr(B, "_lib", None)
+    monkeypatch.setattr(B, "LIB_PATH", "/nonexistent/libmoe_b200.so")
+    with pytest.raises(RuntimeError, match="missing"):
+        B.lib()
