@@ -1,26 +1,603 @@
-// Tensor-core (tcgen05 / TMEM / TMA) GEMMs of the bf16 path.
+// Tensor-core GEMMs of the bf16 path on sm_100a: tcgen05.mma with fp32
+// accumulators in TMEM, operands staged in shared memory by TMA.
+//
+// Orientation ("swap AB"): the weight rows are the UMMA M operand (128
+// output features per MMA) and the routed token rows are the N operand
+// (16..256 rows, rounded up to 16).  Expert segments are ragged (about 128
+// rows per expert at the LongCat shape), so putting tokens on N wastes at most
+// 15 padded rows per segment instead of up to 127 with tokens on M, and every
+// weight tile is streamed from HBM exactly once per (expert, 256-row chunk).
+//
+// One persistent CTA per SM, 6 warps:
+//   warp 0      TMA producer (one lane): A0, A1 weight tiles + B token tile per stage
+//   warp 1      MMA issuer (one lane); also allocates/frees the 512 TMEM columns
+//   warps 2..5  epilogue: TMEM -> registers -> (SwiGLU | copy) -> shared -> global
+// Pipeline: kStages shared-memory stages guarded by full/empty mbarriers, one
+// TMEM accumulator pair guarded by tmem_full/tmem_empty.  Every wait is bounded
+// in time; on expiry the CTA raises MOE_DEV_PIPELINE_TIMEOUT, drains what it
+// issued and returns.
+//
+// Tile = (row chunk of <= 256 token rows of one expert, feature block):
+//   gated mode  (first half of the SwiGLU expert): D0 = W1 rows f0..f0+127,
+//               D1 = W3 rows f0..f0+127, out h = SiLU(D0) * D1 (bf16)
+//   plain modes (second half, router): D0 = rows f0..f0+127, D1 = rows
+//               f0+128..f0+255 of one weight matrix; out bf16 or fp32 (+offset)
 #pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstdio>
 
 #include "common.cuh"
 
 namespace moe {
 namespace tc {
 
-inline bool router_supported(const moe_shape&) { return false; }
-inline bool ffn_supported(const moe_shape&) { return false; }
+constexpr int kBK = 64;                          // K elements per stage = one 128-byte row
+constexpr int kFeat = 128;                       // UMMA M
+constexpr int kNMax = 256;                       // token rows per tile (UMMA N <= 256)
+constexpr int kBoxRows = 32;                     // rows per token TMA box
+constexpr int kStages = 3;
+constexpr int kABytes = kFeat * kBK * 2;         // 16 KiB
+constexpr int kBoxBytes = kBoxRows * kBK * 2;    // 4 KiB
+constexpr int kBBytes = kNMax * kBK * 2;         // 32 KiB
+constexpr int kStageBytes = 2 * kABytes + kBBytes;
+constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;
+constexpr int kStagingPitch = 36;                // 32-bit words per staging row (32 + pad)
+constexpr int kStagingBytes = kEpiWarps * 32 * kStagingPitch * 4;
+constexpr int kTmemCols = 512;
+constexpr int kNumBars = 2 * kStages + 3;        // full[], empty[], tmem_full, tmem_empty, drain
+constexpr int kCtrlBytes = 256;                  // barriers + tmem slot + abort flag
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kStagingBytes + kCtrlBytes +
+                           (kMaxExperts + 1 + 33) * 4;
+constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;  // 4 s
+constexpr unsigned long long kDrainTimeoutNs = 200000000ull;  // 0.2 s
 
-inline moe_status launch_router_gemm(const moe_shape&, const void*, const void*, const float*,
-                                     float*, int, cudaStream_t, char*, size_t) {
-  return MOE_ERR_UNSUPPORTED;
+enum Mode { kGated = 0, kPlainBf16 = 1, kPlainF32 = 2 };
+
+struct Args {
+  const int32_t* seg_offsets;  // [nseg+1] routed-row offsets, or NULL for one segment
+  int nseg;                    // experts (or 1)
+  int single_rows;             // rows of the single segment when seg_offsets == NULL
+  int max_rows;                // rows of the token matrix (bound for offsets)
+  int n_out;                   // output features (row stride of `out`)
+  int k_dim;                   // reduction length (multiple of 64)
+  int a_seg_rows;              // weight rows per expert in the 2-D weight view
+  int a1_row_off;              // D1 weight rows = D0 rows + this (plain modes)
+  int feat_per_tile;           // 128 (gated) or 256 (plain)
+  void* out;
+  const float* add;            // fp32 addend [rows, n_out] (router logit offset) or NULL
+  uint32_t* status;
+};
+
+// --- PTX wrappers --------------------------------------------------------------
+MOE_DEV uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-inline moe_status launch_gate_up(const moe_shape&, const void*, const void*, const void*,
-                                 const int32_t*, void*, uint32_t*, int, cudaStream_t, char*,
-                                 size_t) {
-  return MOE_ERR_UNSUPPORTED;
+MOE_DEV uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
 }
-inline moe_status launch_down(const moe_shape&, const void*, const void*, const int32_t*, void*,
-                              uint32_t*, int, cudaStream_t, char*, size_t) {
-  return MOE_ERR_UNSUPPORTED;
+MOE_DEV void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+MOE_DEV void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+MOE_DEV void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+MOE_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false when the abort flag is raised or the time limit passes
+// (then the flag is raised and the status word records the timeout).
+MOE_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                       uint32_t* status, unsigned long long limit_ns = kWaitTimeoutNs,
+                       bool honour_abort = true) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 31) == 31) {
+      if (honour_abort && *abort_flag) return false;
+      const uint64_t now = globaltimer();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > limit_ns) {
+        *abort_flag = 1;
+        set_status(status, MOE_DEV_PIPELINE_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+MOE_DEV void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+MOE_DEV void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+MOE_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+MOE_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, K-major operand in the 128-byte swizzle
+// layout: rows of 128 bytes, 8-row (1024-byte) swizzle atoms stacked densely.
+//   bits  0-13 start address >> 4     bits 16-29 leading byte offset >> 4 (unused: 1)
+//   bits 32-45 stride byte offset >> 4 (1024 B between 8-row groups)
+//   bits 46-47 version (1 on sm_100)  bits 61-63 layout (2 = 128-byte swizzle)
+MOE_DEV uint64_t smem_desc_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3fff);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// Instruction descriptor of kind::f16: fp32 D, bf16 A and B, both K-major.
+//   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
+//   15/16 A/B major (0 = K), 17-22 N >> 3, 24-28 M >> 4.
+MOE_DEV uint32_t idesc_bf16(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(m >> 4) << 24);
+}
+MOE_DEV void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+MOE_DEV void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+// 32 lanes x 32 consecutive 32-bit TMEM columns: thread i gets row (lane base + i).
+MOE_DEV void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+MOE_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// --- tile decoding ---------------------------------------------------------------
+struct Tile {
+  int seg, r0, n, f0;
+};
+
+MOE_DEV Tile decode_tile(int tile, int n_fblk, const Args& a, const int* prefix) {
+  Tile t;
+  const int chunk = tile / n_fblk;
+  const int fb = tile - chunk * n_fblk;
+  int lo, hi, c0;
+  if (a.seg_offsets) {
+    t.seg = find_expert(prefix, a.nseg, chunk);
+    lo = a.seg_offsets[t.seg];
+    hi = a.seg_offsets[t.seg + 1];
+    c0 = prefix[t.seg];
+  } else {
+    t.seg = 0;
+    lo = 0;
+    hi = a.single_rows;
+    c0 = 0;
+  }
+  t.r0 = lo + (chunk - c0) * kNMax;
+  t.n = min(kNMax, hi - t.r0);
+  t.f0 = fb * a.feat_per_tile;
+  return t;
+}
+
+// --- the kernel ------------------------------------------------------------------
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+               const __grid_constant__ CUtensorMap tmB, const Args args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* stages = smem;
+  uint32_t* staging = reinterpret_cast<uint32_t*>(smem + kStages * kStageBytes);
+  uint8_t* ctrl = smem + kStages * kStageBytes + kStagingBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ctrl);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 8 * kNumBars + 4);
+  volatile int* consumed_sh = reinterpret_cast<volatile int*>(ctrl + 8 * kNumBars + 8);
+  int* prefix = reinterpret_cast<int*>(ctrl + kCtrlBytes);
+  int* scan_tmp = prefix + kMaxExperts + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t full0 = smem_u32(&bars[0]);
+  const uint32_t empty0 = smem_u32(&bars[kStages]);
+  const uint32_t tmem_full = smem_u32(&bars[2 * kStages]);
+  const uint32_t tmem_empty = smem_u32(&bars[2 * kStages + 1]);
+  const uint32_t drain_bar = smem_u32(&bars[2 * kStages + 2]);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 1);
+    }
+    mbar_init(tmem_full, 1);
+    mbar_init(tmem_empty, kEpiWarps * 32);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *consumed_sh = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmA1);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (args.seg_offsets) {
+    build_chunk_prefix(args.seg_offsets, args.nseg, args.max_rows, kNMax, prefix, scan_tmp,
+                       args.status);
+  } else if (threadIdx.x == 0) {
+    prefix[0] = 0;
+    prefix[1] = (args.single_rows + kNMax - 1) / kNMax;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int nseg = args.seg_offsets ? args.nseg : 1;
+  const int n_fblk = (args.n_out + args.feat_per_tile - 1) / args.feat_per_tile;
+  const int total = prefix[nseg] * n_fblk;
+  const int nk = args.k_dim / kBK;
+  int issued = 0;  // producer: stages issued
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const Tile t = decode_tile(tile, n_fblk, args, prefix);
+        const int nbox = (t.n + kBoxRows - 1) / kBoxRows;
+        const uint32_t tx = 2 * kABytes + nbox * kBoxBytes;
+        const int a_row0 = t.seg * args.a_seg_rows + t.f0;
+        const int a_row1 = a_row0 + args.a1_row_off;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = full0 + 8 * stage;
+          const uint32_t sa0 = smem_u32(stages + stage * kStageBytes);
+          mbar_arrive_expect_tx(fb, tx);
+          tma_load_2d(sa0, &tmA0, kb * kBK, a_row0, fb);
+          tma_load_2d(sa0 + kABytes, &tmA1, kb * kBK, a_row1, fb);
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(sa0 + 2 * kABytes + b * kBoxBytes, &tmB, kb * kBK, t.r0 + b * kBoxRows,
+                        fb);
+          ++issued;
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      uint32_t stage = 0, phase = 0, acc_phase = 0;
+      bool ok = true;
+      int consumed = 0;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const Tile t = decode_tile(tile, n_fblk, args, prefix);
+        int n16 = ((t.n + 15) >> 4) << 4;
+        if (n16 < 16) n16 = 16;
+        const uint32_t idesc = idesc_bf16(kFeat, n16);
+        if (!mbar_wait(tmem_empty, acc_phase ^ 1, abort_flag, args.status)) break;
+        acc_phase ^= 1;
+        tc_fence_after();
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa0 = smem_u32(stages + stage * kStageBytes);
+          const uint64_t da0 = smem_desc_sw128(sa0);
+          const uint64_t da1 = smem_desc_sw128(sa0 + kABytes);
+          const uint64_t db = smem_desc_sw128(sa0 + 2 * kABytes);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            // advance 16 bf16 = 32 bytes along K inside the swizzled row
+            const uint32_t acc = (kb | k) != 0;
+            umma_bf16(tmem_base, da0 + 2 * k, db + 2 * k, idesc, acc);
+            umma_bf16(tmem_base + kNMax, da1 + 2 * k, db + 2 * k, idesc, acc);
+          }
+          umma_commit(empty0 + 8 * stage);
+          ++consumed;
+          *consumed_sh = consumed;
+          if (++stage == kStages) { stage = 0; phase ^= 1; }
+        }
+        if (ok) umma_commit(tmem_full);
+      }
+      // every MMA issued so far completes before TMEM is released
+      umma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, abort_flag, args.status, kDrainTimeoutNs, false);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;                      // TMEM lane quarter this warp may access
+    uint32_t* stg = staging + (warp - 2) * 32 * kStagingPitch;
+    uint32_t acc_phase = 0;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const Tile t = decode_tile(tile, n_fblk, args, prefix);
+      if (!mbar_wait(tmem_full, acc_phase, abort_flag, args.status)) break;
+      acc_phase ^= 1;
+      tc_fence_after();
+      const int nhalves = (kMode == kGated) ? 1 : 2;
+      for (int hf = 0; hf < nhalves; ++hf) {
+        const int fbase = t.f0 + hf * kFeat + 32 * q;   // first feature of this warp
+        for (int j0 = 0; j0 < t.n; j0 += 32) {
+          uint32_t v0[32];
+          tmem_ld_32x32b_x32(tmem_base + lane_base + hf * kNMax + j0, v0);
+          if (kMode == kGated) {
+            uint32_t v1[32];
+            tmem_ld_32x32b_x32(tmem_base + lane_base + kNMax + j0, v1);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              float a0 = silu(__uint_as_float(v0[j])) * __uint_as_float(v1[j]);
+              float a1 = silu(__uint_as_float(v0[j + 1])) * __uint_as_float(v1[j + 1]);
+              v0[j] = pack_bf16x2(a0, a1);
+            }
+          } else {
+            tmem_wait_ld();
+            if (kMode == kPlainBf16) {
+#pragma unroll
+              for (int j = 0; j < 32; j += 2)
+                v0[j] = pack_bf16x2(__uint_as_float(v0[j]), __uint_as_float(v0[j + 1]));
+            }
+          }
+          // transpose through shared memory: stg[token j][feature lane]
+          if (kMode == kPlainF32) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) stg[j * kStagingPitch + lane] = v0[j];
+          } else {
+            uint16_t* s16 = reinterpret_cast<uint16_t*>(stg);
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              s16[j * 2 * kStagingPitch + lane] = (uint16_t)(v0[j] & 0xffffu);
+              s16[(j + 1) * 2 * kStagingPitch + lane] = (uint16_t)(v0[j] >> 16);
+            }
+          }
+          __syncwarp();
+          // each token row of this warp: 32 features = 64 B (bf16) or 128 B (fp32)
+          constexpr int kVecPerRow = (kMode == kPlainF32) ? 8 : 4;
+#pragma unroll
+          for (int it = 0; it < kVecPerRow; ++it) {
+            const int vec = it * 32 + lane;
+            const int j = vec / kVecPerRow, c = vec % kVecPerRow;
+            const int row = t.r0 + j0 + j;
+            const int f = fbase + c * (kMode == kPlainF32 ? 4 : 8);
+            if (j0 + j < t.n && f < args.n_out) {
+              if (kMode == kPlainF32) {
+                uint4 w = *reinterpret_cast<const uint4*>(&stg[j * kStagingPitch + c * 4]);
+                float* o = static_cast<float*>(args.out) + (size_t)row * args.n_out + f;
+                if (args.add) {
+                  const float4 ad =
+                      *reinterpret_cast<const float4*>(args.add + (size_t)row * args.n_out + f);
+                  w.x = __float_as_uint(__uint_as_float(w.x) + ad.x);
+                  w.y = __float_as_uint(__uint_as_float(w.y) + ad.y);
+                  w.z = __float_as_uint(__uint_as_float(w.z) + ad.z);
+                  w.w = __float_as_uint(__uint_as_float(w.w) + ad.w);
+                }
+                *reinterpret_cast<uint4*>(o) = w;
+              } else {
+                const uint16_t* s16 = reinterpret_cast<const uint16_t*>(stg);
+                const uint4 w = *reinterpret_cast<const uint4*>(&s16[j * 2 * kStagingPitch + c * 8]);
+                __nv_bfloat16* o =
+                    static_cast<__nv_bfloat16*>(args.out) + (size_t)row * args.n_out + f;
+                *reinterpret_cast<uint4*>(o) = w;
+              }
+            }
+          }
+          __syncwarp();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tmem_empty);
+    }
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {
+    // drain copies still in flight into shared memory (bounded)
+    const int consumed = *consumed_sh;
+    for (int i = consumed; i < issued; ++i)
+      mbar_wait(full0 + 8 * (i % kStages), (uint32_t)((i / kStages) & 1), abort_flag,
+                args.status, kDrainTimeoutNs, false);
+  }
+  __syncwarp();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// --- host side -------------------------------------------------------------------
+inline bool router_supported(const moe_shape& s) {
+  const int E = s.N + s.Z;
+  return s.dtype == MOE_BF16 && s.d % kBK == 0 && E % 8 == 0;
+}
+inline bool ffn_supported(const moe_shape& s) {
+  return s.dtype == MOE_BF16 && s.d % kBK == 0 && s.I % kBK == 0;
+}
+
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 row-major [rows, cols] view, box = box_rows x 64 columns, 128-byte swizzle.
+inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols,
+                     uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int kMode>
+inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+                         const Args& args, long long max_tiles, int sms, cudaStream_t st,
+                         char* err, size_t errn) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kMode>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) {
+      snprintf(err, errn, "tcgen05 gemm smem attribute: %s", cudaGetErrorString(e));
+      return MOE_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  long long grid = max_tiles < sms ? max_tiles : sms;
+  if (grid < 1) grid = 1;
+  gemm_tc_kernel<kMode><<<(int)grid, kThreads, kSmemBytes, st>>>(a0, a1, b, args);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    snprintf(err, errn, "tcgen05 gemm launch: %s", cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+inline moe_status map_error(char* err, size_t errn, const char* what) {
+  snprintf(err, errn, "cuTensorMapEncodeTiled failed for %s", what);
+  return MOE_ERR_CUDA;
+}
+
+// Upper bound of (row chunk, feature block) tiles for routed rows.
+inline long long routed_tiles(const moe_shape& s, int n_out, int feat) {
+  const long long rows = (long long)s.T * s.K;
+  const long long chunks = s.N + (rows + kNMax - 1) / kNMax;
+  return chunks * ((n_out + feat - 1) / feat);
+}
+
+inline moe_status launch_gate_up(const moe_shape& s, const void* x_perm, const void* w1,
+                                 const void* w3, const int32_t* offsets, void* h,
+                                 uint32_t* status, int sms, cudaStream_t st, char* err,
+                                 size_t errn) {
+  CUtensorMap a0, a1, b;
+  const uint64_t rows = (uint64_t)s.T * s.K;
+  if (!make_map(&a0, w1, (uint64_t)s.N * s.I, s.d, kFeat)) return map_error(err, errn, "w1");
+  if (!make_map(&a1, w3, (uint64_t)s.N * s.I, s.d, kFeat)) return map_error(err, errn, "w3");
+  if (!make_map(&b, x_perm, rows, s.d, kBoxRows)) return map_error(err, errn, "x_perm");
+  Args a{};
+  a.seg_offsets = offsets;
+  a.nseg = s.N;
+  a.max_rows = (int)rows;
+  a.n_out = s.I;
+  a.k_dim = s.d;
+  a.a_seg_rows = s.I;
+  a.a1_row_off = 0;
+  a.feat_per_tile = kFeat;
+  a.out = h;
+  a.status = status;
+  return launch<kGated>(a0, a1, b, a, routed_tiles(s, s.I, kFeat), sms, st, err, errn);
+}
+
+inline moe_status launch_down(const moe_shape& s, const void* h, const void* w2,
+                              const int32_t* offsets, void* y_perm, uint32_t* status, int sms,
+                              cudaStream_t st, char* err, size_t errn) {
+  CUtensorMap a, b;
+  const uint64_t rows = (uint64_t)s.T * s.K;
+  if (!make_map(&a, w2, (uint64_t)s.N * s.d, s.I, kFeat)) return map_error(err, errn, "w2");
+  if (!make_map(&b, h, rows, s.I, kBoxRows)) return map_error(err, errn, "h");
+  Args g{};
+  g.seg_offsets = offsets;
+  g.nseg = s.N;
+  g.max_rows = (int)rows;
+  g.n_out = s.d;
+  g.k_dim = s.I;
+  g.a_seg_rows = s.d;
+  g.a1_row_off = kFeat;
+  g.feat_per_tile = 2 * kFeat;
+  g.out = y_perm;
+  g.status = status;
+  return launch<kPlainBf16>(a, a, b, g, routed_tiles(s, s.d, 2 * kFeat), sms, st, err, errn);
+}
+
+inline moe_status launch_router_gemm(const moe_shape& s, const void* x, const void* w,
+                                     const float* offset, float* logits, int sms,
+                                     cudaStream_t st, char* err, size_t errn) {
+  CUtensorMap a, b;
+  const int E = s.N + s.Z;
+  if (!make_map(&a, w, (uint64_t)E, s.d, kFeat)) return map_error(err, errn, "w_router");
+  if (!make_map(&b, x, (uint64_t)s.T, s.d, kBoxRows)) return map_error(err, errn, "x");
+  Args g{};
+  g.seg_offsets = nullptr;
+  g.nseg = 1;
+  g.single_rows = s.T;
+  g.max_rows = s.T;
+  g.n_out = E;
+  g.k_dim = s.d;
+  g.a_seg_rows = 0;
+  g.a1_row_off = kFeat;
+  g.feat_per_tile = 2 * kFeat;
+  g.out = logits;
+  g.add = offset;
+  g.status = nullptr;
+  const long long tiles = (long long)((s.T + kNMax - 1) / kNMax) * ((E + 2 * kFeat - 1) / (2 * kFeat));
+  return launch<kPlainF32>(a, a, b, g, tiles, sms, st, err, errn);
 }
 
 }  // namespace tc

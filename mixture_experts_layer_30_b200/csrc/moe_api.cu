@@ -134,7 +134,8 @@ moe_status route_impl(const moe_shape& s, const void* x, const void* w, const fl
   float* logits = at<float>(ws, L.logits);
   int32_t* hist = at<int32_t>(ws, L.route_hist);
   if (s.T > 0) {
-    if (s.dtype == MOE_BF16 && moe::tc::router_supported(s)) {
+    if (s.dtype == MOE_BF16 && moe::tc::router_supported(s) &&
+        reinterpret_cast<uintptr_t>(off) % 16 == 0) {
       MOE_TRY(moe::tc::launch_router_gemm(s, x, w, off, logits, sm_count(), st, g_err,
                                           sizeof(g_err)));
     } else {
