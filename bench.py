@@ -1,0 +1,430 @@
+"""Benchmark of the MoE layer with zero-computation experts on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step is one pass of the whole path on one batch: route (router GEMM +
+softmax + biased top-K + counts) -> dispatch to FFN experts -> SwiGLU expert
+GEMMs (gate/up, down) -> combine with the identity experts -> expert-bias
+update.  With N > 1 (torchrun) every rank processes its own batch with a full
+weight replica (weak scaling); the count histograms are summed over ranks with
+NCCL before the bias update, the one exchange step of the method.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
+oracle instead, on a bounded sample of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mixture_experts_layer_30_b200 import binding as B  # noqa: E402
+from mixture_experts_layer_30_b200 import configs as C  # noqa: E402
+from mixture_experts_layer_30_b200 import inputs as IN  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec at LongCat shape (bf16) + % of tensor/HBM roofline"
+DEFAULT_WORKLOAD = C.LONGCAT_PREFILL.name
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+TC_SOURCE = os.path.join(ROOT, "mixture_experts_layer_30_b200", "csrc", "gemm_tc.cuh")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest(path=TC_SOURCE):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def committed_traffic(kernel, workload):
+    """dram bytes per launch of ``kernel`` from the committed ncu summary, if it
+    was taken on the current kernel source; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("source_sha") != source_digest() or e.get("workload") != workload:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx, self.proc = gpu_index, None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args, rank, world, local_rank):
+    cfg = C.CONFIGS[args.workload]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    shape = B.shape_of(cfg)
+    L = IN.make_layer_inputs(cfg, device=dev, base_seed=0)
+    # every rank routes its own batch: x drawn with a per-rank seed
+    if rank:
+        L["x"] = IN.make_x(cfg, dev, seed=rank * 1000 + 0 + 7_000_000)
+    buf = B.LayerBuffers(shape, device=dev)
+    bias = L["bias"].clone()
+    counts_global = torch.empty_like(buf.counts)
+    T_all = cfg.T * world
+    K_e, mu = float(np.float32(cfg.K_e)), float(np.float32(cfg.mu))
+    if world > 1:
+        import torch.distributed as dist
+
+    def step(x, ev=None):
+        s = shape
+        if ev: ev[0].record(stream)
+        B.route(s, x, L["w_router"], bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts,
+                buf.n_ffn)
+        if ev: ev[1].record(stream)
+        B.permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
+                  buf.x_perm, buf.ws)
+        if ev: ev[2].record(stream)
+        B.expert_gate_up(s, buf.x_perm, L["w1"], L["w3"], buf.offsets, buf.h, buf.ws)
+        if ev: ev[3].record(stream)
+        B.expert_down(s, buf.h, L["w2"], buf.offsets, buf.y_perm, buf.ws)
+        if ev: ev[4].record(stream)
+        B.combine(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, cfg.gamma, buf.out)
+        if ev: ev[5].record(stream)
+        if world > 1:
+            counts_global.copy_(buf.counts)
+            dist.all_reduce(counts_global)
+            c = counts_global
+        else:
+            c = buf.counts
+        B.bias_update(cfg.N, cfg.Z, c, T_all, cfg.K, K_e, mu, bias)
+        if ev: ev[6].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    x = L["x"]
+    for _ in range(args.warmup):
+        step(x)
+    barrier()
+    st = B.device_status(buf.ws)
+    if st:
+        raise RuntimeError(f"device status 0x{st:x} after warm-up")
+
+    # ---- device-resident timing ----
+    n_ev = 7
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    props = torch.cuda.get_device_properties(dev)
+    clocks = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else local_rank)
+    launches0 = B.kernel_launches()
+    barrier()
+    clocks.start()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(x, evs[i])
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    launches = B.kernel_launches() - launches0
+    ms_total = t0.elapsed_time(t1)
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n_ev - 1)]
+                    for i in range(args.steps)])
+    ms_step_local = ms_total / args.steps
+    if world > 1:
+        tt = torch.tensor([ms_step_local], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_step = float(tt.item())
+    else:
+        ms_step = ms_step_local
+
+    # ---- end to end through the public API with host buffers ----
+    x_host = torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+    x_host.copy_(x.cpu())
+    out_host = torch.empty(buf.out.shape, dtype=buf.out.dtype, pin_memory=True)
+    x_dev = torch.empty_like(x)
+    e2e_steps = max(3, args.steps // 2)
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        out_host.copy_(buf.out, non_blocking=True)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev.copy_(x_host, non_blocking=True)
+        step(x_dev)
+        out_host.copy_(buf.out, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    st = B.device_status(buf.ws)
+    if st:
+        raise RuntimeError(f"device status 0x{st:x} after timing")
+
+    # ---- algorithmic work of the routed batch (counts of the last step) ----
+    counts = buf.counts.cpu().numpy().astype(np.int64)
+    R = int(counts[:cfg.N].sum())
+    touched = int((counts[:cfg.N] > 0).sum())
+    esz = 2 if cfg.dtype == "bf16" else 4
+    w13_bytes = touched * 2 * cfg.I * cfg.d * esz
+    w2_bytes = touched * cfg.d * cfg.I * esz
+    gate_up_bytes = w13_bytes + R * cfg.d * esz + R * cfg.I * esz
+    down_bytes = w2_bytes + R * cfg.I * esz + R * cfg.d * esz
+    gate_up_flops = 4.0 * cfg.d * cfg.I * R
+    down_flops = 2.0 * cfg.d * cfg.I * R
+    router_flops = 2.0 * cfg.d * cfg.E * cfg.T
+    layer_flops = gate_up_flops + down_flops + router_flops
+    layer_bytes = (w13_bytes + w2_bytes + cfg.E * cfg.d * esz + 2 * cfg.T * cfg.d * esz)
+    med = np.median(per, axis=0)
+    peaks, peak_kind = load_peaks()
+    hbm_peak = peaks["hbm_gbs"]
+    tflops_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    gu_ms = float(per[:, 2].mean())
+    achieved = gate_up_bytes / (gu_ms * 1e-3) / 1e9
+    traffic = committed_traffic("gate_up", cfg.name)
+    ffn_ms = float((per[:, 2] + per[:, 3]).mean())
+
+    if rank != 0:
+        return None, L
+    tokens_per_s = cfg.T * world / (ms_step * 1e-3)
+    line = {
+        "metric": METRIC,
+        "value": round(tokens_per_s, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": cfg.dtype,
+        "data": "synthetic (seeded N(0,1) activations, random-init weights of the stated shape)",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "N": cfg.N, "Z": cfg.Z,
+                   "K": cfg.K, "I": cfg.I, "K_e": cfg.K_e, "tokens_per_rank": cfg.T,
+                   "parallelism": f"token-dp{world} (weights replicated, counts all-reduced)",
+                   "l2": "inputs larger than L2 (38.7 GB of expert weights streamed per step)"},
+        "roofline": {"kernel": "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)",
+                     "bound": "hbm", "achieved": round(achieved, 1),
+                     "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": gate_up_bytes,
+                     "avg_launch_ms": round(gu_ms, 4)},
+        "layer": {
+            "routed_rows": R, "touched_experts": touched,
+            "ffn_tflops": round((gate_up_flops + down_flops) / (ffn_ms * 1e-3) / 1e12, 2),
+            "tensor_frac_of_sustained": round(layer_flops / (ms_step * 1e-3) / 1e12 / tflops_peak, 4),
+            "hbm_frac": round(layer_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak, 4),
+            "roofline_frac": round(max(layer_flops / (tflops_peak * 1e12),
+                                       layer_bytes / (hbm_peak * 1e9)) / (ms_step * 1e-3), 4),
+            "per_call_ms_median": {k: round(float(v), 4) for k, v in zip(
+                ["route", "permute", "gate_up", "down", "combine", "bias_update"], med)},
+        },
+        "e2e": {"value": round(cfg.T * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                "d2h_bytes_per_step": int(buf.out.numel() * buf.out.element_size())},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    return line, L
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (CPU baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        blas = [i["num_threads"] for i in info if i.get("user_api") == "blas"]
+        if blas:
+            return int(blas[0])
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_sample(cfg, L, t_begin, n_tok):
+    """Host copies of everything the oracle needs for tokens [t_begin, t_begin+n_tok)."""
+    from oracle import moe_oracle as orc
+
+    def bits(t):
+        t = t.detach().cpu().contiguous()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 \
+            else t.numpy()
+    dec = orc.bf16_bits_to_f64 if cfg.dtype == "bf16" else orc.as_f64
+    x = bits(L["x"][t_begin:t_begin + n_tok])
+    wr = bits(L["w_router"])
+    bias = L["bias"].detach().cpu().numpy()
+    # experts the sample can reach: route it once to find them (not timed)
+    probs = orc.softmax_rows(orc.router_logits(dec(x), dec(wr)))
+    idx, _ = orc.biased_topk(probs, bias, cfg.K)
+    touched = sorted(set(int(e) for e in idx.reshape(-1) if e < cfg.N))
+    w1 = {e: bits(L["w1"][e]) for e in touched}
+    w3 = {e: bits(L["w3"][e]) for e in touched}
+    w2 = {e: bits(L["w2"][e]) for e in touched}
+    return dict(x=x, wr=wr, bias=bias, w1=w1, w3=w3, w2=w2, dec=dec, touched=len(touched))
+
+
+def time_oracle(cfg, S):
+    """Seconds for the oracle's full layer (decode, route, dispatch, FFN, combine)."""
+    from oracle import moe_oracle as orc
+    t = time.perf_counter()
+    orc.moe_layer(S["dec"](S["x"]), S["dec"](S["wr"]), S["w1"], S["w3"], S["w2"], S["bias"],
+                  N=cfg.N, K=cfg.K, gamma=cfg.gamma, decode=S["dec"])
+    return time.perf_counter() - t
+
+
+def cpu_baseline(cfg, L, n_tok):
+    S = oracle_sample(cfg, L, 0, n_tok)
+    sec = time_oracle(cfg, S)
+    return {"value": round(n_tok / sec, 4), "unit": "tokens/s", "cores": oracle_threads(),
+            "kind": "oracle",
+            "sample": f"first {n_tok} tokens of the {cfg.name} batch through the whole fp64 "
+                      f"oracle layer ({S['touched']} experts decoded from bf16), {sec:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """--impl reference: the fp64 CPU oracle on the host cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    cfg = C.CONFIGS[args.workload]
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    if cfg.dtype == "bf16" and dev.type != "cuda":
+        return {"impl": "reference", "unavailable": "the bf16 workload is drawn on the GPU"}
+    L = IN.make_layer_inputs(cfg, device=dev)
+    n_tok = args.ref_tokens
+    for w in range(args.warmup):
+        time_oracle(cfg, oracle_sample(cfg, L, (w * n_tok) % cfg.T, n_tok))
+    secs = []
+    for i in range(args.steps):
+        S = oracle_sample(cfg, L, ((args.warmup + i) * n_tok) % cfg.T, n_tok)
+        secs.append(time_oracle(cfg, S))
+    sec = sum(secs) / len(secs)
+    v = round(n_tok / sec, 4)
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same seeded workload as the GPU arm)",
+        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "N": cfg.N, "Z": cfg.Z,
+                   "K": cfg.K, "I": cfg.I, "parallelism": "host cores"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle_threads(),
+                         "kind": "oracle",
+                         "sample": f"each step: {n_tok} consecutive tokens of the batch through "
+                                   "the whole fp64 oracle layer"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(C.CONFIGS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-baseline-tokens", type=int, default=4)
+    ap.add_argument("--ref-tokens", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line, L = run_gpu(args, rank, world, local_rank)
+        if line is not None:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(C.CONFIGS[args.workload], L,
+                                                    args.cpu_baseline_tokens)
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

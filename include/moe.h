@@ -159,6 +159,10 @@ moe_status moe_get_device_status(void* ws, void* stream, uint32_t* status_out);
 /* Message of the last error on the calling thread ("" if none). */
 const char* moe_last_error(void);
 
+/* Number of CUDA kernels this library has launched in the calling process
+ * (all devices, all threads).  Instrumentation only. */
+uint64_t moe_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

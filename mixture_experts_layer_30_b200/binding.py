@@ -42,6 +42,7 @@ SIGNATURES = {
     "moe_bias_update": (ctypes.c_int, [_i32, _i32, _vp, _i64, _i32, _f32, _f32, _vp, _vp]),
     "moe_get_device_status": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "moe_last_error": (ctypes.c_char_p, []),
+    "moe_kernel_launches": (ctypes.c_uint64, []),
 }
 
 _lib = None
@@ -179,6 +180,11 @@ def bias_update(N, Z, counts, T_all, K, K_e, mu, bias, stream=None):
     _check(lib().moe_bias_update(N, Z, _p(counts, torch.int32, "counts"), int(T_all), K,
                                  float(K_e), float(mu), _p(bias, torch.float32, "bias"),
                                  _stream(stream)))
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process."""
+    return int(lib().moe_kernel_launches())
 
 
 def device_status(ws, stream=None) -> int:

@@ -9,7 +9,16 @@
 
 #define MOE_DEV __device__ __forceinline__
 
+#include <atomic>
+
 namespace moe {
+
+// Process-wide count of kernel launches issued by this library.
+inline std::atomic<unsigned long long>& launch_counter() {
+  static std::atomic<unsigned long long> n{0};
+  return n;
+}
+inline void note_launch() { launch_counter().fetch_add(1, std::memory_order_relaxed); }
 
 constexpr int kMaxExperts = 1024;   // E = N + Z upper bound (one warp holds <= 32 per lane)
 constexpr int kPermChunk = 256;     // tokens per dispatch chunk (one thread per token)

@@ -512,6 +512,7 @@ inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUt
   long long grid = max_tiles < sms ? max_tiles : sms;
   if (grid < 1) grid = 1;
   gemm_tc_kernel<kMode><<<(int)grid, kThreads, kSmemBytes, st>>>(a0, a1, b, args);
+  note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     snprintf(err, errn, "tcgen05 gemm launch: %s", cudaGetErrorString(e));

@@ -27,6 +27,7 @@ moe_status fail(moe_status st, const char* fmt, ...) {
 }
 
 moe_status check_launch(const char* what) {
+  moe::note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
   return MOE_OK;
@@ -422,5 +423,7 @@ moe_status moe_get_device_status(void* ws, void* stream, uint32_t* status_out) {
 }
 
 const char* moe_last_error(void) { return g_err; }
+
+uint64_t moe_kernel_launches(void) { return moe::launch_counter().load(); }
 
 }  // extern "C"

@@ -15,7 +15,13 @@ from mixture_experts_layer_30_b200 import binding as B
 from oracle import moe_oracle as orc
 
 TIE_BAND = 1e-6
+# Router probabilities: the logits are fp32 sums of d bf16 products (tensor
+# cores accumulate in fp32 with truncated alignment inside each K=16 step).
+# A logit error delta changes p by about p * delta, so the bound is relative:
+# |p_gpu - p| <= PROB_ATOL + PROB_RTOL * p.  The top-K check does not depend
+# on it: it is exact outside the 1e-6 tie band.
 PROB_ATOL = 1e-6
+PROB_RTOL = 3e-5
 BF16_MAX_ABS, BF16_REL_L2 = 2e-2, 1e-2
 F32_MAX_ABS = 1e-4
 
@@ -113,14 +119,15 @@ def check_routing_and_dispatch(g, x64, wr64, bias, N, K, logit_offset=None):
     E = wr64.shape[0]
     off = None if logit_offset is None else logit_offset.detach().cpu().numpy().astype(np.float64)
     probs = orc.softmax_rows(orc.router_logits(x64, wr64, off))
-    np.testing.assert_allclose(g["probs"], probs, rtol=0, atol=PROB_ATOL)
+    np.testing.assert_allclose(g["probs"], probs, rtol=PROB_RTOL, atol=PROB_ATOL)
     b64 = bias.detach().cpu().numpy().astype(np.float64)
     oidx, margin = orc.biased_topk(probs, b64, K)
     ties = check_selection(g["idx"], probs + b64[None, :], oidx, K)
     idx_ref = oidx.copy()
     idx_ref[ties] = g["idx"][ties]
     np.testing.assert_array_equal(g["idx"], idx_ref)
-    np.testing.assert_allclose(g["gate"], orc.gates(probs, idx_ref), rtol=0, atol=PROB_ATOL)
+    np.testing.assert_allclose(g["gate"], orc.gates(probs, idx_ref), rtol=PROB_RTOL,
+                               atol=PROB_ATOL)
     np.testing.assert_array_equal(g["counts"], orc.expert_counts(idx_ref, E))
     np.testing.assert_array_equal(g["n_ffn"], orc.ffn_experts_per_token(idx_ref, N))
     off_o, rt_o, sp_o = orc.canonical_permutation(idx_ref, N)
