@@ -29,6 +29,7 @@ sys.path.insert(0, ROOT)
 
 from mixture_experts_layer_30_b200 import binding as B  # noqa: E402
 from mixture_experts_layer_30_b200 import configs as C  # noqa: E402
+from mixture_experts_layer_30_b200 import dist as MD  # noqa: E402
 from mixture_experts_layer_30_b200 import inputs as IN  # noqa: E402
 
 METRIC = "MoE-layer tokens/sec at LongCat shape (bf16) + % of tensor/HBM roofline"
@@ -125,7 +126,7 @@ def run_gpu(args, rank, world, local_rank):
     L = IN.make_layer_inputs(cfg, device=dev, base_seed=0)
     # every rank routes its own batch: x drawn with a per-rank seed
     if rank:
-        L["x"] = IN.make_x(cfg, dev, seed=rank * 1000 + 0 + 7_000_000)
+        L["x"] = IN.make_x(cfg, dev, seed=7_000_000 + rank)
     buf = B.LayerBuffers(shape, device=dev)
     bias = L["bias"].clone()
     counts_global = torch.empty_like(buf.counts)
@@ -149,12 +150,7 @@ def run_gpu(args, rank, world, local_rank):
         if ev: ev[4].record(stream)
         B.combine(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, cfg.gamma, buf.out)
         if ev: ev[5].record(stream)
-        if world > 1:
-            counts_global.copy_(buf.counts)
-            dist.all_reduce(counts_global)
-            c = counts_global
-        else:
-            c = buf.counts
+        c = MD.global_counts(buf.counts, counts_global) if world > 1 else buf.counts
         B.bias_update(cfg.N, cfg.Z, c, T_all, cfg.K, K_e, mu, bias)
         if ev: ev[6].record(stream)
 

@@ -11,3 +11,9 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) and the built CUDA library")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+
+
+def pytest_sessionstart(session):
+    # Rebuild the CUDA library if a source is newer than it (no-op otherwise).
+    from mixture_experts_layer_30_b200 import build
+    build.build()
