@@ -171,7 +171,8 @@ def test_bad_expert_index_sets_status_without_fault():
     B.route(shape, L["x"], L["w_router"], L["bias"], buf.ws, buf.topk_idx, buf.topk_gate,
             buf.counts, buf.n_ffn)
     bad = buf.topk_idx.clone()
-    bad[5, 1] = 99
+    t, k = [int(v) for v in (bad < shape.N).nonzero()[0]]   # an FFN slot
+    bad[t, k] = 99
     B.permute(shape, L["x"], bad, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
               buf.x_perm, buf.ws)
     st = B.device_status(buf.ws)
