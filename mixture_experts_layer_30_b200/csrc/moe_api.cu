@@ -143,8 +143,8 @@ moe_status route_impl(const moe_shape& s, const void* x, const void* w, const fl
       dim3 g((E + moe::kRgBN - 1) / moe::kRgBN, (s.T + moe::kRgBM - 1) / moe::kRgBM);
       moe::router_gemm_simt_kernel<T><<<g, 256, 0, st>>>(
           static_cast<const T*>(x), static_cast<const T*>(w), off, logits, s.T, E, s.d);
+      MOE_TRY(check_launch("router gemm"));
     }
-    MOE_TRY(check_launch("router gemm"));
     const int vpl = (E + 31) / 32;
     dim3 g(route_ctas(s));
     if (vpl <= 1) launch_topk<1>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
