@@ -22,7 +22,8 @@ inline void note_launch() { launch_counter().fetch_add(1, std::memory_order_rela
 
 constexpr int kMaxExperts = 1024;   // E = N + Z upper bound (one warp holds <= 32 per lane)
 constexpr int kPermChunk = 256;     // tokens per dispatch chunk (one thread per token)
-constexpr int kRouteTokensPerCta = 64;
+constexpr int kRouteTokensPerCta = 32;  // 16 warps x 2 tokens: enough warps to hide latency
+constexpr int kRouteThreads = 512;
 
 MOE_DEV void set_status(uint32_t* st, uint32_t bit) {
   if (st) atomicOr(st, bit);

@@ -130,6 +130,30 @@ MOE_DEV void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
       : "memory");
 }
+// Same copy with an L2 eviction-priority hint (a createpolicy value).
+MOE_DEV void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, int c0, int c1, uint32_t bar,
+                              uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar), "l"(policy)
+      : "memory");
+}
+// Weights are read once per step: evict them first.  Token tiles are re-read by
+// every feature block of their expert: keep them.
+MOE_DEV uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+MOE_DEV uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+// SiLU for the bf16 epilogue: a / (1 + e^-a) with the fast exponential and
+// division intrinsics (relative error ~1e-6, far below the bf16 rounding of h).
+MOE_DEV float silu_fast(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 MOE_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -284,6 +308,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       // ---------------- TMA producer ----------------
       uint32_t stage = 0, phase = 0;
       bool ok = true;
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_last();
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const Tile t = decode_tile(tile, n_fblk, args, prefix);
         const int nbox = (t.n + kBoxRows - 1) / kBoxRows;
@@ -298,11 +324,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
           const uint32_t fb = full0 + 8 * stage;
           const uint32_t sa0 = smem_u32(stages + stage * kStageBytes);
           mbar_arrive_expect_tx(fb, tx);
-          tma_load_2d(sa0, &tmA0, kb * kBK, a_row0, fb);
-          tma_load_2d(sa0 + kABytes, &tmA1, kb * kBK, a_row1, fb);
+          tma_load_2d_hint(sa0, &tmA0, kb * kBK, a_row0, fb, pol_w);
+          tma_load_2d_hint(sa0 + kABytes, &tmA1, kb * kBK, a_row1, fb, pol_w);
           for (int b = 0; b < nbox; ++b)
-            tma_load_2d(sa0 + 2 * kABytes + b * kBoxBytes, &tmB, kb * kBK, t.r0 + b * kBoxRows,
-                        fb);
+            tma_load_2d_hint(sa0 + 2 * kABytes + b * kBoxBytes, &tmB, kb * kBK,
+                             t.r0 + b * kBoxRows, fb, pol_x);
           ++issued;
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
@@ -375,8 +401,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-              float a0 = silu(__uint_as_float(v0[j])) * __uint_as_float(v1[j]);
-              float a1 = silu(__uint_as_float(v0[j + 1])) * __uint_as_float(v1[j + 1]);
+              float a0 = silu_fast(__uint_as_float(v0[j])) * __uint_as_float(v1[j]);
+              float a1 = silu_fast(__uint_as_float(v0[j + 1])) * __uint_as_float(v1[j + 1]);
               v0[j] = pack_bf16x2(a0, a1);
             }
           } else {

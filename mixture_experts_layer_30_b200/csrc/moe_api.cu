@@ -122,8 +122,8 @@ template <int VPL>
 void launch_topk(dim3 grid, cudaStream_t st, const float* logits, const float* bias, int T,
                  int E, int N, int K, int32_t* idx, float* gate, uint8_t* nffn, float* probs,
                  int32_t* hist) {
-  moe::softmax_topk_kernel<VPL><<<grid, 256, 0, st>>>(logits, bias, T, E, N, K, idx, gate,
-                                                      nffn, probs, hist);
+  moe::softmax_topk_kernel<VPL><<<grid, moe::kRouteThreads, 0, st>>>(
+      logits, bias, T, E, N, K, idx, gate, nffn, probs, hist);
 }
 
 template <typename T>
@@ -157,7 +157,7 @@ moe_status route_impl(const moe_shape& s, const void* x, const void* w, const fl
     else launch_topk<32>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
     MOE_TRY(check_launch("softmax/top-K"));
   }
-  moe::reduce_hist_kernel<<<(E + 255) / 256, 256, 0, st>>>(hist, route_ctas(s), E, counts);
+  moe::reduce_hist_kernel<<<(E + 7) / 8, 256, 0, st>>>(hist, route_ctas(s), E, counts);
   return check_launch("count reduce");
 }
 

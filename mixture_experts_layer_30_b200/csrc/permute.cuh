@@ -112,11 +112,13 @@ perm_rank_kernel(const int32_t* __restrict__ topk_idx, int T, int K, int N, int 
   }
 }
 
-// One warp per token; copies x[t] (16-byte vectors) to every row of the token.
+// One warp per token: the x row is read once from HBM, in pieces of 8 x 16 B
+// per lane held in registers, and each piece is stored to every row of the token.
 template <typename T>
 __global__ void __launch_bounds__(256)
 gather_kernel(const T* __restrict__ x, const int32_t* __restrict__ slot_pos, int ntok, int K,
               int d, T* __restrict__ x_perm) {
+  constexpr int kPiece = 8;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= ntok) return;
@@ -124,14 +126,28 @@ gather_kernel(const T* __restrict__ x, const int32_t* __restrict__ slot_pos, int
   const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
   for (int kb = 0; kb < K; kb += 32) {
     // rows of slots kb..kb+31 of this token (lane j holds slot kb+j's row)
-    int my_row = kb + lane < K ? slot_pos[(size_t)t * K + kb + lane] : -1;
-    uint32_t has = __ballot_sync(0xffffffffu, my_row >= 0);
-    while (has) {
-      int j = __ffs(has) - 1;
-      has &= has - 1;
-      int row = __shfl_sync(0xffffffffu, my_row, j);
-      uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * d);
-      for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    const int my_row = kb + lane < K ? slot_pos[(size_t)t * K + kb + lane] : -1;
+    const uint32_t rows = __ballot_sync(0xffffffffu, my_row >= 0);
+    if (!rows) continue;
+    for (int v0 = 0; v0 < nvec; v0 += 32 * kPiece) {
+      uint4 piece[kPiece];
+#pragma unroll
+      for (int i = 0; i < kPiece; ++i) {
+        const int v = v0 + i * 32 + lane;
+        if (v < nvec) piece[i] = __ldg(src + v);
+      }
+      uint32_t has = rows;
+      while (has) {
+        const int j = __ffs(has) - 1;
+        has &= has - 1;
+        const int row = __shfl_sync(0xffffffffu, my_row, j);
+        uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * d);
+#pragma unroll
+        for (int i = 0; i < kPiece; ++i) {
+          const int v = v0 + i * 32 + lane;
+          if (v < nvec) dst[v] = piece[i];
+        }
+      }
     }
   }
 }

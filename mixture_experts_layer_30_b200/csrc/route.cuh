@@ -62,7 +62,7 @@ router_gemm_simt_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
 // One warp per token.  Lane l holds experts e = l + 32*j, j < VPL.
 // Selection key: (R_e + b_e) descending, then e ascending (lower index wins ties).
 template <int VPL>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kRouteThreads)
 softmax_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
                     int E, int N, int K, int32_t* __restrict__ topk_idx,
                     float* __restrict__ topk_gate, uint8_t* __restrict__ n_ffn,
@@ -147,14 +147,19 @@ softmax_topk_kernel(const float* __restrict__ logits, const float* __restrict__ 
     partial_hist[(size_t)blockIdx.x * E + e] = hist[e];
 }
 
-// counts[e] = sum over route CTAs of their partial histograms (fixed order).
-__global__ void reduce_hist_kernel(const int32_t* __restrict__ partial, int nparts, int E,
-                                   int32_t* __restrict__ counts) {
-  int e = blockIdx.x * blockDim.x + threadIdx.x;
+// counts[e] = sum over route CTAs of their partial histograms.  One warp per
+// expert; integer sums, so the result does not depend on the order.
+__global__ void __launch_bounds__(256)
+reduce_hist_kernel(const int32_t* __restrict__ partial, int nparts, int E,
+                   int32_t* __restrict__ counts) {
+  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   if (e >= E) return;
   int c = 0;
-  for (int p = 0; p < nparts; ++p) c += partial[(size_t)p * E + e];
-  counts[e] = c;
+  for (int p = lane; p < nparts; p += 32) c += partial[(size_t)p * E + e];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0) counts[e] = c;
 }
 
 }  // namespace moe
