@@ -113,6 +113,33 @@ moe_status moe_permute(const moe_shape* shape, const void* x, const int32_t* top
                        int32_t* slot_pos, void* x_perm, void* ws, size_t ws_bytes,
                        void* stream);
 
+/* moe_permute without a workspace argument.  The paper has no counterpart:
+ * this entry point exists for callers that cannot give the library scratch
+ * memory -- operator plug-ins whose interface hands over only the input and
+ * output buffers of a call, and runtimes that plan all device memory at
+ * start-up and refuse allocations afterwards.  It computes exactly what
+ * moe_permute computes, with the same arguments minus ws/ws_bytes, and it
+ * allocates nothing.
+ *
+ * Scratch: one 4 MiB array in device memory owned by the library, present on
+ * every device that loads it until the process exits.  Limit:
+ * 2*ceil(T/256)*N*4 + 512 bytes must fit in 4 MiB (for example T <= 131072
+ * tokens at N = 1024); larger shapes return MOE_ERR_UNSUPPORTED with a
+ * message and launch nothing.
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture.
+ * Sharing: every call on a device uses the same array and leaves its contents
+ * behind (each call overwrites what it reads, so nothing carries over).  Calls
+ * whose kernels overlap on the GPU -- on different streams, or from different
+ * host threads -- race on the array and must be serialised by the caller.
+ * Device-side consistency bits (bad expert index, count mismatch) go to the
+ * array's own status word and are not reported; use moe_permute with a
+ * workspace and moe_get_device_status to read them. */
+moe_status moe_permute_noalloc(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                               const int32_t* counts, int32_t* offsets, int32_t* row_token,
+                               int32_t* slot_pos, void* x_perm, void* stream);
+
 /* First half of the SwiGLU experts on the routed rows:
  *   h[r, :] = SiLU(x_perm[r, :] W1_e^T) * (x_perm[r, :] W3_e^T)   for rows r of expert e.
  * x_perm [T*K, d], w1/w3 [N, I, d], offsets [N+1] (from moe_permute),

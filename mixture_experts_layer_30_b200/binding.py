@@ -35,6 +35,7 @@ SIGNATURES = {
     "moe_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
     "moe_route": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_noalloc": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_expert_gate_up": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_down": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_ffn": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -141,6 +142,20 @@ def permute(shape, x, topk_idx, counts, offsets, row_token, slot_pos, x_perm, ws
                              _p(row_token, torch.int32, "row_token"),
                              _p(slot_pos, torch.int32, "slot_pos"), _p(x_perm, dt, "x_perm"),
                              _p(ws), ws.numel(), _stream(stream)))
+
+
+def permute_noalloc(shape, x, topk_idx, counts, offsets, row_token, slot_pos, x_perm,
+                    stream=None):
+    """moe_permute for callers that cannot provide a workspace: the dispatch
+    scratch lives in a fixed 4 MiB device array owned by the library."""
+    dt = torch_dtype(shape)
+    _check(lib().moe_permute_noalloc(ctypes.byref(shape), _p(x, dt, "x"),
+                                     _p(topk_idx, torch.int32, "topk_idx"),
+                                     _p(counts, torch.int32, "counts"),
+                                     _p(offsets, torch.int32, "offsets"),
+                                     _p(row_token, torch.int32, "row_token"),
+                                     _p(slot_pos, torch.int32, "slot_pos"),
+                                     _p(x_perm, dt, "x_perm"), _stream(stream)))
 
 
 def expert_gate_up(shape, x_perm, w1, w3, offsets, h, ws, stream=None):

@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "moe.h"
 #include "common.cuh"
@@ -242,6 +243,47 @@ moe_status down_impl(const moe_shape& s, const void* h, const void* w2, const in
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Dispatch without a caller-provided workspace (moe_permute_noalloc).
+//
+// Some callers cannot give this library any device memory beyond the tensors
+// of the call itself: operator plug-ins of frameworks whose interface passes
+// only input and output buffers, and runtimes that plan every device
+// allocation at start-up and refuse allocations afterwards.  For them the
+// dispatch step keeps its scratch (two [chunks x N] int32 tables and a status
+// word) in one fixed array in device memory that the library owns.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 4u << 20;  // 4 MiB, held on every device until exit
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_dev_ptr[64] = {};  // device address of the array, per device
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device and cached.
+moe_status noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(MOE_ERR_UNSUPPORTED, "device ordinal %d >= 64", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_dev_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress of the dispatch scratch: %s",
+                  cudaGetErrorString(e));
+    g_noalloc_dev_ptr[dev] = p;
+  }
+  *out = g_noalloc_dev_ptr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 size_t moe_workspace_bytes(const moe_shape* shape) {
@@ -306,6 +348,42 @@ moe_status moe_permute(const moe_shape* shape, const void* x, const int32_t* top
                                        x_perm, ws, L, st);
   return permute_impl<float>(s, x, topk_idx, counts, offsets, row_token, slot_pos, x_perm, ws,
                              L, st);
+}
+
+moe_status moe_permute_noalloc(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                               const int32_t* counts, int32_t* offsets, int32_t* row_token,
+                               int32_t* slot_pos, void* x_perm, void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  MOE_TRY(need(offsets, "offsets", 4));
+  if (s.T > 0) {
+    MOE_TRY(need(x, "x", 16));
+    MOE_TRY(need(topk_idx, "topk_idx", 4));
+    MOE_TRY(need(row_token, "row_token", 4));
+    MOE_TRY(need(slot_pos, "slot_pos", 4));
+    MOE_TRY(need(x_perm, "x_perm", 16));
+  }
+  const size_t table = align256((size_t)perm_chunks(s) * s.N * sizeof(int32_t));
+  const size_t bytes = 256 + 2 * table;
+  if (bytes > kNoAllocScratchBytes)
+    return fail(MOE_ERR_UNSUPPORTED,
+                "moe_permute_noalloc: T=%d, N=%d needs %zu bytes of dispatch scratch but the "
+                "built-in array holds %zu (2*ceil(T/256)*N*4 + 512 must fit); use moe_permute "
+                "with a workspace",
+                s.T, s.N, bytes, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  MOE_TRY(noalloc_scratch(&scratch));
+  WsLayout L{};
+  L.status = 0;
+  L.perm_hist = 256;
+  L.perm_base = 256 + table;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.dtype == MOE_BF16)
+    return permute_impl<__nv_bfloat16>(s, x, topk_idx, counts, offsets, row_token, slot_pos,
+                                       x_perm, scratch, L, st);
+  return permute_impl<float>(s, x, topk_idx, counts, offsets, row_token, slot_pos, x_perm,
+                             scratch, L, st);
 }
 
 moe_status moe_expert_gate_up(const moe_shape* shape, const void* x_perm, const void* w1,
