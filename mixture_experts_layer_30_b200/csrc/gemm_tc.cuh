@@ -12,8 +12,8 @@
 //   warp 0      TMA producer (one lane): A0, A1 weight tiles + B token tile per stage
 //   warp 1      MMA issuer (one lane); also allocates/frees the 512 TMEM columns
 //   warps 2..5  epilogue: TMEM -> registers -> (SwiGLU | copy) -> shared -> global
-// Pipeline: kStages shared-memory stages guarded by full/empty mbarriers, one
-// TMEM accumulator pair guarded by tmem_full/tmem_empty.  Every wait is bounded
+// Pipeline: kStages shared-memory stages guarded by full/empty mbarriers, one or
+// two TMEM accumulator pairs guarded by tmem_full/tmem_empty.  Every wait is bounded
 // in time; on expiry the CTA raises MOE_DEV_PIPELINE_TIMEOUT, drains what it
 // issued and returns.
 //
@@ -36,24 +36,38 @@ namespace tc {
 
 constexpr int kBK = 64;                          // K elements per stage = one 128-byte row
 constexpr int kFeat = 128;                       // UMMA M
-constexpr int kNMax = 256;                       // token rows per tile (UMMA N <= 256)
 constexpr int kBoxRows = 32;                     // rows per token TMA box
-constexpr int kStages = 3;
 constexpr int kABytes = kFeat * kBK * 2;         // 16 KiB
 constexpr int kBoxBytes = kBoxRows * kBK * 2;    // 4 KiB
-constexpr int kBBytes = kNMax * kBK * 2;         // 32 KiB
-constexpr int kStageBytes = 2 * kABytes + kBBytes;
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
 constexpr int kStagingPitch = 36;                // 32-bit words per staging row (32 + pad)
 constexpr int kStagingBytes = kEpiWarps * 32 * kStagingPitch * 4;
-constexpr int kTmemCols = 512;
-constexpr int kNumBars = 2 * kStages + 3;        // full[], empty[], tmem_full, tmem_empty, drain
 constexpr int kCtrlBytes = 256;                  // barriers + tmem slot + abort flag
-constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kStagingBytes + kCtrlBytes +
-                           (kMaxExperts + 1 + 33) * 4;
 constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;  // 4 s
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;  // 0.2 s
+
+// Tile geometry: up to kNMax token rows per tile (UMMA N), kStages shared-memory
+// stages.  The D0/D1 accumulator pair takes 2*kNMax TMEM columns; when two
+// pairs fit in the 512 columns the accumulators are double-buffered, so the
+// epilogue of one tile overlaps the MMAs of the next.
+template <int NMAX, int STAGES>
+struct TileCfg {
+  static constexpr int kNMax = NMAX;
+  static constexpr int kStages = STAGES;
+  static constexpr int kAccBufs = (4 * NMAX <= 512) ? 2 : 1;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kBBytes = NMAX * kBK * 2;
+  static constexpr int kStageBytes = 2 * kABytes + kBBytes;
+  static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs + 1;  // full, empty, acc full/empty, drain
+  static constexpr int kSmemBytes =
+      1024 + STAGES * kStageBytes + kStagingBytes + kCtrlBytes + (kMaxExperts + 1 + 33) * 4;
+  static_assert(NMAX % kBoxRows == 0 && NMAX <= 256, "token tile");
+  static_assert(8 * kNumBars + 12 <= kCtrlBytes, "control block");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+using CfgWide = TileCfg<256, 3>;    // ragged segments up to 256 rows, one accumulator pair
+using CfgDouble = TileCfg<128, 4>;  // <= 128 rows, double-buffered accumulators
 
 enum Mode { kGated = 0, kPlainBf16 = 1, kPlainF32 = 2 };
 
@@ -215,6 +229,7 @@ struct Tile {
   int seg, r0, n, f0;
 };
 
+template <int kNMax>
 MOE_DEV Tile decode_tile(int tile, int n_fblk, const Args& a, const int* prefix) {
   Tile t;
   const int chunk = tile / n_fblk;
@@ -238,10 +253,13 @@ MOE_DEV Tile decode_tile(int tile, int n_fblk, const Args& a, const int* prefix)
 }
 
 // --- the kernel ------------------------------------------------------------------
-template <int kMode>
+template <int kMode, class Cfg>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                const __grid_constant__ CUtensorMap tmB, const Args args) {
+  constexpr int kNMax = Cfg::kNMax, kStages = Cfg::kStages, kAccBufs = Cfg::kAccBufs;
+  constexpr int kStageBytes = Cfg::kStageBytes, kNumBars = Cfg::kNumBars;
+  constexpr int kTmemCols = Cfg::kTmemCols;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -258,17 +276,19 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(&bars[0]);
   const uint32_t empty0 = smem_u32(&bars[kStages]);
-  const uint32_t tmem_full = smem_u32(&bars[2 * kStages]);
-  const uint32_t tmem_empty = smem_u32(&bars[2 * kStages + 1]);
-  const uint32_t drain_bar = smem_u32(&bars[2 * kStages + 2]);
+  const uint32_t tmem_full0 = smem_u32(&bars[2 * kStages]);             // + 8 * buffer
+  const uint32_t tmem_empty0 = smem_u32(&bars[2 * kStages + kAccBufs]);  // + 8 * buffer
+  const uint32_t drain_bar = smem_u32(&bars[2 * kStages + 2 * kAccBufs]);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
-    mbar_init(tmem_full, 1);
-    mbar_init(tmem_empty, kEpiWarps * 32);
+    for (int b = 0; b < kAccBufs; ++b) {
+      mbar_init(tmem_full0 + 8 * b, 1);
+      mbar_init(tmem_empty0 + 8 * b, kEpiWarps * 32);
+    }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     *consumed_sh = 0;
@@ -311,7 +331,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const Tile t = decode_tile(tile, n_fblk, args, prefix);
+        const Tile t = decode_tile<kNMax>(tile, n_fblk, args, prefix);
         const int nbox = (t.n + kBoxRows - 1) / kBoxRows;
         const uint32_t tx = 2 * kABytes + nbox * kBoxBytes;
         const int a_row0 = t.seg * args.a_seg_rows + t.f0;
@@ -338,16 +358,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      uint32_t stage = 0, phase = 0, acc_phase = 0;
+      uint32_t stage = 0, phase = 0;
       bool ok = true;
-      int consumed = 0;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const Tile t = decode_tile(tile, n_fblk, args, prefix);
+      int consumed = 0, local = 0;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
+        const Tile t = decode_tile<kNMax>(tile, n_fblk, args, prefix);
         int n16 = ((t.n + 15) >> 4) << 4;
         if (n16 < 16) n16 = 16;
         const uint32_t idesc = idesc_bf16(kFeat, n16);
-        if (!mbar_wait(tmem_empty, acc_phase ^ 1, abort_flag, args.status)) break;
-        acc_phase ^= 1;
+        const int buf = local % kAccBufs;
+        const uint32_t acc_parity = (uint32_t)((local / kAccBufs) & 1);
+        const uint32_t d0 = tmem_base + buf * 2 * kNMax;
+        if (!mbar_wait(tmem_empty0 + 8 * buf, acc_parity ^ 1, abort_flag, args.status)) break;
         tc_fence_after();
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.status)) {
@@ -363,15 +385,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
           for (int k = 0; k < kBK / 16; ++k) {
             // advance 16 bf16 = 32 bytes along K inside the swizzled row
             const uint32_t acc = (kb | k) != 0;
-            umma_bf16(tmem_base, da0 + 2 * k, db + 2 * k, idesc, acc);
-            umma_bf16(tmem_base + kNMax, da1 + 2 * k, db + 2 * k, idesc, acc);
+            umma_bf16(d0, da0 + 2 * k, db + 2 * k, idesc, acc);
+            umma_bf16(d0 + kNMax, da1 + 2 * k, db + 2 * k, idesc, acc);
           }
           umma_commit(empty0 + 8 * stage);
           ++consumed;
           *consumed_sh = consumed;
           if (++stage == kStages) { stage = 0; phase ^= 1; }
         }
-        if (ok) umma_commit(tmem_full);
+        if (ok) umma_commit(tmem_full0 + 8 * buf);
       }
       // every MMA issued so far completes before TMEM is released
       umma_commit(drain_bar);
@@ -382,22 +404,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     // ---------------- epilogue (warps 2..5) ----------------
     const int q = warp & 3;                      // TMEM lane quarter this warp may access
     uint32_t* stg = staging + (warp - 2) * 32 * kStagingPitch;
-    uint32_t acc_phase = 0;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const Tile t = decode_tile(tile, n_fblk, args, prefix);
-      if (!mbar_wait(tmem_full, acc_phase, abort_flag, args.status)) break;
-      acc_phase ^= 1;
+    int local = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
+      const Tile t = decode_tile<kNMax>(tile, n_fblk, args, prefix);
+      const int buf = local % kAccBufs;
+      const uint32_t acc_parity = (uint32_t)((local / kAccBufs) & 1);
+      const uint32_t dbase = tmem_base + lane_base + buf * 2 * kNMax;
+      if (!mbar_wait(tmem_full0 + 8 * buf, acc_parity, abort_flag, args.status)) break;
       tc_fence_after();
       const int nhalves = (kMode == kGated) ? 1 : 2;
       for (int hf = 0; hf < nhalves; ++hf) {
         const int fbase = t.f0 + hf * kFeat + 32 * q;   // first feature of this warp
         for (int j0 = 0; j0 < t.n; j0 += 32) {
           uint32_t v0[32];
-          tmem_ld_32x32b_x32(tmem_base + lane_base + hf * kNMax + j0, v0);
+          tmem_ld_32x32b_x32(dbase + hf * kNMax + j0, v0);
           if (kMode == kGated) {
             uint32_t v1[32];
-            tmem_ld_32x32b_x32(tmem_base + lane_base + kNMax + j0, v1);
+            tmem_ld_32x32b_x32(dbase + kNMax + j0, v1);
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
@@ -460,7 +484,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
         }
       }
       tc_fence_before();
-      mbar_arrive(tmem_empty);
+      mbar_arrive(tmem_empty0 + 8 * buf);
     }
   }
 
@@ -519,7 +543,7 @@ inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
   return r == CUDA_SUCCESS;
 }
 
-template <int kMode>
+template <int kMode, class Cfg>
 inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                          const Args& args, long long max_tiles, int sms, cudaStream_t st,
                          char* err, size_t errn) {
@@ -527,8 +551,9 @@ inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUt
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kMode>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kMode, Cfg>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Cfg::kSmemBytes);
     if (e != cudaSuccess) {
       snprintf(err, errn, "tcgen05 gemm smem attribute: %s", cudaGetErrorString(e));
       return MOE_ERR_CUDA;
@@ -537,7 +562,7 @@ inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUt
   }
   long long grid = max_tiles < sms ? max_tiles : sms;
   if (grid < 1) grid = 1;
-  gemm_tc_kernel<kMode><<<(int)grid, kThreads, kSmemBytes, st>>>(a0, a1, b, args);
+  gemm_tc_kernel<kMode, Cfg><<<(int)grid, kThreads, Cfg::kSmemBytes, st>>>(a0, a1, b, args);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -553,10 +578,18 @@ inline moe_status map_error(char* err, size_t errn, const char* what) {
 }
 
 // Upper bound of (row chunk, feature block) tiles for routed rows.
-inline long long routed_tiles(const moe_shape& s, int n_out, int feat) {
+inline long long routed_tiles(const moe_shape& s, int n_out, int feat, int nmax) {
   const long long rows = (long long)s.T * s.K;
-  const long long chunks = s.N + (rows + kNMax - 1) / kNMax;
+  const long long chunks = s.N + (rows + nmax - 1) / nmax;
   return chunks * ((n_out + feat - 1) / feat);
+}
+
+// Expert GEMM geometry: the wide tile keeps every segment of up to 256 rows in
+// one tile (each weight tile streamed once); the double-buffered tile is used
+// when segments are short on average.
+constexpr int kDoubleBufferMaxMeanRows = 0;  // mean routed rows per expert at or below: CfgDouble
+inline bool use_double(const moe_shape& s) {
+  return (long long)s.T * s.K <= (long long)kDoubleBufferMaxMeanRows * (s.N + s.Z);
 }
 
 inline moe_status launch_gate_up(const moe_shape& s, const void* x_perm, const void* w1,
@@ -579,7 +612,11 @@ inline moe_status launch_gate_up(const moe_shape& s, const void* x_perm, const v
   a.feat_per_tile = kFeat;
   a.out = h;
   a.status = status;
-  return launch<kGated>(a0, a1, b, a, routed_tiles(s, s.I, kFeat), sms, st, err, errn);
+  if (use_double(s))
+    return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
+                                     sms, st, err, errn);
+  return launch<kGated, CfgWide>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgWide::kNMax), sms,
+                                 st, err, errn);
 }
 
 inline moe_status launch_down(const moe_shape& s, const void* h, const void* w2,
@@ -600,7 +637,12 @@ inline moe_status launch_down(const moe_shape& s, const void* h, const void* w2,
   g.feat_per_tile = 2 * kFeat;
   g.out = y_perm;
   g.status = status;
-  return launch<kPlainBf16>(a, a, b, g, routed_tiles(s, s.d, 2 * kFeat), sms, st, err, errn);
+  if (use_double(s))
+    return launch<kPlainBf16, CfgDouble>(a, a, b, g,
+                                         routed_tiles(s, s.d, 2 * kFeat, CfgDouble::kNMax), sms,
+                                         st, err, errn);
+  return launch<kPlainBf16, CfgWide>(a, a, b, g, routed_tiles(s, s.d, 2 * kFeat, CfgWide::kNMax),
+                                     sms, st, err, errn);
 }
 
 inline moe_status launch_router_gemm(const moe_shape& s, const void* x, const void* w,
@@ -623,8 +665,9 @@ inline moe_status launch_router_gemm(const moe_shape& s, const void* x, const vo
   g.out = logits;
   g.add = offset;
   g.status = nullptr;
-  const long long tiles = (long long)((s.T + kNMax - 1) / kNMax) * ((E + 2 * kFeat - 1) / (2 * kFeat));
-  return launch<kPlainF32>(a, a, b, g, tiles, sms, st, err, errn);
+  const long long tiles =
+      (long long)((s.T + CfgWide::kNMax - 1) / CfgWide::kNMax) * ((E + 2 * kFeat - 1) / (2 * kFeat));
+  return launch<kPlainF32, CfgWide>(a, a, b, g, tiles, sms, st, err, errn);
 }
 
 }  // namespace tc
