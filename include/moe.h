@@ -107,7 +107,10 @@ moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router
  *   or -1 when topk_idx[t, k] >= N;  x_perm[r, :] = x[row_token[r], :].
  * topk_idx [T, K] int32, counts [E] int32 (checked against topk_idx; a mismatch
  * sets MOE_DEV_COUNT_MISMATCH and topk_idx wins), offsets [N+1] int32,
- * row_token [T*K] int32, slot_pos [T, K] int32, x_perm [T*K, d] (dtype). */
+ * row_token [T*K] int32, slot_pos [T, K] int32, x_perm [T*K, d] (dtype).
+ * x_perm may be NULL: the layout (offsets, row_token, slot_pos) is built and
+ * no row is copied; moe_expert_gate_up_gather then reads x through row_token
+ * (x itself may also be NULL in that case). */
 moe_status moe_permute(const moe_shape* shape, const void* x, const int32_t* topk_idx,
                        const int32_t* counts, int32_t* offsets, int32_t* row_token,
                        int32_t* slot_pos, void* x_perm, void* ws, size_t ws_bytes,
@@ -147,6 +150,16 @@ moe_status moe_permute_noalloc(const moe_shape* shape, const void* x, const int3
 moe_status moe_expert_gate_up(const moe_shape* shape, const void* x_perm, const void* w1,
                               const void* w3, const int32_t* offsets, void* h, void* ws,
                               size_t ws_bytes, void* stream);
+
+/* moe_expert_gate_up with the dispatch copy fused in: the token rows are read
+ * from x through row_token (from moe_permute) instead of from x_perm,
+ *   h[r, :] = SiLU(x[row_token[r], :] W1_e^T) * (x[row_token[r], :] W3_e^T).
+ * x [T, d], row_token [T*K] int32; the other arguments as moe_expert_gate_up.
+ * A row_token entry outside [0, T) sets MOE_DEV_BAD_OFFSETS and reads row 0. */
+moe_status moe_expert_gate_up_gather(const moe_shape* shape, const void* x,
+                                     const int32_t* row_token, const void* w1, const void* w3,
+                                     const int32_t* offsets, void* h, void* ws, size_t ws_bytes,
+                                     void* stream);
 
 /* Second half: y_perm[r, :] = h[r, :] W2_e^T.  h [T*K, I], w2 [N, d, I],
  * y_perm [T*K, d] (dtype). */

@@ -37,6 +37,8 @@ SIGNATURES = {
     "moe_permute": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_noalloc": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_expert_gate_up": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_gate_up_gather": (ctypes.c_int,
+                                  [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_down": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_ffn": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_combine": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp]),
@@ -134,6 +136,7 @@ def route(shape, x, w_router, bias, ws, topk_idx, topk_gate, counts, n_ffn,
 
 
 def permute(shape, x, topk_idx, counts, offsets, row_token, slot_pos, x_perm, ws, stream=None):
+    """x_perm=None builds the layout only (no copy of the token rows)."""
     dt = torch_dtype(shape)
     _check(lib().moe_permute(ctypes.byref(shape), _p(x, dt, "x"),
                              _p(topk_idx, torch.int32, "topk_idx"),
@@ -164,6 +167,15 @@ def expert_gate_up(shape, x_perm, w1, w3, offsets, h, ws, stream=None):
                                     _p(w1, dt, "w1"), _p(w3, dt, "w3"),
                                     _p(offsets, torch.int32, "offsets"), _p(h, dt, "h"),
                                     _p(ws), ws.numel(), _stream(stream)))
+
+
+def expert_gate_up_gather(shape, x, row_token, w1, w3, offsets, h, ws, stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_expert_gate_up_gather(ctypes.byref(shape), _p(x, dt, "x"),
+                                           _p(row_token, torch.int32, "row_token"),
+                                           _p(w1, dt, "w1"), _p(w3, dt, "w3"),
+                                           _p(offsets, torch.int32, "offsets"), _p(h, dt, "h"),
+                                           _p(ws), ws.numel(), _stream(stream)))
 
 
 def expert_down(shape, h, w2, offsets, y_perm, ws, stream=None):
@@ -236,14 +248,21 @@ class LayerBuffers:
 
 
 def forward(buf: LayerBuffers, x, w_router, w1, w3, w2, bias, gamma=1.0, logit_offset=None,
-            stream=None, split_ffn=False):
-    """route -> permute -> expert FFN -> combine; returns buf.out."""
+            stream=None, split_ffn=False, fused_gather=False):
+    """route -> permute -> expert FFN -> combine; returns buf.out.
+
+    split_ffn: gate/up and down as two calls (h in buf.h); fused_gather: no
+    x_perm copy, the gate/up GEMM reads x through row_token."""
     s = buf.shape
     route(s, x, w_router, bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts, buf.n_ffn,
           logit_offset=logit_offset, probs_out=buf.probs, stream=stream)
     permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
-            buf.x_perm, buf.ws, stream=stream)
-    if split_ffn:
+            None if fused_gather else buf.x_perm, buf.ws, stream=stream)
+    if fused_gather:
+        expert_gate_up_gather(s, x, buf.row_token, w1, w3, buf.offsets, buf.h, buf.ws,
+                              stream=stream)
+        expert_down(s, buf.h, w2, buf.offsets, buf.y_perm, buf.ws, stream=stream)
+    elif split_ffn:
         expert_gate_up(s, buf.x_perm, w1, w3, buf.offsets, buf.h, buf.ws, stream=stream)
         expert_down(s, buf.h, w2, buf.offsets, buf.y_perm, buf.ws, stream=stream)
     else:

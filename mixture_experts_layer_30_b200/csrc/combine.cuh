@@ -24,25 +24,42 @@ combine_kernel(const T* __restrict__ x, const T* __restrict__ y_perm,
   __shared__ int s_nffn;
   __shared__ float s_zero;
   const int t = blockIdx.x;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < 32) {
+    // Warp 0 reads the K slots 32 at a time, compacts the FFN slots in k order
+    // and sums the zero-expert gates in k order (adding 0 for other slots
+    // leaves the sum unchanged, so the order of the additions is exactly k).
+    const int lane = threadIdx.x;
+    const uint32_t lt = (1u << lane) - 1u;
     int n = 0;
     float zs = 0.f;
-    for (int k = 0; k < K; ++k) {
-      int e = topk_idx[(size_t)t * K + k];
-      float g = topk_gate[(size_t)t * K + k];
-      if (e < 0 || e >= E) { set_status(status, MOE_DEV_BAD_EXPERT_INDEX); continue; }
-      if (e < N) {
-        int r = slot_pos[(size_t)t * K + k];
-        if (r < 0 || r >= max_rows) { set_status(status, MOE_DEV_BAD_OFFSETS); continue; }
-        s_row[n] = r;
-        s_g[n] = g;
-        ++n;
-      } else {
-        zs += g;  // zero-expert gate mass, k order
+    for (int kb = 0; kb < K; kb += 32) {
+      const int k = kb + lane;
+      int e = -1, r = -1;
+      float g = 0.f;
+      if (k < K) {
+        e = topk_idx[(size_t)t * K + k];
+        g = topk_gate[(size_t)t * K + k];
+        if (e >= 0 && e < N) r = slot_pos[(size_t)t * K + k];
       }
+      if (k < K && (e < 0 || e >= E)) set_status(status, MOE_DEV_BAD_EXPERT_INDEX);
+      const bool is_ffn = k < K && e >= 0 && e < N;
+      const bool row_ok = r >= 0 && r < max_rows;
+      if (is_ffn && !row_ok) set_status(status, MOE_DEV_BAD_OFFSETS);
+      const uint32_t take = __ballot_sync(0xffffffffu, is_ffn && row_ok);
+      if (is_ffn && row_ok) {
+        const int pos = n + __popc(take & lt);
+        s_row[pos] = r;
+        s_g[pos] = g;
+      }
+      n += __popc(take);
+      const float gz = (k < K && e >= N && e < E) ? g : 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) zs += __shfl_sync(0xffffffffu, gz, j);
     }
-    s_nffn = n;
-    s_zero = zs;
+    if (lane == 0) {
+      s_nffn = n;
+      s_zero = zs;
+    }
   }
   __syncthreads();
   const int nffn = s_nffn;

@@ -1,6 +1,7 @@
 // Grouped expert GEMMs on CUDA cores (fp32 path; also the small-shape bf16 path).
 //
-// For each FFN expert e with routed rows [offsets[e], offsets[e+1]):
+// For each FFN expert e with routed rows [offsets[e], offsets[e+1]) (row r of
+// A is A[r], or A[a_rows[r]] when the rows are gathered from the token matrix):
 //   gated (first half of the SwiGLU expert):
 //       C[r, n] = SiLU(sum_k A[r,k] B0[e][n,k]) * (sum_k A[r,k] B1[e][n,k])
 //   plain (second half):
@@ -22,7 +23,7 @@ __global__ void __launch_bounds__(256)
 grouped_gemm_simt_kernel(const TIn* __restrict__ A, const TIn* __restrict__ B0,
                          const TIn* __restrict__ B1, const int32_t* __restrict__ offsets,
                          int N, int max_rows, int n_out, int k_dim, TIn* __restrict__ C,
-                         uint32_t* status) {
+                         uint32_t* status, const int32_t* __restrict__ a_rows, int a_src_rows) {
   __shared__ int prefix[kMaxExperts + 1];
   __shared__ int scan_tmp[33];
   __shared__ float As[kSgBK][kSgBM + 4];
@@ -47,7 +48,14 @@ grouped_gemm_simt_kernel(const TIn* __restrict__ A, const TIn* __restrict__ B0,
         int r = idx >> 4, c = idx & 15;
         int gk = k0 + c;
         int gr = r0 + r, gn = n0 + r;
-        As[c][r] = (gr < r1 && gk < k_dim) ? Cvt<TIn>::to_f(A[(size_t)gr * k_dim + gk]) : 0.f;
+        float av = 0.f;
+        if (gr < r1 && gk < k_dim) {
+          // A row: routed row gr itself, or the token it came from (a_rows != NULL)
+          int src = a_rows ? a_rows[gr] : gr;
+          if (a_rows && (src < 0 || src >= a_src_rows)) src = -1;
+          if (src >= 0) av = Cvt<TIn>::to_f(A[(size_t)src * k_dim + gk]);
+        }
+        As[c][r] = av;
         bool okb = gn < n_out && gk < k_dim;
         Bs[0][c][r] = okb ? Cvt<TIn>::to_f(b0[(size_t)gn * k_dim + gk]) : 0.f;
         if (kGated) Bs[kGated ? 1 : 0][c][r] = okb ? Cvt<TIn>::to_f(b1[(size_t)gn * k_dim + gk]) : 0.f;

@@ -84,6 +84,10 @@ struct Args {
   void* out;
   const float* add;            // fp32 addend [rows, n_out] (router logit offset) or NULL
   uint32_t* status;
+  const int32_t* gather_rows;  // token of each routed row: B rows are read from x through
+                               // this map with 4-row TMA gathers (tmB is x, box 64 x 1);
+                               // NULL: B rows are rows of tmB itself (tiled boxes)
+  int gather_src_rows;         // rows of x (bound for the gathered tokens)
 };
 
 // --- PTX wrappers --------------------------------------------------------------
@@ -168,6 +172,17 @@ MOE_DEV uint64_t l2_policy_evict_last() {
 // SiLU for the bf16 epilogue: a / (1 + e^-a) with the fast exponential and
 // division intrinsics (relative error ~1e-6, far below the bf16 rounding of h).
 MOE_DEV float silu_fast(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
+// Four rows (row0..row3) x 64 columns of a 2-D map whose box is 64 x 1,
+// placed as four consecutive 128-byte rows at dst (128-byte swizzle applied).
+MOE_DEV void tma_gather4_hint(uint32_t dst, const CUtensorMap* map, int c0, int r0, int r1,
+                              int r2, int r3, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+      "r"(bar), "l"(policy)
+      : "memory");
+}
 MOE_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -323,7 +338,65 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   const int nk = args.k_dim / kBK;
   int issued = 0;  // producer: stages issued
 
-  if (warp == 0) {
+  if (warp == 0 && args.gather_rows) {
+    // ---------------- TMA producer, B rows gathered from x ----------------
+    // Lane 0 waits and posts the expected bytes; every lane then issues the
+    // 4-row gathers of its row groups (g = lane, lane + 32, ...).
+    uint32_t stage = 0, phase = 0;
+    bool ok = true;
+    const uint64_t pol_w = l2_policy_evict_first();
+    const uint64_t pol_x = l2_policy_evict_last();
+    constexpr int kGroups = kNMax / 4;
+    constexpr int kPerLane = (kGroups + 31) / 32;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const Tile t = decode_tile<kNMax>(tile, n_fblk, args, prefix);
+      const int ngroups = (t.n + 3) / 4;
+      const uint32_t tx = 2 * kABytes + ngroups * 4 * kBK * 2;
+      const int a_row0 = t.seg * args.a_seg_rows + t.f0;
+      const int a_row1 = a_row0 + args.a1_row_off;
+      int tok[kPerLane][4];
+#pragma unroll
+      for (int i = 0; i < kPerLane; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          // rows past the segment repeat its last row (their columns are never stored)
+          const int row = min(4 * (lane + 32 * i) + j, t.n - 1);
+          int v = args.gather_rows[t.r0 + row];
+          if (v < 0 || v >= args.gather_src_rows) {
+            set_status(args.status, MOE_DEV_BAD_OFFSETS);
+            v = 0;
+          }
+          tok[i][j] = v;
+        }
+      for (int kb = 0; kb < nk; ++kb) {
+        int go = 1;
+        if (lane == 0) go = mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status);
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (!go) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = full0 + 8 * stage;
+        const uint32_t sa0 = smem_u32(stages + stage * kStageBytes);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(fb, tx);
+          tma_load_2d_hint(sa0, &tmA0, kb * kBK, a_row0, fb, pol_w);
+          tma_load_2d_hint(sa0 + kABytes, &tmA1, kb * kBK, a_row1, fb, pol_w);
+          ++issued;
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < kPerLane; ++i) {
+          const int g = lane + 32 * i;
+          if (g < ngroups)
+            tma_gather4_hint(sa0 + 2 * kABytes + g * 4 * kBK * 2, &tmB, kb * kBK, tok[i][0],
+                             tok[i][1], tok[i][2], tok[i][3], fb, pol_x);
+        }
+        if (++stage == kStages) { stage = 0; phase ^= 1; }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       uint32_t stage = 0, phase = 0;
@@ -612,6 +685,38 @@ inline moe_status launch_gate_up(const moe_shape& s, const void* x_perm, const v
   a.feat_per_tile = kFeat;
   a.out = h;
   a.status = status;
+  if (use_double(s))
+    return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
+                                     sms, st, err, errn);
+  return launch<kGated, CfgWide>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgWide::kNMax), sms,
+                                 st, err, errn);
+}
+
+// Gate/up GEMM reading its token rows straight from x through row_token
+// (4-row TMA gathers), so the dispatch needs no x_perm copy.
+inline moe_status launch_gate_up_gather(const moe_shape& s, const void* x,
+                                        const int32_t* row_token, const void* w1,
+                                        const void* w3, const int32_t* offsets, void* h,
+                                        uint32_t* status, int sms, cudaStream_t st, char* err,
+                                        size_t errn) {
+  CUtensorMap a0, a1, b;
+  const uint64_t rows = (uint64_t)s.T * s.K;
+  if (!make_map(&a0, w1, (uint64_t)s.N * s.I, s.d, kFeat)) return map_error(err, errn, "w1");
+  if (!make_map(&a1, w3, (uint64_t)s.N * s.I, s.d, kFeat)) return map_error(err, errn, "w3");
+  if (!make_map(&b, x, (uint64_t)s.T, s.d, 1)) return map_error(err, errn, "x");
+  Args a{};
+  a.seg_offsets = offsets;
+  a.nseg = s.N;
+  a.max_rows = (int)rows;
+  a.n_out = s.I;
+  a.k_dim = s.d;
+  a.a_seg_rows = s.I;
+  a.a1_row_off = 0;
+  a.feat_per_tile = kFeat;
+  a.out = h;
+  a.status = status;
+  a.gather_rows = row_token;
+  a.gather_src_rows = s.T;
   if (use_double(s))
     return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
                                      sms, st, err, errn);

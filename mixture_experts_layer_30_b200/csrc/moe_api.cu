@@ -192,9 +192,11 @@ moe_status permute_impl(const moe_shape& s, const void* x, const int32_t* idx,
     moe::perm_rank_kernel<<<nch, 256, smem, st>>>(idx, s.T, s.K, s.N, E, cbase, row_token,
                                                    slot_pos);
     MOE_TRY(check_launch("dispatch rank"));
-    moe::gather_kernel<T><<<(s.T + 7) / 8, 256, 0, st>>>(
-        static_cast<const T*>(x), slot_pos, s.T, s.K, s.d, static_cast<T*>(x_perm));
-    MOE_TRY(check_launch("dispatch gather"));
+    if (x_perm) {
+      moe::gather_kernel<T><<<(s.T + 7) / 8, 256, 0, st>>>(
+          static_cast<const T*>(x), slot_pos, s.T, s.K, s.d, static_cast<T*>(x_perm));
+      MOE_TRY(check_launch("dispatch gather"));
+    }
   }
   return MOE_OK;
 }
@@ -202,7 +204,7 @@ moe_status permute_impl(const moe_shape& s, const void* x, const int32_t* idx,
 template <typename T, bool kGated>
 moe_status grouped_simt(const moe_shape& s, const void* A, const void* B0, const void* B1,
                         const int32_t* offsets, int n_out, int k_dim, void* C,
-                        uint32_t* status, cudaStream_t st) {
+                        uint32_t* status, cudaStream_t st, const int32_t* a_rows = nullptr) {
   const long long max_rows = (long long)s.T * s.K;
   const long long ncol = (n_out + moe::kSgBN - 1) / moe::kSgBN;
   const long long max_chunks = s.N + (max_rows + moe::kSgBM - 1) / moe::kSgBM;
@@ -212,7 +214,7 @@ moe_status grouped_simt(const moe_shape& s, const void* A, const void* B0, const
   if (grid < 1) grid = 1;
   moe::grouped_gemm_simt_kernel<T, kGated><<<(int)grid, 256, 0, st>>>(
       static_cast<const T*>(A), static_cast<const T*>(B0), static_cast<const T*>(B1), offsets,
-      s.N, (int)max_rows, n_out, k_dim, static_cast<T*>(C), status);
+      s.N, (int)max_rows, n_out, k_dim, static_cast<T*>(C), status, a_rows, s.T);
   return check_launch(kGated ? "gate/up grouped gemm" : "down grouped gemm");
 }
 
@@ -226,6 +228,20 @@ moe_status gate_up_impl(const moe_shape& s, const void* x_perm, const void* w1, 
     return grouped_simt<__nv_bfloat16, true>(s, x_perm, w1, w3, offsets, s.I, s.d, h, status, st);
   }
   return grouped_simt<float, true>(s, x_perm, w1, w3, offsets, s.I, s.d, h, status, st);
+}
+
+moe_status gate_up_gather_impl(const moe_shape& s, const void* x, const int32_t* row_token,
+                               const void* w1, const void* w3, const int32_t* offsets, void* h,
+                               uint32_t* status, cudaStream_t st) {
+  if (s.T == 0) return MOE_OK;
+  if (s.dtype == MOE_BF16) {
+    if (moe::tc::ffn_supported(s))
+      return moe::tc::launch_gate_up_gather(s, x, row_token, w1, w3, offsets, h, status,
+                                            sm_count(), st, g_err, sizeof(g_err));
+    return grouped_simt<__nv_bfloat16, true>(s, x, w1, w3, offsets, s.I, s.d, h, status, st,
+                                             row_token);
+  }
+  return grouped_simt<float, true>(s, x, w1, w3, offsets, s.I, s.d, h, status, st, row_token);
 }
 
 moe_status down_impl(const moe_shape& s, const void* h, const void* w2, const int32_t* offsets,
@@ -336,11 +352,13 @@ moe_status moe_permute(const moe_shape* shape, const void* x, const int32_t* top
   MOE_TRY(check_ws(s, ws, ws_bytes, &L));
   MOE_TRY(need(offsets, "offsets", 4));
   if (s.T > 0) {
-    MOE_TRY(need(x, "x", 16));
     MOE_TRY(need(topk_idx, "topk_idx", 4));
     MOE_TRY(need(row_token, "row_token", 4));
     MOE_TRY(need(slot_pos, "slot_pos", 4));
-    MOE_TRY(need(x_perm, "x_perm", 16));
+    if (x_perm) {
+      MOE_TRY(need(x, "x", 16));
+      MOE_TRY(need(x_perm, "x_perm", 16));
+    }
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (s.dtype == MOE_BF16)
@@ -401,6 +419,25 @@ moe_status moe_expert_gate_up(const moe_shape* shape, const void* x_perm, const 
   MOE_TRY(need(h, "h", 16));
   return gate_up_impl(s, x_perm, w1, w3, offsets, h, at<uint32_t>(ws, L.status),
                       static_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_gate_up_gather(const moe_shape* shape, const void* x,
+                                     const int32_t* row_token, const void* w1, const void* w3,
+                                     const int32_t* offsets, void* h, void* ws, size_t ws_bytes,
+                                     void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  WsLayout L;
+  MOE_TRY(check_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(x, "x", 16));
+  MOE_TRY(need(row_token, "row_token", 4));
+  MOE_TRY(need(w1, "w1", 16));
+  MOE_TRY(need(w3, "w3", 16));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(h, "h", 16));
+  return gate_up_gather_impl(s, x, row_token, w1, w3, offsets, h, at<uint32_t>(ws, L.status),
+                             static_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_expert_down(const moe_shape* shape, const void* h, const void* w2,

@@ -95,10 +95,11 @@ class GpuRun:
     """Runs the layer through the C ABI and keeps every intermediate."""
 
     def __init__(self, shape, x, w_router, w1, w3, w2, bias, gamma=1.0, logit_offset=None,
-                 split_ffn=False):
+                 split_ffn=False, fused_gather=False):
         self.buf = B.LayerBuffers(shape, device=x.device, with_probs=True)
+        self.fused_gather = fused_gather
         B.forward(self.buf, x, w_router, w1, w3, w2, bias, gamma=gamma,
-                  logit_offset=logit_offset, split_ffn=split_ffn)
+                  logit_offset=logit_offset, split_ffn=split_ffn, fused_gather=fused_gather)
         torch.cuda.synchronize()
         self.status = B.device_status(self.buf.ws)
 
@@ -109,7 +110,8 @@ class GpuRun:
                     idx=b.topk_idx.cpu().numpy(), gate=b.topk_gate.cpu().numpy().astype(np.float64),
                     counts=b.counts.cpu().numpy(), n_ffn=b.n_ffn.cpu().numpy(),
                     offsets=b.offsets.cpu().numpy(), row_token=b.row_token[:R].cpu().numpy(),
-                    slot_pos=b.slot_pos.cpu().numpy(), x_perm=to_f64(b.x_perm[:R]),
+                    slot_pos=b.slot_pos.cpu().numpy(),
+                    x_perm=None if self.fused_gather else to_f64(b.x_perm[:R]),
                     y_perm=to_f64(b.y_perm[:R]), out=to_f64(b.out), R=R)
 
 
@@ -135,8 +137,9 @@ def check_routing_and_dispatch(g, x64, wr64, bias, N, K, logit_offset=None):
     np.testing.assert_array_equal(g["row_token"], rt_o)
     np.testing.assert_array_equal(g["slot_pos"], sp_o)
     assert g["R"] == off_o[-1]
-    # the copies are exact
-    assert np.array_equal(g["x_perm"], x64[rt_o])
+    # the copies are exact (absent when the dispatch copy is fused into the GEMM)
+    if g["x_perm"] is not None:
+        assert np.array_equal(g["x_perm"], x64[rt_o])
     return idx_ref, probs, len(ties)
 
 

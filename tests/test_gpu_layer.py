@@ -13,9 +13,10 @@ pytestmark = pytest.mark.gpu
 
 
 def _run_and_check(shape, dtype, L, N, K, gamma=1.0, logit_offset=None, split_ffn=False,
-                   experts=None):
+                   experts=None, fused_gather=False):
     run = P.GpuRun(shape, L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"],
-                   gamma=gamma, logit_offset=logit_offset, split_ffn=split_ffn)
+                   gamma=gamma, logit_offset=logit_offset, split_ffn=split_ffn,
+                   fused_gather=fused_gather)
     assert run.status == 0, hex(run.status)
     g = run.host()
     x64 = P.to_f64(L["x"])
@@ -73,6 +74,21 @@ def test_mid_bf16_layer():
 def test_decode_bf16(cfg):
     L = _cfg_inputs(cfg)
     _run_and_check(B.shape_of(cfg), "bf16", L, cfg.N, cfg.K, split_ffn=True)
+
+
+@pytest.mark.parametrize("cfg", [C.TINY_F32, C.MID_BF16, C.DECODE_T16, C.DECODE_T256],
+                         ids=lambda c: c.name)
+def test_fused_gather_layer(cfg):
+    """Dispatch without the x_perm copy: the gate/up GEMM reads x through row_token."""
+    L = _cfg_inputs(cfg)
+    _run_and_check(B.shape_of(cfg), cfg.dtype, L, cfg.N, cfg.K, fused_gather=True)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [1, 13, 700])
+def test_fused_gather_ragged(dtype, T):
+    shape, L = _small(T, 128, 12, 4, 3, 64, dtype, seed=100 + T)
+    _run_and_check(shape, dtype, L, 12, 3, fused_gather=True)
 
 
 def _small(T, d, N, Z, K, I, dtype, seed=0, bias=None, w_std=0.05):
