@@ -142,10 +142,9 @@ def run_gpu(args, rank, world, local_rank):
                 buf.n_ffn)
         if ev: ev[1].record(stream)
         B.permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
-                  None, buf.ws)
+                  buf.x_perm, buf.ws)
         if ev: ev[2].record(stream)
-        B.expert_gate_up_gather(s, x, buf.row_token, L["w1"], L["w3"], buf.offsets, buf.h,
-                                buf.ws)
+        B.expert_gate_up(s, buf.x_perm, L["w1"], L["w3"], buf.offsets, buf.h, buf.ws)
         if ev: ev[3].record(stream)
         B.expert_down(s, buf.h, L["w2"], buf.offsets, buf.y_perm, buf.ws)
         if ev: ev[4].record(stream)
@@ -224,9 +223,8 @@ def run_gpu(args, rank, world, local_rank):
             B.route(s, x_dev[j], L["w_router"], bias, buf.ws, buf.topk_idx, buf.topk_gate,
                     buf.counts, buf.n_ffn)
             B.permute(s, x_dev[j], buf.topk_idx, buf.counts, buf.offsets, buf.row_token,
-                      buf.slot_pos, None, buf.ws)
-            B.expert_gate_up_gather(s, x_dev[j], buf.row_token, L["w1"], L["w3"], buf.offsets,
-                                    buf.h, buf.ws)
+                      buf.slot_pos, buf.x_perm, buf.ws)
+            B.expert_gate_up(s, buf.x_perm, L["w1"], L["w3"], buf.offsets, buf.h, buf.ws)
             B.expert_down(s, buf.h, L["w2"], buf.offsets, buf.y_perm, buf.ws)
             B.combine(s, x_dev[j], buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos,
                       cfg.gamma, out_dev[j])
@@ -264,7 +262,7 @@ def run_gpu(args, rank, world, local_rank):
     esz = 2 if cfg.dtype == "bf16" else 4
     w13_bytes = touched * 2 * cfg.I * cfg.d * esz
     w2_bytes = touched * cfg.d * cfg.I * esz
-    # gate/up reads every routed token row once (gathered from x) and writes h
+    # gate/up reads every routed row of x_perm once and writes h
     gate_up_bytes = w13_bytes + R * cfg.d * esz + R * cfg.I * esz
     down_bytes = w2_bytes + R * cfg.I * esz + R * cfg.d * esz
     gate_up_flops = 4.0 * cfg.d * cfg.I * R
@@ -301,7 +299,7 @@ def run_gpu(args, rank, world, local_rank):
                    "K": cfg.K, "I": cfg.I, "K_e": cfg.K_e, "tokens_per_rank": cfg.T,
                    "parallelism": f"token-dp{world} (weights replicated, counts all-reduced)",
                    "l2": "inputs larger than L2 (38.7 GB of expert weights streamed per step)"},
-        "roofline": {"kernel": "moe_expert_gate_up_gather (tcgen05 grouped GEMM, TMA row gather, SwiGLU)",
+        "roofline": {"kernel": "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)",
                      "bound": "hbm", "achieved": round(achieved, 1),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
