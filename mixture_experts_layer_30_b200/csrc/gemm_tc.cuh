@@ -41,8 +41,10 @@ constexpr int kABytes = kFeat * kBK * 2;         // 16 KiB
 constexpr int kBoxBytes = kBoxRows * kBK * 2;    // 4 KiB
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
-constexpr int kStagingPitch = 36;                // 32-bit words per staging row (32 + pad)
-constexpr int kStagingBytes = kEpiWarps * 32 * kStagingPitch * 4;
+constexpr int kStagingPitch = 36;                // fp32 staging row: 32 words + pad
+constexpr int kStagingPitch16 = 40;              // bf16 staging row: 32 halves + pad (80 B)
+constexpr int kStagingBytesF32 = kEpiWarps * 32 * kStagingPitch * 4;
+constexpr int kStagingBytesBf16 = kEpiWarps * 32 * kStagingPitch16 * 2;
 constexpr int kCtrlBytes = 256;                  // barriers + tmem slot + abort flag
 constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;  // 4 s
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;  // 0.2 s
@@ -60,14 +62,22 @@ struct TileCfg {
   static constexpr int kBBytes = NMAX * kBK * 2;
   static constexpr int kStageBytes = 2 * kABytes + kBBytes;
   static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs + 1;  // full, empty, acc full/empty, drain
-  static constexpr int kSmemBytes =
-      1024 + STAGES * kStageBytes + kStagingBytes + kCtrlBytes + (kMaxExperts + 1 + 33) * 4;
+  // shared memory for an epilogue whose staging area takes `staging` bytes
+  __host__ __device__ static constexpr int smem_bytes(int staging) {
+    return 1024 + STAGES * kStageBytes + staging + kCtrlBytes + (kMaxExperts + 1 + 33) * 4;
+  }
   static_assert(NMAX % kBoxRows == 0 && NMAX <= 256, "token tile");
   static_assert(8 * kNumBars + 12 <= kCtrlBytes, "control block");
-  static_assert(kSmemBytes <= 232448, "shared memory");
+  static_assert(smem_bytes(kStagingBytesBf16) <= 232448, "shared memory");
 };
-using CfgWide = TileCfg<256, 3>;    // ragged segments up to 256 rows, one accumulator pair
+using CfgWide = TileCfg<256, 3>;    // segments up to 256 rows in one tile, 3 stages
+using CfgN160 = TileCfg<160, 4>;    // segments up to 160 rows, 4 stages (more bytes in flight)
 using CfgDouble = TileCfg<128, 4>;  // <= 128 rows, double-buffered accumulators
+static_assert(CfgWide::smem_bytes(kStagingBytesF32) <= 232448, "router tile");
+
+template <int kMode> __host__ __device__ constexpr int staging_bytes() {
+  return kMode == 2 ? kStagingBytesF32 : kStagingBytesBf16;
+}
 
 enum Mode { kGated = 0, kPlainBf16 = 1, kPlainF32 = 2 };
 
@@ -275,6 +285,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   constexpr int kNMax = Cfg::kNMax, kStages = Cfg::kStages, kAccBufs = Cfg::kAccBufs;
   constexpr int kStageBytes = Cfg::kStageBytes, kNumBars = Cfg::kNumBars;
   constexpr int kTmemCols = Cfg::kTmemCols;
+  constexpr int kStagingBytes = staging_bytes<kMode>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -476,7 +487,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
     const int q = warp & 3;                      // TMEM lane quarter this warp may access
-    uint32_t* stg = staging + (warp - 2) * 32 * kStagingPitch;
+    uint32_t* stg = staging + (warp - 2) * (kStagingBytes / kEpiWarps / 4);
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int local = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
@@ -518,8 +529,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
             uint16_t* s16 = reinterpret_cast<uint16_t*>(stg);
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-              s16[j * 2 * kStagingPitch + lane] = (uint16_t)(v0[j] & 0xffffu);
-              s16[(j + 1) * 2 * kStagingPitch + lane] = (uint16_t)(v0[j] >> 16);
+              s16[j * kStagingPitch16 + lane] = (uint16_t)(v0[j] & 0xffffu);
+              s16[(j + 1) * kStagingPitch16 + lane] = (uint16_t)(v0[j] >> 16);
             }
           }
           __syncwarp();
@@ -546,7 +557,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
                 *reinterpret_cast<uint4*>(o) = w;
               } else {
                 const uint16_t* s16 = reinterpret_cast<const uint16_t*>(stg);
-                const uint4 w = *reinterpret_cast<const uint4*>(&s16[j * 2 * kStagingPitch + c * 8]);
+                const uint4 w = *reinterpret_cast<const uint4*>(&s16[j * kStagingPitch16 + c * 8]);
                 __nv_bfloat16* o =
                     static_cast<__nv_bfloat16*>(args.out) + (size_t)row * args.n_out + f;
                 *reinterpret_cast<uint4*>(o) = w;
@@ -626,7 +637,7 @@ inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUt
   if (dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kMode, Cfg>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg::kSmemBytes);
+                                         Cfg::smem_bytes(staging_bytes<kMode>()));
     if (e != cudaSuccess) {
       snprintf(err, errn, "tcgen05 gemm smem attribute: %s", cudaGetErrorString(e));
       return MOE_ERR_CUDA;
@@ -635,7 +646,8 @@ inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUt
   }
   long long grid = max_tiles < sms ? max_tiles : sms;
   if (grid < 1) grid = 1;
-  gemm_tc_kernel<kMode, Cfg><<<(int)grid, kThreads, Cfg::kSmemBytes, st>>>(a0, a1, b, args);
+  gemm_tc_kernel<kMode, Cfg>
+      <<<(int)grid, kThreads, Cfg::smem_bytes(staging_bytes<kMode>()), st>>>(a0, a1, b, args);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -657,12 +669,19 @@ inline long long routed_tiles(const moe_shape& s, int n_out, int feat, int nmax)
   return chunks * ((n_out + feat - 1) / feat);
 }
 
-// Expert GEMM geometry: the wide tile keeps every segment of up to 256 rows in
-// one tile (each weight tile streamed once); the double-buffered tile is used
-// when segments are short on average.
-constexpr int kDoubleBufferMaxMeanRows = 0;  // mean routed rows per expert at or below: CfgDouble
+// Expert GEMM geometry.  A segment longer than the tile is split into chunks
+// and each chunk streams the expert's weights again, so the tile must hold
+// nearly every segment.  With uniform routing the rows per FFN expert have
+// mean T*K/(N+Z); up to a mean of 128 (LongCat: exactly 128, spread ~11)
+// the 160-row tile with four stages keeps more weight bytes in flight;
+// longer segments use the 256-row tile with three stages.
+constexpr int kDoubleBufferMaxMeanRows = 0;  // mean rows at or below which CfgDouble is used
+constexpr int kN160MaxMeanRows = 128;
 inline bool use_double(const moe_shape& s) {
   return (long long)s.T * s.K <= (long long)kDoubleBufferMaxMeanRows * (s.N + s.Z);
+}
+inline bool use_n160(const moe_shape& s) {
+  return (long long)s.T * s.K <= (long long)kN160MaxMeanRows * (s.N + s.Z);
 }
 
 inline moe_status launch_gate_up(const moe_shape& s, const void* x_perm, const void* w1,
@@ -688,6 +707,9 @@ inline moe_status launch_gate_up(const moe_shape& s, const void* x_perm, const v
   if (use_double(s))
     return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
                                      sms, st, err, errn);
+  if (use_n160(s))
+    return launch<kGated, CfgN160>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgN160::kNMax),
+                                   sms, st, err, errn);
   return launch<kGated, CfgWide>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgWide::kNMax), sms,
                                  st, err, errn);
 }
@@ -720,6 +742,9 @@ inline moe_status launch_gate_up_gather(const moe_shape& s, const void* x,
   if (use_double(s))
     return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
                                      sms, st, err, errn);
+  if (use_n160(s))
+    return launch<kGated, CfgN160>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgN160::kNMax),
+                                   sms, st, err, errn);
   return launch<kGated, CfgWide>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgWide::kNMax), sms,
                                  st, err, errn);
 }
@@ -746,6 +771,10 @@ inline moe_status launch_down(const moe_shape& s, const void* h, const void* w2,
     return launch<kPlainBf16, CfgDouble>(a, a, b, g,
                                          routed_tiles(s, s.d, 2 * kFeat, CfgDouble::kNMax), sms,
                                          st, err, errn);
+  if (use_n160(s))
+    return launch<kPlainBf16, CfgN160>(a, a, b, g,
+                                       routed_tiles(s, s.d, 2 * kFeat, CfgN160::kNMax), sms, st,
+                                       err, errn);
   return launch<kPlainBf16, CfgWide>(a, a, b, g, routed_tiles(s, s.d, 2 * kFeat, CfgWide::kNMax),
                                      sms, st, err, errn);
 }
