@@ -51,11 +51,21 @@ extern "C" {
 
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
+/* Storage order of the expert weights w1, w3, w2.
+ * MOE_WEIGHTS_ROW_MAJOR: [N, rows, cols] row-major (linear-layer layout).
+ * MOE_WEIGHTS_TILED: the same matrices cut into 128-row x 64-column tiles,
+ *   each tile stored as 16 KiB of contiguous row-major bf16, tiles ordered
+ *   (expert, row block, column block); see moe_pack_weights.  Every weight
+ *   tile the expert GEMMs stream is then one contiguous block of HBM.
+ *   Requires bf16, d % 128 == 0 and I % 128 == 0. */
+typedef enum { MOE_WEIGHTS_ROW_MAJOR = 0, MOE_WEIGHTS_TILED = 1 } moe_weight_layout;
+
 /* T tokens, d hidden size, N FFN experts, Z zero-computation experts,
  * K experts per token (1 <= K <= N+Z <= 1024), I expert intermediate size. */
 typedef struct {
   int32_t T, d, N, Z, K, I;
-  int32_t dtype; /* moe_dtype */
+  int32_t dtype;         /* moe_dtype */
+  int32_t weight_layout; /* moe_weight_layout of w1, w3, w2 (w_router is always row-major) */
 } moe_shape;
 
 typedef enum {
@@ -72,6 +82,15 @@ typedef enum {
 #define MOE_DEV_COUNT_MISMATCH 0x2u    /* counts[] disagrees with topk_idx */
 #define MOE_DEV_BAD_OFFSETS 0x4u       /* offsets not monotone or beyond T*K */
 #define MOE_DEV_PIPELINE_TIMEOUT 0x8u  /* a bounded wait inside a GEMM gave up */
+
+/* Repacks n_mats bf16 matrices [rows, cols] (row-major, contiguous) into the
+ * MOE_WEIGHTS_TILED order: dst tile (m, rb, cb) = rows rb*128..+127, columns
+ * cb*64..+63 of matrix m, stored at tile index (m*rows/128 + rb)*cols/64 + cb.
+ * w1 and w3 are packed as N matrices [I, d], w2 as N matrices [d, I].
+ * rows % 128 == 0, cols % 64 == 0; src and dst must not overlap; dtype must be
+ * MOE_BF16.  Done once when the weights are loaded. */
+moe_status moe_pack_weights(int32_t n_mats, int32_t rows, int32_t cols, int32_t dtype,
+                            const void* src, void* dst, void* stream);
 
 /* Bytes of device workspace the calls below need for this shape.  One
  * workspace may serve every call of a layer instance, used in stream order.

@@ -23,14 +23,18 @@ _vp, _i32, _i64, _f32, _sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ct
     ctypes.c_size_t
 
 
+WEIGHTS_ROW_MAJOR, WEIGHTS_TILED = 0, 1
+
+
 class Shape(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("N", ctypes.c_int32),
                 ("Z", ctypes.c_int32), ("K", ctypes.c_int32), ("I", ctypes.c_int32),
-                ("dtype", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("weight_layout", ctypes.c_int32)]
 
 
 _SP = ctypes.POINTER(Shape)
 SIGNATURES = {
+    "moe_pack_weights": (ctypes.c_int, [_i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_workspace_bytes": (_sz, [_SP]),
     "moe_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
     "moe_route": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -77,14 +81,27 @@ def _check(code):
         raise MoEError(code, lib().moe_last_error().decode())
 
 
-def make_shape(T, d, N, Z, K, I, dtype) -> Shape:
+def make_shape(T, d, N, Z, K, I, dtype, weight_layout=WEIGHTS_ROW_MAJOR) -> Shape:
     code = {"f32": MOE_F32, "bf16": MOE_BF16, torch.float32: MOE_F32,
             torch.bfloat16: MOE_BF16}[dtype]
-    return Shape(T, d, N, Z, K, I, code)
+    return Shape(T, d, N, Z, K, I, code, weight_layout)
 
 
-def shape_of(cfg, T=None) -> Shape:
-    return make_shape(cfg.T if T is None else T, cfg.d, cfg.N, cfg.Z, cfg.K, cfg.I, cfg.dtype)
+def shape_of(cfg, T=None, weight_layout=WEIGHTS_ROW_MAJOR) -> Shape:
+    return make_shape(cfg.T if T is None else T, cfg.d, cfg.N, cfg.Z, cfg.K, cfg.I, cfg.dtype,
+                      weight_layout)
+
+
+def pack_weights(w: torch.Tensor, out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """MOE_WEIGHTS_TILED copy of bf16 weights [n, rows, cols] (or [rows, cols])."""
+    if w.dim() == 2:
+        w = w.unsqueeze(0)
+    n, rows, cols = w.shape
+    if out is None:
+        out = torch.empty_like(w)
+    _check(lib().moe_pack_weights(n, rows, cols, MOE_BF16, _p(w, torch.bfloat16, "w"),
+                                  _p(out, torch.bfloat16, "out"), _stream(stream)))
+    return out
 
 
 def torch_dtype(shape: Shape):

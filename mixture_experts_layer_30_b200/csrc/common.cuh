@@ -142,4 +142,25 @@ MOE_DEV int find_expert(const int* prefix, int N, int c) {
   return lo;
 }
 
+// One CTA per 128 x 64 bf16 tile (16 KiB): copies tile (m, rb, cb) of the
+// row-major matrices [rows, cols] to position (m*rows/128 + rb)*cols/64 + cb
+// of the tiled order, row-major inside the tile.  16-byte vectors.
+__global__ void __launch_bounds__(256)
+pack_tiles_kernel(const uint4* __restrict__ src, int rows, int cols, uint4* __restrict__ dst) {
+  const long long tile = blockIdx.x;
+  const int cb_n = cols / 64, rb_n = rows / 128;
+  const int cb = (int)(tile % cb_n);
+  const long long mr = tile / cb_n;  // m * rb_n + rb
+  const int rb = (int)(mr % rb_n);
+  const long long m = mr / rb_n;
+  const size_t vec_per_row = (size_t)cols / 8;  // 8 bf16 per 16-byte vector
+  const uint4* s = src + ((size_t)m * rows + (size_t)rb * 128) * vec_per_row + (size_t)cb * 8;
+  uint4* d = dst + (size_t)tile * 1024;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int v = threadIdx.x + i * 256;  // 0..1023: row v/8, vector v%8 of the tile
+    d[v] = s[(size_t)(v >> 3) * vec_per_row + (v & 7)];
+  }
+}
+
 }  // namespace moe

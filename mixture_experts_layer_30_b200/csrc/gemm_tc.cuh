@@ -98,7 +98,16 @@ struct Args {
                                // this map with 4-row TMA gathers (tmB is x, box 64 x 1);
                                // NULL: B rows are rows of tmB itself (tiled boxes)
   int gather_src_rows;         // rows of x (bound for the gathered tokens)
+  int a_tiled;                 // weights in MOE_WEIGHTS_TILED order: the A tile of weight rows
+                               // r..r+127 (r % 128 == 0), columns kb*64.. is row (r/128*nk+kb)*128
+                               // of a [tiles*128, 64] view
 };
+
+// TMA coordinates (column, row) of the weight tile whose first row is `row`
+// (a multiple of 128 when tiled) for K block kb.
+MOE_DEV int2 a_coord(const Args& a, int row, int kb, int nk) {
+  return a.a_tiled ? make_int2(0, ((row >> 7) * nk + kb) << 7) : make_int2(kb * kBK, row);
+}
 
 // --- PTX wrappers --------------------------------------------------------------
 MOE_DEV uint32_t smem_u32(const void* p) {
@@ -391,8 +400,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
         const uint32_t sa0 = smem_u32(stages + stage * kStageBytes);
         if (lane == 0) {
           mbar_arrive_expect_tx(fb, tx);
-          tma_load_2d_hint(sa0, &tmA0, kb * kBK, a_row0, fb, pol_w);
-          tma_load_2d_hint(sa0 + kABytes, &tmA1, kb * kBK, a_row1, fb, pol_w);
+          const int2 c0 = a_coord(args, a_row0, kb, nk), c1 = a_coord(args, a_row1, kb, nk);
+          tma_load_2d_hint(sa0, &tmA0, c0.x, c0.y, fb, pol_w);
+          tma_load_2d_hint(sa0 + kABytes, &tmA1, c1.x, c1.y, fb, pol_w);
           ++issued;
         }
         __syncwarp();
@@ -428,8 +438,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
           const uint32_t fb = full0 + 8 * stage;
           const uint32_t sa0 = smem_u32(stages + stage * kStageBytes);
           mbar_arrive_expect_tx(fb, tx);
-          tma_load_2d_hint(sa0, &tmA0, kb * kBK, a_row0, fb, pol_w);
-          tma_load_2d_hint(sa0 + kABytes, &tmA1, kb * kBK, a_row1, fb, pol_w);
+          const int2 c0 = a_coord(args, a_row0, kb, nk), c1 = a_coord(args, a_row1, kb, nk);
+          tma_load_2d_hint(sa0, &tmA0, c0.x, c0.y, fb, pol_w);
+          tma_load_2d_hint(sa0 + kABytes, &tmA1, c1.x, c1.y, fb, pol_w);
           for (int b = 0; b < nbox; ++b)
             tma_load_2d_hint(sa0 + 2 * kABytes + b * kBoxBytes, &tmB, kb * kBK,
                              t.r0 + b * kBoxRows, fb, pol_x);
@@ -657,6 +668,14 @@ inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUt
   return MOE_OK;
 }
 
+// Map of n_mats weight matrices [rows, cols]: row-major, or the tiled order
+// seen as [n_mats*rows*cols/64, 64] (each 128 x 64 tile = 128 consecutive rows).
+inline bool make_weight_map(CUtensorMap* m, const void* base, uint64_t n_mats, uint64_t rows,
+                            uint64_t cols, bool tiled) {
+  if (tiled) return make_map(m, base, n_mats * rows * cols / kBK, kBK, kFeat);
+  return make_map(m, base, n_mats * rows, cols, kFeat);
+}
+
 inline moe_status map_error(char* err, size_t errn, const char* what) {
   snprintf(err, errn, "cuTensorMapEncodeTiled failed for %s", what);
   return MOE_ERR_CUDA;
@@ -690,8 +709,9 @@ inline moe_status launch_gate_up(const moe_shape& s, const void* x_perm, const v
                                  size_t errn) {
   CUtensorMap a0, a1, b;
   const uint64_t rows = (uint64_t)s.T * s.K;
-  if (!make_map(&a0, w1, (uint64_t)s.N * s.I, s.d, kFeat)) return map_error(err, errn, "w1");
-  if (!make_map(&a1, w3, (uint64_t)s.N * s.I, s.d, kFeat)) return map_error(err, errn, "w3");
+  const bool tiled = s.weight_layout == MOE_WEIGHTS_TILED;
+  if (!make_weight_map(&a0, w1, s.N, s.I, s.d, tiled)) return map_error(err, errn, "w1");
+  if (!make_weight_map(&a1, w3, s.N, s.I, s.d, tiled)) return map_error(err, errn, "w3");
   if (!make_map(&b, x_perm, rows, s.d, kBoxRows)) return map_error(err, errn, "x_perm");
   Args a{};
   a.seg_offsets = offsets;
@@ -704,6 +724,7 @@ inline moe_status launch_gate_up(const moe_shape& s, const void* x_perm, const v
   a.feat_per_tile = kFeat;
   a.out = h;
   a.status = status;
+  a.a_tiled = tiled;
   if (use_double(s))
     return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
                                      sms, st, err, errn);
@@ -723,8 +744,9 @@ inline moe_status launch_gate_up_gather(const moe_shape& s, const void* x,
                                         size_t errn) {
   CUtensorMap a0, a1, b;
   const uint64_t rows = (uint64_t)s.T * s.K;
-  if (!make_map(&a0, w1, (uint64_t)s.N * s.I, s.d, kFeat)) return map_error(err, errn, "w1");
-  if (!make_map(&a1, w3, (uint64_t)s.N * s.I, s.d, kFeat)) return map_error(err, errn, "w3");
+  const bool tiled = s.weight_layout == MOE_WEIGHTS_TILED;
+  if (!make_weight_map(&a0, w1, s.N, s.I, s.d, tiled)) return map_error(err, errn, "w1");
+  if (!make_weight_map(&a1, w3, s.N, s.I, s.d, tiled)) return map_error(err, errn, "w3");
   if (!make_map(&b, x, (uint64_t)s.T, s.d, 1)) return map_error(err, errn, "x");
   Args a{};
   a.seg_offsets = offsets;
@@ -739,6 +761,7 @@ inline moe_status launch_gate_up_gather(const moe_shape& s, const void* x,
   a.status = status;
   a.gather_rows = row_token;
   a.gather_src_rows = s.T;
+  a.a_tiled = tiled;
   if (use_double(s))
     return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
                                      sms, st, err, errn);
@@ -754,7 +777,8 @@ inline moe_status launch_down(const moe_shape& s, const void* h, const void* w2,
                               cudaStream_t st, char* err, size_t errn) {
   CUtensorMap a, b;
   const uint64_t rows = (uint64_t)s.T * s.K;
-  if (!make_map(&a, w2, (uint64_t)s.N * s.d, s.I, kFeat)) return map_error(err, errn, "w2");
+  const bool tiled = s.weight_layout == MOE_WEIGHTS_TILED;
+  if (!make_weight_map(&a, w2, s.N, s.d, s.I, tiled)) return map_error(err, errn, "w2");
   if (!make_map(&b, h, rows, s.I, kBoxRows)) return map_error(err, errn, "h");
   Args g{};
   g.seg_offsets = offsets;
@@ -767,6 +791,7 @@ inline moe_status launch_down(const moe_shape& s, const void* h, const void* w2,
   g.feat_per_tile = 2 * kFeat;
   g.out = y_perm;
   g.status = status;
+  g.a_tiled = tiled;
   if (use_double(s))
     return launch<kPlainBf16, CfgDouble>(a, a, b, g,
                                          routed_tiles(s, s.d, 2 * kFeat, CfgDouble::kNMax), sms,

@@ -67,6 +67,13 @@ moe_status validate_shape(const moe_shape* sp) {
   const int vec = 16 / elem_bytes(s);
   if (s.d % vec)
     return fail(MOE_ERR_UNSUPPORTED, "d=%d must be a multiple of %d for 16-byte rows", s.d, vec);
+  if (s.weight_layout != MOE_WEIGHTS_ROW_MAJOR && s.weight_layout != MOE_WEIGHTS_TILED)
+    return fail(MOE_ERR_INVALID_ARG, "weight_layout %d is not a moe_weight_layout",
+                s.weight_layout);
+  if (s.weight_layout == MOE_WEIGHTS_TILED &&
+      (s.dtype != MOE_BF16 || s.d % 128 || s.I % 128))
+    return fail(MOE_ERR_UNSUPPORTED,
+                "MOE_WEIGHTS_TILED needs bf16 and d, I multiples of 128 (d=%d, I=%d)", s.d, s.I);
   return MOE_OK;
 }
 
@@ -305,6 +312,28 @@ extern "C" {
 size_t moe_workspace_bytes(const moe_shape* shape) {
   if (validate_shape(shape) != MOE_OK) return 0;
   return layout_of(*shape).total;
+}
+
+moe_status moe_pack_weights(int32_t n_mats, int32_t rows, int32_t cols, int32_t dtype,
+                            const void* src, void* dst, void* stream) {
+  g_err[0] = 0;
+  if (dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "moe_pack_weights packs bf16 only");
+  if (n_mats < 0 || rows < 0 || cols < 0 || rows % 128 || cols % 64)
+    return fail(MOE_ERR_INVALID_ARG,
+                "moe_pack_weights: rows=%d must be a multiple of 128, cols=%d of 64", rows, cols);
+  const long long tiles = (long long)n_mats * (rows / 128) * (cols / 64);
+  if (tiles == 0) return MOE_OK;
+  MOE_TRY(need(src, "src", 16));
+  MOE_TRY(need(dst, "dst", 16));
+  const size_t bytes = (size_t)tiles * 128 * 64 * 2;
+  const char* a = static_cast<const char*>(src);
+  const char* b = static_cast<const char*>(dst);
+  if (a < b + bytes && b < a + bytes)
+    return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: src and dst overlap");
+  if (tiles > 0x7fffffffLL) return fail(MOE_ERR_UNSUPPORTED, "moe_pack_weights: too many tiles");
+  moe::pack_tiles_kernel<<<(unsigned)tiles, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(src), rows, cols, static_cast<uint4*>(dst));
+  return check_launch("weight pack");
 }
 
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {

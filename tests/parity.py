@@ -98,8 +98,12 @@ class GpuRun:
                  split_ffn=False, fused_gather=False):
         self.buf = B.LayerBuffers(shape, device=x.device, with_probs=True)
         self.fused_gather = fused_gather
+        if shape.weight_layout == B.WEIGHTS_TILED:
+            # the library repacks; the oracle keeps the row-major originals
+            w1, w3, w2 = B.pack_weights(w1), B.pack_weights(w3), B.pack_weights(w2)
         B.forward(self.buf, x, w_router, w1, w3, w2, bias, gamma=gamma,
                   logit_offset=logit_offset, split_ffn=split_ffn, fused_gather=fused_gather)
+        del w1, w3, w2
         torch.cuda.synchronize()
         self.status = B.device_status(self.buf.ws)
 

@@ -76,6 +76,34 @@ def test_decode_bf16(cfg):
     _run_and_check(B.shape_of(cfg), "bf16", L, cfg.N, cfg.K, split_ffn=True)
 
 
+def test_pack_weights_layout():
+    """Tiled order: tile (m, rb, cb) = rows rb*128.., columns cb*64.. of matrix m,
+    stored contiguously at tile index (m*rows/128 + rb)*cols/64 + cb."""
+    g = torch.Generator(device="cpu").manual_seed(9)
+    for (n, rows, cols) in ((3, 256, 192), (1, 128, 64), (2, 384, 1024)):
+        w = torch.randn((n, rows, cols), generator=g).to(torch.bfloat16).cuda()
+        got = B.pack_weights(w)
+        want = w.view(n, rows // 128, 128, cols // 64, 64).permute(0, 1, 3, 2, 4).contiguous()
+        assert torch.equal(got.view(-1), want.view(-1))
+
+
+@pytest.mark.parametrize("cfg", [C.MID_BF16, C.DECODE_T16, C.DECODE_T64, C.DECODE_T256],
+                         ids=lambda c: c.name)
+@pytest.mark.parametrize("mode", ["split", "ffn", "gather"])
+def test_tiled_weights_layer(cfg, mode):
+    """The expert GEMMs on weights repacked by moe_pack_weights."""
+    L = _cfg_inputs(cfg)
+    _run_and_check(B.shape_of(cfg, weight_layout=B.WEIGHTS_TILED), "bf16", L, cfg.N, cfg.K,
+                   split_ffn=mode == "split", fused_gather=mode == "gather")
+
+
+@pytest.mark.parametrize("T", [1, 200, 777])
+def test_tiled_weights_ragged(T):
+    shape, L = _small(T, 256, 12, 4, 3, 128, "bf16", seed=300 + T)
+    shape.weight_layout = B.WEIGHTS_TILED
+    _run_and_check(shape, "bf16", L, 12, 3, split_ffn=True)
+
+
 @pytest.mark.parametrize("cfg", [C.TINY_F32, C.MID_BF16, C.DECODE_T16, C.DECODE_T256],
                          ids=lambda c: c.name)
 def test_fused_gather_layer(cfg):

@@ -51,6 +51,23 @@ def test_workspace_bytes_and_validation(lib):
         assert lib.moe_workspace_bytes(ctypes.byref(bad)) == 0
 
 
+def test_tiled_layout_validation(lib):
+    ok = B.make_shape(16, 256, 4, 2, 2, 128, "bf16", B.WEIGHTS_TILED)
+    assert lib.moe_workspace_bytes(ctypes.byref(ok)) > 0
+    for bad in (B.make_shape(16, 256, 4, 2, 2, 128, "f32", B.WEIGHTS_TILED),   # bf16 only
+                B.make_shape(16, 192, 4, 2, 2, 128, "bf16", B.WEIGHTS_TILED),  # d % 128
+                B.make_shape(16, 256, 4, 2, 2, 64, "bf16", B.WEIGHTS_TILED),   # I % 128
+                B.make_shape(16, 256, 4, 2, 2, 128, "bf16", 5)):               # unknown
+        assert lib.moe_workspace_bytes(ctypes.byref(bad)) == 0
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.moe_pack_weights(2, 100, 64, B.MOE_BF16, fake, fake, None) == 1   # rows % 128
+    assert lib.moe_pack_weights(2, 128, 96, B.MOE_BF16, fake, fake, None) == 1   # cols % 64
+    assert lib.moe_pack_weights(2, 128, 64, B.MOE_F32, fake, fake, None) == 2    # bf16 only
+    assert lib.moe_pack_weights(2, 128, 64, B.MOE_BF16, fake, ctypes.c_void_p(0x10000 + 4096),
+                                None) == 1                                      # overlap
+    assert b"overlap" in lib.moe_last_error()
+
+
 def test_invalid_arguments_return_codes(lib):
     s = B.make_shape(16, 64, 4, 2, 2, 32, "f32")
     nb = B.workspace_bytes(s)
