@@ -178,17 +178,35 @@ def run_gpu(args, rank, world, local_rank):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     props = torch.cuda.get_device_properties(dev)
     clocks = ClockSampler(f"GPU-{props.uuid}" if getattr(props, "uuid", None) else local_rank)
+    graph = None
+    if args.graph:
+        # one step captured once and replayed: no host launch cost per kernel
+        graph = torch.cuda.CUDAGraph()
+        n0 = B.kernel_launches()
+        with torch.cuda.graph(graph):
+            step(x)
+        per_step_launches = B.kernel_launches() - n0
+        graph.replay()
+        barrier()
     launches0 = B.kernel_launches()
     barrier()
     clocks.start()
     t0.record(stream)
     for i in range(args.steps):
-        step(x, evs[i])
+        if graph is None:
+            step(x, evs[i])
+        else:
+            graph.replay()
     t1.record(stream)
     barrier()
     clk = clocks.stop()
-    launches = B.kernel_launches() - launches0
+    launches = (B.kernel_launches() - launches0) if graph is None else per_step_launches * args.steps
     ms_total = t0.elapsed_time(t1)
+    if graph is not None:
+        # per-call breakdown from a separate eager pass
+        for i in range(args.steps):
+            step(x, evs[i])
+        barrier()
     per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n_ev - 1)]
                     for i in range(args.steps)])
     ms_step_local = ms_total / args.steps
@@ -325,6 +343,7 @@ def run_gpu(args, rank, world, local_rank):
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(buf.out.numel() * buf.out.element_size())},
         "gpu_launches": int(launches),
+        "cuda_graph": graph is not None,
         "clocks": clk,
     }
     return line, L
@@ -430,9 +449,13 @@ def main():
     ap.add_argument("--cpu-baseline-tokens", type=int, default=4)
     ap.add_argument("--ref-tokens", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay one captured CUDA graph per step (single GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.graph and int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        ap.error("--graph is single-GPU only")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
