@@ -15,6 +15,8 @@ It follows "LongCat-Flash Technical Report" (Chinese translation):
   * §2.1.1 Computation-budget control, Eq. (2): the per-step bias increment
         Delta b_i = mu (K_e/K * 1/N - T_i/(K T_all))  for i <= N, 0 otherwise.
   * §2.3.2 Eq. (8): the optional output scale gamma on the whole sum.
+  * §2.1.2, Eq. (3)-(5): the device-level load-balance statistics f_j, P_j
+    with all zero-computation experts as one extra group.
 
 Readings taken where the pages are silent (each is also listed in the design
 notes): the router has no bias term and no temperature, and its softmax covers
@@ -220,6 +222,41 @@ def bias_update(bias, counts, N, K, K_e, mu, T_all):
     share = Ti / (float(K) * float(T_all))
     b[:N] = b[:N] + float(mu) * (target - share)
     return b
+
+
+# ---------------------------------------------------------------------------
+# Device-level load balance with the zero-expert group: §2.1.2, Eq. (3)-(5)
+# ---------------------------------------------------------------------------
+
+def lb_statistics(probs, idx, N, D, K, K_e):
+    """f_j and P_j of Eq. (4)-(5) for the D groups of G = N/D FFN experts and
+    the extra group j = D+1 that holds all zero-computation experts.
+
+      P_j = (1/T) sum_t sum_{i in group j} R(x_t)_i
+      f_j = D/(K_e T) * #(selections of FFN group j)          (j <= D)
+      f_{D+1} = 1/((K - K_e) T) * #(selections of zero experts)
+
+    "token t selects group j" is counted once per selected expert of the
+    group, so that every f_j equals 1 when the selections match K_e (FFN,
+    spread evenly over the groups) and K - K_e (zero experts) per token.
+    Returns (f, P) as float64 arrays of length D+1.
+    """
+    T, E = probs.shape
+    G = N // D
+    f = np.zeros(D + 1)
+    P = np.zeros(D + 1)
+    for j in range(D):
+        members = (idx >= j * G) & (idx < (j + 1) * G)
+        f[j] = float(D) / (float(K_e) * T) * members.sum()
+        P[j] = probs[:, j * G:(j + 1) * G].sum() / T
+    f[D] = 1.0 / ((float(K) - float(K_e)) * T) * (idx >= N).sum()
+    P[D] = probs[:, N:].sum() / T
+    return f, P
+
+
+def lb_loss(f, P, alpha):
+    """Eq. (3): L_LB = alpha * sum_{j=1}^{D+1} f_j P_j."""
+    return float(alpha) * float((f * P).sum())
 
 
 # ---------------------------------------------------------------------------

@@ -282,6 +282,51 @@ def check_bias_update_closed_form(orc, seed=6):
     assert (b1 == 0).all()
 
 
+def check_worked_lb_statistics(orc):
+    g = load_golden("worked_example_lb_statistics.json")
+    ex = g["expected"]
+    f, P = orc.lb_statistics(np.array(g["probs"]), np.array(g["topk_idx"]), g["N"], g["D"],
+                             g["K"], g["K_e"])
+    np.testing.assert_allclose(f, ex["f"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(P, ex["P"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(orc.lb_loss(f, P, g["alpha"]), ex["loss"], rtol=0, atol=1e-15)
+
+
+def check_lb_statistics_closed_forms(orc, seed=7):
+    rng = np.random.default_rng(seed)
+    for _ in range(30):
+        D = int(rng.integers(1, 5))
+        G = int(rng.integers(1, 4))
+        N, Z = D * G, int(rng.integers(1, 5))
+        E = N + Z
+        K = int(rng.integers(2, E + 1))
+        K_e = float(rng.uniform(0.5, K - 0.5))
+        T = int(rng.integers(1, 40))
+        probs = orc.softmax_rows(rng.normal(size=(T, E)))
+        idx = np.stack([rng.permutation(E)[:K] for _ in range(T)])
+        f, P = orc.lb_statistics(probs, idx, N, D, K, K_e)
+        # the groups partition all experts: the P_j sum to 1
+        np.testing.assert_allclose(P.sum(), 1.0, rtol=0, atol=1e-12)
+        # every selection is counted once: sum_j f_j * (its normaliser) = K T
+        total = f[:D].sum() * K_e * T / D + f[D] * (K - K_e) * T
+        np.testing.assert_allclose(total, K * T, rtol=1e-12)
+        # brute force over tokens and slots
+        sel = np.zeros(D + 1)
+        for t in range(T):
+            for k in range(K):
+                e = int(idx[t, k])
+                sel[D if e >= N else e // G] += 1
+        want_f = np.concatenate([sel[:D] * D / (K_e * T), [sel[D] / ((K - K_e) * T)]])
+        np.testing.assert_allclose(f, want_f, rtol=1e-14)
+    # balance point: every token picks one expert per FFN group and K - D zero experts
+    D, G, Z, T = 3, 2, 4, 5
+    N, K = D * G, D + 2
+    idx = np.array([[j * G + (t % G) for j in range(D)] + [N + (t % Z), N + ((t + 1) % Z)]
+                    for t in range(T)])
+    f, _ = orc.lb_statistics(np.full((T, N + Z), 1.0 / (N + Z)), idx, N, D, K, float(D))
+    np.testing.assert_allclose(f, 1.0, rtol=0, atol=1e-15)
+
+
 def check_bf16_decode(orc):
     bits = np.array([0x3F80, 0xC000, 0x3F81, 0x7F7F, 0x0001, 0x8000, 0x4049], dtype=np.uint16)
     want = [1.0, -2.0, 1.0 + 2.0 ** -7, (2 - 2.0 ** -7) * 2.0 ** 127, 2.0 ** -133, -0.0,
@@ -295,4 +340,5 @@ ALL_CHECKS = [check_worked_tiny_layer, check_worked_swiglu, check_worked_bias_up
               check_worked_zero_experts, check_softmax_closed_forms, check_topk_brute_force,
               check_dense_reduction, check_all_zero_experts_fixed_point,
               check_k_equals_e_fixed_point, check_permutation_invariants,
-              check_bias_update_closed_form, check_bf16_decode]
+              check_bias_update_closed_form, check_bf16_decode, check_worked_lb_statistics,
+              check_lb_statistics_closed_forms]

@@ -115,7 +115,33 @@ def _mut_gamma_only_ffn(mp):
     mp.setattr(orc, "combine", combine)
 
 
-MUTATIONS = [_mut_gate_renormalised, _mut_combine_drops_zero_term, _mut_bias_sign,
+def _mut_lb_indicator_per_token(mp):
+    """'selects group j' as a 0/1 indicator per token instead of a count."""
+    def lb_statistics(probs, idx, N, D, K, K_e):
+        T, E = probs.shape
+        G = N // D
+        f, P = np.zeros(D + 1), np.zeros(D + 1)
+        for j in range(D):
+            hit = ((idx >= j * G) & (idx < (j + 1) * G)).any(axis=1)
+            f[j] = D / (K_e * T) * hit.sum()
+            P[j] = probs[:, j * G:(j + 1) * G].sum() / T
+        f[D] = (idx >= N).any(axis=1).sum() / ((K - K_e) * T)
+        P[D] = probs[:, N:].sum() / T
+        return f, P
+    mp.setattr(orc, "lb_statistics", lb_statistics)
+
+
+def _mut_lb_zero_group_normaliser(mp):
+    real = orc.lb_statistics
+
+    def lb_statistics(probs, idx, N, D, K, K_e):
+        f, P = real(probs, idx, N, D, K, K_e)
+        f[D] *= (K - K_e) / K_e  # K_e in place of K - K_e
+        return f, P
+    mp.setattr(orc, "lb_statistics", lb_statistics)
+
+
+MUTATIONS = [_mut_lb_indicator_per_token, _mut_lb_zero_group_normaliser, _mut_gate_renormalised, _mut_combine_drops_zero_term, _mut_bias_sign,
              _mut_bias_updates_zero_experts, _mut_tie_to_high_index, _mut_select_by_unbiased,
              _mut_no_silu, _mut_swapped_gate_up, _mut_descending_tokens,
              _mut_softmax_no_max_shift_wrong_axis, _mut_gamma_only_ffn]
