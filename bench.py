@@ -140,11 +140,23 @@ def run_gpu(args, rank, world, local_rank):
     if world > 1:
         import torch.distributed as dist
 
+    lb = None
+    if args.lb_stats:
+        D_groups = 32 if cfg.N % 32 == 0 else 1
+        lb = dict(D=D_groups, prob_sum=torch.empty(cfg.E, dtype=torch.float32, device=dev),
+                  f=torch.empty(D_groups + 1, dtype=torch.float32, device=dev),
+                  P=torch.empty(D_groups + 1, dtype=torch.float32, device=dev),
+                  loss=torch.empty(1, dtype=torch.float32, device=dev))
+
     def step(x, ev=None):
         s = shape
         if ev: ev[0].record(stream)
         B.route(s, x, L["w_router"], bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts,
-                buf.n_ffn)
+                buf.n_ffn, prob_sum=None if lb is None else lb["prob_sum"])
+        if lb is not None:
+            # Eq. (3)-(5) statistics on this rank's batch
+            B.lb_stats(cfg.N, cfg.Z, lb["D"], buf.counts, lb["prob_sum"], cfg.T, cfg.K, K_e,
+                       0.001, lb["f"], lb["P"], lb["loss"])
         if ev: ev[1].record(stream)
         B.permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
                   buf.x_perm, buf.ws)
@@ -344,6 +356,7 @@ def run_gpu(args, rank, world, local_rank):
                 "d2h_bytes_per_step": int(buf.out.numel() * buf.out.element_size())},
         "gpu_launches": int(launches),
         "cuda_graph": graph is not None,
+        "lb_stats": lb is not None,
         "clocks": clk,
     }
     return line, L
@@ -449,6 +462,8 @@ def main():
     ap.add_argument("--cpu-baseline-tokens", type=int, default=4)
     ap.add_argument("--ref-tokens", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--lb-stats", action="store_true",
+                    help="also compute the device-level load-balance statistics each step")
     ap.add_argument("--graph", action="store_true",
                     help="replay one captured CUDA graph per step (single GPU)")
     args = ap.parse_args()

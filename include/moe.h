@@ -111,12 +111,14 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
  * x [T, d] (dtype), w_router [E, d] (dtype), bias [E] fp32,
  * logit_offset [T, E] fp32 or NULL (an additive input, used by tests and
  * skewed-routing workloads), topk_idx [T, K] int32, topk_gate [T, K] fp32,
- * counts [E] int32, n_ffn [T] uint8, probs_out [T, E] fp32 or NULL.
+ * counts [E] int32, n_ffn [T] uint8, probs_out [T, E] fp32 or NULL,
+ * prob_sum [E] fp32 or NULL: prob_sum[i] = sum_t R[t, i] (the per-expert
+ * probability mass of Eq. (4), summed in a fixed order).
  * bias entries must be finite. */
 moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router,
                      const float* bias, const float* logit_offset, int32_t* topk_idx,
                      float* topk_gate, int32_t* counts, uint8_t* n_ffn, float* probs_out,
-                     void* ws, size_t ws_bytes, void* stream);
+                     float* prob_sum, void* ws, size_t ws_bytes, void* stream);
 
 /* Dispatch to the FFN experts only (zero-computation experts get no rows).
  *   offsets[e] = sum_{e' < e} counts[e'] over FFN experts, e in [0, N];
@@ -212,6 +214,21 @@ moe_status moe_combine(const moe_shape* shape, const void* x, const void* y_perm
  * fp32. */
 moe_status moe_bias_update(int32_t N, int32_t Z, const int32_t* counts, int64_t T_all,
                            int32_t K, float K_e, float mu, float* bias, void* stream);
+
+/* Device-level load-balance statistics with the zero-expert group,
+ * §2.1.2, Eq. (3)-(5).  The N FFN experts form D groups of G = N/D
+ * consecutive experts; the Z zero-computation experts form group D.
+ *   f[j] = D/(K_e T) * (selections of group j)       j < D
+ *   f[D] = 1/((K - K_e) T) * (selections of zero experts)
+ *   P[j] = (1/T) * sum_{i in group j} prob_sum[i]
+ *   *loss = alpha * sum_{j <= D} f[j] P[j]             (loss may be NULL)
+ * A token's selections of a group are counted once per selected expert of
+ * that group, so f[j] = 1 at the balance point.  counts [N+Z] and prob_sum
+ * [N+Z] come from moe_route over the T tokens (sum them over ranks first for a
+ * global batch); f, P [D+1] fp32.  D must divide N, 0 < K_e < K, Z >= 1. */
+moe_status moe_lb_stats(int32_t N, int32_t Z, int32_t D, const int32_t* counts,
+                        const float* prob_sum, int64_t T, int32_t K, float K_e, float alpha,
+                        float* f, float* P, float* loss, void* stream);
 
 /* Synchronises `stream`, reads the workspace status word into *status_out
  * (may be NULL) and clears it.  Returns MOE_ERR_DEVICE_STATUS when it was

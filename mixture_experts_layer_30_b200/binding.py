@@ -37,7 +37,10 @@ SIGNATURES = {
     "moe_pack_weights": (ctypes.c_int, [_i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_workspace_bytes": (_sz, [_SP]),
     "moe_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
-    "moe_route": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_route": (ctypes.c_int,
+                  [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_lb_stats": (ctypes.c_int, [_i32, _i32, _i32, _vp, _vp, _i64, _i32, _f32, _f32, _vp, _vp,
+                                    _vp, _vp]),
     "moe_permute": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_noalloc": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_expert_gate_up": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -140,7 +143,7 @@ def new_workspace(shape: Shape, device="cuda", stream=None) -> torch.Tensor:
 
 
 def route(shape, x, w_router, bias, ws, topk_idx, topk_gate, counts, n_ffn,
-          logit_offset=None, probs_out=None, stream=None):
+          logit_offset=None, probs_out=None, prob_sum=None, stream=None):
     dt = torch_dtype(shape)
     _check(lib().moe_route(ctypes.byref(shape), _p(x, dt, "x"), _p(w_router, dt, "w_router"),
                            _p(bias, torch.float32, "bias"),
@@ -148,8 +151,18 @@ def route(shape, x, w_router, bias, ws, topk_idx, topk_gate, counts, n_ffn,
                            _p(topk_idx, torch.int32, "topk_idx"),
                            _p(topk_gate, torch.float32, "topk_gate"),
                            _p(counts, torch.int32, "counts"), _p(n_ffn, torch.uint8, "n_ffn"),
-                           _p(probs_out, torch.float32, "probs_out"), _p(ws), ws.numel(),
+                           _p(probs_out, torch.float32, "probs_out"),
+                           _p(prob_sum, torch.float32, "prob_sum"), _p(ws), ws.numel(),
                            _stream(stream)))
+
+
+def lb_stats(N, Z, D, counts, prob_sum, T, K, K_e, alpha, f, P, loss=None, stream=None):
+    """Eq. (3)-(5) statistics from the route's counts and probability sums."""
+    _check(lib().moe_lb_stats(N, Z, D, _p(counts, torch.int32, "counts"),
+                              _p(prob_sum, torch.float32, "prob_sum"), int(T), K, float(K_e),
+                              float(alpha), _p(f, torch.float32, "f"),
+                              _p(P, torch.float32, "P"), _p(loss, torch.float32, "loss"),
+                              _stream(stream)))
 
 
 def permute(shape, x, topk_idx, counts, offsets, row_token, slot_pos, x_perm, ws, stream=None):

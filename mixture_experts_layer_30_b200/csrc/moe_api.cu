@@ -43,7 +43,7 @@ moe_status check_launch(const char* what) {
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct WsLayout {
-  size_t status, logits, route_hist, perm_hist, perm_base, h, total;
+  size_t status, logits, route_hist, route_psum, perm_hist, perm_base, h, total;
 };
 
 int elem_bytes(const moe_shape& s) { return s.dtype == MOE_BF16 ? 2 : 4; }
@@ -89,6 +89,7 @@ WsLayout layout_of(const moe_shape& s) {
   L.status = take(256);
   L.logits = take((size_t)s.T * E * 4);
   L.route_hist = take((size_t)route_ctas(s) * E * 4);
+  L.route_psum = take((size_t)route_ctas(s) * E * 4);
   L.perm_hist = take((size_t)perm_chunks(s) * s.N * 4);
   L.perm_base = take((size_t)perm_chunks(s) * s.N * 4);
   L.h = take((size_t)s.T * s.K * s.I * elem_bytes(s));
@@ -129,19 +130,20 @@ int sm_count() {
 template <int VPL>
 void launch_topk(dim3 grid, cudaStream_t st, const float* logits, const float* bias, int T,
                  int E, int N, int K, int32_t* idx, float* gate, uint8_t* nffn, float* probs,
-                 int32_t* hist) {
+                 int32_t* hist, float* psum) {
   moe::softmax_topk_kernel<VPL><<<grid, moe::kRouteThreads, 0, st>>>(
-      logits, bias, T, E, N, K, idx, gate, nffn, probs, hist);
+      logits, bias, T, E, N, K, idx, gate, nffn, probs, hist, psum);
 }
 
 template <typename T>
 moe_status route_impl(const moe_shape& s, const void* x, const void* w, const float* bias,
                       const float* off, int32_t* idx, float* gate, int32_t* counts,
-                      uint8_t* nffn, float* probs, void* ws, const WsLayout& L,
+                      uint8_t* nffn, float* probs, float* prob_sum, void* ws, const WsLayout& L,
                       cudaStream_t st) {
   const int E = s.N + s.Z;
   float* logits = at<float>(ws, L.logits);
   int32_t* hist = at<int32_t>(ws, L.route_hist);
+  float* psum = prob_sum ? at<float>(ws, L.route_psum) : nullptr;
   if (s.T > 0) {
     if (s.dtype == MOE_BF16 && moe::tc::router_supported(s) &&
         reinterpret_cast<uintptr_t>(off) % 16 == 0) {
@@ -155,18 +157,24 @@ moe_status route_impl(const moe_shape& s, const void* x, const void* w, const fl
     }
     const int vpl = (E + 31) / 32;
     dim3 g(route_ctas(s));
-    if (vpl <= 1) launch_topk<1>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
-    else if (vpl <= 2) launch_topk<2>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
-    else if (vpl <= 3) launch_topk<3>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
-    else if (vpl <= 4) launch_topk<4>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
-    else if (vpl <= 8) launch_topk<8>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
-    else if (vpl <= 16) launch_topk<16>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
-    else if (vpl <= 24) launch_topk<24>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
-    else launch_topk<32>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist);
+    if (vpl <= 1) launch_topk<1>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 2) launch_topk<2>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 3) launch_topk<3>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 4) launch_topk<4>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 8) launch_topk<8>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 16) launch_topk<16>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 24) launch_topk<24>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else launch_topk<32>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
     MOE_TRY(check_launch("softmax/top-K"));
   }
   moe::reduce_hist_kernel<<<(E + 7) / 8, 256, 0, st>>>(hist, route_ctas(s), E, counts);
-  return check_launch("count reduce");
+  MOE_TRY(check_launch("count reduce"));
+  if (prob_sum) {
+    moe::reduce_psum_kernel<<<(E + 7) / 8, 256, 0, st>>>(psum, s.T > 0 ? route_ctas(s) : 0, E,
+                                                        prob_sum);
+    MOE_TRY(check_launch("probability column sums"));
+  }
+  return MOE_OK;
 }
 
 bool g_rank_attr_set[64] = {};
@@ -347,7 +355,7 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router,
                      const float* bias, const float* logit_offset, int32_t* topk_idx,
                      float* topk_gate, int32_t* counts, uint8_t* n_ffn, float* probs_out,
-                     void* ws, size_t ws_bytes, void* stream) {
+                     float* prob_sum, void* ws, size_t ws_bytes, void* stream) {
   g_err[0] = 0;
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
@@ -365,9 +373,9 @@ moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (s.dtype == MOE_BF16)
     return route_impl<__nv_bfloat16>(s, x, w_router, bias, logit_offset, topk_idx, topk_gate,
-                                     counts, n_ffn, probs_out, ws, L, st);
+                                     counts, n_ffn, probs_out, prob_sum, ws, L, st);
   return route_impl<float>(s, x, w_router, bias, logit_offset, topk_idx, topk_gate, counts,
-                           n_ffn, probs_out, ws, L, st);
+                           n_ffn, probs_out, prob_sum, ws, L, st);
 }
 
 moe_status moe_permute(const moe_shape* shape, const void* x, const int32_t* topk_idx,
@@ -549,6 +557,26 @@ moe_status moe_bias_update(int32_t N, int32_t Z, const int32_t* counts, int64_t 
   moe::bias_update_kernel<<<(N + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       N, counts, (long long)T_all, K, K_e, mu, bias);
   return check_launch("bias update");
+}
+
+moe_status moe_lb_stats(int32_t N, int32_t Z, int32_t D, const int32_t* counts,
+                        const float* prob_sum, int64_t T, int32_t K, float K_e, float alpha,
+                        float* f, float* P, float* loss, void* stream) {
+  g_err[0] = 0;
+  if (N < 1 || Z < 1 || N + Z > moe::kMaxExperts)
+    return fail(MOE_ERR_INVALID_ARG, "moe_lb_stats: needs N >= 1 and Z >= 1 (N=%d Z=%d)", N, Z);
+  if (D < 1 || N % D) return fail(MOE_ERR_INVALID_ARG, "moe_lb_stats: D=%d must divide N=%d", D, N);
+  if (K < 1 || K > N + Z) return fail(MOE_ERR_INVALID_ARG, "moe_lb_stats: K=%d", K);
+  if (!(K_e > 0.f) || !(K_e < (float)K))
+    return fail(MOE_ERR_INVALID_ARG, "moe_lb_stats: K_e=%g must lie in (0, K)", (double)K_e);
+  if (T < 1) return fail(MOE_ERR_INVALID_ARG, "moe_lb_stats: T=%lld", (long long)T);
+  MOE_TRY(need(counts, "counts", 4));
+  MOE_TRY(need(prob_sum, "prob_sum", 4));
+  MOE_TRY(need(f, "f", 4));
+  MOE_TRY(need(P, "P", 4));
+  moe::lb_stats_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+      N, Z, D, counts, prob_sum, (long long)T, K, K_e, alpha, f, P, loss);
+  return check_launch("load-balance statistics");
 }
 
 moe_status moe_get_device_status(void* ws, void* stream, uint32_t* status_out) {

@@ -66,8 +66,13 @@ __global__ void __launch_bounds__(kRouteThreads)
 softmax_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
                     int E, int N, int K, int32_t* __restrict__ topk_idx,
                     float* __restrict__ topk_gate, uint8_t* __restrict__ n_ffn,
-                    float* __restrict__ probs_out, int32_t* __restrict__ partial_hist) {
+                    float* __restrict__ probs_out, int32_t* __restrict__ partial_hist,
+                    float* __restrict__ partial_psum) {
   __shared__ int hist[kMaxExperts];
+  __shared__ float psum_acc[kMaxExperts];
+  float ps[VPL];  // this lane's running sums of R over the warp's tokens
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) ps[j] = 0.f;
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -99,6 +104,7 @@ softmax_topk_kernel(const float* __restrict__ logits, const float* __restrict__ 
     for (int j = 0; j < VPL; ++j) {
       int e = lane + 32 * j;
       p[j] = p[j] / sum;                       // R_e
+      ps[j] += p[j];
       if (e < E) {
         s[j] = p[j] + bias[e];                 // biased score, selection only
         if (probs_out) probs_out[(size_t)t * E + e] = p[j];
@@ -145,6 +151,82 @@ softmax_topk_kernel(const float* __restrict__ logits, const float* __restrict__ 
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     partial_hist[(size_t)blockIdx.x * E + e] = hist[e];
+  if (partial_psum) {
+    // column sums of R over the CTA's tokens, warps added in a fixed order
+    for (int e = threadIdx.x; e < E; e += blockDim.x) psum_acc[e] = 0.f;
+    __syncthreads();
+    for (int w = 0; w < nwarps; ++w) {
+      if (warp == w) {
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+          const int e = lane + 32 * j;
+          if (e < E) psum_acc[e] += ps[j];
+        }
+      }
+      __syncthreads();
+    }
+    for (int e = threadIdx.x; e < E; e += blockDim.x)
+      partial_psum[(size_t)blockIdx.x * E + e] = psum_acc[e];
+  }
+}
+
+// prob_sum[e] = sum over route CTAs of their column sums of R (lane-strided
+// partial sums, then a fixed shuffle tree: the same order on every run).
+__global__ void __launch_bounds__(256)
+reduce_psum_kernel(const float* __restrict__ partial, int nparts, int E,
+                   float* __restrict__ prob_sum) {
+  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (e >= E) return;
+  float c = 0.f;
+  for (int p = lane; p < nparts; p += 32) c += partial[(size_t)p * E + e];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0) prob_sum[e] = c;
+}
+
+// Device-level load-balance statistics with the zero-expert group, Eq. (3)-(5):
+//   f_j = D/(K_e T) * sum_{i in group j} counts[i]      (j < D, groups of G = N/D)
+//   f_D = 1/((K - K_e) T) * sum_{i >= N} counts[i]     (zero-computation experts)
+//   P_j = (1/T) * sum_{i in group j} prob_sum[i],  L = alpha * sum_j f_j P_j
+// One warp per group; integer selection counts, fp64 arithmetic, fp32 outputs.
+__global__ void __launch_bounds__(1024)
+lb_stats_kernel(int N, int Z, int D, const int32_t* __restrict__ counts,
+                const float* __restrict__ prob_sum, long long T, int K, float K_e, float alpha,
+                float* __restrict__ f_out, float* __restrict__ p_out, float* __restrict__ loss) {
+  __shared__ double f_sh[kMaxExperts + 1], p_sh[kMaxExperts + 1];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int G = N / D;
+  for (int j = warp; j <= D; j += nwarps) {
+    const int lo = j < D ? j * G : N, hi = j < D ? lo + G : N + Z;
+    long long sel = 0;
+    double pr = 0.0;
+    for (int i = lo + lane; i < hi; i += 32) {
+      sel += counts[i];
+      pr += (double)prob_sum[i];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sel += __shfl_xor_sync(0xffffffffu, sel, o);
+      pr += __shfl_xor_sync(0xffffffffu, pr, o);
+    }
+    const double denom = j < D ? __dmul_rn((double)K_e, (double)T) / (double)D
+                               : __dmul_rn((double)K - (double)K_e, (double)T);
+    const double f = __ddiv_rn((double)sel, denom);
+    const double P = __ddiv_rn(pr, (double)T);
+    if (lane == 0) {
+      f_out[j] = (float)f;
+      p_out[j] = (float)P;
+      f_sh[j] = f;
+      p_sh[j] = P;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && loss) {
+    double acc = 0.0;
+    for (int j = 0; j <= D; ++j) acc += f_sh[j] * p_sh[j];
+    *loss = (float)((double)alpha * acc);
+  }
 }
 
 // counts[e] = sum over route CTAs of their partial histograms.  One warp per

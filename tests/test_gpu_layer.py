@@ -239,3 +239,45 @@ def test_bias_update_open_loop_bit_exact():
                                T).astype(np.float32)
         assert got.tobytes() == want.tobytes()
         assert got[N:].tobytes() == b0[N:].tobytes()
+
+
+@pytest.mark.parametrize("cfg,D", [(C.TINY_F32, 4), (C.MID_BF16, 8), (C.DECODE_T16, 8),
+                                   (C.SKEWED_BIAS_CONTROL, 2)], ids=lambda v: str(v))
+def test_lb_statistics(cfg, D):
+    """Eq. (3)-(5): probability column sums from the route kernel, then f_j, P_j, L."""
+    if cfg.skewed:
+        x, off = IN.make_skewed_step(cfg, 3, device="cuda")
+        L = IN.make_layer_inputs(cfg, device="cuda", with_x=False)
+        L["x"] = x
+    else:
+        L, off = _cfg_inputs(cfg), None
+    shape = B.shape_of(cfg)
+    buf = B.LayerBuffers(shape, with_probs=True)
+    prob_sum = torch.empty(cfg.E, dtype=torch.float32, device="cuda")
+    B.route(shape, L["x"], L["w_router"], L["bias"], buf.ws, buf.topk_idx, buf.topk_gate,
+            buf.counts, buf.n_ffn, logit_offset=off, probs_out=buf.probs, prob_sum=prob_sum)
+    f = torch.empty(D + 1, dtype=torch.float32, device="cuda")
+    Pg = torch.empty_like(f)
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    K_e, alpha = float(np.float32(cfg.K_e)), 0.01
+    B.lb_stats(cfg.N, cfg.Z, D, buf.counts, prob_sum, cfg.T, cfg.K, K_e, alpha, f, Pg, loss)
+    torch.cuda.synchronize()
+    assert B.device_status(buf.ws) == 0
+    x64, wr64 = P.to_f64(L["x"]), P.to_f64(L["w_router"])
+    g = dict(probs=buf.probs.cpu().numpy().astype(np.float64), idx=buf.topk_idx.cpu().numpy(),
+             gate=buf.topk_gate.cpu().numpy().astype(np.float64), counts=buf.counts.cpu().numpy(),
+             n_ffn=buf.n_ffn.cpu().numpy())
+    probs = orc.softmax_rows(orc.router_logits(x64, wr64, None if off is None else
+                                               off.cpu().numpy().astype(np.float64)))
+    b64 = L["bias"].cpu().numpy().astype(np.float64)
+    oidx, _ = orc.biased_topk(probs, b64, cfg.K)
+    ties = P.check_selection(g["idx"], probs + b64[None, :], oidx, cfg.K)
+    idx_ref = oidx.copy()
+    idx_ref[ties] = g["idx"][ties]
+    np.testing.assert_allclose(prob_sum.cpu().numpy(), probs.sum(axis=0), rtol=2e-5, atol=1e-6)
+    f_o, P_o = orc.lb_statistics(probs, idx_ref, cfg.N, D, cfg.K, K_e)
+    np.testing.assert_allclose(f.cpu().numpy(), f_o, rtol=1e-6, atol=0)
+    np.testing.assert_allclose(Pg.cpu().numpy(), P_o, rtol=2e-5, atol=1e-7)
+    np.testing.assert_allclose(loss.item(), orc.lb_loss(f_o, P_o, alpha), rtol=2e-5)
+    # the groups partition all experts
+    assert abs(Pg.sum().item() - 1.0) < 1e-4

@@ -73,11 +73,11 @@ def test_invalid_arguments_return_codes(lib):
     nb = B.workspace_bytes(s)
     fake = ctypes.c_void_p(0x10000)  # never dereferenced: validation fails first
     # NULL shape
-    assert lib.moe_route(None, fake, fake, fake, None, fake, fake, fake, fake, None, fake, nb,
-                         None) == 1
+    assert lib.moe_route(None, fake, fake, fake, None, fake, fake, fake, fake, None, None, fake,
+                         nb, None) == 1
     # NULL workspace
     assert lib.moe_route(ctypes.byref(s), fake, fake, fake, None, fake, fake, fake, fake, None,
-                         None, nb, None) == 1
+                         None, None, nb, None) == 1
     assert b"workspace" in lib.moe_last_error()
     # workspace too small
     assert lib.moe_permute(ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake, fake,
@@ -96,6 +96,21 @@ def test_invalid_arguments_return_codes(lib):
     # bad dtype code
     bad = B.Shape(16, 64, 4, 2, 2, 32, 7)
     assert lib.moe_combine(ctypes.byref(bad), fake, fake, fake, fake, fake, 1.0, fake, None) == 1
+
+
+def test_lb_stats_validation(lib):
+    fake = ctypes.c_void_p(0x10000)
+    args = dict(N=8, Z=4, D=2, T=16, K=3, K_e=2.0)
+
+    def call(**over):
+        a = dict(args, **over)
+        return lib.moe_lb_stats(a["N"], a["Z"], a["D"], fake, fake, a["T"], a["K"], a["K_e"],
+                                0.01, fake, fake, None, None)
+    assert call(D=3) == 1        # D must divide N
+    assert call(Z=0) == 1        # the zero-expert group must exist
+    assert call(K_e=3.0) == 1    # K_e < K
+    assert call(K_e=0.0) == 1
+    assert call(T=0) == 1
 
 
 def test_missing_library_fails_loudly(monkeypatch):
