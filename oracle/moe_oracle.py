@@ -260,6 +260,94 @@ def lb_loss(f, P, alpha):
 
 
 # ---------------------------------------------------------------------------
+# FP8 blockwise quantisation of the expert path (deployment note of the
+# LongCat series notes, inference section: expert weights in FP8 with block
+# scales).  Format: E4M3 elements with one power-of-two scale 2^s per 32
+# consecutive values of a row (along the GEMM reduction axis), the shape the
+# sm_100 block-scaled tensor-core instructions consume.  s is the smallest
+# integer with amax <= 448 * 2^s (the block's scale amax/448 rounded up to a
+# power of two), so no element saturates; scaled values round to
+# nearest-even E4M3.  A block of zeros gets s = 0.
+# ---------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+MX_BLOCK = 32
+
+
+def e4m3_values():
+    """All 256 E4M3 codes decoded (NaN codes 0x7F, 0xFF as nan): sign bit 7,
+    exponent bits 6..3 (bias 7), mantissa bits 2..0; exponent field 0 is
+    subnormal (m/8 * 2^-6); there is no infinity."""
+    v = np.zeros(256)
+    for c in range(256):
+        sgn = -1.0 if c & 0x80 else 1.0
+        e, m = (c >> 3) & 0xF, c & 0x7
+        if e == 0xF and m == 0x7:
+            v[c] = np.nan
+        elif e == 0:
+            v[c] = sgn * (m / 8.0) * 2.0 ** -6
+        else:
+            v[c] = sgn * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return v
+
+
+def round_to_e4m3(v):
+    """Nearest E4M3 value to each float64 in v (ties to an even mantissa),
+    saturating at +-448; returns (codes uint8, values float64)."""
+    v = np.asarray(v, dtype=np.float64)
+    table = e4m3_values()
+    pos = np.array([c for c in range(0x7F)])            # 0x00..0x7E: 0 .. 448
+    pos_val = table[pos]
+    a = np.minimum(np.abs(v), E4M3_MAX)
+    j = np.searchsorted(pos_val, a)                     # pos_val[j-1] < a <= pos_val[j]
+    j = np.clip(j, 1, len(pos) - 1)
+    lo, hi = pos_val[j - 1], pos_val[j]
+    pick_hi = (a - lo > hi - a) | ((a - lo == hi - a) & ((pos[j] & 1) == 0))
+    code = np.where(pick_hi, pos[j], pos[j - 1])
+    code = np.where(a == 0.0, 0, code)
+    neg = np.signbit(v)                                 # -0.0 keeps its sign bit
+    code = np.where(neg, code | 0x80, code).astype(np.uint8)
+    return code, np.where(neg, -table[code & 0x7F], table[code & 0x7F])
+
+
+def mx_scale_exponent(amax):
+    """Smallest integer s with amax <= 448 * 2^s (0 for an all-zero block)."""
+    amax = np.asarray(amax, dtype=np.float64)
+    with np.errstate(divide="ignore"):
+        s = np.ceil(np.log2(np.where(amax > 0, amax, E4M3_MAX) / E4M3_MAX))
+    # exact at the boundaries: correct any rounding of log2
+    s = np.where(E4M3_MAX * 2.0 ** s < amax, s + 1, s)
+    s = np.where(E4M3_MAX * 2.0 ** (s - 1) >= amax, s - 1, s)
+    return np.where(amax > 0, s, 0).astype(np.int64)
+
+
+def mxfp8_quantize(a):
+    """MXFP8 of a [..., K] array (K % 32 == 0) along its last axis.
+
+    Returns (codes uint8 [..., K], scale exponents int64 [..., K/32],
+    dequantised values float64 [..., K])."""
+    a = np.asarray(a, dtype=np.float64)
+    K = a.shape[-1]
+    blocks = a.reshape(a.shape[:-1] + (K // MX_BLOCK, MX_BLOCK))
+    s = mx_scale_exponent(np.abs(blocks).max(axis=-1))
+    scaled = blocks / (2.0 ** s)[..., None]
+    codes, vals = round_to_e4m3(scaled)
+    deq = vals * (2.0 ** s)[..., None]
+    return codes.reshape(a.shape), s, deq.reshape(a.shape)
+
+
+def expert_ffn_mxfp8(x_rows, w1, w3, w2):
+    """FFN_e with MXFP8 operands: x, W1, W3 quantised along d, the SwiGLU
+    hidden h quantised along I, W2 along I; products and sums in float64 on
+    the dequantised values.  Returns (y, h before its quantisation)."""
+    xq = mxfp8_quantize(x_rows)[2]
+    a = xq @ mxfp8_quantize(w1)[2].T
+    u = xq @ mxfp8_quantize(w3)[2].T
+    h = silu(a) * u
+    return mxfp8_quantize(h)[2] @ mxfp8_quantize(w2)[2].T, h
+
+
+# ---------------------------------------------------------------------------
 # The whole layer
 # ---------------------------------------------------------------------------
 

@@ -336,7 +336,87 @@ def check_bf16_decode(orc):
     assert math.copysign(1.0, got[5]) == -1.0
 
 
-ALL_CHECKS = [check_worked_tiny_layer, check_worked_swiglu, check_worked_bias_update,
+def check_e4m3_table(orc):
+    """Values fixed by the E4M3 definition (sign, 4-bit exponent with bias 7,
+    3-bit mantissa, subnormals, 0x7F/0xFF NaN, no infinity)."""
+    t = orc.e4m3_values()
+    assert t[0x7E] == 448.0 and t[0x08] == 2.0 ** -6 and t[0x01] == 2.0 ** -9
+    assert t[0x38] == 1.0 and t[0x40] == 2.0 and t[0x3F] == 1.875 and t[0x07] == 7 * 2.0 ** -9
+    assert t[0xB8] == -1.0 and t[0x80] == 0.0 and np.isnan(t[0x7F]) and np.isnan(t[0xFF])
+    finite = t[~np.isnan(t)]
+    assert len(np.unique(finite)) == 253  # +-0 coincide
+
+
+def brute_force_e4m3(v):
+    """Nearest finite E4M3 code by exhaustive search; ties to the even code."""
+    t = e4m3_table_cache()
+    a = min(abs(v), 448.0)
+    best = None
+    for c in range(0x7F):
+        d = abs(t[c] - a)
+        if best is None or d < best[0] or (d == best[0] and c % 2 == 0):
+            best = (d, c)
+    c = best[1]
+    if math.copysign(1.0, v) < 0:
+        c |= 0x80
+    return c
+
+
+_E4M3 = None
+
+
+def e4m3_table_cache():
+    global _E4M3
+    if _E4M3 is None:
+        vals = []
+        for c in range(256):
+            e, m = (c >> 3) & 0xF, c & 7
+            mag = (m / 8.0) * 2.0 ** -6 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+            vals.append(-mag if c & 0x80 else mag)
+        _E4M3 = vals
+    return _E4M3
+
+
+def check_e4m3_rounding_brute_force(orc, seed=8):
+    rng = np.random.default_rng(seed)
+    t = e4m3_table_cache()
+    mids = [(t[c] + t[c + 1]) / 2 for c in range(0x7E)]           # exact ties
+    vals = list(rng.normal(size=300) * 50) + list(rng.uniform(-1e-3, 1e-3, 100)) + mids + \
+        [-m for m in mids] + [0.0, -0.0, 500.0, -1e6, 448.0, 2.0 ** -10]
+    codes, deq = orc.round_to_e4m3(np.array(vals))
+    for v, c, dv in zip(vals, codes, deq):
+        want = brute_force_e4m3(v)
+        assert int(c) == want, (v, int(c), want)
+        assert dv == t[want & 0x7F] * (-1 if want & 0x80 else 1)
+
+
+def check_mxfp8_block_quantization(orc, seed=9):
+    rng = np.random.default_rng(seed)
+    a = rng.normal(size=(7, 96)) * np.exp(rng.normal(size=(7, 1)) * 3)
+    a[3, 32:64] = 0.0                                               # an all-zero block
+    codes, s, deq = orc.mxfp8_quantize(a)
+    blocks = np.abs(a).reshape(7, 3, 32)
+    amax = blocks.max(axis=-1)
+    nz = amax > 0
+    # the scale puts every block's largest magnitude in (224, 448] before rounding:
+    # the smallest power of two that avoids saturation
+    assert ((amax[nz] / 2.0 ** s[nz] > 224) & (amax[nz] / 2.0 ** s[nz] <= 448)).all()
+    assert (s[~nz] == 0).all() and (deq[3, 32:64] == 0).all()
+    # exact powers-of-two boundaries: 448 * 2^k maps to s = k, just above it to k + 1
+    sb = orc.mx_scale_exponent(np.array([448.0, 448.0 * 2 ** -5, 448.0 * 2 ** 3 * (1 + 2 ** -40),
+                                         1.0, 0.0]))
+    assert list(sb) == [0, -5, 4, -8, 0]
+    # normal-range elements are within half an E4M3 step (2^-4 relative)
+    big = np.abs(a) >= (2.0 ** np.repeat(s, 32, axis=1)) * 2.0 ** -6
+    rel = np.abs(deq - a)[big] / np.abs(a)[big]
+    assert rel.max() <= 2.0 ** -4 + 1e-12
+    # quantising a quantised array changes nothing
+    _, s2, deq2 = orc.mxfp8_quantize(deq)
+    assert np.array_equal(deq2, deq)
+
+
+ALL_CHECKS = [check_e4m3_table, check_e4m3_rounding_brute_force,
+              check_mxfp8_block_quantization, check_worked_tiny_layer, check_worked_swiglu, check_worked_bias_update,
               check_worked_zero_experts, check_softmax_closed_forms, check_topk_brute_force,
               check_dense_reduction, check_all_zero_experts_fixed_point,
               check_k_equals_e_fixed_point, check_permutation_invariants,

@@ -141,7 +141,22 @@ def _mut_lb_zero_group_normaliser(mp):
     mp.setattr(orc, "lb_statistics", lb_statistics)
 
 
-MUTATIONS = [_mut_lb_indicator_per_token, _mut_lb_zero_group_normaliser, _mut_gate_renormalised, _mut_combine_drops_zero_term, _mut_bias_sign,
+def _mut_e4m3_ties_away(mp):
+    real = orc.round_to_e4m3
+
+    def round_to_e4m3(v):
+        v = np.asarray(v, dtype=np.float64)
+        codes, vals = real(v * (1 + 1e-15))     # nudges exact ties upward
+        return codes, vals
+    mp.setattr(orc, "round_to_e4m3", round_to_e4m3)
+
+
+def _mut_mx_scale_off_by_one(mp):
+    real = orc.mx_scale_exponent
+    mp.setattr(orc, "mx_scale_exponent", lambda amax: real(amax) - 1)
+
+
+MUTATIONS = [_mut_e4m3_ties_away, _mut_mx_scale_off_by_one, _mut_lb_indicator_per_token, _mut_lb_zero_group_normaliser, _mut_gate_renormalised, _mut_combine_drops_zero_term, _mut_bias_sign,
              _mut_bias_updates_zero_experts, _mut_tie_to_high_index, _mut_select_by_unbiased,
              _mut_no_silu, _mut_swapped_gate_up, _mut_descending_tokens,
              _mut_softmax_no_max_shift_wrong_axis, _mut_gamma_only_ffn]
