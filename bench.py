@@ -128,9 +128,14 @@ def run_gpu(args, rank, world, local_rank):
     # every rank routes its own batch: x drawn with a per-rank seed
     if rank:
         L["x"] = IN.make_x(cfg, dev, seed=7_000_000 + rank)
-    # expert weights repacked once into the tiled order (untimed set-up); the
-    # row-major originals stay for the oracle baseline
-    W = {k: (B.pack_weights(L[k]) if tiled else L[k]) for k in ("w1", "w3", "w2")}
+    # expert weights repacked once into the tiled order, or quantised to MXFP8
+    # (untimed set-up); the row-major originals stay for the oracle baseline
+    fp8 = args.fp8_experts
+    if fp8:
+        W = {k: B.quantize_weights_mxfp8(L[k]) for k in ("w1", "w3", "w2")}
+        fbuf = B.Mxfp8Buffers(shape, device=dev)
+    else:
+        W = {k: (B.pack_weights(L[k]) if tiled else L[k]) for k in ("w1", "w3", "w2")}
     torch.cuda.synchronize()
     buf = B.LayerBuffers(shape, device=dev)
     bias = L["bias"].clone()
@@ -158,12 +163,21 @@ def run_gpu(args, rank, world, local_rank):
             B.lb_stats(cfg.N, cfg.Z, lb["D"], buf.counts, lb["prob_sum"], cfg.T, cfg.K, K_e,
                        0.001, lb["f"], lb["P"], lb["loss"])
         if ev: ev[1].record(stream)
-        B.permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
-                  buf.x_perm, buf.ws)
-        if ev: ev[2].record(stream)
-        B.expert_gate_up(s, buf.x_perm, W["w1"], W["w3"], buf.offsets, buf.h, buf.ws)
-        if ev: ev[3].record(stream)
-        B.expert_down(s, buf.h, W["w2"], buf.offsets, buf.y_perm, buf.ws)
+        if fp8:
+            B.permute_mxfp8(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token,
+                            buf.slot_pos, fbuf.x_perm_q, fbuf.x_perm_sf, buf.ws)
+            if ev: ev[2].record(stream)
+            B.expert_gate_up_mxfp8(s, fbuf.x_perm_q, fbuf.x_perm_sf, W["w1"], W["w3"],
+                                   buf.offsets, fbuf.h_q, fbuf.h_sf, buf.ws)
+            if ev: ev[3].record(stream)
+            B.expert_down_mxfp8(s, fbuf.h_q, fbuf.h_sf, W["w2"], buf.offsets, buf.y_perm, buf.ws)
+        else:
+            B.permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
+                      buf.x_perm, buf.ws)
+            if ev: ev[2].record(stream)
+            B.expert_gate_up(s, buf.x_perm, W["w1"], W["w3"], buf.offsets, buf.h, buf.ws)
+            if ev: ev[3].record(stream)
+            B.expert_down(s, buf.h, W["w2"], buf.offsets, buf.y_perm, buf.ws)
         if ev: ev[4].record(stream)
         B.combine(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, cfg.gamma, buf.out)
         if ev: ev[5].record(stream)
@@ -257,10 +271,19 @@ def run_gpu(args, rank, world, local_rank):
             s = shape
             B.route(s, x_dev[j], L["w_router"], bias, buf.ws, buf.topk_idx, buf.topk_gate,
                     buf.counts, buf.n_ffn)
-            B.permute(s, x_dev[j], buf.topk_idx, buf.counts, buf.offsets, buf.row_token,
-                      buf.slot_pos, buf.x_perm, buf.ws)
-            B.expert_gate_up(s, buf.x_perm, W["w1"], W["w3"], buf.offsets, buf.h, buf.ws)
-            B.expert_down(s, buf.h, W["w2"], buf.offsets, buf.y_perm, buf.ws)
+            if fp8:
+                B.permute_mxfp8(s, x_dev[j], buf.topk_idx, buf.counts, buf.offsets,
+                                buf.row_token, buf.slot_pos, fbuf.x_perm_q, fbuf.x_perm_sf,
+                                buf.ws)
+                B.expert_gate_up_mxfp8(s, fbuf.x_perm_q, fbuf.x_perm_sf, W["w1"], W["w3"],
+                                       buf.offsets, fbuf.h_q, fbuf.h_sf, buf.ws)
+                B.expert_down_mxfp8(s, fbuf.h_q, fbuf.h_sf, W["w2"], buf.offsets, buf.y_perm,
+                                    buf.ws)
+            else:
+                B.permute(s, x_dev[j], buf.topk_idx, buf.counts, buf.offsets, buf.row_token,
+                          buf.slot_pos, buf.x_perm, buf.ws)
+                B.expert_gate_up(s, buf.x_perm, W["w1"], W["w3"], buf.offsets, buf.h, buf.ws)
+                B.expert_down(s, buf.h, W["w2"], buf.offsets, buf.y_perm, buf.ws)
             B.combine(s, x_dev[j], buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos,
                       cfg.gamma, out_dev[j])
             x_free[j].record(stream)
@@ -295,11 +318,13 @@ def run_gpu(args, rank, world, local_rank):
     R = int(counts[:cfg.N].sum())
     touched = int((counts[:cfg.N] > 0).sum())
     esz = 2 if cfg.dtype == "bf16" else 4
-    w13_bytes = touched * 2 * cfg.I * cfg.d * esz
-    w2_bytes = touched * cfg.d * cfg.I * esz
+    # expert operands: bf16/fp32, or MXFP8 (1 byte + a scale byte per 32 values)
+    wsz = (1 + 1 / 32) if fp8 else esz
+    w13_bytes = touched * 2 * cfg.I * cfg.d * wsz
+    w2_bytes = touched * cfg.d * cfg.I * wsz
     # gate/up reads every routed row of x_perm once and writes h
-    gate_up_bytes = w13_bytes + R * cfg.d * esz + R * cfg.I * esz
-    down_bytes = w2_bytes + R * cfg.I * esz + R * cfg.d * esz
+    gate_up_bytes = w13_bytes + R * cfg.d * wsz + R * cfg.I * wsz
+    down_bytes = w2_bytes + R * cfg.I * wsz + R * cfg.d * esz
     gate_up_flops = 4.0 * cfg.d * cfg.I * R
     down_flops = 2.0 * cfg.d * cfg.I * R
     router_flops = 2.0 * cfg.d * cfg.E * cfg.T
@@ -332,14 +357,16 @@ def run_gpu(args, rank, world, local_rank):
         "data": "synthetic (seeded N(0,1) activations, random-init weights of the stated shape)",
         "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "N": cfg.N, "Z": cfg.Z,
                    "K": cfg.K, "I": cfg.I, "K_e": cfg.K_e, "tokens_per_rank": cfg.T,
-                   "expert_weights": "tiled (moe_pack_weights)" if tiled else "row-major",
+                   "expert_weights": ("mxfp8 (moe_quantize_weights_mxfp8)" if args.fp8_experts
+                                      else "tiled (moe_pack_weights)" if tiled else "row-major"),
                    "parallelism": f"token-dp{world} (weights replicated, counts all-reduced)",
                    "l2": "inputs larger than L2 (38.7 GB of expert weights streamed per step)"},
-        "roofline": {"kernel": "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)",
+        "roofline": {"kernel": ("moe_expert_gate_up_mxfp8 (tcgen05 block-scaled grouped GEMM)"
+                                if fp8 else "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)"),
                      "bound": "hbm", "achieved": round(achieved, 1),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
-                     "algorithmic_bytes_per_launch": gate_up_bytes,
+                     "algorithmic_bytes_per_launch": int(gate_up_bytes),
                      "avg_launch_ms": round(gu_ms, 4)},
         "layer": {
             "routed_rows": R, "touched_experts": touched,
@@ -357,6 +384,7 @@ def run_gpu(args, rank, world, local_rank):
         "gpu_launches": int(launches),
         "cuda_graph": graph is not None,
         "lb_stats": lb is not None,
+        "expert_format": "mxfp8" if fp8 else cfg.dtype,
         "clocks": clk,
     }
     return line, L
@@ -464,6 +492,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--lb-stats", action="store_true",
                     help="also compute the device-level load-balance statistics each step")
+    ap.add_argument("--fp8-experts", action="store_true",
+                    help="expert weights and routed activations in MXFP8 (block-scaled E4M3)")
     ap.add_argument("--graph", action="store_true",
                     help="replay one captured CUDA graph per step (single GPU)")
     args = ap.parse_args()

@@ -197,6 +197,46 @@ moe_status moe_expert_ffn(const moe_shape* shape, const void* x_perm, const void
                           const void* w3, const void* w2, const int32_t* offsets,
                           void* y_perm, void* ws, size_t ws_bytes, void* stream);
 
+/* ---- MXFP8 expert path ------------------------------------------------
+ * FP8 blockwise-quantised experts (the LongCat series notes: FP8 with block
+ * scales at inference).  Format MXFP8: E4M3 values with one power-of-two
+ * scale 2^s per 32 consecutive values of a row along the GEMM reduction
+ * axis; s is the smallest integer with amax <= 448 * 2^s (no saturation),
+ * stored as the byte s + 127.  The expert GEMMs use the sm_100a block-scaled
+ * tensor-core instructions.  Requires dtype MOE_BF16 (x, y_perm, out stay
+ * bf16), d % 256 == 0 and I % 128 == 0.  The shape's weight_layout is ignored.
+ */
+
+/* Quantises n_mats bf16 matrices [rows, cols] (row-major, reduction axis =
+ * cols) to MXFP8.  dst_q: rows*cols bytes per matrix, 128 x 128 tiles of 16 KiB
+ * (row-major inside a tile) at tile index (m*rows/128 + rb)*cols/128 + cb.
+ * dst_sf: one 512-byte atom per tile; byte 16*(r%32) + 4*(r/32) + b is the
+ * scale of tile row r, 32-column block b.  w1/w3 are quantised as N matrices
+ * [I, d], w2 as N matrices [d, I].  rows % 128 == 0, cols % 128 == 0. */
+moe_status moe_quantize_weights_mxfp8(int32_t n_mats, int32_t rows, int32_t cols,
+                                      const void* src, void* dst_q, void* dst_sf, void* stream);
+
+/* moe_permute whose copy quantises: x_perm_q [T*K, d] E4M3 bytes and
+ * x_perm_sf [T*K, d/32] scale bytes (row-major) for every routed row; the
+ * layout outputs are those of moe_permute. */
+moe_status moe_permute_mxfp8(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                             const int32_t* counts, int32_t* offsets, int32_t* row_token,
+                             int32_t* slot_pos, void* x_perm_q, void* x_perm_sf, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* h = SiLU(x_perm W1_e^T) * (x_perm W3_e^T) on MXFP8 operands (fp32
+ * accumulation), written as MXFP8: h_q [T*K, I] bytes, h_sf [T*K, I/32]. */
+moe_status moe_expert_gate_up_mxfp8(const moe_shape* shape, const void* x_perm_q,
+                                    const void* x_perm_sf, const void* w1_q, const void* w1_sf,
+                                    const void* w3_q, const void* w3_sf, const int32_t* offsets,
+                                    void* h_q, void* h_sf, void* ws, size_t ws_bytes,
+                                    void* stream);
+
+/* y_perm = h W2_e^T on MXFP8 operands, written as bf16 [T*K, d]. */
+moe_status moe_expert_down_mxfp8(const moe_shape* shape, const void* h_q, const void* h_sf,
+                                 const void* w2_q, const void* w2_sf, const int32_t* offsets,
+                                 void* y_perm, void* ws, size_t ws_bytes, void* stream);
+
 /* Weighted sum of Eq. (1) with the zero-computation experts folded in:
  *   out[t, :] = gamma * ( sum_{k: idx < N} gate[t,k] * y_perm[slot_pos[t,k], :]
  *                         + (sum_{k: idx >= N} gate[t,k]) * x[t, :] )

@@ -35,6 +35,12 @@ class Shape(ctypes.Structure):
 _SP = ctypes.POINTER(Shape)
 SIGNATURES = {
     "moe_pack_weights": (ctypes.c_int, [_i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moe_quantize_weights_mxfp8": (ctypes.c_int, [_i32, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "moe_permute_mxfp8": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                         _vp]),
+    "moe_expert_gate_up_mxfp8": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                                _vp, _sz, _vp]),
+    "moe_expert_down_mxfp8": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_workspace_bytes": (_sz, [_SP]),
     "moe_workspace_init": (ctypes.c_int, [_vp, _sz, _vp]),
     "moe_route": (ctypes.c_int,
@@ -127,6 +133,78 @@ def _p(t, dtype=None, name="tensor"):
 def _stream(stream=None):
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def quantize_weights_mxfp8(w: torch.Tensor, stream=None):
+    """MXFP8 of bf16 weights [n, rows, cols] (reduction axis = cols): returns
+    (codes uint8 [n*rows*cols] in 128x128 tiles, scales uint8 [n*rows*cols/32]
+    in 512-byte atoms)."""
+    if w.dim() == 2:
+        w = w.unsqueeze(0)
+    n, rows, cols = w.shape
+    q = torch.empty(n * rows * cols, dtype=torch.uint8, device=w.device)
+    sf = torch.empty(n * rows * cols // 32, dtype=torch.uint8, device=w.device)
+    _check(lib().moe_quantize_weights_mxfp8(n, rows, cols, _p(w, torch.bfloat16, "w"), _p(q),
+                                            _p(sf), _stream(stream)))
+    return q, sf
+
+
+def permute_mxfp8(shape, x, topk_idx, counts, offsets, row_token, slot_pos, x_perm_q, x_perm_sf,
+                  ws, stream=None):
+    _check(lib().moe_permute_mxfp8(ctypes.byref(shape), _p(x, torch.bfloat16, "x"),
+                                   _p(topk_idx, torch.int32, "topk_idx"),
+                                   _p(counts, torch.int32, "counts"),
+                                   _p(offsets, torch.int32, "offsets"),
+                                   _p(row_token, torch.int32, "row_token"),
+                                   _p(slot_pos, torch.int32, "slot_pos"),
+                                   _p(x_perm_q, torch.uint8, "x_perm_q"),
+                                   _p(x_perm_sf, torch.uint8, "x_perm_sf"), _p(ws), ws.numel(),
+                                   _stream(stream)))
+
+
+def expert_gate_up_mxfp8(shape, x_perm_q, x_perm_sf, w1, w3, offsets, h_q, h_sf, ws,
+                         stream=None):
+    """w1, w3: (codes, scales) pairs from quantize_weights_mxfp8."""
+    _check(lib().moe_expert_gate_up_mxfp8(
+        ctypes.byref(shape), _p(x_perm_q, torch.uint8, "x_perm_q"),
+        _p(x_perm_sf, torch.uint8, "x_perm_sf"), _p(w1[0]), _p(w1[1]), _p(w3[0]), _p(w3[1]),
+        _p(offsets, torch.int32, "offsets"), _p(h_q, torch.uint8, "h_q"),
+        _p(h_sf, torch.uint8, "h_sf"), _p(ws), ws.numel(), _stream(stream)))
+
+
+def expert_down_mxfp8(shape, h_q, h_sf, w2, offsets, y_perm, ws, stream=None):
+    _check(lib().moe_expert_down_mxfp8(
+        ctypes.byref(shape), _p(h_q, torch.uint8, "h_q"), _p(h_sf, torch.uint8, "h_sf"),
+        _p(w2[0]), _p(w2[1]), _p(offsets, torch.int32, "offsets"),
+        _p(y_perm, torch.bfloat16, "y_perm"), _p(ws), ws.numel(), _stream(stream)))
+
+
+class Mxfp8Buffers:
+    """Routed-row buffers of the MXFP8 expert path for one shape."""
+
+    def __init__(self, shape: Shape, device="cuda"):
+        R = max(shape.T * shape.K, 1)
+        kw = dict(dtype=torch.uint8, device=device)
+        self.x_perm_q = torch.empty((R, shape.d), **kw)
+        self.x_perm_sf = torch.empty((R, shape.d // 32), **kw)
+        self.h_q = torch.empty((R, shape.I), **kw)
+        self.h_sf = torch.empty((R, shape.I // 32), **kw)
+
+
+def forward_mxfp8(buf: "LayerBuffers", fb: Mxfp8Buffers, x, w_router, w1, w3, w2, bias,
+                  gamma=1.0, logit_offset=None, stream=None):
+    """The layer with MXFP8 experts: w1, w3, w2 are (codes, scales) pairs."""
+    s = buf.shape
+    route(s, x, w_router, bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts, buf.n_ffn,
+          logit_offset=logit_offset, probs_out=buf.probs, stream=stream)
+    permute_mxfp8(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
+                  fb.x_perm_q, fb.x_perm_sf, buf.ws, stream=stream)
+    expert_gate_up_mxfp8(s, fb.x_perm_q, fb.x_perm_sf, w1, w3, buf.offsets, fb.h_q, fb.h_sf,
+                         buf.ws, stream=stream)
+    expert_down_mxfp8(s, fb.h_q, fb.h_sf, w2, buf.offsets, buf.y_perm, buf.ws, stream=stream)
+    combine(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, gamma, buf.out,
+            stream=stream)
+    return buf.out
 
 
 def workspace_bytes(shape: Shape) -> int:

@@ -13,6 +13,8 @@
 #include "permute.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_fp8.cuh"
+#include "quant.cuh"
 #include "combine.cuh"
 
 namespace {
@@ -344,6 +346,26 @@ moe_status moe_pack_weights(int32_t n_mats, int32_t rows, int32_t cols, int32_t 
   return check_launch("weight pack");
 }
 
+moe_status moe_quantize_weights_mxfp8(int32_t n_mats, int32_t rows, int32_t cols,
+                                      const void* src, void* dst_q, void* dst_sf, void* stream) {
+  g_err[0] = 0;
+  if (n_mats < 0 || rows < 0 || cols < 0 || rows % 128 || cols % 128)
+    return fail(MOE_ERR_INVALID_ARG,
+                "moe_quantize_weights_mxfp8: rows=%d and cols=%d must be multiples of 128", rows,
+                cols);
+  const long long tiles = (long long)n_mats * (rows / 128) * (cols / 128);
+  if (tiles == 0) return MOE_OK;
+  if (tiles > 0x7fffffffLL) return fail(MOE_ERR_UNSUPPORTED, "too many weight tiles");
+  MOE_TRY(need(src, "src", 16));
+  MOE_TRY(need(dst_q, "dst_q", 16));
+  MOE_TRY(need(dst_sf, "dst_sf", 16));
+  moe::quantize_weights_mxfp8_kernel<<<(unsigned)tiles, 256, 0,
+                                       static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(src), rows, cols, static_cast<uint8_t*>(dst_q),
+      static_cast<uint8_t*>(dst_sf));
+  return check_launch("mxfp8 weight quantisation");
+}
+
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   g_err[0] = 0;
   if (!ws || ws_bytes < 256) return fail(MOE_ERR_INVALID_ARG, "workspace NULL or < 256 bytes");
@@ -439,6 +461,90 @@ moe_status moe_permute_noalloc(const moe_shape* shape, const void* x, const int3
                                        x_perm, scratch, L, st);
   return permute_impl<float>(s, x, topk_idx, counts, offsets, row_token, slot_pos, x_perm,
                              scratch, L, st);
+}
+
+static moe_status check_mxfp8_shape(const moe_shape* shape) {
+  MOE_TRY(validate_shape(shape));
+  if (!moe::f8::supported(*shape))
+    return fail(MOE_ERR_UNSUPPORTED,
+                "the MXFP8 path needs bf16, d %% 256 == 0 and I %% 128 == 0 (d=%d, I=%d)",
+                shape->d, shape->I);
+  return MOE_OK;
+}
+
+moe_status moe_permute_mxfp8(const moe_shape* shape, const void* x, const int32_t* topk_idx,
+                             const int32_t* counts, int32_t* offsets, int32_t* row_token,
+                             int32_t* slot_pos, void* x_perm_q, void* x_perm_sf, void* ws,
+                             size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(check_mxfp8_shape(shape));
+  const moe_shape& s = *shape;
+  WsLayout L;
+  MOE_TRY(check_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(offsets, "offsets", 4));
+  if (s.T > 0) {
+    MOE_TRY(need(x, "x", 16));
+    MOE_TRY(need(topk_idx, "topk_idx", 4));
+    MOE_TRY(need(row_token, "row_token", 4));
+    MOE_TRY(need(slot_pos, "slot_pos", 4));
+    MOE_TRY(need(x_perm_q, "x_perm_q", 16));
+    MOE_TRY(need(x_perm_sf, "x_perm_sf", 16));
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_TRY(permute_impl<__nv_bfloat16>(s, x, topk_idx, counts, offsets, row_token, slot_pos,
+                                      nullptr, ws, L, st));
+  if (s.T > 0) {
+    moe::gather_quant_kernel<<<(s.T + 7) / 8, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), slot_pos, s.T, s.K, s.d,
+        static_cast<uint8_t*>(x_perm_q), static_cast<uint8_t*>(x_perm_sf));
+    MOE_TRY(check_launch("quantising dispatch copy"));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_expert_gate_up_mxfp8(const moe_shape* shape, const void* x_perm_q,
+                                    const void* x_perm_sf, const void* w1_q, const void* w1_sf,
+                                    const void* w3_q, const void* w3_sf, const int32_t* offsets,
+                                    void* h_q, void* h_sf, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(check_mxfp8_shape(shape));
+  const moe_shape& s = *shape;
+  WsLayout L;
+  MOE_TRY(check_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(x_perm_q, "x_perm_q", 16));
+  MOE_TRY(need(x_perm_sf, "x_perm_sf", 16));
+  MOE_TRY(need(w1_q, "w1_q", 16));
+  MOE_TRY(need(w1_sf, "w1_sf", 16));
+  MOE_TRY(need(w3_q, "w3_q", 16));
+  MOE_TRY(need(w3_sf, "w3_sf", 16));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(h_q, "h_q", 16));
+  MOE_TRY(need(h_sf, "h_sf", 4));
+  if (s.T == 0) return MOE_OK;
+  return moe::f8::launch_gate_up(s, x_perm_q, x_perm_sf, w1_q, w1_sf, w3_q, w3_sf, offsets, h_q,
+                                 h_sf, at<uint32_t>(ws, L.status), sm_count(),
+                                 static_cast<cudaStream_t>(stream), g_err, sizeof(g_err));
+}
+
+moe_status moe_expert_down_mxfp8(const moe_shape* shape, const void* h_q, const void* h_sf,
+                                 const void* w2_q, const void* w2_sf, const int32_t* offsets,
+                                 void* y_perm, void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(check_mxfp8_shape(shape));
+  const moe_shape& s = *shape;
+  WsLayout L;
+  MOE_TRY(check_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(h_q, "h_q", 16));
+  MOE_TRY(need(h_sf, "h_sf", 16));
+  MOE_TRY(need(w2_q, "w2_q", 16));
+  MOE_TRY(need(w2_sf, "w2_sf", 16));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(y_perm, "y_perm", 16));
+  if (s.T == 0) return MOE_OK;
+  return moe::f8::launch_down(s, h_q, h_sf, w2_q, w2_sf, offsets, y_perm,
+                              at<uint32_t>(ws, L.status), sm_count(),
+                              static_cast<cudaStream_t>(stream), g_err, sizeof(g_err));
 }
 
 moe_status moe_expert_gate_up(const moe_shape* shape, const void* x_perm, const void* w1,
