@@ -310,7 +310,7 @@ gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
               const uint32_t am = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(h)));
               const int s = mx_scale_exp(__uint_as_float(am));
               if (lane == j) my_s = s;
-              stg[j * kPitchH + lane] = mx_quant(h, s);
+              stg[j * kPitchH + lane] = mx_quant_inv(h, mx_inv_scale(s));
             }
             __syncwarp();
             // 32 tokens x 32 bytes: two 16-byte stores per lane

@@ -32,7 +32,18 @@ MOE_DEV int mx_scale_exp(float amax) {
 
 MOE_DEV uint8_t mx_scale_byte(int s) { return (uint8_t)min(254, max(0, s + 127)); }
 
+// 2^-s as a float: exact for -126 <= -s <= 127 (built from the exponent bits),
+// ldexpf outside that range.
+MOE_DEV float mx_inv_scale(int s) {
+  const int e = 127 - s;
+  return (e >= 1 && e <= 254) ? __uint_as_float((uint32_t)e << 23) : ldexpf(1.0f, -s);
+}
+
 // E4M3 code of v * 2^-s, round to nearest even (|v| <= 448 * 2^s never saturates).
+// Multiplying by a power of two is exact, so this is the rounding of v / 2^s.
+MOE_DEV uint8_t mx_quant_inv(float v, float inv) {
+  return (uint8_t)__nv_cvt_float_to_fp8(v * inv, __NV_SATFINITE, __NV_E4M3);
+}
 MOE_DEV uint8_t mx_quant(float v, int s) {
   return (uint8_t)__nv_cvt_float_to_fp8(ldexpf(v, -s), __NV_SATFINITE, __NV_E4M3);
 }
@@ -47,11 +58,13 @@ MOE_DEV int mx_quant_block_bf16(const uint4 (&in)[4], uint4 (&q)[2]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(f[i]));
   const int s = mx_scale_exp(amax);
+  const float inv = mx_inv_scale(s);
   uint32_t w[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
-    w[i] = (uint32_t)mx_quant(f[4 * i], s) | ((uint32_t)mx_quant(f[4 * i + 1], s) << 8) |
-           ((uint32_t)mx_quant(f[4 * i + 2], s) << 16) | ((uint32_t)mx_quant(f[4 * i + 3], s) << 24);
+    w[i] = (uint32_t)mx_quant_inv(f[4 * i], inv) | ((uint32_t)mx_quant_inv(f[4 * i + 1], inv) << 8) |
+           ((uint32_t)mx_quant_inv(f[4 * i + 2], inv) << 16) |
+           ((uint32_t)mx_quant_inv(f[4 * i + 3], inv) << 24);
   q[0] = make_uint4(w[0], w[1], w[2], w[3]);
   q[1] = make_uint4(w[4], w[5], w[6], w[7]);
   return s;
