@@ -53,6 +53,10 @@ MID_BF16 = MoEConfig("mid_bf16_T4096_d2048_N64_Z32_K6_I1024", T=4096, d=2048, N=
 LONGCAT_PREFILL = MoEConfig("longcat_prefill_bf16_T8192_d6144_N512_Z256_K12_I2048", T=8192,
                             d=6144, N=512, Z=256, K=12, I=2048, dtype="bf16",
                             w_std=0.006, bias_kind="zero")
+# The LongCat expert geometry (d=6144, I=2048, K=12, ~128 rows per expert) on
+# 32 FFN experts: a few GB, for profiling captures and quick parity runs.
+LONGCAT_SLICE = MoEConfig("longcat_slice_bf16_T512_d6144_N32_Z16_K12_I2048", T=512, d=6144,
+                          N=32, Z=16, K=12, I=2048, dtype="bf16", w_std=0.006, bias_kind="zero")
 DECODE_T16 = MID_BF16.with_T(16, "decode_bf16_T16_d2048_N64_Z32_K6_I1024")
 DECODE_T64 = MID_BF16.with_T(64, "decode_bf16_T64_d2048_N64_Z32_K6_I1024")
 DECODE_T256 = MID_BF16.with_T(256, "decode_bf16_T256_d2048_N64_Z32_K6_I1024")
@@ -60,4 +64,4 @@ SKEWED_BIAS_CONTROL = replace(TINY_F32, name="skewed_f32_T16384_d256_N16_Z8_K4_s
                               T=16384, steps=200, skewed=True)
 
 CONFIGS = {c.name: c for c in (TINY_F32, MID_BF16, LONGCAT_PREFILL, DECODE_T16, DECODE_T64,
-                               DECODE_T256, SKEWED_BIAS_CONTROL)}
+                               DECODE_T256, SKEWED_BIAS_CONTROL, LONGCAT_SLICE)}

@@ -55,7 +55,7 @@ def _fp8_layer(cfg, T=None):
     return L, shape, buf, fb
 
 
-@pytest.mark.parametrize("cfg", [C.MID_BF16, C.DECODE_T16, C.DECODE_T256],
+@pytest.mark.parametrize("cfg", [C.MID_BF16, C.DECODE_T16, C.DECODE_T256, C.LONGCAT_SLICE],
                          ids=lambda c: c.name)
 def test_mxfp8_layer(cfg):
     L, shape, buf, fb = _fp8_layer(cfg)
