@@ -196,6 +196,12 @@ gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
 #pragma unroll
       for (int c = 0; c < kNMax / 32; ++c)
         sfb_src[c] = args.sfb + (size_t)(t.r0 + min(32 * c + lane, t.n - 1)) * sfb_row;
+      const uint8_t* sfb_rot[4];  // row group (i + lane/8) % 4 of copy i
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = (i + (lane >> 3)) & 3;
+        sfb_rot[i] = args.sfb + (size_t)(t.r0 + min(32 * c + lane, t.n - 1)) * sfb_row;
+      }
       for (int kb = 0; kb < nk; ++kb) {
         int go = 1;
         if (lane == 0) go = mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status);
@@ -219,9 +225,15 @@ gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
           bulk_load_hint(sf + 512, args.sfa1 + (size_t)i1 * 512, 512, fb, pol_w);
           ++issued;
         }
-        // token scales: 4 bytes (the stage's four K steps) per row
+        // token scales: 4 bytes (the stage's four K steps) per row.  Row groups
+        // 0-3 rotate with the lane so the 32 writes of one copy hit 32 banks.
 #pragma unroll
-        for (int c = 0; c < kNMax / 32; ++c)
+        for (int i = 0; i < 4; ++i) {
+          const int c = (i + (lane >> 3)) & 3;
+          cp_async_4(sf + 1024 + lane * 16 + c * 4, sfb_rot[i] + 4 * kb);
+        }
+#pragma unroll
+        for (int c = 4; c < kNMax / 32; ++c)
           cp_async_4(sf + 1024 + (c >> 2) * 512 + lane * 16 + (c & 3) * 4, sfb_src[c] + 4 * kb);
         cp_async_arrive_noinc(fb);
         if (++stage == kStages) { stage = 0; phase ^= 1; }
@@ -303,15 +315,31 @@ gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
             tmem_wait_ld();
             // h = SiLU(gate) * up for this lane's feature, tokens j0..j0+31, then
             // MXFP8: the warp's 32 features of one token are one scale block
-            int my_s = 0;
+            float hv[32], am[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const float h = silu_fast(__uint_as_float(v0[j])) * __uint_as_float(v1[j]);
-              const uint32_t am = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(h)));
-              const int s = mx_scale_exp(__uint_as_float(am));
-              if (lane == j) my_s = s;
-              stg[j * kPitchH + lane] = mx_quant_inv(h, mx_inv_scale(s));
+              hv[j] = silu_fast(__uint_as_float(v0[j])) * __uint_as_float(v1[j]);
+              am[j] = fabsf(hv[j]);
             }
+            // per-token amax over the 32 lanes by a butterfly transpose-reduce:
+            // each round a lane keeps half of its tokens and merges the partner's
+            // half; afterwards am[0] of lane j is the amax of token j
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) {
+              const bool upper = (lane & off) != 0;
+#pragma unroll
+              for (int i = 0; i < off; ++i) {
+                const float send = upper ? am[i] : am[i + off];
+                const float keep = upper ? am[i + off] : am[i];
+                am[i] = fmaxf(keep, __shfl_xor_sync(0xffffffffu, send, off));
+              }
+            }
+            const int my_s = mx_scale_exp(am[0]);           // scale of token j0 + lane
+            const float my_inv = mx_inv_scale(my_s);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              stg[j * kPitchH + lane] =
+                  mx_quant_inv(hv[j], __shfl_sync(0xffffffffu, my_inv, j));
             __syncwarp();
             // 32 tokens x 32 bytes: two 16-byte stores per lane
 #pragma unroll
