@@ -61,6 +61,46 @@ router_gemm_simt_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
 // --- softmax + biased top-K + per-CTA histogram -----------------------------
 // One warp per token.  Lane l holds experts e = l + 32*j, j < VPL.
 // Selection key: (R_e + b_e) descending, then e ascending (lower index wins ties).
+
+// Order-preserving map of a float to an unsigned key (larger float -> larger
+// key); -0 is folded into +0 first.  Keys are > 0 for every float, so 0 means
+// "no candidate".
+MOE_DEV uint32_t ordered_key(float x) {
+  const uint32_t u = __float_as_uint(x + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Insert (v, j) into a lane's descending top-3 list; equal values keep the
+// earlier (lower) j first.
+struct Top3 {
+  float v[3];
+  float p[3];
+  int j[3];
+  MOE_DEV void clear() {
+#pragma unroll
+    for (int i = 0; i < 3; ++i) { v[i] = -INFINITY; p[i] = 0.f; j[i] = -1; }
+  }
+  MOE_DEV void insert(float vv, float pp, int jj) {
+    if (j[2] >= 0 && !(vv > v[2])) return;
+    if (j[1] < 0 || vv > v[1]) {
+      v[2] = v[1]; p[2] = p[1]; j[2] = j[1];
+      if (j[0] < 0 || vv > v[0]) {
+        v[1] = v[0]; p[1] = p[0]; j[1] = j[0];
+        v[0] = vv; p[0] = pp; j[0] = jj;
+      } else {
+        v[1] = vv; p[1] = pp; j[1] = jj;
+      }
+    } else {
+      v[2] = vv; p[2] = pp; j[2] = jj;
+    }
+  }
+  MOE_DEV void pop() {
+    v[0] = v[1]; p[0] = p[1]; j[0] = j[1];
+    v[1] = v[2]; p[1] = p[2]; j[1] = j[2];
+    v[2] = -INFINITY; p[2] = 0.f; j[2] = -1;
+  }
+};
+
 template <int VPL>
 __global__ void __launch_bounds__(kRouteThreads)
 softmax_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
@@ -94,51 +134,48 @@ softmax_topk_kernel(const float* __restrict__ logits, const float* __restrict__ 
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
       int e = lane + 32 * j;
-      p[j] = e < E ? expf(p[j] - m) : 0.f;
+      p[j] = e < E ? __expf(p[j] - m) : 0.f;
       sum += p[j];
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    uint32_t taken = 0;
+    const float inv = 1.0f / sum;
+    Top3 top;
+    top.clear();
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
       int e = lane + 32 * j;
-      p[j] = p[j] / sum;                       // R_e
+      p[j] *= inv;                             // R_e
       ps[j] += p[j];
       if (e < E) {
-        s[j] = p[j] + bias[e];                 // biased score, selection only
+        s[j] = p[j] + __ldg(bias + e);         // biased score, selection only
         if (probs_out) probs_out[(size_t)t * E + e] = p[j];
+        top.insert(s[j], p[j], j);
       } else {
-        taken |= 1u << j;                      // padding never selected
         s[j] = -INFINITY;
       }
     }
+    uint32_t taken = 0;
     int nf = 0;
     for (int k = 0; k < K; ++k) {
-      // lane-local best among untaken: larger s, then smaller e (= smaller j)
-      float bs = -INFINITY;
-      int bj = -1;
+      // warp arg-max: largest score, then the smallest expert index among equals
+      const uint32_t key = top.j[0] >= 0 ? ordered_key(top.v[0]) : 0u;
+      const uint32_t mkey = __reduce_max_sync(0xffffffffu, key);
+      const uint32_t cand =
+          (key == mkey && top.j[0] >= 0) ? (uint32_t)(lane + 32 * top.j[0]) : 0xffffffffu;
+      const int be = (int)__reduce_min_sync(0xffffffffu, cand);
+      const int owner = be & 31;
+      const float gate = __shfl_sync(0xffffffffu, top.p[0], owner);
+      if (lane == owner) {
+        taken |= 1u << top.j[0];
+        top.pop();
+        if (top.j[0] < 0) {
+          // this lane's three best are used up: rebuild from what is left
 #pragma unroll
-      for (int j = 0; j < VPL; ++j) {
-        if (!(taken >> j & 1u) && (bj < 0 || s[j] > bs)) { bs = s[j]; bj = j; }
-      }
-      int be = bj >= 0 ? lane + 32 * bj : 0x7fffffff;
-      // warp arg-max on (s desc, e asc)
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        float os = __shfl_xor_sync(0xffffffffu, bs, o);
-        int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (oe != 0x7fffffff && (be == 0x7fffffff || os > bs || (os == bs && oe < be))) {
-          bs = os; be = oe;
+          for (int j = 0; j < VPL; ++j)
+            if (!(taken >> j & 1u) && lane + 32 * j < E) top.insert(s[j], p[j], j);
         }
       }
-      const int owner = be & 31, oj = be >> 5;
-      float gate = 0.f;
-#pragma unroll
-      for (int j = 0; j < VPL; ++j)
-        if (j == oj) gate = p[j];
-      gate = __shfl_sync(0xffffffffu, gate, owner);
-      if (lane == owner) taken |= 1u << oj;
       if (lane == 0) {
         topk_idx[(size_t)t * K + k] = be;
         topk_gate[(size_t)t * K + k] = gate;
