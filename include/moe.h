@@ -177,9 +177,9 @@ moe_status moe_expert_gate_up(const moe_shape* shape, const void* x_perm, const 
  *   h[r, :] = SiLU(x[row_token[r], :] W1_e^T) * (x[row_token[r], :] W3_e^T).
  * x [T, d], row_token [T*K] int32; the other arguments as moe_expert_gate_up.
  * A row_token entry outside [0, T) sets MOE_DEV_BAD_OFFSETS and reads row 0.
- * It saves the x_perm buffer (T*K*d elements) at the price of one 4-row
- * gather per 4 token rows per 64-wide K step; on the LongCat prefill shape the
- * copy plus moe_expert_gate_up is the faster pair. */
+ * The token rows are copied into shared memory by the GEMM's producer
+ * (16-byte asynchronous copies), so the x_perm buffer (T*K*d elements) and
+ * its write and read are not needed. */
 moe_status moe_expert_gate_up_gather(const moe_shape* shape, const void* x,
                                      const int32_t* row_token, const void* w1, const void* w3,
                                      const int32_t* offsets, void* h, void* ws, size_t ws_bytes,

@@ -109,9 +109,6 @@ MOE_DEV void bulk_load_hint(uint32_t dst, const void* src, uint32_t bytes, uint3
 MOE_DEV void cp_async_4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
-MOE_DEV void cp_async_arrive_noinc(uint32_t bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
 
 // --- the kernel --------------------------------------------------------------
 template <bool kGatedOut>

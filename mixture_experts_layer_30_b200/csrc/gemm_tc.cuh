@@ -73,7 +73,9 @@ struct TileCfg {
 using CfgWide = TileCfg<256, 3>;    // segments up to 256 rows in one tile, 3 stages
 using CfgN160 = TileCfg<160, 4>;    // segments up to 160 rows, 4 stages (more bytes in flight)
 using CfgDouble = TileCfg<128, 4>;  // <= 128 rows, double-buffered accumulators
+using CfgR192 = TileCfg<192, 3>;    // router: 192 token rows, one wave at T = 8192, E = 768
 static_assert(CfgWide::smem_bytes(kStagingBytesF32) <= 232448, "router tile");
+static_assert(CfgR192::smem_bytes(kStagingBytesF32) <= 232448, "router tile");
 
 template <int kMode> __host__ __device__ constexpr int staging_bytes() {
   return kMode == 2 ? kStagingBytesF32 : kStagingBytesBf16;
@@ -94,10 +96,11 @@ struct Args {
   void* out;
   const float* add;            // fp32 addend [rows, n_out] (router logit offset) or NULL
   uint32_t* status;
-  const int32_t* gather_rows;  // token of each routed row: B rows are read from x through
-                               // this map with 4-row TMA gathers (tmB is x, box 64 x 1);
-                               // NULL: B rows are rows of tmB itself (tiled boxes)
+  const int32_t* gather_rows;  // token of each routed row: B rows are copied from x through
+                               // this map by the producer lanes (cp.async, 16 bytes each);
+                               // NULL: B rows are rows of tmB itself (TMA boxes)
   int gather_src_rows;         // rows of x (bound for the gathered tokens)
+  const void* gather_src;      // x [gather_src_rows, k_dim] bf16 when gathering
   int a_tiled;                 // weights in MOE_WEIGHTS_TILED order: the A tile of weight rows
                                // r..r+127 (r % 128 == 0), columns kb*64.. is row (r/128*nk+kb)*128
                                // of a [tiles*128, 64] view
@@ -191,16 +194,15 @@ MOE_DEV uint64_t l2_policy_evict_last() {
 // SiLU for the bf16 epilogue: a / (1 + e^-a) with the fast exponential and
 // division intrinsics (relative error ~1e-6, far below the bf16 rounding of h).
 MOE_DEV float silu_fast(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
-// Four rows (row0..row3) x 64 columns of a 2-D map whose box is 64 x 1,
-// placed as four consecutive 128-byte rows at dst (128-byte swizzle applied).
-MOE_DEV void tma_gather4_hint(uint32_t dst, const CUtensorMap* map, int c0, int r0, int r1,
-                              int r2, int r3, uint32_t bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3, %4, %5, %6}], [%7], %8;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-      "r"(bar), "l"(policy)
-      : "memory");
+// 16-byte asynchronous copy global -> shared through L2 with an eviction hint,
+// and the arrival on an mbarrier once all of this thread's copies have landed.
+MOE_DEV void cp_async_16_hint(uint32_t dst, const void* src, uint64_t policy) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst),
+               "l"(src), "l"(policy)
+               : "memory");
+}
+MOE_DEV void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 MOE_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -317,7 +319,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
+      // gathered B rows: the producer's expect_tx plus one cp.async arrival per lane
+      mbar_init(full0 + 8 * s, args.gather_rows ? 1 + 32 : 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int b = 0; b < kAccBufs; ++b) {
@@ -359,35 +362,35 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   int issued = 0;  // producer: stages issued
 
   if (warp == 0 && args.gather_rows) {
-    // ---------------- TMA producer, B rows gathered from x ----------------
-    // Lane 0 waits and posts the expected bytes; every lane then issues the
-    // 4-row gathers of its row groups (g = lane, lane + 32, ...).
+    // ---------------- producer, B rows gathered from x with cp.async ----------------
+    // Lane 0 waits for the stage and loads the two weight tiles by TMA; every
+    // lane then copies the K slice of its token rows (rows lane, lane + 32, ...)
+    // into the 128-byte-swizzled B tile, 16 bytes per copy, and arrives on the
+    // stage barrier once its copies have landed.
     uint32_t stage = 0, phase = 0;
     bool ok = true;
     const uint64_t pol_w = l2_policy_evict_first();
     const uint64_t pol_x = l2_policy_evict_last();
-    constexpr int kGroups = kNMax / 4;
-    constexpr int kPerLane = (kGroups + 31) / 32;
+    constexpr int kRowsPerLane = kNMax / 32;
+    const __nv_bfloat16* xsrc = static_cast<const __nv_bfloat16*>(args.gather_src);
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       const Tile t = decode_tile<kNMax>(tile, n_fblk, args, prefix);
-      const int ngroups = (t.n + 3) / 4;
-      const uint32_t tx = 2 * kABytes + ngroups * 4 * kBK * 2;
       const int a_row0 = t.seg * args.a_seg_rows + t.f0;
       const int a_row1 = a_row0 + args.a1_row_off;
-      int tok[kPerLane][4];
+      const __nv_bfloat16* src[kRowsPerLane];
 #pragma unroll
-      for (int i = 0; i < kPerLane; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          // rows past the segment repeat its last row (their columns are never stored)
-          const int row = min(4 * (lane + 32 * i) + j, t.n - 1);
-          int v = args.gather_rows[t.r0 + row];
+      for (int i = 0; i < kRowsPerLane; ++i) {
+        const int row = lane + 32 * i;
+        int v = 0;
+        if (row < t.n) {
+          v = args.gather_rows[t.r0 + row];
           if (v < 0 || v >= args.gather_src_rows) {
             set_status(args.status, MOE_DEV_BAD_OFFSETS);
             v = 0;
           }
-          tok[i][j] = v;
         }
+        src[i] = xsrc + (size_t)v * args.k_dim;
+      }
       for (int kb = 0; kb < nk; ++kb) {
         int go = 1;
         if (lane == 0) go = mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status);
@@ -399,20 +402,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
         const uint32_t fb = full0 + 8 * stage;
         const uint32_t sa0 = smem_u32(stages + stage * kStageBytes);
         if (lane == 0) {
-          mbar_arrive_expect_tx(fb, tx);
+          mbar_arrive_expect_tx(fb, 2 * kABytes);
           const int2 c0 = a_coord(args, a_row0, kb, nk), c1 = a_coord(args, a_row1, kb, nk);
           tma_load_2d_hint(sa0, &tmA0, c0.x, c0.y, fb, pol_w);
           tma_load_2d_hint(sa0 + kABytes, &tmA1, c1.x, c1.y, fb, pol_w);
           ++issued;
         }
-        __syncwarp();
+        const uint32_t sb = sa0 + 2 * kABytes;
 #pragma unroll
-        for (int i = 0; i < kPerLane; ++i) {
-          const int g = lane + 32 * i;
-          if (g < ngroups)
-            tma_gather4_hint(sa0 + 2 * kABytes + g * 4 * kBK * 2, &tmB, kb * kBK, tok[i][0],
-                             tok[i][1], tok[i][2], tok[i][3], fb, pol_x);
+        for (int i = 0; i < kRowsPerLane; ++i) {
+          const int row = lane + 32 * i;
+          if (row < t.n) {
+            const __nv_bfloat16* g = src[i] + kb * kBK;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)  // 16-byte chunk c of the row, swizzled position
+              cp_async_16_hint(sb + row * 128 + ((c ^ (row & 7)) << 4), g + c * 8, pol_x);
+          }
         }
+        cp_async_arrive_noinc(fb);
         if (++stage == kStages) { stage = 0; phase ^= 1; }
       }
     }
@@ -472,6 +479,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
             break;
           }
           tc_fence_after();
+          // gathered B rows arrive through the generic proxy (cp.async)
+          if (args.gather_rows) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           const uint32_t sa0 = smem_u32(stages + stage * kStageBytes);
           const uint64_t da0 = smem_desc_sw128(sa0);
           const uint64_t da1 = smem_desc_sw128(sa0 + kABytes);
@@ -736,7 +745,8 @@ inline moe_status launch_gate_up(const moe_shape& s, const void* x_perm, const v
 }
 
 // Gate/up GEMM reading its token rows straight from x through row_token
-// (4-row TMA gathers), so the dispatch needs no x_perm copy.
+// (cp.async row copies by the producer lanes), so the dispatch needs no
+// x_perm copy.
 inline moe_status launch_gate_up_gather(const moe_shape& s, const void* x,
                                         const int32_t* row_token, const void* w1,
                                         const void* w3, const int32_t* offsets, void* h,
@@ -747,7 +757,7 @@ inline moe_status launch_gate_up_gather(const moe_shape& s, const void* x,
   const bool tiled = s.weight_layout == MOE_WEIGHTS_TILED;
   if (!make_weight_map(&a0, w1, s.N, s.I, s.d, tiled)) return map_error(err, errn, "w1");
   if (!make_weight_map(&a1, w3, s.N, s.I, s.d, tiled)) return map_error(err, errn, "w3");
-  if (!make_map(&b, x, (uint64_t)s.T, s.d, 1)) return map_error(err, errn, "x");
+  if (!make_map(&b, x, (uint64_t)s.T, s.d, kBoxRows)) return map_error(err, errn, "x");
   Args a{};
   a.seg_offsets = offsets;
   a.nseg = s.N;
@@ -761,6 +771,7 @@ inline moe_status launch_gate_up_gather(const moe_shape& s, const void* x,
   a.status = status;
   a.gather_rows = row_token;
   a.gather_src_rows = s.T;
+  a.gather_src = x;
   a.a_tiled = tiled;
   if (use_double(s))
     return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
@@ -824,9 +835,14 @@ inline moe_status launch_router_gemm(const moe_shape& s, const void* x, const vo
   g.out = logits;
   g.add = offset;
   g.status = nullptr;
-  const long long tiles =
-      (long long)((s.T + CfgWide::kNMax - 1) / CfgWide::kNMax) * ((E + 2 * kFeat - 1) / (2 * kFeat));
-  return launch<kPlainF32, CfgWide>(a, a, b, g, tiles, sms, st, err, errn);
+  // The router is one dense GEMM: pick the token tile so that all tiles run
+  // in one wave when 256-row tiles would leave SMs idle.
+  const long long fblk = (E + 2 * kFeat - 1) / (2 * kFeat);
+  const long long tiles256 = (long long)((s.T + 255) / 256) * fblk;
+  const long long tiles192 = (long long)((s.T + 191) / 192) * fblk;
+  if (tiles256 < sms && tiles192 <= sms)
+    return launch<kPlainF32, CfgR192>(a, a, b, g, tiles192, sms, st, err, errn);
+  return launch<kPlainF32, CfgWide>(a, a, b, g, tiles256, sms, st, err, errn);
 }
 
 }  // namespace tc
