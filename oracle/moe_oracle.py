@@ -17,6 +17,9 @@ It follows "LongCat-Flash Technical Report" (Chinese translation):
   * §2.3.2 Eq. (8): the optional output scale gamma on the whole sum.
   * §2.1.2, Eq. (3)-(5): the device-level load-balance statistics f_j, P_j
     with all zero-computation experts as one extra group.
+  * The backward pass of Eq. (1) (the training half of the same layer): the
+    chain rule through the gates, the SwiGLU experts, the identity experts
+    and the softmax router, with the selection held fixed.
 
 Readings taken where the pages are silent (each is also listed in the design
 notes): the router has no bias term and no temperature, and its softmax covers
@@ -32,7 +35,9 @@ matmul, exp, sort and bincount are the only library steps.
 Parity status: every function here is pinned by the CPU tests
 (brute-force top-K, the Z=0 dense top-K MoE reduction, the all-zero-expert
 and K=E fixed points, closed forms of softmax, SwiGLU and Eq. (2), and the
-hand-derived worked examples under tests/golden/).
+hand-derived worked examples under tests/golden/); the backward pass by
+central finite differences of the forward and by torch autograd through an
+independently written dense top-K layer.
 """
 import numpy as np
 
@@ -257,6 +262,95 @@ def lb_statistics(probs, idx, N, D, K, K_e):
 def lb_loss(f, P, alpha):
     """Eq. (3): L_LB = alpha * sum_{j=1}^{D+1} f_j P_j."""
     return float(alpha) * float((f * P).sum())
+
+
+# ---------------------------------------------------------------------------
+# Backward pass of the layer (the training half of the same path)
+# ---------------------------------------------------------------------------
+# The selection is piecewise constant in the inputs, so gradients flow
+# through the gates g = R_i of the selected experts, the FFN experts, the
+# identity experts and the router softmax; the bias b (selection only) has
+# no gradient.  For a loss L with dL/dout = dout:
+#   dy_k = gamma g_k dout_t,   dg_k = gamma <dout_t, E_k(x_t)>
+#   dx_t = gamma (sum of zero-expert gates) dout_t + sum_k dFFN_k + router term
+#   SwiGLU: a = W1 x, u = W3 x, h = SiLU(a) u, y = W2 h
+#     dh = W2^T dy, da = dh u SiLU'(a), du = dh SiLU(a),
+#     dW2 = dy h^T, dW1 = da x^T, dW3 = du x^T, dx = W1^T da + W3^T du
+#     SiLU'(a) = sigma(a) (1 + a (1 - sigma(a)))
+#   softmax: dlogits = R (dR - <R, dR>),  dWr = dlogits^T x,  dx += dlogits Wr
+
+def sigmoid(a):
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-a))
+
+
+def softmax_backward(probs, dR):
+    """Vector-Jacobian product of the row softmax: R (dR - <R, dR>)."""
+    return probs * (dR - (probs * dR).sum(axis=1, keepdims=True))
+
+
+def expert_backward(x_rows, w1, w3, w2, dy):
+    """Gradients of FFN_e on rows x_rows for upstream dy: (dx, dW1, dW3, dW2)."""
+    w1, w3, w2 = as_f64(w1), as_f64(w3), as_f64(w2)
+    a = x_rows @ w1.T
+    u = x_rows @ w3.T
+    sg = sigmoid(a)
+    h = a * sg * u
+    dh = dy @ w2
+    da = dh * u * sg * (1.0 + a * (1.0 - sg))
+    du = dh * a * sg
+    return da @ w1 + du @ w3, da.T @ x_rows, du.T @ x_rows, dy.T @ h
+
+
+def moe_layer_backward(x, w_router, w1, w3, w2, bias, N, K, dout, gamma=1.0,
+                       logit_offset=None, decode=as_f64):
+    """Forward intermediates plus dx, dw_router, dw1, dw3, dw2 (all float64)
+    and the per-slot dgate [T, K] and dy_perm [R, d]."""
+    f = moe_layer(x, w_router, w1, w3, w2, bias, N, K, gamma, logit_offset, decode)
+    x = as_f64(x)
+    dout = as_f64(dout)
+    T, d = x.shape
+    idx, g, probs = f["idx"], f["gate"], f["probs"]
+    off, slot_pos, x_perm, y_perm = f["offsets"], f["slot_pos"], f["x_perm"], f["y_perm"]
+    E = probs.shape[1]
+    # combine
+    R = int(off[-1])
+    dy_perm = np.zeros((R, d))
+    dgate = np.zeros((T, K))
+    dx = np.zeros_like(x)
+    for k in range(K):
+        for t in range(T):
+            e, r = int(idx[t, k]), int(slot_pos[t, k])
+            if e < N:
+                dy_perm[r] = gamma * g[t, k] * dout[t]
+                dgate[t, k] = gamma * float(dout[t] @ y_perm[r])
+            else:
+                dgate[t, k] = gamma * float(dout[t] @ x[t])
+                dx[t] += gamma * g[t, k] * dout[t]
+    # experts
+    dw1 = np.zeros((N,) + np.shape(w1[0])) if N else None
+    dw3 = np.zeros_like(dw1)
+    dw2 = np.zeros((N,) + np.shape(w2[0]))
+    dx_perm = np.zeros((R, d))
+    for e in range(N):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi > lo:
+            dxe, dw1[e], dw3[e], dw2[e] = expert_backward(x_perm[lo:hi], decode(w1[e]),
+                                                          decode(w3[e]), decode(w2[e]),
+                                                          dy_perm[lo:hi])
+            dx_perm[lo:hi] = dxe
+    for k in range(K):
+        ffn = idx[:, k] < N
+        dx[ffn] += dx_perm[slot_pos[ffn, k]]
+    # router
+    dR = np.zeros((T, E))
+    np.put_along_axis(dR, idx.astype(np.int64), dgate, axis=1)
+    dlogits = softmax_backward(probs, dR)
+    wr = as_f64(w_router)
+    dx += dlogits @ wr
+    f.update(dx=dx, dw_router=dlogits.T @ x, dw1=dw1, dw3=dw3, dw2=dw2, dgate=dgate,
+             dy_perm=dy_perm, dx_perm=dx_perm, dlogits=dlogits)
+    return f
 
 
 # ---------------------------------------------------------------------------

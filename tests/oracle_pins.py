@@ -415,7 +415,74 @@ def check_mxfp8_block_quantization(orc, seed=9):
     assert np.array_equal(deq2, deq)
 
 
-ALL_CHECKS = [check_e4m3_table, check_e4m3_rounding_brute_force,
+def _loss_and_grads(orc, L, N, K, gamma, dout):
+    r = orc.moe_layer_backward(L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"],
+                               N=N, K=K, dout=dout, gamma=gamma)
+    return r
+
+
+def check_backward_finite_differences(orc, seed=10):
+    """Central differences of L = <dout, out> in float64 against every gradient
+    (inputs drawn so that no small step changes the top-K selection)."""
+    rng = np.random.default_rng(seed)
+    T, d, N, Z, K, I, gamma = 5, 4, 3, 2, 3, 3, 1.5
+    L = _rand_layer(rng, T, d, N, Z, I, 0.2)
+    dout = rng.normal(size=(T, d))
+    r = _loss_and_grads(orc, L, N, K, gamma, dout)
+    assert r["margin"].min() > 1e-4
+
+    def loss(LL):
+        o = orc.moe_layer(LL["x"], LL["w_router"], LL["w1"], LL["w3"], LL["w2"], LL["bias"],
+                          N=N, K=K, gamma=gamma)["out"]
+        return float((o * dout).sum())
+    eps = 1e-6
+    for name, grad in (("x", "dx"), ("w_router", "dw_router"), ("w1", "dw1"), ("w3", "dw3"),
+                       ("w2", "dw2")):
+        base = L[name]
+        fd = np.zeros_like(base)
+        for ix in np.ndindex(base.shape):
+            Lp = dict(L); Lm = dict(L)
+            Lp[name] = base.copy(); Lp[name][ix] += eps
+            Lm[name] = base.copy(); Lm[name][ix] -= eps
+            fd[ix] = (loss(Lp) - loss(Lm)) / (2 * eps)
+        np.testing.assert_allclose(r[grad], fd, rtol=1e-5, atol=1e-7, err_msg=name)
+
+
+def check_backward_against_autograd(orc, seed=11):
+    """The dense top-K MoE written with torch float64 ops, differentiated by
+    torch autograd, against the oracle's hand-written backward."""
+    rng = np.random.default_rng(seed)
+    T, d, N, Z, K, I, gamma = 9, 6, 5, 3, 4, 7, 0.7
+    L = _rand_layer(rng, T, d, N, Z, I, 0.1)
+    dout = rng.normal(size=(T, d))
+    r = _loss_and_grads(orc, L, N, K, gamma, dout)
+    tens = {k: torch.tensor(L[k], dtype=torch.float64, requires_grad=True)
+            for k in ("x", "w_router", "w1", "w3", "w2")}
+    F = torch.nn.functional
+    p = torch.softmax(F.linear(tens["x"], tens["w_router"]), dim=1)
+    s_ = p.detach() + torch.tensor(L["bias"])[None, :]
+    out = torch.zeros_like(tens["x"])
+    rows = []
+    for t in range(T):
+        chosen = sorted(range(N + Z), key=lambda i: (-float(s_[t, i]), i))[:K]
+        acc = torch.zeros(d, dtype=torch.float64)
+        for i in chosen:
+            if i < N:
+                y = F.linear(F.silu(F.linear(tens["x"][t], tens["w1"][i])) *
+                             F.linear(tens["x"][t], tens["w3"][i]), tens["w2"][i])
+            else:
+                y = tens["x"][t]
+            acc = acc + p[t, i] * y
+        rows.append(gamma * acc)
+    out = torch.stack(rows)
+    (out * torch.tensor(dout)).sum().backward()
+    for name, grad in (("x", "dx"), ("w_router", "dw_router"), ("w1", "dw1"), ("w3", "dw3"),
+                       ("w2", "dw2")):
+        np.testing.assert_allclose(r[grad], tens[name].grad.numpy(), rtol=1e-10, atol=1e-12,
+                                   err_msg=name)
+
+
+ALL_CHECKS = [check_backward_finite_differences, check_backward_against_autograd, check_e4m3_table, check_e4m3_rounding_brute_force,
               check_mxfp8_block_quantization, check_worked_tiny_layer, check_worked_swiglu, check_worked_bias_update,
               check_worked_zero_experts, check_softmax_closed_forms, check_topk_brute_force,
               check_dense_reduction, check_all_zero_experts_fixed_point,

@@ -156,7 +156,25 @@ def _mut_mx_scale_off_by_one(mp):
     mp.setattr(orc, "mx_scale_exponent", lambda amax: real(amax) - 1)
 
 
-MUTATIONS = [_mut_e4m3_ties_away, _mut_mx_scale_off_by_one, _mut_lb_indicator_per_token, _mut_lb_zero_group_normaliser, _mut_gate_renormalised, _mut_combine_drops_zero_term, _mut_bias_sign,
+def _mut_silu_derivative_sigma_only(mp):
+    """SiLU'(a) taken as sigma(a), the derivative of SiLU mistaken for the gate."""
+    def expert_backward(x_rows, w1, w3, w2, dy):
+        w1, w3, w2 = (np.asarray(w, dtype=np.float64) for w in (w1, w3, w2))
+        a, u = x_rows @ w1.T, x_rows @ w3.T
+        sg = orc.sigmoid(a)
+        h = a * sg * u
+        dh = dy @ w2
+        da, du = dh * u * sg, dh * a * sg
+        return da @ w1 + du @ w3, da.T @ x_rows, du.T @ x_rows, dy.T @ h
+    mp.setattr(orc, "expert_backward", expert_backward)
+
+
+def _mut_softmax_backward_no_centering(mp):
+    mp.setattr(orc, "softmax_backward", lambda probs, dR: probs * dR)
+
+
+MUTATIONS = [_mut_silu_derivative_sigma_only, _mut_softmax_backward_no_centering,
+             _mut_e4m3_ties_away, _mut_mx_scale_off_by_one, _mut_lb_indicator_per_token, _mut_lb_zero_group_normaliser, _mut_gate_renormalised, _mut_combine_drops_zero_term, _mut_bias_sign,
              _mut_bias_updates_zero_experts, _mut_tie_to_high_index, _mut_select_by_unbiased,
              _mut_no_silu, _mut_swapped_gate_up, _mut_descending_tokens,
              _mut_softmax_no_max_shift_wrong_axis, _mut_gamma_only_ffn]
