@@ -270,6 +270,95 @@ moe_status moe_lb_stats(int32_t N, int32_t Z, int32_t D, const int32_t* counts,
                         const float* prob_sum, int64_t T, int32_t K, float K_e, float alpha,
                         float* f, float* P, float* loss, void* stream);
 
+/* ---- Backward pass (the training half of the same layer) ---------------
+ * Gradients of Eq. (1) for an upstream gradient dout = dL/d out [T, d].  The
+ * top-K selection is piecewise constant in the inputs, so it is held fixed
+ * and the gradient flows through the gates g = R(x)_i of the selected
+ * experts, the SwiGLU experts, the identity experts and the softmax router;
+ * the expert bias b (used for selection only) receives none.  With
+ * a = x W1^T, u = x W3^T, h = SiLU(a) * u, y = h W2^T per routed row:
+ *   dy       = gamma g dout_t                         (FFN slot of token t)
+ *   dgate    = gamma <dout_t, y>  (FFN slot),  gamma <dout_t, x_t>  (zero slot)
+ *   dh       = dy W2,   da = dh u SiLU'(a),   du = dh SiLU(a)
+ *   SiLU'(a) = sigma(a) (1 + a (1 - sigma(a)))
+ *   dx_row   = da W1 + du W3;  dW1 = da^T x, dW3 = du^T x, dW2 = dy^T h (per expert)
+ *   dlogits  = R (dR - <R, dR>),  dR = dgate scattered to the selected experts
+ *   dW_r     = dlogits^T x;      dx = gamma (sum of zero gates) dout + sum_k dx_row
+ *                                     + dlogits W_r
+ * One backward pass is, on one stream, after moe_expert_gate_up_save was used
+ * for the forward gate/up half:
+ *   moe_combine_backward -> moe_route_backward -> moe_expert_ffn_backward
+ *   -> moe_permute_backward
+ * Every reduction runs in a fixed order, so results are bit-reproducible: the
+ * token gradient is gathered per token (no atomic scatter-add).  Gradients of
+ * bf16 weights are bf16 (rounded once from fp32 sums), row-major in the
+ * linear-layer layout whatever the shape's weight_layout. */
+
+/* Bytes of device workspace the backward calls need for this shape (status
+ * word, router-logit gradient [T, E], SwiGLU gradient [T*K, 2I]).  Clear it
+ * once with moe_workspace_init.  Returns 0 for an invalid shape. */
+size_t moe_backward_workspace_bytes(const moe_shape* shape);
+
+/* moe_expert_gate_up that also keeps what the backward pass needs: besides
+ * h it writes the pre-activations au[r, 0:I] = a = x_perm[r] W1_e^T and
+ * au[r, I:2I] = u = x_perm[r] W3_e^T (dtype, bf16 rounded once from the fp32
+ * accumulators; h is formed from the unrounded a, u as in
+ * moe_expert_gate_up).  au [T*K, 2I]; other arguments as moe_expert_gate_up
+ * (forward workspace). */
+moe_status moe_expert_gate_up_save(const moe_shape* shape, const void* x_perm, const void* w1,
+                                   const void* w3, const int32_t* offsets, void* h, void* au,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of moe_combine (Eq. (1) weighted sum and Eq. (8) gamma):
+ *   dy_perm[slot_pos[t,k], :] = gamma * gate[t,k] * dout[t, :]   (FFN slots)
+ *   dgate[t, k] = gamma * <dout[t], y_perm[slot_pos[t,k]]>       (FFN slots)
+ *               = gamma * <dout[t], x[t]>                        (zero slots)
+ * Dot products are fp32 sums in a fixed order.  x, dout [T, d], y_perm,
+ * dy_perm [T*K, d] (dtype), dgate [T, K] fp32; the routing arrays are those
+ * of the forward pass.  Rows of dy_perm >= offsets[N] are not written. */
+moe_status moe_combine_backward(const moe_shape* shape, const void* x, const void* y_perm,
+                                const int32_t* topk_idx, const float* topk_gate,
+                                const int32_t* slot_pos, const void* dout, float gamma,
+                                void* dy_perm, float* dgate, void* stream);
+
+/* Backward of the router (Eq. (1): g_i = R_i with R = softmax of x W_r^T):
+ *   dlogits[t, :] = R[t, :] * (dR[t, :] - <R[t, :], dR[t, :]>), dR[t, idx[t,k]] = dgate[t,k]
+ *   dw_router     = dlogits^T x          [E, d] (dtype)
+ *   dx_router     = dlogits w_router     [T, d] fp32
+ * probs [T, E] fp32 are the forward probabilities (moe_route's probs_out).
+ * dlogits is kept in the backward workspace (bf16 for MOE_BF16). */
+moe_status moe_route_backward(const moe_shape* shape, const void* x, const void* w_router,
+                              const float* probs, const int32_t* topk_idx, const float* dgate,
+                              void* dw_router, float* dx_router, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Backward of the SwiGLU experts over the routed rows (per expert segment):
+ *   dh = dy_perm W2_e;  da = dh u SiLU'(a);  du = dh SiLU(a)   (kept in the
+ *                                                backward workspace, dtype)
+ *   dx_perm = da W1_e + du W3_e                 [T*K, d]
+ *   dw1[e] = da^T x_perm,  dw3[e] = du^T x_perm [N, I, d]
+ *   dw2[e] = dy_perm^T h                        [N, d, I]
+ * x_perm, h, au from the forward pass (moe_permute, moe_expert_gate_up_save),
+ * offsets [N+1].  An expert with no rows gets zero weight gradients.  Rows of
+ * dx_perm >= offsets[N] are not written.  For MOE_BF16 the tensor-core path
+ * needs d % 128 == 0 and I % 128 == 0. */
+moe_status moe_expert_ffn_backward(const moe_shape* shape, const void* x_perm, const void* w1,
+                                   const void* w3, const void* w2, const int32_t* offsets,
+                                   const void* h, const void* au, const void* dy_perm,
+                                   void* dx_perm, void* dw1, void* dw3, void* dw2, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* Token gradient, gathered per token in a fixed order (the deterministic
+ * form of the scatter-add back through the dispatch):
+ *   dx[t] = sum_{k: idx < N, in k order} dx_perm[slot_pos[t,k]]
+ *           + gamma * (sum_{k: idx >= N} gate[t,k]) * dout[t]  (+ dx_router[t])
+ * accumulated in fp32 and rounded once.  dout, dx [T, d] (dtype), dx_perm
+ * [T*K, d] (dtype), dx_router [T, d] fp32 or NULL. */
+moe_status moe_permute_backward(const moe_shape* shape, const void* dout,
+                                const int32_t* topk_idx, const float* topk_gate,
+                                const int32_t* slot_pos, const void* dx_perm,
+                                const float* dx_router, float gamma, void* dx, void* stream);
+
 /* Synchronises `stream`, reads the workspace status word into *status_out
  * (may be NULL) and clears it.  Returns MOE_ERR_DEVICE_STATUS when it was
  * non-zero. */

@@ -56,6 +56,14 @@ SIGNATURES = {
     "moe_expert_ffn": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_combine": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp]),
     "moe_bias_update": (ctypes.c_int, [_i32, _i32, _vp, _i64, _i32, _f32, _f32, _vp, _vp]),
+    "moe_backward_workspace_bytes": (_sz, [_SP]),
+    "moe_expert_gate_up_save": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_combine_backward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp,
+                                            _vp]),
+    "moe_route_backward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_expert_ffn_backward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                               _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_permute_backward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp]),
     "moe_get_device_status": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_kernel_launches": (ctypes.c_uint64, []),
@@ -378,3 +386,130 @@ def forward(buf: LayerBuffers, x, w_router, w1, w3, w2, bias, gamma=1.0, logit_o
     combine(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, gamma, buf.out,
             stream=stream)
     return buf.out
+
+
+# ---------------------------------------------------------------------------
+# Backward pass
+# ---------------------------------------------------------------------------
+
+def backward_workspace_bytes(shape: Shape) -> int:
+    n = lib().moe_backward_workspace_bytes(ctypes.byref(shape))
+    if n == 0:
+        raise MoEError(1, "invalid shape")
+    return n
+
+
+def new_backward_workspace(shape: Shape, device="cuda", stream=None) -> torch.Tensor:
+    ws = torch.empty(backward_workspace_bytes(shape), dtype=torch.uint8, device=device)
+    _check(lib().moe_workspace_init(_p(ws), ws.numel(), _stream(stream)))
+    return ws
+
+
+def expert_gate_up_save(shape, x_perm, w1, w3, offsets, h, au, ws, stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_expert_gate_up_save(ctypes.byref(shape), _p(x_perm, dt, "x_perm"),
+                                         _p(w1, dt, "w1"), _p(w3, dt, "w3"),
+                                         _p(offsets, torch.int32, "offsets"), _p(h, dt, "h"),
+                                         _p(au, dt, "au"), _p(ws), ws.numel(), _stream(stream)))
+
+
+def combine_backward(shape, x, y_perm, topk_idx, topk_gate, slot_pos, dout, gamma, dy_perm,
+                     dgate, stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_combine_backward(ctypes.byref(shape), _p(x, dt, "x"),
+                                      _p(y_perm, dt, "y_perm"),
+                                      _p(topk_idx, torch.int32, "topk_idx"),
+                                      _p(topk_gate, torch.float32, "topk_gate"),
+                                      _p(slot_pos, torch.int32, "slot_pos"), _p(dout, dt, "dout"),
+                                      float(gamma), _p(dy_perm, dt, "dy_perm"),
+                                      _p(dgate, torch.float32, "dgate"), _stream(stream)))
+
+
+def route_backward(shape, x, w_router, probs, topk_idx, dgate, dw_router, dx_router, bws,
+                   stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_route_backward(ctypes.byref(shape), _p(x, dt, "x"),
+                                    _p(w_router, dt, "w_router"),
+                                    _p(probs, torch.float32, "probs"),
+                                    _p(topk_idx, torch.int32, "topk_idx"),
+                                    _p(dgate, torch.float32, "dgate"),
+                                    _p(dw_router, dt, "dw_router"),
+                                    _p(dx_router, torch.float32, "dx_router"), _p(bws),
+                                    bws.numel(), _stream(stream)))
+
+
+def expert_ffn_backward(shape, x_perm, w1, w3, w2, offsets, h, au, dy_perm, dx_perm, dw1, dw3,
+                        dw2, bws, stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_expert_ffn_backward(
+        ctypes.byref(shape), _p(x_perm, dt, "x_perm"), _p(w1, dt, "w1"), _p(w3, dt, "w3"),
+        _p(w2, dt, "w2"), _p(offsets, torch.int32, "offsets"), _p(h, dt, "h"), _p(au, dt, "au"),
+        _p(dy_perm, dt, "dy_perm"), _p(dx_perm, dt, "dx_perm"), _p(dw1, dt, "dw1"),
+        _p(dw3, dt, "dw3"), _p(dw2, dt, "dw2"), _p(bws), bws.numel(), _stream(stream)))
+
+
+def permute_backward(shape, dout, topk_idx, topk_gate, slot_pos, dx_perm, dx_router, gamma, dx,
+                     stream=None):
+    dt = torch_dtype(shape)
+    _check(lib().moe_permute_backward(ctypes.byref(shape), _p(dout, dt, "dout"),
+                                      _p(topk_idx, torch.int32, "topk_idx"),
+                                      _p(topk_gate, torch.float32, "topk_gate"),
+                                      _p(slot_pos, torch.int32, "slot_pos"),
+                                      _p(dx_perm, dt, "dx_perm"),
+                                      _p(dx_router, torch.float32, "dx_router"), float(gamma),
+                                      _p(dx, dt, "dx"), _stream(stream)))
+
+
+class BackwardBuffers:
+    """Buffers of one training step (forward intermediates kept for the
+    backward pass, and every gradient) for a shape, allocated once by torch."""
+
+    def __init__(self, shape: Shape, device="cuda"):
+        T, K, d, I, N, E = shape.T, shape.K, shape.d, shape.I, shape.N, shape.N + shape.Z
+        dt = torch_dtype(shape)
+        R = max(T * K, 1)
+        kw = dict(device=device)
+        self.bws = new_backward_workspace(shape, device)
+        self.au = torch.empty((R, 2 * I), dtype=dt, **kw)
+        self.dy_perm = torch.empty((R, d), dtype=dt, **kw)
+        self.dgate = torch.empty((T, K), dtype=torch.float32, **kw)
+        self.dx_router = torch.empty((T, d), dtype=torch.float32, **kw)
+        self.dx_perm = torch.empty((R, d), dtype=dt, **kw)
+        self.dx = torch.empty((T, d), dtype=dt, **kw)
+        self.dw_router = torch.empty((E, d), dtype=dt, **kw)
+        self.dw1 = torch.empty((N, I, d), dtype=dt, **kw)
+        self.dw3 = torch.empty((N, I, d), dtype=dt, **kw)
+        self.dw2 = torch.empty((N, d, I), dtype=dt, **kw)
+
+
+def forward_train(buf: LayerBuffers, bb: BackwardBuffers, x, w_router, w1, w3, w2, bias,
+                  gamma=1.0, logit_offset=None, stream=None):
+    """The forward pass keeping what the backward pass needs (probs, x_perm,
+    h, and the pre-activations a | u in bb.au); returns buf.out."""
+    s = buf.shape
+    if buf.probs is None:
+        raise ValueError("forward_train needs LayerBuffers(with_probs=True)")
+    route(s, x, w_router, bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts, buf.n_ffn,
+          logit_offset=logit_offset, probs_out=buf.probs, stream=stream)
+    permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
+            buf.x_perm, buf.ws, stream=stream)
+    expert_gate_up_save(s, buf.x_perm, w1, w3, buf.offsets, buf.h, bb.au, buf.ws, stream=stream)
+    expert_down(s, buf.h, w2, buf.offsets, buf.y_perm, buf.ws, stream=stream)
+    combine(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, gamma, buf.out,
+            stream=stream)
+    return buf.out
+
+
+def backward(buf: LayerBuffers, bb: BackwardBuffers, x, w_router, w1, w3, w2, dout, gamma=1.0,
+             stream=None):
+    """Gradients of the layer for upstream gradient dout, after forward_train:
+    bb.dx, bb.dw_router, bb.dw1, bb.dw3, bb.dw2 (the selection held fixed)."""
+    s = buf.shape
+    combine_backward(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, dout, gamma,
+                     bb.dy_perm, bb.dgate, stream=stream)
+    route_backward(s, x, w_router, buf.probs, buf.topk_idx, bb.dgate, bb.dw_router,
+                   bb.dx_router, bb.bws, stream=stream)
+    expert_ffn_backward(s, buf.x_perm, w1, w3, w2, buf.offsets, buf.h, bb.au, bb.dy_perm,
+                        bb.dx_perm, bb.dw1, bb.dw3, bb.dw2, bb.bws, stream=stream)
+    permute_backward(s, dout, buf.topk_idx, buf.topk_gate, buf.slot_pos, bb.dx_perm,
+                     bb.dx_router, gamma, bb.dx, stream=stream)

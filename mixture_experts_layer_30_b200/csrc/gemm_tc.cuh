@@ -77,11 +77,18 @@ using CfgR192 = TileCfg<192, 3>;    // router: 192 token rows, one wave at T = 8
 static_assert(CfgWide::smem_bytes(kStagingBytesF32) <= 232448, "router tile");
 static_assert(CfgR192::smem_bytes(kStagingBytesF32) <= 232448, "router tile");
 
-template <int kMode> __host__ __device__ constexpr int staging_bytes() {
-  return kMode == 2 ? kStagingBytesF32 : kStagingBytesBf16;
-}
+// Epilogue modes.
+//   kGated      h = SiLU(D0) * D1 (bf16)                      forward gate/up
+//   kPlainBf16  D0 | D1 as features f0.. / f0+128.. (bf16)    forward down, backward dx
+//   kPlainF32   the same in fp32 (+ optional addend)          router logits, router dx
+//   kSwigluBwd  D = dh; with a, u read from `au`:             backward of SiLU(a) * u
+//               da = dh u s (1 + a (1 - s)), du = dh a s, s = sigmoid(a)
+//   kGatedSave  kGated that also writes a = D0 and u = D1 to `aux_out`
+enum Mode { kGated = 0, kPlainBf16 = 1, kPlainF32 = 2, kSwigluBwd = 3, kGatedSave = 4 };
 
-enum Mode { kGated = 0, kPlainBf16 = 1, kPlainF32 = 2 };
+template <int kMode> __host__ __device__ constexpr int staging_bytes() {
+  return (kMode == kPlainF32 || kMode == kSwigluBwd) ? kStagingBytesF32 : kStagingBytesBf16;
+}
 
 struct Args {
   const int32_t* seg_offsets;  // [nseg+1] routed-row offsets, or NULL for one segment
@@ -104,12 +111,28 @@ struct Args {
   int a_tiled;                 // weights in MOE_WEIGHTS_TILED order: the A tile of weight rows
                                // r..r+127 (r % 128 == 0), columns kb*64.. is row (r/128*nk+kb)*128
                                // of a [tiles*128, 64] view
+  // MN-major A (the kernel's kAMN form: the output features are the weight's
+  // columns, the reduction runs over its rows).  K block kb reads weight rows
+  // seg*a_seg_rows + kb*64 .. +63 of tmA0, or of tmA1 from K block a_k_split on
+  // (rows counted from that block); D0 = columns f0..f0+127, D1 = columns
+  // f0+a1_row_off..+127.  0: no split.
+  int a_k_split;
+  const void* au;              // kSwigluBwd: pre-activations [rows, 2*n_out] (a | u)
+  void* aux_out;               // kGatedSave: a | u output [rows, 2*n_out]
 };
 
 // TMA coordinates (column, row) of the weight tile whose first row is `row`
 // (a multiple of 128 when tiled) for K block kb.
 MOE_DEV int2 a_coord(const Args& a, int row, int kb, int nk) {
   return a.a_tiled ? make_int2(0, ((row >> 7) * nk + kb) << 7) : make_int2(kb * kBK, row);
+}
+// MN-major form: the 64 x 64 box of weight rows krow..krow+63 (krow % 64 == 0)
+// and columns col..col+63.  In the tiled order the box lies inside tile
+// (krow/128, col/64) of a matrix with n_out columns.
+MOE_DEV int2 a_mn_coord(const Args& a, int krow, int col) {
+  return a.a_tiled
+             ? make_int2(0, (((krow >> 7) * (a.n_out >> 6) + (col >> 6)) << 7) + (krow & 127))
+             : make_int2(col, krow);
 }
 
 // --- PTX wrappers --------------------------------------------------------------
@@ -224,12 +247,27 @@ MOE_DEV uint64_t smem_desc_sw128(uint32_t addr) {
   d |= (uint64_t)2 << 61;
   return d;
 }
-// Instruction descriptor of kind::f16: fp32 D, bf16 A and B, both K-major.
+// MN-major operand in the 128-byte swizzle layout, as TMA writes 64 x 64 boxes
+// (64 K rows of 128 bytes = 64 MN elements): 8 K rows form a 1024-byte
+// swizzle atom, consecutive atoms along K are 1024 bytes apart (stride byte
+// offset) and the next 64 MN elements start 8192 bytes further on (leading
+// byte offset, the second box).  One K = 16 step advances 2048 bytes.
+constexpr int kMnBoxBytes = 8192;
+MOE_DEV uint64_t smem_desc_mn_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3fff);
+  d |= (uint64_t)(kMnBoxBytes >> 4) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+// Instruction descriptor of kind::f16: fp32 D, bf16 A and B.
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
-//   15/16 A/B major (0 = K), 17-22 N >> 3, 24-28 M >> 4.
-MOE_DEV uint32_t idesc_bf16(int m, int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
-         ((uint32_t)(m >> 4) << 24);
+//   15/16 A/B major (0 = K, 1 = MN), 17-22 N >> 3, 24-28 M >> 4.
+MOE_DEV uint32_t idesc_bf16(int m, int n, bool a_mn = false, bool b_mn = false) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
+         ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 MOE_DEV void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                        uint32_t accumulate) {
@@ -288,8 +326,37 @@ MOE_DEV Tile decode_tile(int tile, int n_fblk, const Args& a, const int* prefix)
   return t;
 }
 
+// --- epilogue helpers --------------------------------------------------------------
+MOE_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+MOE_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+MOE_DEV float sigmoid_fast(float a) { return __fdividef(1.0f, 1.0f + __expf(-a)); }
+
+// 32 tokens x this warp's 32 features, bf16 pairs packed along tokens
+// (pk[j/2] = tokens j, j+1 of this lane's feature): transposed through the
+// warp's staging rows and stored as 16-byte row pieces of out[row0 + j, fbase..].
+MOE_DEV void stage_store_bf16x32(const uint32_t (&pk)[16], uint16_t* s16, int lane,
+                                 __nv_bfloat16* out, size_t ld, int row0, int nrows, int fbase,
+                                 int fmax) {
+#pragma unroll
+  for (int j = 0; j < 32; j += 2) {
+    s16[j * kStagingPitch16 + lane] = (uint16_t)(pk[j >> 1] & 0xffffu);
+    s16[(j + 1) * kStagingPitch16 + lane] = (uint16_t)(pk[j >> 1] >> 16);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int vec = it * 32 + lane;
+    const int j = vec >> 2, c = vec & 3;
+    const int f = fbase + c * 8;
+    if (j < nrows && f < fmax)
+      *reinterpret_cast<uint4*>(out + (size_t)(row0 + j) * ld + f) =
+          *reinterpret_cast<const uint4*>(&s16[j * kStagingPitch16 + c * 8]);
+  }
+  __syncwarp();
+}
+
 // --- the kernel ------------------------------------------------------------------
-template <int kMode, class Cfg>
+template <int kMode, class Cfg, bool kAMN = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                const __grid_constant__ CUtensorMap tmB, const Args args) {
@@ -445,9 +512,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
           const uint32_t fb = full0 + 8 * stage;
           const uint32_t sa0 = smem_u32(stages + stage * kStageBytes);
           mbar_arrive_expect_tx(fb, tx);
-          const int2 c0 = a_coord(args, a_row0, kb, nk), c1 = a_coord(args, a_row1, kb, nk);
-          tma_load_2d_hint(sa0, &tmA0, c0.x, c0.y, fb, pol_w);
-          tma_load_2d_hint(sa0 + kABytes, &tmA1, c1.x, c1.y, fb, pol_w);
+          if constexpr (kAMN) {
+            // four 64 x 64 boxes: D0 columns f0, f0+64; D1 columns f0+a1_row_off, +64
+            const bool second = args.a_k_split > 0 && kb >= args.a_k_split;
+            const CUtensorMap* am = second ? &tmA1 : &tmA0;
+            const int krow = t.seg * args.a_seg_rows + (second ? kb - args.a_k_split : kb) * kBK;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int2 c0 = a_mn_coord(args, krow, t.f0 + 64 * h);
+              const int2 c1 = a_mn_coord(args, krow, t.f0 + args.a1_row_off + 64 * h);
+              tma_load_2d_hint(sa0 + h * kMnBoxBytes, am, c0.x, c0.y, fb, pol_w);
+              tma_load_2d_hint(sa0 + kABytes + h * kMnBoxBytes, am, c1.x, c1.y, fb, pol_w);
+            }
+          } else {
+            const int2 c0 = a_coord(args, a_row0, kb, nk), c1 = a_coord(args, a_row1, kb, nk);
+            tma_load_2d_hint(sa0, &tmA0, c0.x, c0.y, fb, pol_w);
+            tma_load_2d_hint(sa0 + kABytes, &tmA1, c1.x, c1.y, fb, pol_w);
+          }
           for (int b = 0; b < nbox; ++b)
             tma_load_2d_hint(sa0 + 2 * kABytes + b * kBoxBytes, &tmB, kb * kBK,
                              t.r0 + b * kBoxRows, fb, pol_x);
@@ -467,7 +548,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
         const Tile t = decode_tile<kNMax>(tile, n_fblk, args, prefix);
         int n16 = ((t.n + 15) >> 4) << 4;
         if (n16 < 16) n16 = 16;
-        const uint32_t idesc = idesc_bf16(kFeat, n16);
+        const uint32_t idesc = idesc_bf16(kFeat, n16, kAMN);
         const int buf = local % kAccBufs;
         const uint32_t acc_parity = (uint32_t)((local / kAccBufs) & 1);
         const uint32_t d0 = tmem_base + buf * 2 * kNMax;
@@ -482,15 +563,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
           // gathered B rows arrive through the generic proxy (cp.async)
           if (args.gather_rows) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
           const uint32_t sa0 = smem_u32(stages + stage * kStageBytes);
-          const uint64_t da0 = smem_desc_sw128(sa0);
-          const uint64_t da1 = smem_desc_sw128(sa0 + kABytes);
+          const uint64_t da0 = kAMN ? smem_desc_mn_sw128(sa0) : smem_desc_sw128(sa0);
+          const uint64_t da1 = kAMN ? smem_desc_mn_sw128(sa0 + kABytes) : smem_desc_sw128(sa0 + kABytes);
           const uint64_t db = smem_desc_sw128(sa0 + 2 * kABytes);
+          // K = 16 step: 32 bytes inside the swizzled K-major row (encoded +2), or
+          // 16 K rows = 2048 bytes of the MN-major tile (encoded +128)
+          constexpr uint64_t kAStep = kAMN ? 128 : 2;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
-            // advance 16 bf16 = 32 bytes along K inside the swizzled row
             const uint32_t acc = (kb | k) != 0;
-            umma_bf16(d0, da0 + 2 * k, db + 2 * k, idesc, acc);
-            umma_bf16(d0 + kNMax, da1 + 2 * k, db + 2 * k, idesc, acc);
+            umma_bf16(d0, da0 + kAStep * k, db + 2 * k, idesc, acc);
+            umma_bf16(d0 + kNMax, da1 + kAStep * k, db + 2 * k, idesc, acc);
           }
           umma_commit(empty0 + 8 * stage);
           ++consumed;
@@ -517,6 +600,77 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       const uint32_t dbase = tmem_base + lane_base + buf * 2 * kNMax;
       if (!mbar_wait(tmem_full0 + 8 * buf, acc_parity, abort_flag, args.status)) break;
       tc_fence_after();
+      if constexpr (kMode == kSwigluBwd) {
+        // D0 | D1 = dh of features f0.. / f0+128..; a, u from au; da | du to out
+        const __nv_bfloat16* au = static_cast<const __nv_bfloat16*>(args.au);
+        __nv_bfloat16* dau = static_cast<__nv_bfloat16*>(args.out);
+        const size_t ld = 2 * (size_t)args.n_out;
+        for (int hf = 0; hf < 2; ++hf) {
+          const int fbase = t.f0 + hf * kFeat + 32 * q;
+          for (int j0 = 0; j0 < t.n; j0 += 32) {
+            uint32_t v0[32];
+            tmem_ld_32x32b_x32(dbase + hf * kNMax + j0, v0);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) stg[j * kStagingPitch + lane] = v0[j];
+            __syncwarp();
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int vec = it * 32 + lane;
+              const int j = vec >> 3, c = vec & 7;
+              const int f = fbase + c * 4;
+              if (j0 + j < t.n && f < args.n_out) {
+                const size_t row = (size_t)(t.r0 + j0 + j);
+                const float4 dh = *reinterpret_cast<const float4*>(&stg[j * kStagingPitch + c * 4]);
+                const uint2 ar = *reinterpret_cast<const uint2*>(au + row * ld + f);
+                const uint2 ur = *reinterpret_cast<const uint2*>(au + row * ld + args.n_out + f);
+                const float a[4] = {bf16_lo(ar.x), bf16_hi(ar.x), bf16_lo(ar.y), bf16_hi(ar.y)};
+                const float u[4] = {bf16_lo(ur.x), bf16_hi(ur.x), bf16_lo(ur.y), bf16_hi(ur.y)};
+                const float g[4] = {dh.x, dh.y, dh.z, dh.w};
+                float da[4], du[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const float sg = sigmoid_fast(a[i]);
+                  da[i] = g[i] * u[i] * sg * (1.0f + a[i] * (1.0f - sg));
+                  du[i] = g[i] * a[i] * sg;
+                }
+                *reinterpret_cast<uint2*>(dau + row * ld + f) =
+                    make_uint2(pack_bf16x2(da[0], da[1]), pack_bf16x2(da[2], da[3]));
+                *reinterpret_cast<uint2*>(dau + row * ld + args.n_out + f) =
+                    make_uint2(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]));
+              }
+            }
+            __syncwarp();
+          }
+        }
+      } else if constexpr (kMode == kGatedSave) {
+        // h = SiLU(a) * u as in kGated, plus a and u themselves (bf16)
+        const int fbase = t.f0 + 32 * q;
+        uint16_t* s16 = reinterpret_cast<uint16_t*>(stg);
+        __nv_bfloat16* hout = static_cast<__nv_bfloat16*>(args.out);
+        __nv_bfloat16* aux = static_cast<__nv_bfloat16*>(args.aux_out);
+        const size_t lda = 2 * (size_t)args.n_out;
+        for (int j0 = 0; j0 < t.n; j0 += 32) {
+          uint32_t v0[32], v1[32];
+          tmem_ld_32x32b_x32(dbase + j0, v0);
+          tmem_ld_32x32b_x32(dbase + kNMax + j0, v1);
+          tmem_wait_ld();
+          uint32_t hp[16], ap[16], up[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float a0 = __uint_as_float(v0[j]), a1 = __uint_as_float(v0[j + 1]);
+            const float u0 = __uint_as_float(v1[j]), u1 = __uint_as_float(v1[j + 1]);
+            hp[j >> 1] = pack_bf16x2(silu_fast(a0) * u0, silu_fast(a1) * u1);
+            ap[j >> 1] = pack_bf16x2(a0, a1);
+            up[j >> 1] = pack_bf16x2(u0, u1);
+          }
+          const int row0 = t.r0 + j0, nrows = t.n - j0;
+          stage_store_bf16x32(hp, s16, lane, hout, args.n_out, row0, nrows, fbase, args.n_out);
+          stage_store_bf16x32(ap, s16, lane, aux, lda, row0, nrows, fbase, args.n_out);
+          stage_store_bf16x32(up, s16, lane, aux + args.n_out, lda, row0, nrows, fbase,
+                              args.n_out);
+        }
+      } else {
       const int nhalves = (kMode == kGated) ? 1 : 2;
       for (int hf = 0; hf < nhalves; ++hf) {
         const int fbase = t.f0 + hf * kFeat + 32 * q;   // first feature of this warp
@@ -587,6 +741,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
           __syncwarp();
         }
       }
+      }
       tc_fence_before();
       mbar_arrive(tmem_empty0 + 8 * buf);
     }
@@ -647,7 +802,7 @@ inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
   return r == CUDA_SUCCESS;
 }
 
-template <int kMode, class Cfg>
+template <int kMode, class Cfg, bool kAMN = false>
 inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                          const Args& args, long long max_tiles, int sms, cudaStream_t st,
                          char* err, size_t errn) {
@@ -655,7 +810,7 @@ inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUt
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kMode, Cfg>,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kMode, Cfg, kAMN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Cfg::smem_bytes(staging_bytes<kMode>()));
     if (e != cudaSuccess) {
@@ -666,7 +821,7 @@ inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUt
   }
   long long grid = max_tiles < sms ? max_tiles : sms;
   if (grid < 1) grid = 1;
-  gemm_tc_kernel<kMode, Cfg>
+  gemm_tc_kernel<kMode, Cfg, kAMN>
       <<<(int)grid, kThreads, Cfg::smem_bytes(staging_bytes<kMode>()), st>>>(a0, a1, b, args);
   note_launch();
   cudaError_t e = cudaGetLastError();
@@ -843,6 +998,138 @@ inline moe_status launch_router_gemm(const moe_shape& s, const void* x, const vo
   if (tiles256 < sms && tiles192 <= sms)
     return launch<kPlainF32, CfgR192>(a, a, b, g, tiles192, sms, st, err, errn);
   return launch<kPlainF32, CfgWide>(a, a, b, g, tiles256, sms, st, err, errn);
+}
+
+// Forward gate/up for training: h as launch_gate_up, and a | u to au [rows, 2I].
+inline moe_status launch_gate_up_save(const moe_shape& s, const void* x_perm, const void* w1,
+                                      const void* w3, const int32_t* offsets, void* h, void* au,
+                                      uint32_t* status, int sms, cudaStream_t st, char* err,
+                                      size_t errn) {
+  CUtensorMap a0, a1, b;
+  const uint64_t rows = (uint64_t)s.T * s.K;
+  const bool tiled = s.weight_layout == MOE_WEIGHTS_TILED;
+  if (!make_weight_map(&a0, w1, s.N, s.I, s.d, tiled)) return map_error(err, errn, "w1");
+  if (!make_weight_map(&a1, w3, s.N, s.I, s.d, tiled)) return map_error(err, errn, "w3");
+  if (!make_map(&b, x_perm, rows, s.d, kBoxRows)) return map_error(err, errn, "x_perm");
+  Args a{};
+  a.seg_offsets = offsets;
+  a.nseg = s.N;
+  a.max_rows = (int)rows;
+  a.n_out = s.I;
+  a.k_dim = s.d;
+  a.a_seg_rows = s.I;
+  a.feat_per_tile = kFeat;
+  a.out = h;
+  a.aux_out = au;
+  a.status = status;
+  a.a_tiled = tiled;
+  if (use_n160(s))
+    return launch<kGatedSave, CfgN160>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgN160::kNMax),
+                                       sms, st, err, errn);
+  return launch<kGatedSave, CfgWide>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgWide::kNMax),
+                                     sms, st, err, errn);
+}
+
+// MN-major view of n_mats weight matrices [rows, cols] for 64 x 64 boxes:
+// row-major [n_mats*rows, cols], or the tiled order seen as [n_mats*rows*cols/64, 64].
+inline bool make_weight_map_mn(CUtensorMap* m, const void* base, uint64_t n_mats, uint64_t rows,
+                               uint64_t cols, bool tiled) {
+  if (tiled) return make_map(m, base, n_mats * rows * cols / kBK, kBK, 64);
+  return make_map(m, base, n_mats * rows, cols, 64);
+}
+
+// Backward through the down projection and the SwiGLU:
+//   dh = dy_perm W2_e (reduction over d; W2_e [d, I] read MN-major), then
+//   da = dh u SiLU'(a), du = dh SiLU(a) written to dau [rows, 2I].
+inline moe_status launch_dgrad_h(const moe_shape& s, const void* dy, const void* w2,
+                                 const int32_t* offsets, const void* au, void* dau,
+                                 uint32_t* status, int sms, cudaStream_t st, char* err,
+                                 size_t errn) {
+  CUtensorMap a, b;
+  const uint64_t rows = (uint64_t)s.T * s.K;
+  const bool tiled = s.weight_layout == MOE_WEIGHTS_TILED;
+  if (!make_weight_map_mn(&a, w2, s.N, s.d, s.I, tiled)) return map_error(err, errn, "w2");
+  if (!make_map(&b, dy, rows, s.d, kBoxRows)) return map_error(err, errn, "dy_perm");
+  Args g{};
+  g.seg_offsets = offsets;
+  g.nseg = s.N;
+  g.max_rows = (int)rows;
+  g.n_out = s.I;
+  g.k_dim = s.d;
+  g.a_seg_rows = s.d;
+  g.a1_row_off = kFeat;
+  g.feat_per_tile = 2 * kFeat;
+  g.out = dau;
+  g.au = au;
+  g.status = status;
+  g.a_tiled = tiled;
+  return launch<kSwigluBwd, CfgWide, true>(a, a, b, g,
+                                           routed_tiles(s, s.I, 2 * kFeat, CfgWide::kNMax), sms,
+                                           st, err, errn);
+}
+
+// dx_perm = da W1_e + du W3_e: one reduction over 2I (K blocks of W1, then of
+// W3), W1_e / W3_e [I, d] read MN-major, dau [rows, 2I] the token operand.
+inline moe_status launch_dgrad_x(const moe_shape& s, const void* dau, const void* w1,
+                                 const void* w3, const int32_t* offsets, void* dx_perm,
+                                 uint32_t* status, int sms, cudaStream_t st, char* err,
+                                 size_t errn) {
+  CUtensorMap a0, a1, b;
+  const uint64_t rows = (uint64_t)s.T * s.K;
+  const bool tiled = s.weight_layout == MOE_WEIGHTS_TILED;
+  if (!make_weight_map_mn(&a0, w1, s.N, s.I, s.d, tiled)) return map_error(err, errn, "w1");
+  if (!make_weight_map_mn(&a1, w3, s.N, s.I, s.d, tiled)) return map_error(err, errn, "w3");
+  if (!make_map(&b, dau, rows, 2 * (uint64_t)s.I, kBoxRows)) return map_error(err, errn, "dau");
+  Args g{};
+  g.seg_offsets = offsets;
+  g.nseg = s.N;
+  g.max_rows = (int)rows;
+  g.n_out = s.d;
+  g.k_dim = 2 * s.I;
+  g.a_seg_rows = s.I;
+  g.a_k_split = s.I / kBK;
+  g.a1_row_off = kFeat;
+  g.feat_per_tile = 2 * kFeat;
+  g.out = dx_perm;
+  g.status = status;
+  g.a_tiled = tiled;
+  if (use_n160(s))
+    return launch<kPlainBf16, CfgN160, true>(a0, a1, b, g,
+                                             routed_tiles(s, s.d, 2 * kFeat, CfgN160::kNMax),
+                                             sms, st, err, errn);
+  return launch<kPlainBf16, CfgWide, true>(a0, a1, b, g,
+                                           routed_tiles(s, s.d, 2 * kFeat, CfgWide::kNMax), sms,
+                                           st, err, errn);
+}
+
+// dx_router = dlogits W_r [T, d] fp32: reduction over the E experts (W_r [E, d]
+// read MN-major, the K tail past E zero-filled by TMA).
+inline moe_status launch_router_dx(const moe_shape& s, const void* dlogits, const void* w,
+                                   float* dx_router, uint32_t* status, int sms, cudaStream_t st,
+                                   char* err, size_t errn) {
+  CUtensorMap a, b;
+  const int E = s.N + s.Z;
+  if (!make_map(&a, w, (uint64_t)E, s.d, 64)) return map_error(err, errn, "w_router");
+  if (!make_map(&b, dlogits, (uint64_t)s.T, E, kBoxRows)) return map_error(err, errn, "dlogits");
+  Args g{};
+  g.seg_offsets = nullptr;
+  g.nseg = 1;
+  g.single_rows = s.T;
+  g.max_rows = s.T;
+  g.n_out = s.d;
+  g.k_dim = (E + kBK - 1) / kBK * kBK;
+  g.a_seg_rows = 0;
+  g.a1_row_off = kFeat;
+  g.feat_per_tile = 2 * kFeat;
+  g.out = dx_router;
+  g.status = status;
+  const long long tiles = (long long)((s.T + 255) / 256) * ((s.d + 2 * kFeat - 1) / (2 * kFeat));
+  return launch<kPlainF32, CfgWide, true>(a, a, b, g, tiles, sms, st, err, errn);
+}
+
+// Tensor-core backward needs whole 128-feature tiles on both expert axes.
+inline bool bwd_supported(const moe_shape& s) {
+  return s.dtype == MOE_BF16 && s.d % 128 == 0 && s.I % 128 == 0;
 }
 
 }  // namespace tc

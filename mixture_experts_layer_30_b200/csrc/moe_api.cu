@@ -16,6 +16,9 @@
 #include "gemm_fp8.cuh"
 #include "quant.cuh"
 #include "combine.cuh"
+#include "backward.cuh"
+#include "gemm_simt_bwd.cuh"
+#include "gemm_wgrad.cuh"
 
 namespace {
 
@@ -259,6 +262,69 @@ moe_status gate_up_gather_impl(const moe_shape& s, const void* x, const int32_t*
                                              row_token);
   }
   return grouped_simt<float, true>(s, x, w1, w3, offsets, s.I, s.d, h, status, st, row_token);
+}
+
+// --- backward ---------------------------------------------------------------
+
+struct BwdLayout {
+  size_t status, dlogits, dau, total;
+};
+
+BwdLayout bwd_layout_of(const moe_shape& s) {
+  BwdLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align256(off + bytes);
+    return o;
+  };
+  L.status = take(256);
+  L.dlogits = take((size_t)s.T * (s.N + s.Z) * elem_bytes(s));
+  L.dau = take((size_t)s.T * s.K * 2 * s.I * elem_bytes(s));
+  L.total = off;
+  return L;
+}
+
+moe_status check_bwd_ws(const moe_shape& s, void* ws, size_t ws_bytes, BwdLayout* L) {
+  *L = bwd_layout_of(s);
+  if (!ws) return fail(MOE_ERR_INVALID_ARG, "backward workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % 256)
+    return fail(MOE_ERR_INVALID_ARG, "backward workspace must be 256-byte aligned");
+  if (ws_bytes < L->total)
+    return fail(MOE_ERR_WORKSPACE, "backward workspace has %zu bytes, needs %zu", ws_bytes,
+                L->total);
+  return MOE_OK;
+}
+
+// The backward pass runs on the tensor cores for bf16 (d, I multiples of 128,
+// E multiple of 8) and on CUDA cores for fp32.
+moe_status check_bwd_shape(const moe_shape& s) {
+  if (s.dtype == MOE_BF16 &&
+      !(moe::tc::bwd_supported(s) && moe::tc::router_supported(s)))
+    return fail(MOE_ERR_UNSUPPORTED,
+                "bf16 backward needs d %% 128 == 0, I %% 128 == 0 and (N+Z) %% 8 == 0 "
+                "(d=%d, I=%d, N+Z=%d)",
+                s.d, s.I, s.N + s.Z);
+  return MOE_OK;
+}
+
+template <bool kKSeg, bool kSwiglu>
+moe_status simt_bwd(const moe::SimtBwdArgs& a, long long tiles, cudaStream_t st,
+                    const char* what) {
+  long long grid = tiles;
+  const long long cap = (long long)sm_count() * 8;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  moe::gemm_simt_bwd_kernel<float, kKSeg, kSwiglu><<<(int)grid, 256, 0, st>>>(a);
+  return check_launch(what);
+}
+
+long long simt_row_tiles(const moe_shape& s, int n_out) {
+  const long long rows = (long long)s.T * s.K;
+  return (s.N + (rows + moe::kSbBM - 1) / moe::kSbBM) * ((n_out + moe::kSbBN - 1) / moe::kSbBN);
+}
+long long simt_kseg_tiles(int nseg, int m, int n) {
+  return (long long)nseg * ((m + moe::kSbBM - 1) / moe::kSbBM) * ((n + moe::kSbBN - 1) / moe::kSbBN);
 }
 
 moe_status down_impl(const moe_shape& s, const void* h, const void* w2, const int32_t* offsets,
@@ -683,6 +749,314 @@ moe_status moe_lb_stats(int32_t N, int32_t Z, int32_t D, const int32_t* counts,
   moe::lb_stats_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
       N, Z, D, counts, prob_sum, (long long)T, K, K_e, alpha, f, P, loss);
   return check_launch("load-balance statistics");
+}
+
+// --- backward pass ----------------------------------------------------------
+
+size_t moe_backward_workspace_bytes(const moe_shape* shape) {
+  if (validate_shape(shape) != MOE_OK) return 0;
+  return bwd_layout_of(*shape).total;
+}
+
+moe_status moe_expert_gate_up_save(const moe_shape* shape, const void* x_perm, const void* w1,
+                                   const void* w3, const int32_t* offsets, void* h, void* au,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  WsLayout L;
+  MOE_TRY(check_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(x_perm, "x_perm", 16));
+  MOE_TRY(need(w1, "w1", 16));
+  MOE_TRY(need(w3, "w3", 16));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(h, "h", 16));
+  MOE_TRY(need(au, "au", 16));
+  if (s.T == 0) return MOE_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  if (s.dtype == MOE_BF16 && moe::tc::ffn_supported(s))
+    return moe::tc::launch_gate_up_save(s, x_perm, w1, w3, offsets, h, au, status, sm_count(),
+                                        st, g_err, sizeof(g_err));
+  if (s.dtype == MOE_BF16)
+    return fail(MOE_ERR_UNSUPPORTED, "bf16 moe_expert_gate_up_save needs d, I multiples of 64");
+  // fp32: h by the gated kernel, a and u by two plain products into au
+  MOE_TRY(gate_up_impl(s, x_perm, w1, w3, offsets, h, status, st));
+  moe::SimtBwdArgs a{};
+  a.A = x_perm;
+  a.a_sm = s.d;
+  a.a_sk = 1;
+  a.b_sk = 1;
+  a.b_sn = s.d;
+  a.b_seg = (long long)s.I * s.d;
+  a.c_sm = 2LL * s.I;
+  a.offsets = offsets;
+  a.nseg = s.N;
+  a.max_rows = s.T * s.K;
+  a.N = s.I;
+  a.Kd = s.d;
+  a.status = status;
+  a.B0 = w1;
+  a.C = au;
+  MOE_TRY((simt_bwd<false, false>(a, simt_row_tiles(s, s.I), st, "pre-activation a")));
+  a.B0 = w3;
+  a.C = static_cast<float*>(au) + s.I;
+  return simt_bwd<false, false>(a, simt_row_tiles(s, s.I), st, "pre-activation u");
+}
+
+moe_status moe_combine_backward(const moe_shape* shape, const void* x, const void* y_perm,
+                                const int32_t* topk_idx, const float* topk_gate,
+                                const int32_t* slot_pos, const void* dout, float gamma,
+                                void* dy_perm, float* dgate, void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  if (s.T == 0) return MOE_OK;
+  MOE_TRY(need(x, "x", 16));
+  MOE_TRY(need(y_perm, "y_perm", 16));
+  MOE_TRY(need(topk_idx, "topk_idx", 4));
+  MOE_TRY(need(topk_gate, "topk_gate", 4));
+  MOE_TRY(need(slot_pos, "slot_pos", 4));
+  MOE_TRY(need(dout, "dout", 16));
+  MOE_TRY(need(dy_perm, "dy_perm", 16));
+  MOE_TRY(need(dgate, "dgate", 4));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int E = s.N + s.Z;
+  const int nvec = s.d * elem_bytes(s) / 16;
+  int threads = ((nvec + 31) / 32) * 32;
+  if (threads > 256) threads = 256;
+  const int max_rows = s.T * s.K;
+  if (s.dtype == MOE_BF16)
+    moe::combine_backward_kernel<__nv_bfloat16><<<s.T, threads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y_perm),
+        topk_idx, topk_gate, slot_pos, static_cast<const __nv_bfloat16*>(dout), s.K, s.N, E,
+        s.d, max_rows, gamma, static_cast<__nv_bfloat16*>(dy_perm), dgate, nullptr);
+  else
+    moe::combine_backward_kernel<float><<<s.T, threads, 0, st>>>(
+        static_cast<const float*>(x), static_cast<const float*>(y_perm), topk_idx, topk_gate,
+        slot_pos, static_cast<const float*>(dout), s.K, s.N, E, s.d, max_rows, gamma,
+        static_cast<float*>(dy_perm), dgate, nullptr);
+  return check_launch("combine backward");
+}
+
+moe_status moe_route_backward(const moe_shape* shape, const void* x, const void* w_router,
+                              const float* probs, const int32_t* topk_idx, const float* dgate,
+                              void* dw_router, float* dx_router, void* ws, size_t ws_bytes,
+                              void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  MOE_TRY(check_bwd_shape(s));
+  BwdLayout L;
+  MOE_TRY(check_bwd_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(w_router, "w_router", 16));
+  MOE_TRY(need(dw_router, "dw_router", 16));
+  const int E = s.N + s.Z;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.T == 0) {
+    // no tokens: the router weight gradient is zero
+    cudaError_t e = cudaMemsetAsync(dw_router, 0, (size_t)E * s.d * elem_bytes(s), st);
+    if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+    return MOE_OK;
+  }
+  MOE_TRY(need(x, "x", 16));
+  MOE_TRY(need(probs, "probs", 4));
+  MOE_TRY(need(topk_idx, "topk_idx", 4));
+  MOE_TRY(need(dgate, "dgate", 4));
+  MOE_TRY(need(dx_router, "dx_router", 16));
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  void* dlogits = at<char>(ws, L.dlogits);
+  const int sms = sm_count();
+  if (s.dtype == MOE_BF16) {
+    moe::dlogits_kernel<__nv_bfloat16><<<(s.T + 7) / 8, 256, 0, st>>>(
+        probs, topk_idx, dgate, s.T, E, s.K, static_cast<__nv_bfloat16*>(dlogits), status);
+    MOE_TRY(check_launch("router logit gradient"));
+    MOE_TRY(moe::tc::launch_router_wgrad(s, dlogits, x, dw_router, status, sms, st, g_err,
+                                         sizeof(g_err)));
+    return moe::tc::launch_router_dx(s, dlogits, w_router, dx_router, status, sms, st, g_err,
+                                     sizeof(g_err));
+  }
+  moe::dlogits_kernel<float><<<(s.T + 7) / 8, 256, 0, st>>>(
+      probs, topk_idx, dgate, s.T, E, s.K, static_cast<float*>(dlogits), status);
+  MOE_TRY(check_launch("router logit gradient"));
+  moe::SimtBwdArgs a{};
+  // dW_r[i, j] = sum_t dlogits[t, i] x[t, j]
+  a.A = dlogits;
+  a.a_sm = 1;
+  a.a_sk = E;
+  a.B0 = x;
+  a.b_sk = s.d;
+  a.b_sn = 1;
+  a.C = dw_router;
+  a.c_sm = s.d;
+  a.single_rows = s.T;
+  a.max_rows = s.T;
+  a.M = E;
+  a.N = s.d;
+  a.status = status;
+  MOE_TRY((simt_bwd<true, false>(a, simt_kseg_tiles(1, E, s.d), st, "router weight gradient")));
+  // dx_router[t, j] = sum_i dlogits[t, i] W_r[i, j]
+  moe::SimtBwdArgs b{};
+  b.A = dlogits;
+  b.a_sm = E;
+  b.a_sk = 1;
+  b.B0 = w_router;
+  b.b_sk = s.d;
+  b.b_sn = 1;
+  b.C = dx_router;
+  b.c_sm = s.d;
+  b.single_rows = s.T;
+  b.max_rows = s.T;
+  b.N = s.d;
+  b.Kd = E;
+  b.status = status;
+  const long long tiles = (long long)((s.T + moe::kSbBM - 1) / moe::kSbBM) *
+                          ((s.d + moe::kSbBN - 1) / moe::kSbBN);
+  return simt_bwd<false, false>(b, tiles, st, "router input gradient");
+}
+
+moe_status moe_expert_ffn_backward(const moe_shape* shape, const void* x_perm, const void* w1,
+                                   const void* w3, const void* w2, const int32_t* offsets,
+                                   const void* h, const void* au, const void* dy_perm,
+                                   void* dx_perm, void* dw1, void* dw3, void* dw2, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  MOE_TRY(check_bwd_shape(s));
+  BwdLayout L;
+  MOE_TRY(check_bwd_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(x_perm, "x_perm", 16));
+  MOE_TRY(need(w1, "w1", 16));
+  MOE_TRY(need(w3, "w3", 16));
+  MOE_TRY(need(w2, "w2", 16));
+  MOE_TRY(need(offsets, "offsets", 4));
+  MOE_TRY(need(h, "h", 16));
+  MOE_TRY(need(au, "au", 16));
+  MOE_TRY(need(dy_perm, "dy_perm", 16));
+  MOE_TRY(need(dx_perm, "dx_perm", 16));
+  MOE_TRY(need(dw1, "dw1", 16));
+  MOE_TRY(need(dw3, "dw3", 16));
+  MOE_TRY(need(dw2, "dw2", 16));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* status = at<uint32_t>(ws, L.status);
+  void* dau = at<char>(ws, L.dau);
+  const int sms = sm_count();
+  const int rows = s.T * s.K;
+  if (s.dtype == MOE_BF16) {
+    if (s.T > 0) {
+      MOE_TRY(moe::tc::launch_dgrad_h(s, dy_perm, w2, offsets, au, dau, status, sms, st, g_err,
+                                      sizeof(g_err)));
+      MOE_TRY(moe::tc::launch_dgrad_x(s, dau, w1, w3, offsets, dx_perm, status, sms, st, g_err,
+                                      sizeof(g_err)));
+    }
+    return moe::tc::launch_expert_wgrad(s, x_perm, h, dy_perm, dau, offsets, dw1, dw3, dw2,
+                                        status, sms, st, g_err, sizeof(g_err));
+  }
+  moe::SimtBwdArgs a{};
+  a.offsets = offsets;
+  a.nseg = s.N;
+  a.max_rows = rows;
+  a.status = status;
+  if (s.T > 0) {
+    // dh = dy W2_e, then the SwiGLU backward into dau
+    a.A = dy_perm;
+    a.a_sm = s.d;
+    a.a_sk = 1;
+    a.B0 = w2;
+    a.b_seg = (long long)s.d * s.I;
+    a.b_sk = s.I;
+    a.b_sn = 1;
+    a.C = dau;
+    a.N = s.I;
+    a.Kd = s.d;
+    a.au = au;
+    MOE_TRY((simt_bwd<false, true>(a, simt_row_tiles(s, s.I), st, "expert dh")));
+    // dx_perm = da W1_e + du W3_e (one reduction over 2I)
+    moe::SimtBwdArgs b = a;
+    b.A = dau;
+    b.a_sm = 2LL * s.I;
+    b.a_sk = 1;
+    b.B0 = w1;
+    b.B1 = w3;
+    b.k_split = s.I;
+    b.b_seg = (long long)s.I * s.d;
+    b.b_sk = s.d;
+    b.b_sn = 1;
+    b.C = dx_perm;
+    b.c_sm = s.d;
+    b.N = s.d;
+    b.Kd = 2 * s.I;
+    b.au = nullptr;
+    MOE_TRY((simt_bwd<false, false>(b, simt_row_tiles(s, s.d), st, "expert dx")));
+  }
+  // weight gradients: reductions over each expert's rows
+  moe::SimtBwdArgs w{};
+  w.offsets = offsets;
+  w.nseg = s.N;
+  w.max_rows = rows;
+  w.status = status;
+  w.A = dau;  // dW1[e][i, j] = sum_r da[r, i] x_perm[r, j]
+  w.a_sm = 1;
+  w.a_sk = 2LL * s.I;
+  w.B0 = x_perm;
+  w.b_sk = s.d;
+  w.b_sn = 1;
+  w.C = dw1;
+  w.c_seg = (long long)s.I * s.d;
+  w.c_sm = s.d;
+  w.M = s.I;
+  w.N = s.d;
+  MOE_TRY((simt_bwd<true, false>(w, simt_kseg_tiles(s.N, s.I, s.d), st, "dW1")));
+  w.A = static_cast<const float*>(dau) + s.I;  // du
+  w.C = dw3;
+  MOE_TRY((simt_bwd<true, false>(w, simt_kseg_tiles(s.N, s.I, s.d), st, "dW3")));
+  w.A = dy_perm;  // dW2[e][j, i] = sum_r dy[r, j] h[r, i]
+  w.a_sm = 1;
+  w.a_sk = s.d;
+  w.B0 = h;
+  w.b_sk = s.I;
+  w.b_sn = 1;
+  w.C = dw2;
+  w.c_seg = (long long)s.d * s.I;
+  w.c_sm = s.I;
+  w.M = s.d;
+  w.N = s.I;
+  return simt_bwd<true, false>(w, simt_kseg_tiles(s.N, s.d, s.I), st, "dW2");
+}
+
+moe_status moe_permute_backward(const moe_shape* shape, const void* dout,
+                                const int32_t* topk_idx, const float* topk_gate,
+                                const int32_t* slot_pos, const void* dx_perm,
+                                const float* dx_router, float gamma, void* dx, void* stream) {
+  g_err[0] = 0;
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  if (s.T == 0) return MOE_OK;
+  MOE_TRY(need(dout, "dout", 16));
+  MOE_TRY(need(topk_idx, "topk_idx", 4));
+  MOE_TRY(need(topk_gate, "topk_gate", 4));
+  MOE_TRY(need(slot_pos, "slot_pos", 4));
+  MOE_TRY(need(dx_perm, "dx_perm", 16));
+  MOE_TRY(need(dx, "dx", 16));
+  if (dx_router) MOE_TRY(need(dx_router, "dx_router", 16));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int E = s.N + s.Z;
+  const int nvec = s.d * elem_bytes(s) / 16;
+  int threads = ((nvec + 31) / 32) * 32;
+  if (threads > 256) threads = 256;
+  const int max_rows = s.T * s.K;
+  if (s.dtype == MOE_BF16)
+    moe::permute_backward_kernel<__nv_bfloat16><<<s.T, threads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(dout), topk_idx, topk_gate, slot_pos,
+        static_cast<const __nv_bfloat16*>(dx_perm), dx_router, s.K, s.N, E, s.d, max_rows, gamma,
+        static_cast<__nv_bfloat16*>(dx));
+  else
+    moe::permute_backward_kernel<float><<<s.T, threads, 0, st>>>(
+        static_cast<const float*>(dout), topk_idx, topk_gate, slot_pos,
+        static_cast<const float*>(dx_perm), dx_router, s.K, s.N, E, s.d, max_rows, gamma,
+        static_cast<float*>(dx));
+  return check_launch("permute backward");
 }
 
 moe_status moe_get_device_status(void* ws, void* stream, uint32_t* status_out) {

@@ -303,10 +303,10 @@ def expert_backward(x_rows, w1, w3, w2, dy):
 
 
 def moe_layer_backward(x, w_router, w1, w3, w2, bias, N, K, dout, gamma=1.0,
-                       logit_offset=None, decode=as_f64):
+                       logit_offset=None, decode=as_f64, selection=None):
     """Forward intermediates plus dx, dw_router, dw1, dw3, dw2 (all float64)
     and the per-slot dgate [T, K] and dy_perm [R, d]."""
-    f = moe_layer(x, w_router, w1, w3, w2, bias, N, K, gamma, logit_offset, decode)
+    f = moe_layer(x, w_router, w1, w3, w2, bias, N, K, gamma, logit_offset, decode, selection)
     x = as_f64(x)
     dout = as_f64(dout)
     T, d = x.shape
@@ -446,16 +446,23 @@ def expert_ffn_mxfp8(x_rows, w1, w3, w2):
 # ---------------------------------------------------------------------------
 
 def moe_layer(x, w_router, w1, w3, w2, bias, N, K, gamma=1.0, logit_offset=None,
-              decode=as_f64):
+              decode=as_f64, selection=None):
     """Every intermediate of one forward pass of the layer, in float64.
 
     ``x`` and ``w_router`` are float64-convertible arrays (decode bf16 first);
     ``w1/w3/w2`` are per-expert arrays passed through ``decode``.
+    ``selection`` [T, K], when given, replaces the biased top-K (a comparison
+    whose rows lie inside the tie band takes the other side's valid ordering
+    there and re-derives every later stage from it).
     """
     x = as_f64(x)
     logits = router_logits(x, w_router, logit_offset)
     probs = softmax_rows(logits)
-    idx, margin = biased_topk(probs, bias, K)
+    if selection is None:
+        idx, margin = biased_topk(probs, bias, K)
+    else:
+        idx = np.asarray(selection).astype(np.int32)
+        margin = np.full(idx.shape[0], np.nan)
     g = gates(probs, idx)
     E = probs.shape[1]
     counts = expert_counts(idx, E)

@@ -118,3 +118,35 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(B, "LIB_PATH", "/nonexistent/libmoe_b200.so")
     with pytest.raises(RuntimeError, match="missing"):
         B.lib()
+
+
+def test_backward_validation(lib):
+    fake = ctypes.c_void_p(0x10000)
+    s = B.make_shape(64, 256, 12, 4, 4, 128, "bf16")
+    nb = lib.moe_backward_workspace_bytes(ctypes.byref(s))
+    # status word + dlogits [T, E] + dau [T*K, 2I] (bf16)
+    assert nb >= 256 + 64 * 16 * 2 + 64 * 4 * 2 * 128 * 2
+    # bf16 backward needs d and I multiples of 128 and E multiple of 8
+    for bad in (B.make_shape(64, 192, 12, 4, 4, 128, "bf16"),
+                B.make_shape(64, 256, 12, 4, 4, 64, "bf16"),
+                B.make_shape(64, 256, 12, 2, 4, 128, "bf16")):
+        nbb = lib.moe_backward_workspace_bytes(ctypes.byref(bad))
+        assert lib.moe_expert_ffn_backward(ctypes.byref(bad), fake, fake, fake, fake, fake, fake,
+                                           fake, fake, fake, fake, fake, fake, fake, nbb,
+                                           None) == 2
+        assert lib.moe_route_backward(ctypes.byref(bad), fake, fake, fake, fake, fake, fake,
+                                      fake, fake, nbb, None) == 2
+    # workspace too small, NULL operand
+    assert lib.moe_expert_ffn_backward(ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake,
+                                       fake, fake, fake, fake, fake, fake, nb - 256, None) == 3
+    assert lib.moe_expert_ffn_backward(ctypes.byref(s), fake, fake, fake, fake, fake, fake, None,
+                                       fake, fake, fake, fake, fake, fake, nb, None) == 1
+    assert b"au" in lib.moe_last_error()
+    assert lib.moe_combine_backward(ctypes.byref(s), fake, fake, fake, fake, fake, None, 1.0,
+                                    fake, fake, None) == 1
+    assert b"dout" in lib.moe_last_error()
+    assert lib.moe_permute_backward(ctypes.byref(s), fake, fake, fake, fake, fake,
+                                    ctypes.c_void_p(0x10004), 1.0, fake, None) == 1
+    assert b"dx_router" in lib.moe_last_error()
+    assert lib.moe_expert_gate_up_save(ctypes.byref(s), fake, fake, fake, fake, fake, None,
+                                       fake, B.workspace_bytes(s), None) == 1
