@@ -340,6 +340,8 @@ def run_gpu(args, rank, world, local_rank):
     ffn_ms = float((per[:, 2] + per[:, 3]).mean())
 
     if rank != 0:
+        if args.backward:
+            time_training(args, cfg, shape, L, W, dev, stream, L["bias"].clone())
         return None, L
     tokens_per_s = cfg.T * world / (ms_step * 1e-3)
     line = {
@@ -387,7 +389,106 @@ def run_gpu(args, rank, world, local_rank):
         "expert_format": "mxfp8" if fp8 else cfg.dtype,
         "clocks": clk,
     }
+    if args.backward:
+        line["training"] = time_training(args, cfg, shape, L, W, dev, stream, L["bias"].clone())
     return line, L
+
+
+# ---------------------------------------------------------------------------
+# training step (forward keeping the pre-activations + backward), --backward
+# ---------------------------------------------------------------------------
+
+def time_training(args, cfg, shape, L, W, dev, stream, bias):
+    """Per-step time of forward_train + backward on the same batch, with the
+    per-call split and the roofline of the expert backward call."""
+    buf = B.LayerBuffers(shape, device=dev, with_probs=True)
+    bb = B.BackwardBuffers(shape, device=dev)
+    dout = IN.make_x(cfg, dev, seed=424242)  # synthetic upstream gradient, N(0, 1)
+    x = L["x"]
+    K_e, mu = float(np.float32(cfg.K_e)), float(np.float32(cfg.mu))
+    names = ["route", "permute", "gate_up_save", "down", "combine", "combine_bwd", "route_bwd",
+             "expert_ffn_bwd", "permute_bwd"]
+
+    def tstep(ev=None):
+        s = shape
+        if ev: ev[0].record(stream)
+        B.route(s, x, L["w_router"], bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts,
+                buf.n_ffn, probs_out=buf.probs)
+        if ev: ev[1].record(stream)
+        B.permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
+                  buf.x_perm, buf.ws)
+        if ev: ev[2].record(stream)
+        B.expert_gate_up_save(s, buf.x_perm, W["w1"], W["w3"], buf.offsets, buf.h, bb.au, buf.ws)
+        if ev: ev[3].record(stream)
+        B.expert_down(s, buf.h, W["w2"], buf.offsets, buf.y_perm, buf.ws)
+        if ev: ev[4].record(stream)
+        B.combine(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, cfg.gamma, buf.out)
+        if ev: ev[5].record(stream)
+        B.combine_backward(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, dout,
+                           cfg.gamma, bb.dy_perm, bb.dgate)
+        if ev: ev[6].record(stream)
+        B.route_backward(s, x, L["w_router"], buf.probs, buf.topk_idx, bb.dgate, bb.dw_router,
+                         bb.dx_router, bb.bws)
+        if ev: ev[7].record(stream)
+        B.expert_ffn_backward(s, buf.x_perm, W["w1"], W["w3"], W["w2"], buf.offsets, buf.h,
+                              bb.au, bb.dy_perm, bb.dx_perm, bb.dw1, bb.dw3, bb.dw2, bb.bws)
+        if ev: ev[8].record(stream)
+        B.permute_backward(s, dout, buf.topk_idx, buf.topk_gate, buf.slot_pos, bb.dx_perm,
+                           bb.dx_router, cfg.gamma, bb.dx)
+        if ev: ev[9].record(stream)
+        B.bias_update(cfg.N, cfg.Z, buf.counts, cfg.T, cfg.K, K_e, mu, bias)
+
+    for _ in range(args.warmup):
+        tstep()
+    torch.cuda.synchronize()
+    for ws in (buf.ws, bb.bws):
+        st = B.device_status(ws)
+        if st:
+            raise RuntimeError(f"device status 0x{st:x} in the training step")
+    n = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(10)] for _ in range(n)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(n):
+        tstep()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / n
+    for i in range(n):
+        tstep(evs[i])
+    torch.cuda.synchronize()
+    per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(9)] for i in range(n)])
+    med = np.median(per, axis=0)
+    counts = buf.counts.cpu().numpy().astype(np.int64)
+    R = int(counts[:cfg.N].sum())
+    touched = int((counts[:cfg.N] > 0).sum())
+    esz = 2 if cfg.dtype == "bf16" else 4
+    wbytes = touched * 3 * cfg.I * cfg.d * esz   # W1, W3, W2 of the touched experts
+    gbytes = cfg.N * 3 * cfg.I * cfg.d * esz     # dW1, dW3, dW2 written (every expert)
+    # token-row operands: dy (read twice), a|u, h, x_perm read; da|du written and
+    # read twice; dx_perm written
+    rows = R * esz * (2 * cfg.d + 2 * cfg.I + cfg.I + cfg.d + 3 * 2 * cfg.I + cfg.d)
+    ffn_bwd_bytes = wbytes + gbytes + rows
+    ffn_bwd_flops = 12.0 * cfg.d * cfg.I * R
+    bwd_ms = float(per[:, 7].mean())
+    peaks, peak_kind = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    tfl = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    achieved = ffn_bwd_bytes / (bwd_ms * 1e-3) / 1e9
+    return {
+        "ms_per_step": round(ms, 4),
+        "tokens_per_s": round(cfg.T / (ms * 1e-3), 1),
+        "dout": "synthetic N(0, 1) upstream gradient",
+        "per_call_ms_median": {k: round(float(v), 4) for k, v in zip(names, med)},
+        "expert_ffn_backward": {
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "peak_source": f"{peak_kind} hbm_gbs",
+            "algorithmic_bytes_per_launch": int(ffn_bwd_bytes),
+            "tflops": round(ffn_bwd_flops / (bwd_ms * 1e-3) / 1e12, 2),
+            "tensor_frac_of_sustained": round(ffn_bwd_flops / (bwd_ms * 1e-3) / 1e12 / tfl, 4),
+            "avg_launch_ms": round(bwd_ms, 4)},
+    }
 
 
 # ---------------------------------------------------------------------------
@@ -494,6 +595,9 @@ def main():
                     help="also compute the device-level load-balance statistics each step")
     ap.add_argument("--fp8-experts", action="store_true",
                     help="expert weights and routed activations in MXFP8 (block-scaled E4M3)")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time a training step (forward keeping pre-activations + "
+                         "backward pass) and report it under \"training\"")
     ap.add_argument("--graph", action="store_true",
                     help="replay one captured CUDA graph per step (single GPU)")
     args = ap.parse_args()
@@ -501,6 +605,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.graph and int(os.environ.get("WORLD_SIZE", "1")) > 1:
         ap.error("--graph is single-GPU only")
+    if args.backward and args.fp8_experts:
+        ap.error("--backward runs on bf16 experts")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
