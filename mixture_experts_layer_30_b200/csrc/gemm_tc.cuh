@@ -45,6 +45,7 @@ constexpr int kStagingPitch = 36;                // fp32 staging row: 32 words +
 constexpr int kStagingPitch16 = 40;              // bf16 staging row: 32 halves + pad (80 B)
 constexpr int kStagingBytesF32 = kEpiWarps * 32 * kStagingPitch * 4;
 constexpr int kStagingBytesBf16 = kEpiWarps * 32 * kStagingPitch16 * 2;
+constexpr int kStagingBytesF32Half = kEpiWarps * 16 * kStagingPitch * 4;  // 16 token rows
 constexpr int kCtrlBytes = 256;                  // barriers + tmem slot + abort flag
 constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;  // 4 s
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;  // 0.2 s
@@ -76,6 +77,7 @@ using CfgDouble = TileCfg<128, 4>;  // <= 128 rows, double-buffered accumulators
 using CfgR192 = TileCfg<192, 3>;    // router: 192 token rows, one wave at T = 8192, E = 768
 static_assert(CfgWide::smem_bytes(kStagingBytesF32) <= 232448, "router tile");
 static_assert(CfgR192::smem_bytes(kStagingBytesF32) <= 232448, "router tile");
+static_assert(CfgN160::smem_bytes(kStagingBytesF32Half) <= 232448, "SwiGLU backward tile");
 
 // Epilogue modes.
 //   kGated      h = SiLU(D0) * D1 (bf16)                      forward gate/up
@@ -87,7 +89,8 @@ static_assert(CfgR192::smem_bytes(kStagingBytesF32) <= 232448, "router tile");
 enum Mode { kGated = 0, kPlainBf16 = 1, kPlainF32 = 2, kSwigluBwd = 3, kGatedSave = 4 };
 
 template <int kMode> __host__ __device__ constexpr int staging_bytes() {
-  return (kMode == kPlainF32 || kMode == kSwigluBwd) ? kStagingBytesF32 : kStagingBytesBf16;
+  return kMode == kPlainF32 ? kStagingBytesF32
+                            : kMode == kSwigluBwd ? kStagingBytesF32Half : kStagingBytesBf16;
 }
 
 struct Args {
@@ -226,6 +229,10 @@ MOE_DEV void cp_async_16_hint(uint32_t dst, const void* src, uint64_t policy) {
 }
 MOE_DEV void cp_async_arrive_noinc(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2.
+MOE_DEV void l2_prefetch_bulk(const void* p, int bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 MOE_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -501,6 +508,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const Tile t = decode_tile<kNMax>(tile, n_fblk, args, prefix);
         const int nbox = (t.n + kBoxRows - 1) / kBoxRows;
+        if constexpr (kMode == kSwigluBwd) {
+          // the epilogue of this tile reads a and u of its rows and 256 features:
+          // bring them into L2 while the main loop streams the weights
+          const int nf = min(2 * kFeat, args.n_out - t.f0) * 2;  // bytes per row and half
+          const char* au = static_cast<const char*>(args.au);
+          for (int j = 0; j < t.n; ++j) {
+            const char* row = au + ((size_t)(t.r0 + j) * 2 * args.n_out + t.f0) * 2;
+            l2_prefetch_bulk(row, nf);
+            l2_prefetch_bulk(row + (size_t)args.n_out * 2, nf);
+          }
+        }
         const uint32_t tx = 2 * kABytes + nbox * kBoxBytes;
         const int a_row0 = t.seg * args.a_seg_rows + t.f0;
         const int a_row1 = a_row0 + args.a1_row_off;
@@ -601,46 +619,85 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       if (!mbar_wait(tmem_full0 + 8 * buf, acc_parity, abort_flag, args.status)) break;
       tc_fence_after();
       if constexpr (kMode == kSwigluBwd) {
-        // D0 | D1 = dh of features f0.. / f0+128..; a, u from au; da | du to out
+        // D0 | D1 = dh of features f0.. / f0+128..; a, u from au; da | du to out.
+        // dh is transposed through shared memory in fp32, 16 token rows per
+        // round; the a, u loads of round r+1 are issued before round r is
+        // computed (the producer prefetched the tile's a, u rows into L2).
         const __nv_bfloat16* au = static_cast<const __nv_bfloat16*>(args.au);
         __nv_bfloat16* dau = static_cast<__nv_bfloat16*>(args.out);
         const size_t ld = 2 * (size_t)args.n_out;
-        for (int hf = 0; hf < 2; ++hf) {
-          const int fbase = t.f0 + hf * kFeat + 32 * q;
-          for (int j0 = 0; j0 < t.n; j0 += 32) {
-            uint32_t v0[32];
-            tmem_ld_32x32b_x32(dbase + hf * kNMax + j0, v0);
+        const int nr16 = (t.n + 15) >> 4;  // rounds per accumulator half
+        const int nrounds = 2 * nr16;
+        auto load_round = [&](int r, uint2 (&ar)[4], uint2 (&ur)[4]) {
+          const int hf = r >= nr16 ? 1 : 0;
+          const int jr = (r - hf * nr16) << 4;
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int vec = it * 32 + lane;
+            const int j = vec >> 3, c = vec & 7;
+            const int f = t.f0 + hf * kFeat + 32 * q + c * 4;
+            ar[it] = ur[it] = make_uint2(0, 0);
+            if (jr + j < t.n && f < args.n_out) {
+              const size_t row = (size_t)(t.r0 + jr + j);
+              ar[it] = __ldg(reinterpret_cast<const uint2*>(au + row * ld + f));
+              ur[it] = __ldg(reinterpret_cast<const uint2*>(au + row * ld + args.n_out + f));
+            }
+          }
+        };
+        uint2 ca[4], cu[4], na[4], nu[4];
+        uint32_t v0[32];
+        if (nrounds > 0) load_round(0, ca, cu);
+        for (int r = 0; r < nrounds; ++r) {
+          const int hf = r >= nr16 ? 1 : 0;
+          const int jr = (r - hf * nr16) << 4;
+          if ((jr & 31) == 0) {
+            tmem_ld_32x32b_x32(dbase + hf * kNMax + jr, v0);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) stg[j * kStagingPitch + lane] = v0[j];
-            __syncwarp();
+            for (int j = 0; j < 16; ++j) stg[j * kStagingPitch + lane] = v0[j];
+          } else {
 #pragma unroll
-            for (int it = 0; it < 8; ++it) {
-              const int vec = it * 32 + lane;
-              const int j = vec >> 3, c = vec & 7;
-              const int f = fbase + c * 4;
-              if (j0 + j < t.n && f < args.n_out) {
-                const size_t row = (size_t)(t.r0 + j0 + j);
-                const float4 dh = *reinterpret_cast<const float4*>(&stg[j * kStagingPitch + c * 4]);
-                const uint2 ar = *reinterpret_cast<const uint2*>(au + row * ld + f);
-                const uint2 ur = *reinterpret_cast<const uint2*>(au + row * ld + args.n_out + f);
-                const float a[4] = {bf16_lo(ar.x), bf16_hi(ar.x), bf16_lo(ar.y), bf16_hi(ar.y)};
-                const float u[4] = {bf16_lo(ur.x), bf16_hi(ur.x), bf16_lo(ur.y), bf16_hi(ur.y)};
-                const float g[4] = {dh.x, dh.y, dh.z, dh.w};
-                float da[4], du[4];
+            for (int j = 0; j < 16; ++j) stg[j * kStagingPitch + lane] = v0[16 + j];
+          }
+          __syncwarp();
+          if (r + 1 < nrounds) load_round(r + 1, na, nu);
+          float g[4][4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const float sg = sigmoid_fast(a[i]);
-                  da[i] = g[i] * u[i] * sg * (1.0f + a[i] * (1.0f - sg));
-                  du[i] = g[i] * a[i] * sg;
-                }
-                *reinterpret_cast<uint2*>(dau + row * ld + f) =
-                    make_uint2(pack_bf16x2(da[0], da[1]), pack_bf16x2(da[2], da[3]));
-                *reinterpret_cast<uint2*>(dau + row * ld + args.n_out + f) =
-                    make_uint2(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]));
+          for (int it = 0; it < 4; ++it) {
+            const int vec = it * 32 + lane;
+            const int j = vec >> 3, c = vec & 7;
+            const float4 dh = *reinterpret_cast<const float4*>(&stg[j * kStagingPitch + c * 4]);
+            g[it][0] = dh.x; g[it][1] = dh.y; g[it][2] = dh.z; g[it][3] = dh.w;
+          }
+          __syncwarp();
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int vec = it * 32 + lane;
+            const int j = vec >> 3, c = vec & 7;
+            const int f = t.f0 + hf * kFeat + 32 * q + c * 4;
+            if (jr + j < t.n && f < args.n_out) {
+              const size_t row = (size_t)(t.r0 + jr + j);
+              const float a[4] = {bf16_lo(ca[it].x), bf16_hi(ca[it].x), bf16_lo(ca[it].y),
+                                  bf16_hi(ca[it].y)};
+              const float u[4] = {bf16_lo(cu[it].x), bf16_hi(cu[it].x), bf16_lo(cu[it].y),
+                                  bf16_hi(cu[it].y)};
+              float da[4], du[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float sg = sigmoid_fast(a[i]);
+                da[i] = g[it][i] * u[i] * sg * (1.0f + a[i] * (1.0f - sg));
+                du[i] = g[it][i] * a[i] * sg;
               }
+              *reinterpret_cast<uint2*>(dau + row * ld + f) =
+                  make_uint2(pack_bf16x2(da[0], da[1]), pack_bf16x2(da[2], da[3]));
+              *reinterpret_cast<uint2*>(dau + row * ld + args.n_out + f) =
+                  make_uint2(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]));
             }
-            __syncwarp();
+          }
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            ca[it] = na[it];
+            cu[it] = nu[it];
           }
         }
       } else if constexpr (kMode == kGatedSave) {
@@ -1063,6 +1120,10 @@ inline moe_status launch_dgrad_h(const moe_shape& s, const void* dy, const void*
   g.au = au;
   g.status = status;
   g.a_tiled = tiled;
+  if (use_n160(s))
+    return launch<kSwigluBwd, CfgN160, true>(a, a, b, g,
+                                             routed_tiles(s, s.I, 2 * kFeat, CfgN160::kNMax),
+                                             sms, st, err, errn);
   return launch<kSwigluBwd, CfgWide, true>(a, a, b, g,
                                            routed_tiles(s, s.I, 2 * kFeat, CfgWide::kNMax), sms,
                                            st, err, errn);

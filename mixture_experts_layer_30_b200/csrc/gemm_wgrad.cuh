@@ -13,12 +13,16 @@
 // Two accumulator pairs fill the 512 TMEM columns, so the epilogue of one
 // tile overlaps the MMAs of the next.
 //
-// One persistent CTA per SM, 6 warps:
+// One persistent CTA per SM, 10 warps:
 //   warp 0      TMA producer (one lane): six 64 x 64 boxes per stage (A0, A1, B)
 //   warp 1      MMA warp: zeroes the K rows past the segment end in the last
 //               stage of a segment (generic stores + proxy fence), lane 0 issues
-//   warps 2..5  epilogue: TMEM -> registers -> bf16 -> swizzled staging box ->
-//               TMA store (32 rows x 64 columns per store)
+//   warps 2..9  epilogue, two warps per TMEM lane quarter (warps 2..5: D0,
+//               6..9: D1): all 128 columns of its 32 rows loaded behind one
+//               wait -> bf16 -> swizzled staging box -> TMA store (32 rows x
+//               64 columns per store, two staging boxes per warp)
+// A tile writes 64 KiB of bf16 and performs only 2*R_e*256*128 FLOPs (R_e ~
+// 128 routed rows), so the epilogue's store rate sets the pace.
 // Waits are bounded as in gemm_tc.cuh; on expiry the status word records
 // MOE_DEV_PIPELINE_TIMEOUT and the CTA drains and returns.
 #pragma once
@@ -28,11 +32,13 @@
 namespace moe {
 namespace tc {
 
-constexpr int kWgStages = 4;
+constexpr int kWgStages = 3;
+constexpr int kWgThreads = 320;
+constexpr int kWgEpiWarps = 8;
 constexpr int kWgN = 128;                         // output columns per tile (UMMA N)
 constexpr int kWgStageBytes = 6 * kMnBoxBytes;    // A0, A1, B: two 64 x 64 boxes each
 constexpr int kWgStoreBox = 32 * 128;             // 32 rows x 64 bf16 output columns
-constexpr int kWgStagingBytes = kEpiWarps * 2 * kWgStoreBox;
+constexpr int kWgStagingBytes = kWgEpiWarps * 2 * kWgStoreBox;
 constexpr int kWgNumBars = 2 * kWgStages + 2 * 2 + 1;
 constexpr int kWgSmemBytes = 1024 + kWgStages * kWgStageBytes + kWgStagingBytes + kCtrlBytes;
 static_assert(kWgSmemBytes <= 232448, "wgrad shared memory");
@@ -86,7 +92,7 @@ MOE_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "mem
 MOE_DEV void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kWgThreads, 1)
 gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmO0,
                   const __grid_constant__ CUtensorMap tmO1, const WgArgs args) {
@@ -115,7 +121,7 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tmem_full0 + 8 * b, 1);
-      mbar_init(tmem_empty0 + 8 * b, kEpiWarps * 32);
+      mbar_init(tmem_empty0 + 8 * b, kWgEpiWarps * 32);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -240,10 +246,12 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
-    const int q = warp & 3;  // TMEM lane quarter = output rows 32q..32q+31 of a half
+    // ---------------- epilogue (warps 2..9) ----------------
+    const int q = warp & 3;         // TMEM lane quarter = output rows 32q..32q+31 of a half
+    const int hf = (warp - 2) >> 2; // accumulator D0 or D1
     const uint32_t stg0 = smem_u32(staging + (warp - 2) * 2 * kWgStoreBox);
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const CUtensorMap* om = hf ? &tmO1 : &tmO0;
     int local = 0, nstore = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
       const WgTile t = wg_decode(tile, args, mblk, nblk);
@@ -251,26 +259,27 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       const uint32_t acc_parity = (uint32_t)((local >> 1) & 1);
       if (!mbar_wait(tmem_full0 + 8 * buf, acc_parity, abort_flag, args.status)) break;
       tc_fence_after();
-      const bool empty_seg = t.rows <= 0;
-#pragma unroll 1
-      for (int hf = 0; hf < 2; ++hf) {
-        const int r = (hf ? t.m0 + args.out1_row_off : t.m0) + 32 * q;  // first output row
-        if (r >= args.m_out) continue;
-        const CUtensorMap* om = hf ? &tmO1 : &tmO0;
-#pragma unroll 1
+      const int r = (hf ? t.m0 + args.out1_row_off : t.m0) + 32 * q;  // first output row
+      if (r < args.m_out) {
+        // the warp's 32 rows x 128 columns: four loads, one wait
+        uint32_t v[4][32];
+        if (t.rows > 0) {
+          const uint32_t ta = tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(ta + 32 * c, v[c]);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[c][i] = 0u;
+        }
+        tc_fence_before();
+        mbar_arrive(tmem_empty0 + 8 * buf);  // TMEM is free once the loads landed
+#pragma unroll
         for (int c = 0; c < kWgN / 64; ++c) {
           const int col = t.n0 + 64 * c;
           if (col >= args.n_out) continue;
-          uint32_t va[32], vb[32];
-          if (!empty_seg) {
-            const uint32_t ta = tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN + 64 * c;
-            tmem_ld_32x32b_x32(ta, va);
-            tmem_ld_32x32b_x32(ta + 32, vb);
-            tmem_wait_ld();
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) va[i] = vb[i] = 0u;
-          }
           // this lane's output row: 64 columns -> 32 bf16 pairs -> 8 16-byte pieces,
           // written to the 128-byte-swizzled staging box (piece p at p ^ (row & 7))
           const uint32_t sb = stg0 + (nstore & 1) * kWgStoreBox;
@@ -278,11 +287,11 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           __syncwarp();
 #pragma unroll
           for (int p = 0; p < 8; ++p) {
-            const uint32_t* v = p < 4 ? va + 8 * p : vb + 8 * (p - 4);
-            const uint32_t w0 = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
-            const uint32_t w1 = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
-            const uint32_t w2 = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
-            const uint32_t w3 = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
+            const uint32_t* w = &v[2 * c + (p >> 2)][8 * (p & 3)];
+            const uint32_t w0 = pack_bf16x2(__uint_as_float(w[0]), __uint_as_float(w[1]));
+            const uint32_t w1 = pack_bf16x2(__uint_as_float(w[2]), __uint_as_float(w[3]));
+            const uint32_t w2 = pack_bf16x2(__uint_as_float(w[4]), __uint_as_float(w[5]));
+            const uint32_t w3 = pack_bf16x2(__uint_as_float(w[6]), __uint_as_float(w[7]));
             const uint32_t addr = sb + lane * 128 + ((p ^ (lane & 7)) << 4);
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
                          "r"(w2), "r"(w3)
@@ -296,9 +305,10 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
           }
           ++nstore;
         }
+      } else {
+        tc_fence_before();
+        mbar_arrive(tmem_empty0 + 8 * buf);
       }
-      tc_fence_before();
-      mbar_arrive(tmem_empty0 + 8 * buf);
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
@@ -357,7 +367,7 @@ inline moe_status launch_wgrad(const CUtensorMap& a, const CUtensorMap& b, const
                           ((args.n_out + kWgN - 1) / kWgN);
   long long grid = tiles < sms ? tiles : sms;
   if (grid < 1) grid = 1;
-  gemm_wgrad_kernel<<<(int)grid, kThreads, kWgSmemBytes, st>>>(a, b, o0, o1, args);
+  gemm_wgrad_kernel<<<(int)grid, kWgThreads, kWgSmemBytes, st>>>(a, b, o0, o1, args);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
