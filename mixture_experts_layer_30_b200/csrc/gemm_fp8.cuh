@@ -430,10 +430,10 @@ inline bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_
 }
 
 template <bool kGatedOut>
-inline moe_status launch_f8(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+static inline moe_status launch_f8(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                             const ArgsF8& args, long long max_tiles, int sms, cudaStream_t st,
                             char* err, size_t errn) {
-  static bool attr_set[64] = {};
+  static bool attr_set[64] = {};  // per device; internal linkage (one per loaded library)
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {

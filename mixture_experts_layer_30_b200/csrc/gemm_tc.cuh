@@ -860,10 +860,10 @@ inline bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t c
 }
 
 template <int kMode, class Cfg, bool kAMN = false>
-inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
+static inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& b,
                          const Args& args, long long max_tiles, int sms, cudaStream_t st,
                          char* err, size_t errn) {
-  static bool attr_set[64] = {};
+  static bool attr_set[64] = {};  // per device; internal linkage (one per loaded library)
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {

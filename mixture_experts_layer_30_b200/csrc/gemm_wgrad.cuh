@@ -92,6 +92,79 @@ MOE_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "mem
 MOE_DEV void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// One accumulator half of a finished tile: the warp's 32 output rows x 128
+// columns.  TMEM (address `ta`: lane quarter, buffer and half applied) is read
+// with four loads behind one wait and released on `tmem_empty` before the
+// stores; each 64-column piece goes bf16 -> swizzled staging box -> TMA store.
+// has_data false: the segment had no rows and the gradient is zero.
+MOE_DEV void wg_store_half(const CUtensorMap* om, uint32_t ta, bool has_data, bool row_ok,
+                           int out_row, int n0, int n_out, uint32_t stg0, int lane, int& nstore,
+                           uint32_t tmem_empty) {
+  if (!row_ok) {
+    tc_fence_before();
+    mbar_arrive(tmem_empty);
+    return;
+  }
+  uint32_t v[4][32];
+  if (has_data) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(ta + 32 * c, v[c]);
+    tmem_wait_ld();
+  } else {
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[c][i] = 0u;
+  }
+  tc_fence_before();
+  mbar_arrive(tmem_empty);  // TMEM is free once the loads landed
+#pragma unroll
+  for (int c = 0; c < kWgN / 64; ++c) {
+    const int col = n0 + 64 * c;
+    if (col >= n_out) continue;
+    // this lane's output row: 64 columns -> 32 bf16 pairs -> 8 16-byte pieces,
+    // written to the 128-byte-swizzled staging box (piece p at p ^ (row & 7))
+    const uint32_t sb = stg0 + (nstore & 1) * kWgStoreBox;
+    if (lane == 0) bulk_wait_read1();
+    __syncwarp();
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      const uint32_t* w = &v[2 * c + (p >> 2)][8 * (p & 3)];
+      const uint32_t w0 = pack_bf16x2(__uint_as_float(w[0]), __uint_as_float(w[1]));
+      const uint32_t w1 = pack_bf16x2(__uint_as_float(w[2]), __uint_as_float(w[3]));
+      const uint32_t w2 = pack_bf16x2(__uint_as_float(w[4]), __uint_as_float(w[5]));
+      const uint32_t w3 = pack_bf16x2(__uint_as_float(w[6]), __uint_as_float(w[7]));
+      const uint32_t addr = sb + lane * 128 + ((p ^ (lane & 7)) << 4);
+      asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
+                   "r"(w2), "r"(w3)
+                   : "memory");
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(om, sb, col, out_row);
+      bulk_commit();
+    }
+    ++nstore;
+  }
+}
+
+// Zero K rows nv .. 16*ceil(nv/16)-1 of `nbox` consecutive 64 x 64 boxes at
+// shared address `base` (whole 128-byte rows, so the swizzle does not matter),
+// then make the stores visible to the tensor cores.  The whole warp calls.
+MOE_DEV void wg_zero_tail(uint32_t base, int nbox, int nv, int lane) {
+  const int zrows = ((nv + 15) & ~15) - nv;
+  if (zrows <= 0) return;
+  const int per_box = zrows * 8;  // 16-byte pieces per box
+  for (int i = lane; i < nbox * per_box; i += 32) {
+    const int box = i / per_box, piece = i - box * per_box;
+    const uint32_t addr = base + box * kMnBoxBytes + nv * 128 + piece * 16;
+    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncwarp();
+}
+
 __global__ void __launch_bounds__(kWgThreads, 1)
 gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmO0,
@@ -208,19 +281,7 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const uint32_t sa = smem_u32(stages + stage * kWgStageBytes);
         const int nv = min(kBK, t.rows - kb * kBK);  // live K rows of this block
         const int ksteps = (nv + 15) >> 4;
-        const int zrows = ksteps * 16 - nv;           // rows the last K step reads past the segment
-        if (zrows > 0) {
-          // zero K rows nv .. 16*ksteps-1 of the six boxes (128 bytes each)
-          const int per_box = zrows * 8;              // 16-byte pieces per box
-          for (int i = lane; i < 6 * per_box; i += 32) {
-            const int box = i / per_box, piece = i - box * per_box;
-            const uint32_t addr = sa + box * kMnBoxBytes + nv * 128 + piece * 16;
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u)
-                         : "memory");
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-        }
+        wg_zero_tail(sa, 6, nv, lane);
         if (lane == 0) {
           const uint64_t da0 = smem_desc_mn_sw128(sa);
           const uint64_t da1 = smem_desc_mn_sw128(sa + 2 * kMnBoxBytes);
@@ -260,55 +321,9 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       if (!mbar_wait(tmem_full0 + 8 * buf, acc_parity, abort_flag, args.status)) break;
       tc_fence_after();
       const int r = (hf ? t.m0 + args.out1_row_off : t.m0) + 32 * q;  // first output row
-      if (r < args.m_out) {
-        // the warp's 32 rows x 128 columns: four loads, one wait
-        uint32_t v[4][32];
-        if (t.rows > 0) {
-          const uint32_t ta = tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(ta + 32 * c, v[c]);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[c][i] = 0u;
-        }
-        tc_fence_before();
-        mbar_arrive(tmem_empty0 + 8 * buf);  // TMEM is free once the loads landed
-#pragma unroll
-        for (int c = 0; c < kWgN / 64; ++c) {
-          const int col = t.n0 + 64 * c;
-          if (col >= args.n_out) continue;
-          // this lane's output row: 64 columns -> 32 bf16 pairs -> 8 16-byte pieces,
-          // written to the 128-byte-swizzled staging box (piece p at p ^ (row & 7))
-          const uint32_t sb = stg0 + (nstore & 1) * kWgStoreBox;
-          if (lane == 0) bulk_wait_read1();
-          __syncwarp();
-#pragma unroll
-          for (int p = 0; p < 8; ++p) {
-            const uint32_t* w = &v[2 * c + (p >> 2)][8 * (p & 3)];
-            const uint32_t w0 = pack_bf16x2(__uint_as_float(w[0]), __uint_as_float(w[1]));
-            const uint32_t w1 = pack_bf16x2(__uint_as_float(w[2]), __uint_as_float(w[3]));
-            const uint32_t w2 = pack_bf16x2(__uint_as_float(w[4]), __uint_as_float(w[5]));
-            const uint32_t w3 = pack_bf16x2(__uint_as_float(w[6]), __uint_as_float(w[7]));
-            const uint32_t addr = sb + lane * 128 + ((p ^ (lane & 7)) << 4);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1),
-                         "r"(w2), "r"(w3)
-                         : "memory");
-          }
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(om, sb, col, t.seg * args.m_out + r);
-            bulk_commit();
-          }
-          ++nstore;
-        }
-      } else {
-        tc_fence_before();
-        mbar_arrive(tmem_empty0 + 8 * buf);
-      }
+      wg_store_half(om, tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, t.rows > 0,
+                    r < args.m_out, t.seg * args.m_out + r, t.n0, args.n_out, stg0, lane, nstore,
+                    tmem_empty0 + 8 * buf);
     }
     if (lane == 0) bulk_wait_all();
     __syncwarp();
@@ -319,6 +334,294 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     const int consumed = *consumed_sh;
     for (int i = consumed; i < issued; ++i)
       mbar_wait(full0 + 8 * (i % kWgStages), (uint32_t)((i / kWgStages) & 1), abort_flag,
+                args.status, kDrainTimeoutNs, false);
+  }
+  __syncwarp();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(512)
+                 : "memory");
+  }
+}
+
+// --- expert weight gradients with the A operand resident -------------------------
+// Work unit = (expert e, m-block): the A rows of the segment (da | du, or dy:
+// 256 columns x R_e rows) are loaded once into up to kAsSlots resident blocks
+// and every n-block of the unit streams only its B block (x_perm or h, 128
+// columns x R_e rows), so the token rows cross L2 ~3x less often than with a
+// (A, B) pair per tile.  A unit whose segment is longer than the resident
+// blocks hold streams A with B, block by block, through the same slots.
+constexpr int kAsSlots = 3;                       // resident A blocks: segments up to 192 rows
+constexpr int kAsSlotBytes = 4 * kMnBoxBytes;     // A0 and A1, two 64 x 64 boxes each
+constexpr int kAsBStages = 4;
+constexpr int kAsBBytes = 2 * kMnBoxBytes;        // B: two 64 x 64 boxes
+constexpr int kAsNumBars = 2 * kAsSlots + 2 * kAsBStages + 2 * 2 + 1;
+constexpr int kAsSmemBytes = 1024 + kAsSlots * kAsSlotBytes + kAsBStages * kAsBBytes +
+                             kWgStagingBytes + kCtrlBytes;
+static_assert(kAsSmemBytes <= 232448, "A-stationary wgrad shared memory");
+static_assert(8 * kAsNumBars + 16 <= kCtrlBytes, "A-stationary wgrad control block");
+
+struct AsUnit {
+  int seg, m0, lo, rows, nk;
+  bool stat;
+};
+
+MOE_DEV AsUnit as_decode(int unit, const WgArgs& a, int mblk) {
+  AsUnit u;
+  u.seg = unit / mblk;
+  u.m0 = (unit - u.seg * mblk) * a.m_step;
+  int lo = a.seg_offsets[u.seg], hi = a.seg_offsets[u.seg + 1];
+  if (lo < 0 || hi < lo || hi > a.max_rows) {
+    set_status(a.status, MOE_DEV_BAD_OFFSETS);
+    lo = hi = 0;
+  }
+  u.lo = lo;
+  u.rows = hi - lo;
+  u.nk = (u.rows + kBK - 1) / kBK;
+  u.stat = u.nk <= kAsSlots;
+  return u;
+}
+
+__global__ void __launch_bounds__(kWgThreads, 1)
+gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmO0,
+                     const __grid_constant__ CUtensorMap tmO1, const WgArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* aslots = smem;
+  uint8_t* bstages = aslots + kAsSlots * kAsSlotBytes;
+  uint8_t* staging = bstages + kAsBStages * kAsBBytes;
+  uint8_t* ctrl = staging + kWgStagingBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ctrl);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * kAsNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 8 * kAsNumBars + 4);
+  volatile int* a_seen_sh = reinterpret_cast<volatile int*>(ctrl + 8 * kAsNumBars + 8);
+  volatile int* b_seen_sh = reinterpret_cast<volatile int*>(ctrl + 8 * kAsNumBars + 12);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t a_full0 = smem_u32(&bars[0]);
+  const uint32_t a_empty0 = smem_u32(&bars[kAsSlots]);
+  const uint32_t b_full0 = smem_u32(&bars[2 * kAsSlots]);
+  const uint32_t b_empty0 = smem_u32(&bars[2 * kAsSlots + kAsBStages]);
+  const uint32_t tmem_full0 = smem_u32(&bars[2 * kAsSlots + 2 * kAsBStages]);
+  const uint32_t tmem_empty0 = smem_u32(&bars[2 * kAsSlots + 2 * kAsBStages + 2]);
+  const uint32_t drain_bar = smem_u32(&bars[2 * kAsSlots + 2 * kAsBStages + 4]);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kAsSlots; ++i) {
+      mbar_init(a_full0 + 8 * i, 1);
+      mbar_init(a_empty0 + 8 * i, 1);
+    }
+    for (int i = 0; i < kAsBStages; ++i) {
+      mbar_init(b_full0 + 8 * i, 1);
+      mbar_init(b_empty0 + 8 * i, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tmem_full0 + 8 * b, 1);
+      mbar_init(tmem_empty0 + 8 * b, kWgEpiWarps * 32);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    *a_seen_sh = 0;
+    *b_seen_sh = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmO0);
+    tma_prefetch_desc(&tmO1);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int mblk = (args.m_out + args.m_step - 1) / args.m_step;
+  const int nblk = (args.n_out + kWgN - 1) / kWgN;
+  const int units = args.nseg * mblk;
+  int a_issued = 0, b_issued = 0;  // producer: A and B fills
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      bool ok = true;
+      auto fill_a = [&](const AsUnit& u, int kb) -> bool {
+        const int slot = a_issued % kAsSlots;
+        const uint32_t par = (uint32_t)((a_issued / kAsSlots) & 1);
+        if (!mbar_wait(a_empty0 + 8 * slot, par ^ 1, abort_flag, args.status)) return false;
+        const uint32_t fb = a_full0 + 8 * slot;
+        const uint32_t sa = smem_u32(aslots + slot * kAsSlotBytes);
+        const int row = u.lo + kb * kBK;
+        mbar_arrive_expect_tx(fb, kAsSlotBytes);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          tma_load_2d(sa + h * kMnBoxBytes, &tmA, u.m0 + 64 * h, row, fb);
+          tma_load_2d(sa + 2 * kMnBoxBytes + h * kMnBoxBytes, &tmA,
+                      u.m0 + args.a1_col_off + 64 * h, row, fb);
+        }
+        ++a_issued;
+        return true;
+      };
+      auto fill_b = [&](const AsUnit& u, int nb, int kb) -> bool {
+        const int st = b_issued % kAsBStages;
+        const uint32_t par = (uint32_t)((b_issued / kAsBStages) & 1);
+        if (!mbar_wait(b_empty0 + 8 * st, par ^ 1, abort_flag, args.status)) return false;
+        const uint32_t fb = b_full0 + 8 * st;
+        const uint32_t sb = smem_u32(bstages + st * kAsBBytes);
+        const int row = u.lo + kb * kBK;
+        mbar_arrive_expect_tx(fb, kAsBBytes);
+        tma_load_2d(sb, &tmB, nb * kWgN, row, fb);
+        tma_load_2d(sb + kMnBoxBytes, &tmB, nb * kWgN + 64, row, fb);
+        ++b_issued;
+        return true;
+      };
+      for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
+        const AsUnit u = as_decode(unit, args, mblk);
+        if (u.stat) {
+          for (int kb = 0; kb < u.nk && ok; ++kb) ok = fill_a(u, kb);
+          for (int nb = 0; nb < nblk && ok; ++nb)
+            for (int kb = 0; kb < u.nk && ok; ++kb) ok = fill_b(u, nb, kb);
+        } else {
+          for (int nb = 0; nb < nblk && ok; ++nb)
+            for (int kb = 0; kb < u.nk && ok; ++kb) ok = fill_a(u, kb) && fill_b(u, nb, kb);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA warp ----------------
+    bool ok = true;
+    int a_seen = 0, b_seen = 0, local = 0;
+    const uint32_t idesc = idesc_bf16(kFeat, kWgN, true, true);
+    auto wait_bcast = [&](uint32_t bar, uint32_t par) -> bool {
+      int go = 1;
+      if (lane == 0) go = mbar_wait(bar, par, abort_flag, args.status);
+      return __shfl_sync(0xffffffffu, go, 0) != 0;
+    };
+    for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
+      const AsUnit u = as_decode(unit, args, mblk);
+      const int a0 = a_seen;  // first A fill of this unit
+      if (u.stat) {
+        for (int kb = 0; kb < u.nk && ok; ++kb) {
+          const int i = a0 + kb;
+          ok = wait_bcast(a_full0 + 8 * (i % kAsSlots), (uint32_t)((i / kAsSlots) & 1));
+        }
+        if (!ok) break;
+        a_seen = a0 + u.nk;
+        if (lane == 0) *a_seen_sh = a_seen;
+      }
+      for (int nb = 0; nb < nblk && ok; ++nb, ++local) {
+        const int buf = local & 1;
+        if (!wait_bcast(tmem_empty0 + 8 * buf, (uint32_t)(((local >> 1) & 1) ^ 1))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + buf * 2 * kWgN;
+        for (int kb = 0; kb < u.nk; ++kb) {
+          int ai;
+          if (u.stat) {
+            ai = a0 + kb;
+          } else {
+            ai = a_seen;
+            if (!wait_bcast(a_full0 + 8 * (ai % kAsSlots), (uint32_t)((ai / kAsSlots) & 1))) {
+              ok = false;
+              break;
+            }
+            ++a_seen;
+          }
+          const int bs = b_seen % kAsBStages;
+          if (!wait_bcast(b_full0 + 8 * bs, (uint32_t)((b_seen / kAsBStages) & 1))) {
+            ok = false;
+            break;
+          }
+          ++b_seen;
+          if (lane == 0) {
+            *a_seen_sh = a_seen;
+            *b_seen_sh = b_seen;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(aslots + (ai % kAsSlots) * kAsSlotBytes);
+          const uint32_t sb = smem_u32(bstages + bs * kAsBBytes);
+          const int nv = min(kBK, u.rows - kb * kBK);
+          const int ksteps = (nv + 15) >> 4;
+          if (!u.stat || nb == 0) wg_zero_tail(sa, 4, nv, lane);  // resident A: zeroed once
+          wg_zero_tail(sb, 2, nv, lane);
+          if (lane == 0) {
+            const uint64_t da0 = smem_desc_mn_sw128(sa);
+            const uint64_t da1 = smem_desc_mn_sw128(sa + 2 * kMnBoxBytes);
+            const uint64_t db = smem_desc_mn_sw128(sb);
+            for (int k = 0; k < ksteps; ++k) {
+              const uint32_t acc = (kb | k) != 0;
+              umma_bf16(d0, da0 + 128 * k, db + 128 * k, idesc, acc);
+              umma_bf16(d0 + kWgN, da1 + 128 * k, db + 128 * k, idesc, acc);
+            }
+            umma_commit(b_empty0 + 8 * bs);
+            if (!u.stat) umma_commit(a_empty0 + 8 * (ai % kAsSlots));
+          }
+          __syncwarp();
+        }
+        if (ok && lane == 0) umma_commit(tmem_full0 + 8 * buf);
+        __syncwarp();
+      }
+      // resident A blocks are released once the unit's last MMAs complete
+      if (ok && u.stat && lane == 0)
+        for (int kb = 0; kb < u.nk; ++kb) umma_commit(a_empty0 + 8 * ((a0 + kb) % kAsSlots));
+      __syncwarp();
+    }
+    if (lane == 0) {
+      umma_commit(drain_bar);
+      mbar_wait(drain_bar, 0, abort_flag, args.status, kDrainTimeoutNs, false);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..9) ----------------
+    const int q = warp & 3;
+    const int hf = (warp - 2) >> 2;
+    const uint32_t stg0 = smem_u32(staging + (warp - 2) * 2 * kWgStoreBox);
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    const CUtensorMap* om = hf ? &tmO1 : &tmO0;
+    int local = 0, nstore = 0;
+    bool ok = true;
+    for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
+      const AsUnit u = as_decode(unit, args, mblk);
+      const int r = (hf ? u.m0 + args.out1_row_off : u.m0) + 32 * q;  // first output row
+      for (int nb = 0; nb < nblk; ++nb, ++local) {
+        const int buf = local & 1;
+        if (!mbar_wait(tmem_full0 + 8 * buf, (uint32_t)((local >> 1) & 1), abort_flag,
+                       args.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        wg_store_half(om, tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, u.rows > 0,
+                      r < args.m_out, u.seg * args.m_out + r, nb * kWgN, args.n_out, stg0, lane,
+                      nstore, tmem_empty0 + 8 * buf);
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) {
+    // drain the copies still in flight into shared memory (bounded)
+    for (int i = *a_seen_sh; i < a_issued; ++i)
+      mbar_wait(a_full0 + 8 * (i % kAsSlots), (uint32_t)((i / kAsSlots) & 1), abort_flag,
+                args.status, kDrainTimeoutNs, false);
+    for (int i = *b_seen_sh; i < b_issued; ++i)
+      mbar_wait(b_full0 + 8 * (i % kAsBStages), (uint32_t)((i / kAsBStages) & 1), abort_flag,
                 args.status, kDrainTimeoutNs, false);
   }
   __syncwarp();
@@ -347,10 +650,10 @@ inline bool make_store_map(CUtensorMap* m, void* base, uint64_t rows, uint64_t c
   return r == CUDA_SUCCESS;
 }
 
-inline moe_status launch_wgrad(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o0,
+static inline moe_status launch_wgrad(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& o0,
                                const CUtensorMap& o1, const WgArgs& args, int sms,
                                cudaStream_t st, char* err, size_t errn) {
-  static bool attr_set[64] = {};
+  static bool attr_set[64] = {};  // per device; internal linkage (one per loaded library)
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !attr_set[dev]) {
@@ -377,12 +680,40 @@ inline moe_status launch_wgrad(const CUtensorMap& a, const CUtensorMap& b, const
   return MOE_OK;
 }
 
-// dW1[e] = da_e^T x_perm_e and dW3[e] = du_e^T x_perm_e (dau = da | du [rows, 2I]),
-// then dW2[e] = dy_e^T h_e.
-inline moe_status launch_expert_wgrad(const moe_shape& s, const void* x_perm, const void* h,
-                                      const void* dy, const void* dau, const int32_t* offsets,
-                                      void* dw1, void* dw3, void* dw2, uint32_t* status, int sms,
-                                      cudaStream_t st, char* err, size_t errn) {
+static inline moe_status launch_wgrad_as(const CUtensorMap& a, const CUtensorMap& b,
+                                  const CUtensorMap& o0, const CUtensorMap& o1,
+                                  const WgArgs& args, int sms, cudaStream_t st, char* err,
+                                  size_t errn) {
+  static bool attr_set[64] = {};  // per device; internal linkage (one per loaded library)
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_wgrad_as_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kAsSmemBytes);
+    if (e != cudaSuccess) {
+      snprintf(err, errn, "wgrad smem attribute: %s", cudaGetErrorString(e));
+      return MOE_ERR_CUDA;
+    }
+    attr_set[dev] = true;
+  }
+  const long long units = (long long)args.nseg * ((args.m_out + args.m_step - 1) / args.m_step);
+  long long grid = units < sms ? units : sms;
+  if (grid < 1) grid = 1;
+  gemm_wgrad_as_kernel<<<(int)grid, kWgThreads, kAsSmemBytes, st>>>(a, b, o0, o1, args);
+  note_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    snprintf(err, errn, "wgrad launch: %s", cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// dW1[e] = da_e^T x_perm_e and dW3[e] = du_e^T x_perm_e (dau = da | du [rows, 2I]).
+inline moe_status launch_wgrad_w13(const moe_shape& s, const void* x_perm, const void* dau,
+                                   const int32_t* offsets, void* dw1, void* dw3,
+                                   uint32_t* status, int sms, cudaStream_t st, char* err,
+                                   size_t errn) {
   const uint64_t rows = (uint64_t)s.T * s.K;
   CUtensorMap a, b, o0, o1;
   if (!make_map(&a, dau, rows, 2 * (uint64_t)s.I, 64)) return map_error(err, errn, "dau");
@@ -399,17 +730,29 @@ inline moe_status launch_expert_wgrad(const moe_shape& s, const void* x_perm, co
   g.a1_col_off = s.I;
   g.out1_row_off = 0;
   g.status = status;
-  moe_status r = launch_wgrad(a, b, o0, o1, g, sms, st, err, errn);
-  if (r != MOE_OK) return r;
+  return launch_wgrad_as(a, b, o0, o1, g, sms, st, err, errn);
+}
+
+// dW2[e] = dy_e^T h_e.
+inline moe_status launch_wgrad_w2(const moe_shape& s, const void* h, const void* dy,
+                                  const int32_t* offsets, void* dw2, uint32_t* status, int sms,
+                                  cudaStream_t st, char* err, size_t errn) {
+  const uint64_t rows = (uint64_t)s.T * s.K;
+  CUtensorMap a, b, o0;
   if (!make_map(&a, dy, rows, s.d, 64)) return map_error(err, errn, "dy_perm");
   if (!make_map(&b, h, rows, s.I, 64)) return map_error(err, errn, "h");
   if (!make_store_map(&o0, dw2, (uint64_t)s.N * s.d, s.I)) return map_error(err, errn, "dw2");
+  WgArgs g{};
+  g.seg_offsets = offsets;
+  g.nseg = s.N;
+  g.max_rows = (int)rows;
   g.m_out = s.d;
   g.n_out = s.I;
   g.m_step = 256;
   g.a1_col_off = 128;
   g.out1_row_off = 128;
-  return launch_wgrad(a, b, o0, o0, g, sms, st, err, errn);
+  g.status = status;
+  return launch_wgrad_as(a, b, o0, o0, g, sms, st, err, errn);
 }
 
 // dW_r = dlogits^T x over all T tokens (one segment).

@@ -944,14 +944,20 @@ moe_status moe_expert_ffn_backward(const moe_shape* shape, const void* x_perm, c
   const int sms = sm_count();
   const int rows = s.T * s.K;
   if (s.dtype == MOE_BF16) {
-    if (s.T > 0) {
-      MOE_TRY(moe::tc::launch_dgrad_h(s, dy_perm, w2, offsets, au, dau, status, sms, st, g_err,
-                                      sizeof(g_err)));
-      MOE_TRY(moe::tc::launch_dgrad_x(s, dau, w1, w3, offsets, dx_perm, status, sms, st, g_err,
-                                      sizeof(g_err)));
-    }
-    return moe::tc::launch_expert_wgrad(s, x_perm, h, dy_perm, dau, offsets, dw1, dw3, dw2,
-                                        status, sms, st, g_err, sizeof(g_err));
+    // data gradients (weights read, dau and dx_perm written), then weight
+    // gradients (dW written).  Running the write-bound weight-gradient GEMMs
+    // beside the read-bound data-gradient GEMMs on split SM partitions measured
+    // no faster than this order.
+    if (s.T > 0)
+      MOE_TRY(moe::tc::launch_dgrad_h(s, dy_perm, w2, offsets, au, dau, status, sms, st,
+                                      g_err, sizeof(g_err)));
+    if (s.T > 0)
+      MOE_TRY(moe::tc::launch_dgrad_x(s, dau, w1, w3, offsets, dx_perm, status, sms, st,
+                                      g_err, sizeof(g_err)));
+    MOE_TRY(moe::tc::launch_wgrad_w2(s, h, dy_perm, offsets, dw2, status, sms, st, g_err,
+                                     sizeof(g_err)));
+    return moe::tc::launch_wgrad_w13(s, x_perm, dau, offsets, dw1, dw3, status, sms, st,
+                                      g_err, sizeof(g_err));
   }
   moe::SimtBwdArgs a{};
   a.offsets = offsets;
