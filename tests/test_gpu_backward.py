@@ -193,3 +193,36 @@ def test_backward_is_deterministic_and_forward_unchanged(dtype):
     assert torch.equal(ref.h[:R], buf1.h[:R])
     assert torch.equal(ref.y_perm[:R], buf1.y_perm[:R])
     assert torch.equal(ref.out, buf1.out)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_k_equals_e(dtype):
+    """Every expert selected: the gates sum to 1 and dlogits covers all E."""
+    N, Z = 12, 4
+    shape, L = _small(60, 256, N, Z, N + Z, 128, dtype, seed=61)
+    check_backward(shape, dtype, L, N, N + Z, seed=61)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_all_slots_to_zero_experts(dtype):
+    """No routed rows: the expert weight gradients are exactly zero and dx is
+    the identity term plus the router term."""
+    N, Z, K = 8, 8, 3
+    bias = [0.0] * N + [10.0] * Z
+    shape, L = _small(70, 256, N, Z, K, 128, dtype, seed=62, bias=bias)
+    buf, bb, _ = check_backward(shape, dtype, L, N, K, gamma=0.8, seed=62)
+    assert int(buf.offsets[-1].item()) == 0
+    assert not bb.dw1.any() and not bb.dw3.any() and not bb.dw2.any()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_no_zero_experts(dtype):
+    shape, L = _small(150, 256, 16, 0, 3, 128, dtype, seed=63)
+    check_backward(shape, dtype, L, 16, 3, seed=63)
+
+
+def test_backward_max_experts_bf16():
+    """E = 1024 experts and K = 40 slots per token."""
+    N, Z, K = 640, 384, 40
+    shape, L = _small(150, 128, N, Z, K, 128, "bf16", seed=64)
+    check_backward(shape, "bf16", L, N, K, seed=64)

@@ -179,6 +179,21 @@ def test_no_zero_experts(dtype):
     _run_and_check(shape, dtype, L, 10, 3)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_max_experts_large_k(dtype):
+    """E = N + Z = 1024, the library's limit (32 scores per lane in the top-K
+    kernel), with K = 40 slots per token (more than one 32-lane pass)."""
+    N, Z, K = 640, 384, 40
+    shape, L = _small(150, 128, N, Z, K, 128, dtype, seed=21)
+    _run_and_check(shape, dtype, L, N, K)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_single_ffn_expert_top1(dtype):
+    shape, L = _small(90, 64, 1, 2, 1, 64, dtype, seed=22)
+    _run_and_check(shape, dtype, L, 1, 1)
+
+
 def test_empty_batch():
     shape, L = _small(0, 64, 6, 2, 2, 64, "f32", seed=1)
     L["x"] = torch.empty((0, 64), device="cuda")
