@@ -943,17 +943,24 @@ moe_status moe_expert_ffn_backward(const moe_shape* shape, const void* x_perm, c
   void* dau = at<char>(ws, L.dau);
   const int sms = sm_count();
   const int rows = s.T * s.K;
+  if (s.T == 0) {
+    // no tokens: every weight gradient is zero
+    const size_t bytes = (size_t)s.N * s.I * s.d * elem_bytes(s);
+    for (void* p : {dw1, dw3, dw2}) {
+      cudaError_t e = cudaMemsetAsync(p, 0, bytes, st);
+      if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+    }
+    return MOE_OK;
+  }
   if (s.dtype == MOE_BF16) {
     // data gradients (weights read, dau and dx_perm written), then weight
     // gradients (dW written).  Running the write-bound weight-gradient GEMMs
     // beside the read-bound data-gradient GEMMs on split SM partitions measured
     // no faster than this order.
-    if (s.T > 0)
-      MOE_TRY(moe::tc::launch_dgrad_h(s, dy_perm, w2, offsets, au, dau, status, sms, st,
-                                      g_err, sizeof(g_err)));
-    if (s.T > 0)
-      MOE_TRY(moe::tc::launch_dgrad_x(s, dau, w1, w3, offsets, dx_perm, status, sms, st,
-                                      g_err, sizeof(g_err)));
+    MOE_TRY(moe::tc::launch_dgrad_h(s, dy_perm, w2, offsets, au, dau, status, sms, st, g_err,
+                                    sizeof(g_err)));
+    MOE_TRY(moe::tc::launch_dgrad_x(s, dau, w1, w3, offsets, dx_perm, status, sms, st, g_err,
+                                    sizeof(g_err)));
     MOE_TRY(moe::tc::launch_wgrad_w2(s, h, dy_perm, offsets, dw2, status, sms, st, g_err,
                                      sizeof(g_err)));
     return moe::tc::launch_wgrad_w13(s, x_perm, dau, offsets, dw1, dw3, status, sms, st,
@@ -964,7 +971,7 @@ moe_status moe_expert_ffn_backward(const moe_shape* shape, const void* x_perm, c
   a.nseg = s.N;
   a.max_rows = rows;
   a.status = status;
-  if (s.T > 0) {
+  {
     // dh = dy W2_e, then the SwiGLU backward into dau
     a.A = dy_perm;
     a.a_sm = s.d;

@@ -226,3 +226,21 @@ def test_backward_max_experts_bf16():
     N, Z, K = 640, 384, 40
     shape, L = _small(150, 128, N, Z, K, 128, "bf16", seed=64)
     check_backward(shape, "bf16", L, N, K, seed=64)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_empty_batch(dtype):
+    """T = 0: every call is a no-op except that the weight gradients are zero."""
+    shape, L = _small(0, 256, 8, 8, 2, 128, dtype, seed=65)
+    L["x"] = torch.empty((0, 256), dtype=L["x"].dtype, device="cuda")
+    dout = torch.empty((0, 256), dtype=L["x"].dtype, device="cuda")
+    buf = B.LayerBuffers(shape, with_probs=True)
+    bb = B.BackwardBuffers(shape)
+    for t in (bb.dw1, bb.dw3, bb.dw2, bb.dw_router):
+        t.fill_(1.0)
+    B.forward_train(buf, bb, L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"])
+    B.backward(buf, bb, L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], dout)
+    torch.cuda.synchronize()
+    assert B.device_status(buf.ws) == 0 and B.device_status(bb.bws) == 0
+    for t in (bb.dw1, bb.dw3, bb.dw2, bb.dw_router):
+        assert not t.any()
