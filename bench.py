@@ -362,7 +362,9 @@ def run_gpu(args, rank, world, local_rank):
                    "expert_weights": ("mxfp8 (moe_quantize_weights_mxfp8)" if args.fp8_experts
                                       else "tiled (moe_pack_weights)" if tiled else "row-major"),
                    "parallelism": f"token-dp{world} (weights replicated, counts all-reduced)",
-                   "l2": "inputs larger than L2 (38.7 GB of expert weights streamed per step)"},
+                   "l2": f"inputs larger than L2 ({cfg.N * 3 * cfg.I * cfg.d * wsz / 1e9:.2f} GB "
+                         "of expert weights, 126 MB L2; the touched experts' weights are "
+                         "streamed every step)"},
         "roofline": {"kernel": ("moe_expert_gate_up_mxfp8 (tcgen05 block-scaled grouped GEMM)"
                                 if fp8 else "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)"),
                      "bound": "hbm", "achieved": round(achieved, 1),

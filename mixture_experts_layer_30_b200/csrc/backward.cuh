@@ -36,6 +36,8 @@ combine_backward_kernel(const T* __restrict__ x, const T* __restrict__ y_perm,
                         const T* __restrict__ dout, int K, int N, int E, int d, int max_rows,
                         float gamma, T* __restrict__ dy_perm, float* __restrict__ dgate,
                         uint32_t* status) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int VN = Vec16<T>::kN;
   __shared__ int s_row[kMaxExperts + 1];  // -1: the x_t source
   __shared__ int s_k[kMaxExperts + 1];
@@ -153,6 +155,8 @@ __global__ void __launch_bounds__(256)
 dlogits_kernel(const float* __restrict__ probs, const int32_t* __restrict__ topk_idx,
                const float* __restrict__ dgate, int T, int E, int K, TOut* __restrict__ dlogits,
                uint32_t* status) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float s_dR[8][kMaxExperts];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x * 8 + warp;
@@ -188,6 +192,8 @@ permute_backward_kernel(const T* __restrict__ dout, const int32_t* __restrict__ 
                         const T* __restrict__ dx_perm, const float* __restrict__ dx_router,
                         int K, int N, int E, int d, int max_rows, float gamma,
                         T* __restrict__ dx) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int VN = Vec16<T>::kN;
   __shared__ int s_row[kMaxExperts];
   __shared__ int s_n;

@@ -18,6 +18,8 @@ combine_kernel(const T* __restrict__ x, const T* __restrict__ y_perm,
                const int32_t* __restrict__ topk_idx, const float* __restrict__ topk_gate,
                const int32_t* __restrict__ slot_pos, int K, int N, int E, int d, int max_rows,
                float gamma, T* __restrict__ out, uint32_t* status) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int VN = Vec16<T>::kN;
   __shared__ int s_row[kMaxExperts];
   __shared__ float s_g[kMaxExperts];
@@ -91,6 +93,8 @@ combine_kernel(const T* __restrict__ x, const T* __restrict__ y_perm,
 // fp64 with explicit round-to-nearest operations (no contraction), one rounding to fp32.
 __global__ void bias_update_kernel(int N, const int32_t* __restrict__ counts, long long T_all,
                                    int K, float K_e, float mu, float* __restrict__ bias) {
+  pdl_trigger();
+  pdl_wait();
   const double target = __ddiv_rn((double)K_e, __dmul_rn((double)K, (double)N));
   const double denom = __dmul_rn((double)K, (double)T_all);
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < N; i += gridDim.x * blockDim.x) {

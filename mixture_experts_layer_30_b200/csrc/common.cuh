@@ -25,6 +25,34 @@ constexpr int kPermChunk = 256;     // tokens per dispatch chunk (one thread per
 constexpr int kRouteTokensPerCta = 32;  // 16 warps x 2 tokens: enough warps to hide latency
 constexpr int kRouteThreads = 512;
 
+// --- programmatic dependent launch ------------------------------------------
+// Every kernel of this library is launched with programmatic stream
+// serialisation (launch_pdl).  A kernel first lets the next kernel on the
+// stream be scheduled (pdl_trigger: once all of this grid's CTAs have started)
+// and then waits for the previous grid to complete and publish its memory
+// (pdl_wait) before its first global-memory read or write; only work on
+// registers, shared memory, barriers and TMEM may come before the wait.  The
+// next kernel's launch and prologue thus overlap this kernel's tail.  Both are
+// no-ops for a kernel launched without the attribute.
+MOE_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+MOE_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 MOE_DEV void set_status(uint32_t* st, uint32_t bit) {
   if (st) atomicOr(st, bit);
 }
@@ -147,6 +175,8 @@ MOE_DEV int find_expert(const int* prefix, int N, int c) {
 // of the tiled order, row-major inside the tile.  16-byte vectors.
 __global__ void __launch_bounds__(256)
 pack_tiles_kernel(const uint4* __restrict__ src, int rows, int cols, uint4* __restrict__ dst) {
+  pdl_trigger();
+  pdl_wait();
   const long long tile = blockIdx.x;
   const int cb_n = cols / 64, rb_n = rows / 128;
   const int cb = (int)(tile % cb_n);

@@ -115,6 +115,7 @@ template <bool kGatedOut>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                  const __grid_constant__ CUtensorMap tmB, const ArgsF8 args) {
+  pdl_trigger();
   constexpr int kStagingBytes = staging<kGatedOut>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -159,6 +160,7 @@ gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  pdl_wait();  // the prologue above touches no global memory
   build_chunk_prefix(args.seg_offsets, args.nseg, args.max_rows, kNMax, prefix, scan_tmp,
                      args.status);
   tc_fence_before();
@@ -448,8 +450,8 @@ static inline moe_status launch_f8(const CUtensorMap& a0, const CUtensorMap& a1,
   }
   long long grid = max_tiles < sms ? max_tiles : sms;
   if (grid < 1) grid = 1;
-  gemm_mxf8_kernel<kGatedOut><<<(int)grid, kThreads, smem_bytes<kGatedOut>(), st>>>(a0, a1, b,
-                                                                                   args);
+  launch_pdl(gemm_mxf8_kernel<kGatedOut>, dim3((unsigned)grid), dim3(kThreads),
+             (size_t)smem_bytes<kGatedOut>(), st, a0, a1, b, args);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

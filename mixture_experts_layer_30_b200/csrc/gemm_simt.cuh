@@ -24,6 +24,8 @@ grouped_gemm_simt_kernel(const TIn* __restrict__ A, const TIn* __restrict__ B0,
                          const TIn* __restrict__ B1, const int32_t* __restrict__ offsets,
                          int N, int max_rows, int n_out, int k_dim, TIn* __restrict__ C,
                          uint32_t* status, const int32_t* __restrict__ a_rows, int a_src_rows) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int prefix[kMaxExperts + 1];
   __shared__ int scan_tmp[33];
   __shared__ float As[kSgBK][kSgBM + 4];

@@ -46,6 +46,8 @@ constexpr int kSbBM = 64, kSbBN = 64, kSbBK = 16;
 
 template <typename T, bool kKSeg, bool kSwiglu>
 __global__ void __launch_bounds__(256) gemm_simt_bwd_kernel(const SimtBwdArgs p) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int prefix[kMaxExperts + 1];
   __shared__ int scan_tmp[33];
   __shared__ float As[kSbBK][kSbBM + 4];

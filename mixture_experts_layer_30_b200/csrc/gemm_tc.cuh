@@ -122,6 +122,11 @@ struct Args {
   int a_k_split;
   const void* au;              // kSwigluBwd: pre-activations [rows, 2*n_out] (a | u)
   void* aux_out;               // kGatedSave: a | u output [rows, 2*n_out]
+  // Split-K (kPlainF32, one segment): K blocks are cut into k_splits ranges;
+  // split s writes its fp32 partial sums at out + s*split_stride (the addend
+  // goes to split 0 only).  0 or 1: no split.
+  int k_splits;
+  long long split_stride;
 };
 
 // TMA coordinates (column, row) of the weight tile whose first row is `row`
@@ -367,6 +372,7 @@ template <int kMode, class Cfg, bool kAMN = false>
 __global__ void __launch_bounds__(kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                const __grid_constant__ CUtensorMap tmB, const Args args) {
+  pdl_trigger();
   constexpr int kNMax = Cfg::kNMax, kStages = Cfg::kStages, kAccBufs = Cfg::kAccBufs;
   constexpr int kStageBytes = Cfg::kStageBytes, kNumBars = Cfg::kNumBars;
   constexpr int kTmemCols = Cfg::kTmemCols;
@@ -417,6 +423,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  pdl_wait();  // the prologue above touches no global memory
   if (args.seg_offsets) {
     build_chunk_prefix(args.seg_offsets, args.nseg, args.max_rows, kNMax, prefix, scan_tmp,
                        args.status);
@@ -431,8 +438,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
 
   const int nseg = args.seg_offsets ? args.nseg : 1;
   const int n_fblk = (args.n_out + args.feat_per_tile - 1) / args.feat_per_tile;
-  const int total = prefix[nseg] * n_fblk;
+  const int ksplit = args.k_splits > 1 ? args.k_splits : 1;
+  const int base_tiles = prefix[nseg] * n_fblk;
+  const int total = base_tiles * ksplit;
   const int nk = args.k_dim / kBK;
+  // tile -> (row chunk, feature block) and its K-block range [kb0, kb1)
+  auto tile_of = [&](int tile, int& sp, int& kb0, int& kb1) {
+    sp = tile / base_tiles;
+    kb0 = sp * nk / ksplit;
+    kb1 = (sp + 1) * nk / ksplit;
+    return decode_tile<kNMax>(tile - sp * base_tiles, n_fblk, args, prefix);
+  };
   int issued = 0;  // producer: stages issued
 
   if (warp == 0 && args.gather_rows) {
@@ -448,7 +464,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     constexpr int kRowsPerLane = kNMax / 32;
     const __nv_bfloat16* xsrc = static_cast<const __nv_bfloat16*>(args.gather_src);
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      const Tile t = decode_tile<kNMax>(tile, n_fblk, args, prefix);
+      int sp, kb0, kb1;
+      const Tile t = tile_of(tile, sp, kb0, kb1);
       const int a_row0 = t.seg * args.a_seg_rows + t.f0;
       const int a_row1 = a_row0 + args.a1_row_off;
       const __nv_bfloat16* src[kRowsPerLane];
@@ -465,7 +482,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
         }
         src[i] = xsrc + (size_t)v * args.k_dim;
       }
-      for (int kb = 0; kb < nk; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         int go = 1;
         if (lane == 0) go = mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status);
         go = __shfl_sync(0xffffffffu, go, 0);
@@ -506,7 +523,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const Tile t = decode_tile<kNMax>(tile, n_fblk, args, prefix);
+        int sp, kb0, kb1;
+        const Tile t = tile_of(tile, sp, kb0, kb1);
         const int nbox = (t.n + kBoxRows - 1) / kBoxRows;
         if constexpr (kMode == kSwigluBwd) {
           // the epilogue of this tile reads a and u of its rows and 256 features:
@@ -522,7 +540,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
         const uint32_t tx = 2 * kABytes + nbox * kBoxBytes;
         const int a_row0 = t.seg * args.a_seg_rows + t.f0;
         const int a_row1 = a_row0 + args.a1_row_off;
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status)) {
             ok = false;
             break;
@@ -563,7 +581,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       bool ok = true;
       int consumed = 0, local = 0;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++local) {
-        const Tile t = decode_tile<kNMax>(tile, n_fblk, args, prefix);
+        int sp, kb0, kb1;
+        const Tile t = tile_of(tile, sp, kb0, kb1);
         int n16 = ((t.n + 15) >> 4) << 4;
         if (n16 < 16) n16 = 16;
         const uint32_t idesc = idesc_bf16(kFeat, n16, kAMN);
@@ -572,7 +591,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
         const uint32_t d0 = tmem_base + buf * 2 * kNMax;
         if (!mbar_wait(tmem_empty0 + 8 * buf, acc_parity ^ 1, abort_flag, args.status)) break;
         tc_fence_after();
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.status)) {
             ok = false;
             break;
@@ -589,7 +608,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
           constexpr uint64_t kAStep = kAMN ? 128 : 2;
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
-            const uint32_t acc = (kb | k) != 0;
+            const uint32_t acc = ((kb - kb0) | k) != 0;
             umma_bf16(d0, da0 + kAStep * k, db + 2 * k, idesc, acc);
             umma_bf16(d0 + kNMax, da1 + kAStep * k, db + 2 * k, idesc, acc);
           }
@@ -612,7 +631,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int local = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++local) {
-      const Tile t = decode_tile<kNMax>(tile, n_fblk, args, prefix);
+      int sp, kb0, kb1;
+      const Tile t = tile_of(tile, sp, kb0, kb1);
       const int buf = local % kAccBufs;
       const uint32_t acc_parity = (uint32_t)((local / kAccBufs) & 1);
       const uint32_t dbase = tmem_base + lane_base + buf * 2 * kNMax;
@@ -776,8 +796,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
             if (j0 + j < t.n && f < args.n_out) {
               if (kMode == kPlainF32) {
                 uint4 w = *reinterpret_cast<const uint4*>(&stg[j * kStagingPitch + c * 4]);
-                float* o = static_cast<float*>(args.out) + (size_t)row * args.n_out + f;
-                if (args.add) {
+                float* o = static_cast<float*>(args.out) + sp * args.split_stride +
+                           (size_t)row * args.n_out + f;
+                if (args.add && sp == 0) {
                   const float4 ad =
                       *reinterpret_cast<const float4*>(args.add + (size_t)row * args.n_out + f);
                   w.x = __float_as_uint(__uint_as_float(w.x) + ad.x);
@@ -878,8 +899,8 @@ static inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, co
   }
   long long grid = max_tiles < sms ? max_tiles : sms;
   if (grid < 1) grid = 1;
-  gemm_tc_kernel<kMode, Cfg, kAMN>
-      <<<(int)grid, kThreads, Cfg::smem_bytes(staging_bytes<kMode>()), st>>>(a0, a1, b, args);
+  launch_pdl(gemm_tc_kernel<kMode, Cfg, kAMN>, dim3((unsigned)grid), dim3(kThreads),
+             (size_t)Cfg::smem_bytes(staging_bytes<kMode>()), st, a0, a1, b, args);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -1027,6 +1048,22 @@ inline moe_status launch_down(const moe_shape& s, const void* h, const void* w2,
                                      sms, st, err, errn);
 }
 
+// K splits of the router GEMM for a shape.  A small batch has few
+// (256-token, 256-expert) tiles, so each would walk all d/64 K blocks on one SM;
+// splitting K spreads it over ~128 CTAs, and the top-K kernel sums the fp32
+// partial logits in split order.  The count depends on the shape only (it sizes
+// the workspace): 1 at the LongCat prefill shape.
+inline int router_splits(const moe_shape& s) {
+  const int E = s.N + s.Z;
+  const long long tiles = (long long)((s.T + 255) / 256) * ((E + 255) / 256);
+  long long sp = tiles > 0 ? 128 / tiles : 1;
+  const int nk = s.d / kBK;
+  if (sp > 32) sp = 32;
+  if (sp > nk) sp = nk;
+  if (sp < 1) sp = 1;
+  return (int)sp;
+}
+
 inline moe_status launch_router_gemm(const moe_shape& s, const void* x, const void* w,
                                      const float* offset, float* logits, int sms,
                                      cudaStream_t st, char* err, size_t errn) {
@@ -1047,9 +1084,16 @@ inline moe_status launch_router_gemm(const moe_shape& s, const void* x, const vo
   g.out = logits;
   g.add = offset;
   g.status = nullptr;
+  const long long fblk = (E + 2 * kFeat - 1) / (2 * kFeat);
+  const int splits = router_splits(s);
+  if (splits > 1) {
+    g.k_splits = splits;
+    g.split_stride = (long long)s.T * E;
+    return launch<kPlainF32, CfgWide>(a, a, b, g, (long long)((s.T + 255) / 256) * fblk * splits,
+                                      sms, st, err, errn);
+  }
   // The router is one dense GEMM: pick the token tile so that all tiles run
   // in one wave when 256-row tiles would leave SMs idle.
-  const long long fblk = (E + 2 * kFeat - 1) / (2 * kFeat);
   const long long tiles256 = (long long)((s.T + 255) / 256) * fblk;
   const long long tiles192 = (long long)((s.T + 191) / 192) * fblk;
   if (tiles256 < sms && tiles192 <= sms)

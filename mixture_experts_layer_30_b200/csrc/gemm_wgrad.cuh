@@ -169,6 +169,7 @@ __global__ void __launch_bounds__(kWgThreads, 1)
 gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmO0,
                   const __grid_constant__ CUtensorMap tmO1, const WgArgs args) {
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -217,6 +218,7 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the prologue above touches no global memory
 
   const int nseg = args.seg_offsets ? args.nseg : 1;
   const int mblk = (args.m_out + args.m_step - 1) / args.m_step;
@@ -389,6 +391,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmO0,
                      const __grid_constant__ CUtensorMap tmO1, const WgArgs args) {
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -446,6 +449,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the prologue above touches no global memory
 
   const int mblk = (args.m_out + args.m_step - 1) / args.m_step;
   const int nblk = (args.n_out + kWgN - 1) / kWgN;
@@ -670,7 +674,8 @@ static inline moe_status launch_wgrad(const CUtensorMap& a, const CUtensorMap& b
                           ((args.n_out + kWgN - 1) / kWgN);
   long long grid = tiles < sms ? tiles : sms;
   if (grid < 1) grid = 1;
-  gemm_wgrad_kernel<<<(int)grid, kWgThreads, kWgSmemBytes, st>>>(a, b, o0, o1, args);
+  launch_pdl(gemm_wgrad_kernel, dim3((unsigned)grid), dim3(kWgThreads), (size_t)kWgSmemBytes, st,
+             a, b, o0, o1, args);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -699,7 +704,8 @@ static inline moe_status launch_wgrad_as(const CUtensorMap& a, const CUtensorMap
   const long long units = (long long)args.nseg * ((args.m_out + args.m_step - 1) / args.m_step);
   long long grid = units < sms ? units : sms;
   if (grid < 1) grid = 1;
-  gemm_wgrad_as_kernel<<<(int)grid, kWgThreads, kAsSmemBytes, st>>>(a, b, o0, o1, args);
+  launch_pdl(gemm_wgrad_as_kernel, dim3((unsigned)grid), dim3(kWgThreads), (size_t)kAsSmemBytes,
+             st, a, b, o0, o1, args);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -82,6 +82,12 @@ moe_status validate_shape(const moe_shape* sp) {
   return MOE_OK;
 }
 
+// K splits of the router GEMM: the tensor-core router splits K for small
+// batches; the CUDA-core router does not split.
+int router_nsplit(const moe_shape& s) {
+  return (s.dtype == MOE_BF16 && moe::tc::router_supported(s)) ? moe::tc::router_splits(s) : 1;
+}
+
 WsLayout layout_of(const moe_shape& s) {
   WsLayout L{};
   size_t off = 0;
@@ -92,7 +98,8 @@ WsLayout layout_of(const moe_shape& s) {
   };
   const size_t E = (size_t)s.N + s.Z;
   L.status = take(256);
-  L.logits = take((size_t)s.T * E * 4);
+  // fp32 logits, one [T, E] slab per K split of the tensor-core router GEMM
+  L.logits = take((size_t)router_nsplit(s) * s.T * E * 4);
   L.route_hist = take((size_t)route_ctas(s) * E * 4);
   L.route_psum = take((size_t)route_ctas(s) * E * 4);
   L.perm_hist = take((size_t)perm_chunks(s) * s.N * 4);
@@ -133,11 +140,11 @@ int sm_count() {
 // --- launches ---------------------------------------------------------------
 
 template <int VPL>
-void launch_topk(dim3 grid, cudaStream_t st, const float* logits, const float* bias, int T,
-                 int E, int N, int K, int32_t* idx, float* gate, uint8_t* nffn, float* probs,
-                 int32_t* hist, float* psum) {
-  moe::softmax_topk_kernel<VPL><<<grid, moe::kRouteThreads, 0, st>>>(
-      logits, bias, T, E, N, K, idx, gate, nffn, probs, hist, psum);
+void launch_topk(dim3 grid, cudaStream_t st, const float* logits, int nsplit, const float* bias,
+                 int T, int E, int N, int K, int32_t* idx, float* gate, uint8_t* nffn,
+                 float* probs, int32_t* hist, float* psum) {
+  moe::launch_pdl(moe::softmax_topk_kernel<VPL>, dim3(grid), dim3(moe::kRouteThreads), 0, st,
+      logits, nsplit, (long long)T * E, bias, T, E, N, K, idx, gate, nffn, probs, hist, psum);
 }
 
 template <typename T>
@@ -149,33 +156,35 @@ moe_status route_impl(const moe_shape& s, const void* x, const void* w, const fl
   float* logits = at<float>(ws, L.logits);
   int32_t* hist = at<int32_t>(ws, L.route_hist);
   float* psum = prob_sum ? at<float>(ws, L.route_psum) : nullptr;
+  int nsplit = 1;
   if (s.T > 0) {
     if (s.dtype == MOE_BF16 && moe::tc::router_supported(s) &&
         reinterpret_cast<uintptr_t>(off) % 16 == 0) {
+      nsplit = moe::tc::router_splits(s);
       MOE_TRY(moe::tc::launch_router_gemm(s, x, w, off, logits, sm_count(), st, g_err,
                                           sizeof(g_err)));
     } else {
       dim3 g((E + moe::kRgBN - 1) / moe::kRgBN, (s.T + moe::kRgBM - 1) / moe::kRgBM);
-      moe::router_gemm_simt_kernel<T><<<g, 256, 0, st>>>(
+      moe::launch_pdl(moe::router_gemm_simt_kernel<T>, dim3(g), dim3(256), 0, st,
           static_cast<const T*>(x), static_cast<const T*>(w), off, logits, s.T, E, s.d);
       MOE_TRY(check_launch("router gemm"));
     }
     const int vpl = (E + 31) / 32;
     dim3 g(route_ctas(s));
-    if (vpl <= 1) launch_topk<1>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 2) launch_topk<2>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 3) launch_topk<3>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 4) launch_topk<4>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 8) launch_topk<8>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 16) launch_topk<16>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 24) launch_topk<24>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else launch_topk<32>(g, st, logits, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    if (vpl <= 1) launch_topk<1>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 2) launch_topk<2>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 3) launch_topk<3>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 4) launch_topk<4>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 8) launch_topk<8>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 16) launch_topk<16>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else if (vpl <= 24) launch_topk<24>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    else launch_topk<32>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
     MOE_TRY(check_launch("softmax/top-K"));
   }
-  moe::reduce_hist_kernel<<<(E + 7) / 8, 256, 0, st>>>(hist, route_ctas(s), E, counts);
+  moe::launch_pdl(moe::reduce_hist_kernel, dim3((E + 7) / 8), dim3(256), 0, st, hist, route_ctas(s), E, counts);
   MOE_TRY(check_launch("count reduce"));
   if (prob_sum) {
-    moe::reduce_psum_kernel<<<(E + 7) / 8, 256, 0, st>>>(psum, s.T > 0 ? route_ctas(s) : 0, E,
+    moe::launch_pdl(moe::reduce_psum_kernel, dim3((E + 7) / 8), dim3(256), 0, st, psum, s.T > 0 ? route_ctas(s) : 0, E,
                                                         prob_sum);
     MOE_TRY(check_launch("probability column sums"));
   }
@@ -193,12 +202,25 @@ moe_status permute_impl(const moe_shape& s, const void* x, const int32_t* idx,
   uint32_t* status = at<uint32_t>(ws, L.status);
   int32_t* chist = at<int32_t>(ws, L.perm_hist);
   int32_t* cbase = at<int32_t>(ws, L.perm_base);
+  const size_t small_smem = (size_t)17 * s.N * sizeof(uint32_t);
+  if (nch == 1 && small_smem <= 48 * 1024) {
+    // one chunk (decode): histogram, scan and rank in one CTA
+    moe::launch_pdl(moe::perm_small_kernel, dim3(1), dim3(256), small_smem, st, idx, s.T, s.K, s.N, E, counts, offsets,
+                                                         row_token, slot_pos, status);
+    MOE_TRY(check_launch("dispatch layout"));
+    if (x_perm) {
+      moe::launch_pdl(moe::gather_kernel<T>, dim3((s.T + 7) / 8), dim3(256), 0, st,
+          static_cast<const T*>(x), slot_pos, s.T, s.K, s.d, static_cast<T*>(x_perm));
+      MOE_TRY(check_launch("dispatch gather"));
+    }
+    return MOE_OK;
+  }
   if (nch > 0) {
-    moe::chunk_hist_kernel<<<nch, 256, s.N * sizeof(int), st>>>(idx, s.T, s.K, s.N, E, chist,
+    moe::launch_pdl(moe::chunk_hist_kernel, dim3(nch), dim3(256), s.N * sizeof(int), st, idx, s.T, s.K, s.N, E, chist,
                                                                  status);
     MOE_TRY(check_launch("dispatch histogram"));
   }
-  moe::perm_scan_kernel<<<1, 1024, 0, st>>>(chist, nch, s.N, counts, offsets, cbase, status);
+  moe::launch_pdl(moe::perm_scan_kernel, dim3(1), dim3(1024), 0, st, chist, nch, s.N, counts, offsets, cbase, status);
   MOE_TRY(check_launch("dispatch scan"));
   if (nch > 0) {
     const size_t smem = (size_t)16 * s.N * sizeof(uint32_t);
@@ -209,11 +231,11 @@ moe_status permute_impl(const moe_shape& s, const void* x, const int32_t* idx,
                            (int)smem);
       g_rank_attr_set[dev] = true;
     }
-    moe::perm_rank_kernel<<<nch, 256, smem, st>>>(idx, s.T, s.K, s.N, E, cbase, row_token,
+    moe::launch_pdl(moe::perm_rank_kernel, dim3(nch), dim3(256), smem, st, idx, s.T, s.K, s.N, E, cbase, row_token,
                                                    slot_pos);
     MOE_TRY(check_launch("dispatch rank"));
     if (x_perm) {
-      moe::gather_kernel<T><<<(s.T + 7) / 8, 256, 0, st>>>(
+      moe::launch_pdl(moe::gather_kernel<T>, dim3((s.T + 7) / 8), dim3(256), 0, st,
           static_cast<const T*>(x), slot_pos, s.T, s.K, s.d, static_cast<T*>(x_perm));
       MOE_TRY(check_launch("dispatch gather"));
     }
@@ -232,7 +254,7 @@ moe_status grouped_simt(const moe_shape& s, const void* A, const void* B0, const
   const long long cap = (long long)sm_count() * 8;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  moe::grouped_gemm_simt_kernel<T, kGated><<<(int)grid, 256, 0, st>>>(
+  moe::launch_pdl(moe::grouped_gemm_simt_kernel<T, kGated>, dim3((int)grid), dim3(256), 0, st,
       static_cast<const T*>(A), static_cast<const T*>(B0), static_cast<const T*>(B1), offsets,
       s.N, (int)max_rows, n_out, k_dim, static_cast<T*>(C), status, a_rows, s.T);
   return check_launch(kGated ? "gate/up grouped gemm" : "down grouped gemm");
@@ -315,7 +337,7 @@ moe_status simt_bwd(const moe::SimtBwdArgs& a, long long tiles, cudaStream_t st,
   const long long cap = (long long)sm_count() * 8;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
-  moe::gemm_simt_bwd_kernel<float, kKSeg, kSwiglu><<<(int)grid, 256, 0, st>>>(a);
+  moe::launch_pdl(moe::gemm_simt_bwd_kernel<float, kKSeg, kSwiglu>, dim3((int)grid), dim3(256), 0, st, a);
   return check_launch(what);
 }
 
@@ -407,7 +429,7 @@ moe_status moe_pack_weights(int32_t n_mats, int32_t rows, int32_t cols, int32_t 
   if (a < b + bytes && b < a + bytes)
     return fail(MOE_ERR_INVALID_ARG, "moe_pack_weights: src and dst overlap");
   if (tiles > 0x7fffffffLL) return fail(MOE_ERR_UNSUPPORTED, "moe_pack_weights: too many tiles");
-  moe::pack_tiles_kernel<<<(unsigned)tiles, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  moe::launch_pdl(moe::pack_tiles_kernel, dim3((unsigned)tiles), dim3(256), 0, static_cast<cudaStream_t>(stream),
       static_cast<const uint4*>(src), rows, cols, static_cast<uint4*>(dst));
   return check_launch("weight pack");
 }
@@ -425,8 +447,7 @@ moe_status moe_quantize_weights_mxfp8(int32_t n_mats, int32_t rows, int32_t cols
   MOE_TRY(need(src, "src", 16));
   MOE_TRY(need(dst_q, "dst_q", 16));
   MOE_TRY(need(dst_sf, "dst_sf", 16));
-  moe::quantize_weights_mxfp8_kernel<<<(unsigned)tiles, 256, 0,
-                                       static_cast<cudaStream_t>(stream)>>>(
+  moe::launch_pdl(moe::quantize_weights_mxfp8_kernel, dim3((unsigned)tiles), dim3(256), 0, static_cast<cudaStream_t>(stream),
       static_cast<const __nv_bfloat16*>(src), rows, cols, static_cast<uint8_t*>(dst_q),
       static_cast<uint8_t*>(dst_sf));
   return check_launch("mxfp8 weight quantisation");
@@ -560,7 +581,7 @@ moe_status moe_permute_mxfp8(const moe_shape* shape, const void* x, const int32_
   MOE_TRY(permute_impl<__nv_bfloat16>(s, x, topk_idx, counts, offsets, row_token, slot_pos,
                                       nullptr, ws, L, st));
   if (s.T > 0) {
-    moe::gather_quant_kernel<<<(s.T + 7) / 8, 256, 0, st>>>(
+    moe::launch_pdl(moe::gather_quant_kernel, dim3((s.T + 7) / 8), dim3(256), 0, st,
         static_cast<const __nv_bfloat16*>(x), slot_pos, s.T, s.K, s.d,
         static_cast<uint8_t*>(x_perm_q), static_cast<uint8_t*>(x_perm_sf));
     MOE_TRY(check_launch("quantising dispatch copy"));
@@ -706,12 +727,12 @@ moe_status moe_combine(const moe_shape* shape, const void* x, const void* y_perm
   if (threads > 256) threads = 256;
   const int max_rows = s.T * s.K;
   if (s.dtype == MOE_BF16)
-    moe::combine_kernel<__nv_bfloat16><<<s.T, threads, 0, st>>>(
+    moe::launch_pdl(moe::combine_kernel<__nv_bfloat16>, dim3(s.T), dim3(threads), 0, st,
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y_perm),
         topk_idx, topk_gate, slot_pos, s.K, s.N, E, s.d, max_rows, gamma,
         static_cast<__nv_bfloat16*>(out), nullptr);
   else
-    moe::combine_kernel<float><<<s.T, threads, 0, st>>>(
+    moe::launch_pdl(moe::combine_kernel<float>, dim3(s.T), dim3(threads), 0, st,
         static_cast<const float*>(x), static_cast<const float*>(y_perm), topk_idx, topk_gate,
         slot_pos, s.K, s.N, E, s.d, max_rows, gamma, static_cast<float*>(out), nullptr);
   return check_launch("combine");
@@ -726,7 +747,7 @@ moe_status moe_bias_update(int32_t N, int32_t Z, const int32_t* counts, int64_t 
   if (T_all < 1) return fail(MOE_ERR_INVALID_ARG, "T_all=%lld must be >= 1", (long long)T_all);
   MOE_TRY(need(counts, "counts", 4));
   MOE_TRY(need(bias, "bias", 4));
-  moe::bias_update_kernel<<<(N + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  moe::launch_pdl(moe::bias_update_kernel, dim3((N + 255) / 256), dim3(256), 0, static_cast<cudaStream_t>(stream),
       N, counts, (long long)T_all, K, K_e, mu, bias);
   return check_launch("bias update");
 }
@@ -746,7 +767,7 @@ moe_status moe_lb_stats(int32_t N, int32_t Z, int32_t D, const int32_t* counts,
   MOE_TRY(need(prob_sum, "prob_sum", 4));
   MOE_TRY(need(f, "f", 4));
   MOE_TRY(need(P, "P", 4));
-  moe::lb_stats_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+  moe::launch_pdl(moe::lb_stats_kernel, dim3(1), dim3(1024), 0, static_cast<cudaStream_t>(stream),
       N, Z, D, counts, prob_sum, (long long)T, K, K_e, alpha, f, P, loss);
   return check_launch("load-balance statistics");
 }
@@ -827,12 +848,12 @@ moe_status moe_combine_backward(const moe_shape* shape, const void* x, const voi
   if (threads > 256) threads = 256;
   const int max_rows = s.T * s.K;
   if (s.dtype == MOE_BF16)
-    moe::combine_backward_kernel<__nv_bfloat16><<<s.T, threads, 0, st>>>(
+    moe::launch_pdl(moe::combine_backward_kernel<__nv_bfloat16>, dim3(s.T), dim3(threads), 0, st,
         static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(y_perm),
         topk_idx, topk_gate, slot_pos, static_cast<const __nv_bfloat16*>(dout), s.K, s.N, E,
         s.d, max_rows, gamma, static_cast<__nv_bfloat16*>(dy_perm), dgate, nullptr);
   else
-    moe::combine_backward_kernel<float><<<s.T, threads, 0, st>>>(
+    moe::launch_pdl(moe::combine_backward_kernel<float>, dim3(s.T), dim3(threads), 0, st,
         static_cast<const float*>(x), static_cast<const float*>(y_perm), topk_idx, topk_gate,
         slot_pos, static_cast<const float*>(dout), s.K, s.N, E, s.d, max_rows, gamma,
         static_cast<float*>(dy_perm), dgate, nullptr);
@@ -868,7 +889,7 @@ moe_status moe_route_backward(const moe_shape* shape, const void* x, const void*
   void* dlogits = at<char>(ws, L.dlogits);
   const int sms = sm_count();
   if (s.dtype == MOE_BF16) {
-    moe::dlogits_kernel<__nv_bfloat16><<<(s.T + 7) / 8, 256, 0, st>>>(
+    moe::launch_pdl(moe::dlogits_kernel<__nv_bfloat16>, dim3((s.T + 7) / 8), dim3(256), 0, st,
         probs, topk_idx, dgate, s.T, E, s.K, static_cast<__nv_bfloat16*>(dlogits), status);
     MOE_TRY(check_launch("router logit gradient"));
     MOE_TRY(moe::tc::launch_router_wgrad(s, dlogits, x, dw_router, status, sms, st, g_err,
@@ -876,7 +897,7 @@ moe_status moe_route_backward(const moe_shape* shape, const void* x, const void*
     return moe::tc::launch_router_dx(s, dlogits, w_router, dx_router, status, sms, st, g_err,
                                      sizeof(g_err));
   }
-  moe::dlogits_kernel<float><<<(s.T + 7) / 8, 256, 0, st>>>(
+  moe::launch_pdl(moe::dlogits_kernel<float>, dim3((s.T + 7) / 8), dim3(256), 0, st,
       probs, topk_idx, dgate, s.T, E, s.K, static_cast<float*>(dlogits), status);
   MOE_TRY(check_launch("router logit gradient"));
   moe::SimtBwdArgs a{};
@@ -1060,12 +1081,12 @@ moe_status moe_permute_backward(const moe_shape* shape, const void* dout,
   if (threads > 256) threads = 256;
   const int max_rows = s.T * s.K;
   if (s.dtype == MOE_BF16)
-    moe::permute_backward_kernel<__nv_bfloat16><<<s.T, threads, 0, st>>>(
+    moe::launch_pdl(moe::permute_backward_kernel<__nv_bfloat16>, dim3(s.T), dim3(threads), 0, st,
         static_cast<const __nv_bfloat16*>(dout), topk_idx, topk_gate, slot_pos,
         static_cast<const __nv_bfloat16*>(dx_perm), dx_router, s.K, s.N, E, s.d, max_rows, gamma,
         static_cast<__nv_bfloat16*>(dx));
   else
-    moe::permute_backward_kernel<float><<<s.T, threads, 0, st>>>(
+    moe::launch_pdl(moe::permute_backward_kernel<float>, dim3(s.T), dim3(threads), 0, st,
         static_cast<const float*>(dout), topk_idx, topk_gate, slot_pos,
         static_cast<const float*>(dx_perm), dx_router, s.K, s.N, E, s.d, max_rows, gamma,
         static_cast<float*>(dx));

@@ -10,6 +10,7 @@
 //   3. rank_kernel        per chunk: row of (t, k) = base[c][e] + #earlier tokens of
 //                         the chunk routed to e (warp bitmaps + popcount)
 //   4. gather_kernel      one warp per token: x row copied to each of its rows.
+// A batch of one chunk (decode) runs 1-3 as one kernel (perm_small_kernel).
 #pragma once
 
 #include "common.cuh"
@@ -19,6 +20,8 @@ namespace moe {
 __global__ void __launch_bounds__(256)
 chunk_hist_kernel(const int32_t* __restrict__ topk_idx, int T, int K, int N, int E,
                   int32_t* __restrict__ chunk_hist, uint32_t* status) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int sh_hist[];  // [N]
   for (int e = threadIdx.x; e < N; e += blockDim.x) sh_hist[e] = 0;
   __syncthreads();
@@ -40,6 +43,8 @@ __global__ void __launch_bounds__(1024)
 perm_scan_kernel(const int32_t* __restrict__ chunk_hist, int nchunks, int N,
                  const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                  int32_t* __restrict__ chunk_base, uint32_t* status) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int scan_tmp[33];
   __shared__ int tot_sh[kMaxExperts];
   // per-expert totals (thread per expert, chunks in order)
@@ -74,6 +79,8 @@ __global__ void __launch_bounds__(256)
 perm_rank_kernel(const int32_t* __restrict__ topk_idx, int T, int K, int N, int E,
                  const int32_t* __restrict__ chunk_base, int32_t* __restrict__ row_token,
                  int32_t* __restrict__ slot_pos) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ uint32_t sh_rank[];
   uint32_t* bits = sh_rank;                                   // [8][N]
   int* wbase = reinterpret_cast<int*>(sh_rank + 8 * N);       // [8][N]
@@ -112,12 +119,81 @@ perm_rank_kernel(const int32_t* __restrict__ topk_idx, int T, int K, int N, int 
   }
 }
 
+// The layout of a batch of one chunk (T <= 256, decode): histogram, scan and
+// rank of the three kernels above in one CTA, one thread per token.
+// Shared: bits[8][N], wbase[8][N], tot[N] (68*N bytes).
+__global__ void __launch_bounds__(256)
+perm_small_kernel(const int32_t* __restrict__ topk_idx, int T, int K, int N, int E,
+                  const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                  int32_t* __restrict__ row_token, int32_t* __restrict__ slot_pos,
+                  uint32_t* status) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ uint32_t sh_small[];
+  __shared__ int scan_tmp[33];
+  uint32_t* bits = sh_small;                                  // [8][N]
+  int* wbase = reinterpret_cast<int*>(sh_small + 8 * N);      // [8][N]
+  int* tot = reinterpret_cast<int*>(sh_small + 16 * N);       // [N]
+  for (int i = threadIdx.x; i < 8 * N; i += blockDim.x) bits[i] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = threadIdx.x;
+  if (t < T) {
+    for (int k = 0; k < K; ++k) {
+      const int e = topk_idx[(size_t)t * K + k];
+      if (e < 0 || e >= E) { set_status(status, MOE_DEV_BAD_EXPERT_INDEX); continue; }
+      if (e < N) atomicOr(&bits[warp * N + e], 1u << lane);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) c += __popc(bits[w * N + e]);
+    tot[e] = c;
+    if (counts && counts[e] != c) set_status(status, MOE_DEV_COUNT_MISMATCH);
+  }
+  __syncthreads();
+  // exclusive scan over experts: each thread owns a run of consecutive experts
+  const int per = (N + blockDim.x - 1) / blockDim.x;
+  const int lo = min(N, (int)threadIdx.x * per), hi = min(N, lo + per);
+  int local = 0;
+  for (int e = lo; e < hi; ++e) local += tot[e];
+  int run = block_exclusive_scan(local, scan_tmp, &scan_tmp[32]);
+  for (int e = lo; e < hi; ++e) {
+    offsets[e] = run;
+    int b = run;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      wbase[w * N + e] = b;
+      b += __popc(bits[w * N + e]);
+    }
+    run += tot[e];
+  }
+  if (threadIdx.x == 0) offsets[N] = scan_tmp[32];
+  __syncthreads();
+  if (t < T) {
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int k = 0; k < K; ++k) {
+      const int e = topk_idx[(size_t)t * K + k];
+      int row = -1;
+      if (e >= 0 && e < N) {
+        row = wbase[warp * N + e] + __popc(bits[warp * N + e] & lt);
+        row_token[row] = t;
+      }
+      slot_pos[(size_t)t * K + k] = row;
+    }
+  }
+}
+
 // One warp per token: the x row is read once from HBM, in pieces of 8 x 16 B
 // per lane held in registers, and each piece is stored to every row of the token.
 template <typename T>
 __global__ void __launch_bounds__(256)
 gather_kernel(const T* __restrict__ x, const int32_t* __restrict__ slot_pos, int ntok, int K,
               int d, T* __restrict__ x_perm) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int kPiece = 8;
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);

@@ -78,6 +78,8 @@ MOE_DEV int mx_quant_block_bf16(const uint4 (&in)[4], uint4 (&q)[2]) {
 __global__ void __launch_bounds__(256)
 quantize_weights_mxfp8_kernel(const __nv_bfloat16* __restrict__ src, int rows, int cols,
                               uint8_t* __restrict__ dst_q, uint8_t* __restrict__ dst_sf) {
+  pdl_trigger();
+  pdl_wait();
   const long long tile = blockIdx.x;
   const int cb_n = cols / 128, rb_n = rows / 128;
   const int cb = (int)(tile % cb_n);
@@ -106,6 +108,8 @@ quantize_weights_mxfp8_kernel(const __nv_bfloat16* __restrict__ src, int rows, i
 __global__ void __launch_bounds__(256)
 gather_quant_kernel(const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ slot_pos,
                     int ntok, int K, int d, uint8_t* __restrict__ xq, uint8_t* __restrict__ xsf) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= ntok) return;

@@ -15,6 +15,8 @@ __global__ void __launch_bounds__(256)
 router_gemm_simt_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
                         const float* __restrict__ offset, float* __restrict__ logits, int T,
                         int E, int d) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float As[kRgBK][kRgBM + 4];
   __shared__ float Bs[kRgBK][kRgBN + 4];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -103,11 +105,14 @@ struct Top3 {
 
 template <int VPL>
 __global__ void __launch_bounds__(kRouteThreads)
-softmax_topk_kernel(const float* __restrict__ logits, const float* __restrict__ bias, int T,
-                    int E, int N, int K, int32_t* __restrict__ topk_idx,
+softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long split_stride,
+                    const float* __restrict__ bias, int T, int E, int N, int K,
+                    int32_t* __restrict__ topk_idx,
                     float* __restrict__ topk_gate, uint8_t* __restrict__ n_ffn,
                     float* __restrict__ probs_out, int32_t* __restrict__ partial_hist,
                     float* __restrict__ partial_psum) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int hist[kMaxExperts];
   __shared__ float psum_acc[kMaxExperts];
   float ps[VPL];  // this lane's running sums of R over the warp's tokens
@@ -125,7 +130,14 @@ softmax_topk_kernel(const float* __restrict__ logits, const float* __restrict__ 
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
       int e = lane + 32 * j;
-      p[j] = e < E ? lrow[e] : -INFINITY;
+      if (e < E) {
+        // split-K partial logits, summed in split order
+        float v = lrow[e];
+        for (int sp = 1; sp < nsplit; ++sp) v += lrow[sp * split_stride + e];
+        p[j] = v;
+      } else {
+        p[j] = -INFINITY;
+      }
       m = fmaxf(m, p[j]);
     }
 #pragma unroll
@@ -212,6 +224,8 @@ softmax_topk_kernel(const float* __restrict__ logits, const float* __restrict__ 
 __global__ void __launch_bounds__(256)
 reduce_psum_kernel(const float* __restrict__ partial, int nparts, int E,
                    float* __restrict__ prob_sum) {
+  pdl_trigger();
+  pdl_wait();
   const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (e >= E) return;
@@ -231,6 +245,8 @@ __global__ void __launch_bounds__(1024)
 lb_stats_kernel(int N, int Z, int D, const int32_t* __restrict__ counts,
                 const float* __restrict__ prob_sum, long long T, int K, float K_e, float alpha,
                 float* __restrict__ f_out, float* __restrict__ p_out, float* __restrict__ loss) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ double f_sh[kMaxExperts + 1], p_sh[kMaxExperts + 1];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const int G = N / D;
@@ -271,6 +287,8 @@ lb_stats_kernel(int N, int Z, int D, const int32_t* __restrict__ counts,
 __global__ void __launch_bounds__(256)
 reduce_hist_kernel(const int32_t* __restrict__ partial, int nparts, int E,
                    int32_t* __restrict__ counts) {
+  pdl_trigger();
+  pdl_wait();
   const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (e >= E) return;
