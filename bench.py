@@ -131,6 +131,7 @@ def run_gpu(args, rank, world, local_rank):
     # expert weights repacked once into the tiled order, or quantised to MXFP8
     # (untimed set-up); the row-major originals stay for the oracle baseline
     fp8 = args.fp8_experts
+    gather = args.fused_gather
     if fp8:
         W = {k: B.quantize_weights_mxfp8(L[k]) for k in ("w1", "w3", "w2")}
         fbuf = B.Mxfp8Buffers(shape, device=dev)
@@ -173,9 +174,13 @@ def run_gpu(args, rank, world, local_rank):
             B.expert_down_mxfp8(s, fbuf.h_q, fbuf.h_sf, W["w2"], buf.offsets, buf.y_perm, buf.ws)
         else:
             B.permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
-                      buf.x_perm, buf.ws)
+                      None if gather else buf.x_perm, buf.ws)
             if ev: ev[2].record(stream)
-            B.expert_gate_up(s, buf.x_perm, W["w1"], W["w3"], buf.offsets, buf.h, buf.ws)
+            if gather:
+                B.expert_gate_up_gather(s, x, buf.row_token, W["w1"], W["w3"], buf.offsets,
+                                        buf.h, buf.ws)
+            else:
+                B.expert_gate_up(s, buf.x_perm, W["w1"], W["w3"], buf.offsets, buf.h, buf.ws)
             if ev: ev[3].record(stream)
             B.expert_down(s, buf.h, W["w2"], buf.offsets, buf.y_perm, buf.ws)
         if ev: ev[4].record(stream)
@@ -281,8 +286,13 @@ def run_gpu(args, rank, world, local_rank):
                                     buf.ws)
             else:
                 B.permute(s, x_dev[j], buf.topk_idx, buf.counts, buf.offsets, buf.row_token,
-                          buf.slot_pos, buf.x_perm, buf.ws)
-                B.expert_gate_up(s, buf.x_perm, W["w1"], W["w3"], buf.offsets, buf.h, buf.ws)
+                          buf.slot_pos, None if gather else buf.x_perm, buf.ws)
+                if gather:
+                    B.expert_gate_up_gather(s, x_dev[j], buf.row_token, W["w1"], W["w3"],
+                                            buf.offsets, buf.h, buf.ws)
+                else:
+                    B.expert_gate_up(s, buf.x_perm, W["w1"], W["w3"], buf.offsets, buf.h,
+                                     buf.ws)
                 B.expert_down(s, buf.h, W["w2"], buf.offsets, buf.y_perm, buf.ws)
             B.combine(s, x_dev[j], buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos,
                       cfg.gamma, out_dev[j])
@@ -389,6 +399,7 @@ def run_gpu(args, rank, world, local_rank):
         "cuda_graph": graph is not None,
         "lb_stats": lb is not None,
         "expert_format": "mxfp8" if fp8 else cfg.dtype,
+        "dispatch": "fused into gate/up (row gather)" if gather else "x_perm copy",
         "clocks": clk,
     }
     if args.backward:
@@ -600,6 +611,9 @@ def main():
     ap.add_argument("--backward", action="store_true",
                     help="also time a training step (forward keeping pre-activations + "
                          "backward pass) and report it under \"training\"")
+    ap.add_argument("--fused-gather", action="store_true",
+                    help="no x_perm copy: the gate/up GEMM reads the token rows from x "
+                         "(moe_expert_gate_up_gather)")
     ap.add_argument("--graph", action="store_true",
                     help="replay one captured CUDA graph per step (single GPU)")
     args = ap.parse_args()
@@ -609,6 +623,8 @@ def main():
         ap.error("--graph is single-GPU only")
     if args.backward and args.fp8_experts:
         ap.error("--backward runs on bf16 experts")
+    if args.fused_gather and args.fp8_experts:
+        ap.error("--fused-gather is a bf16 path")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -139,12 +139,17 @@ int sm_count() {
 
 // --- launches ---------------------------------------------------------------
 
+// The last CTA reduces the partial histograms itself when the grid is this small.
+constexpr int kFusedReduceMaxCtas = 16;
+
 template <int VPL>
 void launch_topk(dim3 grid, cudaStream_t st, const float* logits, int nsplit, const float* bias,
                  int T, int E, int N, int K, int32_t* idx, float* gate, uint8_t* nffn,
-                 float* probs, int32_t* hist, float* psum) {
+                 float* probs, int32_t* hist, float* psum, unsigned int* ticket, int32_t* counts,
+                 float* prob_sum) {
   moe::launch_pdl(moe::softmax_topk_kernel<VPL>, dim3(grid), dim3(moe::kRouteThreads), 0, st,
-      logits, nsplit, (long long)T * E, bias, T, E, N, K, idx, gate, nffn, probs, hist, psum);
+      logits, nsplit, (long long)T * E, bias, T, E, N, K, idx, gate, nffn, probs, hist, psum,
+      ticket, counts, prob_sum);
 }
 
 template <typename T>
@@ -157,6 +162,7 @@ moe_status route_impl(const moe_shape& s, const void* x, const void* w, const fl
   int32_t* hist = at<int32_t>(ws, L.route_hist);
   float* psum = prob_sum ? at<float>(ws, L.route_psum) : nullptr;
   int nsplit = 1;
+  bool fused = false;
   if (s.T > 0) {
     if (s.dtype == MOE_BF16 && moe::tc::router_supported(s) &&
         reinterpret_cast<uintptr_t>(off) % 16 == 0) {
@@ -171,21 +177,26 @@ moe_status route_impl(const moe_shape& s, const void* x, const void* w, const fl
     }
     const int vpl = (E + 31) / 32;
     dim3 g(route_ctas(s));
-    if (vpl <= 1) launch_topk<1>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 2) launch_topk<2>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 3) launch_topk<3>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 4) launch_topk<4>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 8) launch_topk<8>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 16) launch_topk<16>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else if (vpl <= 24) launch_topk<24>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
-    else launch_topk<32>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum);
+    // small grid: partial histograms reduced by the last CTA (ticket in the status block)
+    fused = route_ctas(s) <= kFusedReduceMaxCtas;
+    unsigned int* ticket = fused ? at<unsigned int>(ws, L.status + 4) : nullptr;
+    if (vpl <= 1) launch_topk<1>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
+    else if (vpl <= 2) launch_topk<2>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
+    else if (vpl <= 3) launch_topk<3>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
+    else if (vpl <= 4) launch_topk<4>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
+    else if (vpl <= 8) launch_topk<8>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
+    else if (vpl <= 16) launch_topk<16>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
+    else if (vpl <= 24) launch_topk<24>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
+    else launch_topk<32>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
     MOE_TRY(check_launch("softmax/top-K"));
   }
-  moe::launch_pdl(moe::reduce_hist_kernel, dim3((E + 7) / 8), dim3(256), 0, st, hist, route_ctas(s), E, counts);
+  if (fused) return MOE_OK;  // counts (and prob_sum) written by the top-K kernel
+  moe::launch_pdl(moe::reduce_hist_kernel, dim3((E + 7) / 8), dim3(256), 0, st, hist,
+                  route_ctas(s), E, counts);
   MOE_TRY(check_launch("count reduce"));
   if (prob_sum) {
-    moe::launch_pdl(moe::reduce_psum_kernel, dim3((E + 7) / 8), dim3(256), 0, st, psum, s.T > 0 ? route_ctas(s) : 0, E,
-                                                        prob_sum);
+    moe::launch_pdl(moe::reduce_psum_kernel, dim3((E + 7) / 8), dim3(256), 0, st, psum,
+                    s.T > 0 ? route_ctas(s) : 0, E, prob_sum);
     MOE_TRY(check_launch("probability column sums"));
   }
   return MOE_OK;

@@ -110,7 +110,8 @@ softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long spli
                     int32_t* __restrict__ topk_idx,
                     float* __restrict__ topk_gate, uint8_t* __restrict__ n_ffn,
                     float* __restrict__ probs_out, int32_t* __restrict__ partial_hist,
-                    float* __restrict__ partial_psum) {
+                    float* __restrict__ partial_psum, unsigned int* ticket,
+                    int32_t* __restrict__ counts_out, float* __restrict__ psum_out) {
   pdl_trigger();
   pdl_wait();
   __shared__ int hist[kMaxExperts];
@@ -216,6 +217,37 @@ softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long spli
     }
     for (int e = threadIdx.x; e < E; e += blockDim.x)
       partial_psum[(size_t)blockIdx.x * E + e] = psum_acc[e];
+  }
+  if (ticket) {
+    // Small grids: the CTA that finishes last reduces the per-CTA partials
+    // (the reduce kernels' per-expert order, so the sums are the same bits),
+    // which saves their launch.  The ticket wraps back to 0 after the last CTA.
+    __shared__ unsigned int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicInc(ticket, gridDim.x - 1) == gridDim.x - 1;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      const int nparts = gridDim.x;
+      for (int e = warp; e < E; e += nwarps) {
+        int c = 0;
+        float q = 0.f;
+        for (int p = lane; p < nparts; p += 32) {
+          c += __ldcg(partial_hist + (size_t)p * E + e);
+          if (psum_out) q += __ldcg(partial_psum + (size_t)p * E + e);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          c += __shfl_xor_sync(0xffffffffu, c, o);
+          q += __shfl_xor_sync(0xffffffffu, q, o);
+        }
+        if (lane == 0) {
+          counts_out[e] = c;
+          if (psum_out) psum_out[e] = q;
+        }
+      }
+    }
   }
 }
 
