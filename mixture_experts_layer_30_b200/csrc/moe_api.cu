@@ -147,9 +147,14 @@ void launch_topk(dim3 grid, cudaStream_t st, const float* logits, int nsplit, co
                  int T, int E, int N, int K, int32_t* idx, float* gate, uint8_t* nffn,
                  float* probs, int32_t* hist, float* psum, unsigned int* ticket, int32_t* counts,
                  float* prob_sum) {
-  moe::launch_pdl(moe::softmax_topk_kernel<VPL>, dim3(grid), dim3(moe::kRouteThreads), 0, st,
-      logits, nsplit, (long long)T * E, bias, T, E, N, K, idx, gate, nffn, probs, hist, psum,
-      ticket, counts, prob_sum);
+  if (psum)
+    moe::launch_pdl(moe::softmax_topk_kernel<VPL, true>, dim3(grid), dim3(moe::kRouteThreads),
+                    0, st, logits, nsplit, (long long)T * E, bias, T, E, N, K, idx, gate, nffn,
+                    probs, hist, psum, ticket, counts, prob_sum);
+  else
+    moe::launch_pdl(moe::softmax_topk_kernel<VPL, false>, dim3(grid), dim3(moe::kRouteThreads),
+                    0, st, logits, nsplit, (long long)T * E, bias, T, E, N, K, idx, gate, nffn,
+                    probs, hist, psum, ticket, counts, prob_sum);
 }
 
 template <typename T>

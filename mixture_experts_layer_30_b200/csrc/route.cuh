@@ -103,8 +103,13 @@ struct Top3 {
   }
 };
 
-template <int VPL>
-__global__ void __launch_bounds__(kRouteThreads)
+// kPsum: also accumulate the column sums of R (per-lane registers over the
+// warp's tokens).  The biased scores are recomputed from R and the bias when a
+// lane's top-3 list is rebuilt instead of being kept in registers, so up to 24
+// scores per lane fit 64 registers and two CTAs share an SM (the LongCat shape,
+// 8192 tokens, then runs as one wave).
+template <int VPL, bool kPsum>
+__global__ void __launch_bounds__(kRouteThreads, (kPsum || VPL > 24) ? 1 : 2)
 softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long split_stride,
                     const float* __restrict__ bias, int T, int E, int N, int K,
                     int32_t* __restrict__ topk_idx,
@@ -116,9 +121,9 @@ softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long spli
   pdl_wait();
   __shared__ int hist[kMaxExperts];
   __shared__ float psum_acc[kMaxExperts];
-  float ps[VPL];  // this lane's running sums of R over the warp's tokens
+  float ps[kPsum ? VPL : 1];  // this lane's running sums of R over the warp's tokens
 #pragma unroll
-  for (int j = 0; j < VPL; ++j) ps[j] = 0.f;
+  for (int j = 0; j < (kPsum ? VPL : 1); ++j) ps[j] = 0.f;
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -126,7 +131,7 @@ softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long spli
   const int t_end = min(T, t_begin + kRouteTokensPerCta);
   for (int t = t_begin + warp; t < t_end; t += nwarps) {
     const float* lrow = logits + (size_t)t * E;
-    float p[VPL], s[VPL];
+    float p[VPL];
     float m = -INFINITY;
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
@@ -159,13 +164,10 @@ softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long spli
     for (int j = 0; j < VPL; ++j) {
       int e = lane + 32 * j;
       p[j] *= inv;                             // R_e
-      ps[j] += p[j];
+      if constexpr (kPsum) ps[j] += p[j];
       if (e < E) {
-        s[j] = p[j] + __ldg(bias + e);         // biased score, selection only
         if (probs_out) probs_out[(size_t)t * E + e] = p[j];
-        top.insert(s[j], p[j], j);
-      } else {
-        s[j] = -INFINITY;
+        top.insert(p[j] + __ldg(bias + e), p[j], j);  // biased score, selection only
       }
     }
     uint32_t taken = 0;
@@ -186,7 +188,8 @@ softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long spli
           // this lane's three best are used up: rebuild from what is left
 #pragma unroll
           for (int j = 0; j < VPL; ++j)
-            if (!(taken >> j & 1u) && lane + 32 * j < E) top.insert(s[j], p[j], j);
+            if (!(taken >> j & 1u) && lane + 32 * j < E)
+              top.insert(p[j] + __ldg(bias + lane + 32 * j), p[j], j);
         }
       }
       if (lane == 0) {
@@ -201,7 +204,7 @@ softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long spli
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     partial_hist[(size_t)blockIdx.x * E + e] = hist[e];
-  if (partial_psum) {
+  if (kPsum && partial_psum) {
     // column sums of R over the CTA's tokens, warps added in a fixed order
     for (int e = threadIdx.x; e < E; e += blockDim.x) psum_acc[e] = 0.f;
     __syncthreads();
@@ -210,7 +213,7 @@ softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long spli
 #pragma unroll
         for (int j = 0; j < VPL; ++j) {
           const int e = lane + 32 * j;
-          if (e < E) psum_acc[e] += ps[j];
+          if (e < E) psum_acc[e] += ps[kPsum ? j : 0];
         }
       }
       __syncthreads();
