@@ -296,3 +296,48 @@ def test_lb_statistics(cfg, D):
     np.testing.assert_allclose(loss.item(), orc.lb_loss(f_o, P_o, alpha), rtol=2e-5)
     # the groups partition all experts
     assert abs(Pg.sum().item() - 1.0) < 1e-4
+
+
+@pytest.mark.parametrize("cfg", [C.DECODE_T64, C.MID_BF16], ids=lambda c: c.name)
+def test_cuda_graph_replay_matches_eager(cfg):
+    """The layer captured once in a CUDA graph (programmatic dependent launches
+    become graph edges) and replayed on new inputs gives the eager results bit
+    for bit, bias update included."""
+    L = _cfg_inputs(cfg)
+    s = B.shape_of(cfg)
+    K_e, mu = float(np.float32(cfg.K_e)), float(np.float32(cfg.mu))
+    x_in = L["x"].clone()
+    bias_g = L["bias"].clone()
+    gbuf = B.LayerBuffers(s)
+
+    def step(buf, x, bias):
+        B.forward(buf, x, L["w_router"], L["w1"], L["w3"], L["w2"], bias, split_ffn=True)
+        B.bias_update(cfg.N, cfg.Z, buf.counts, cfg.T, cfg.K, K_e, mu, bias)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step(gbuf, x_in, bias_g)  # warm-up outside the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    bias_g.copy_(L["bias"])
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(gbuf, x_in, bias_g)
+    ebuf = B.LayerBuffers(s)
+    bias_e = L["bias"].clone()
+    gen = torch.Generator(device="cuda").manual_seed(77)
+    for it in range(3):
+        x_new = torch.randn(x_in.shape, generator=gen, device="cuda").to(x_in.dtype)
+        x_in.copy_(x_new)
+        graph.replay()
+        step(ebuf, x_new, bias_e)
+        torch.cuda.synchronize()
+        R = int(ebuf.offsets[-1].item())
+        assert torch.equal(gbuf.topk_idx, ebuf.topk_idx), it
+        assert torch.equal(gbuf.offsets, ebuf.offsets), it
+        assert torch.equal(gbuf.y_perm[:R], ebuf.y_perm[:R]), it
+        assert torch.equal(gbuf.out, ebuf.out), it
+        assert torch.equal(bias_g, bias_e), it
+    assert B.device_status(gbuf.ws) == 0 and B.device_status(ebuf.ws) == 0
+    del graph
