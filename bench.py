@@ -11,6 +11,11 @@ NCCL before the bias update, the one exchange step of the method.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
 oracle instead, on a bounded sample of the same workload.
+
+Options: --graph (replay one captured CUDA graph per step), --fp8-experts
+(MXFP8 expert weights), --fused-gather (no x_perm copy), --lb-stats (the
+load-balance statistics each step), --backward (also time a training step:
+forward keeping the pre-activations, then the backward pass).
 """
 import argparse
 import hashlib
@@ -48,9 +53,17 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_digest(path=TC_SOURCE):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def source_digest(path=TC_SOURCE, text=None):
+    """sha256 prefix of the GEMM source with comments and blank lines removed
+    (a comment edit does not invalidate counters taken on the same code)."""
+    import re
+    if text is None:
+        with open(path) as f:
+            text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def committed_traffic(kernel, workload):

@@ -22,6 +22,15 @@
 //               D1 = W3 rows f0..f0+127, out h = SiLU(D0) * D1 (bf16)
 //   plain modes (second half, router): D0 = rows f0..f0+127, D1 = rows
 //               f0+128..f0+255 of one weight matrix; out bf16 or fp32 (+offset)
+//   gated-save  (training forward): h as the gated mode, plus a = D0, u = D1
+//   SwiGLU backward: D0 | D1 = dh; epilogue da = dh u SiLU'(a), du = dh SiLU(a)
+// MN-major A (template flag, the backward's data gradients and the router's
+// input gradient): the weights are read in their stored order with the output
+// features as their columns -- 64 x 64 TMA boxes and the transpose bit of the
+// instruction descriptor instead of a transposed copy -- and the reduction may
+// switch from tmA0 to tmA1 part-way (dx = da W1 + du W3 in one accumulator).
+// Split-K (the router at small batches): K-block ranges on separate CTAs write
+// fp32 partial sums that the consumer adds in a fixed order.
 #pragma once
 
 #include <cuda.h>
