@@ -194,6 +194,21 @@ def test_single_ffn_expert_top1(dtype):
     _run_and_check(shape, dtype, L, 1, 1)
 
 
+@pytest.mark.parametrize("mode", ["split", "ffn", "gather"])
+def test_bf16_cuda_core_fallback(mode):
+    """bf16 shapes the tensor-core kernels do not take (d = 72, I = 40: not
+    multiples of 64) run the CUDA-core router and grouped GEMMs."""
+    shape, L = _small(130, 72, 9, 3, 3, 40, "bf16", seed=23)
+    _run_and_check(shape, "bf16", L, 9, 3, split_ffn=mode == "split",
+                   fused_gather=mode == "gather")
+
+
+def test_bf16_router_fallback_odd_expert_count():
+    """E = 13 (not a multiple of 8): the CUDA-core router, tensor-core experts."""
+    shape, L = _small(200, 128, 9, 4, 3, 64, "bf16", seed=24)
+    _run_and_check(shape, "bf16", L, 9, 3, split_ffn=True)
+
+
 def test_empty_batch():
     shape, L = _small(0, 64, 6, 2, 2, 64, "f32", seed=1)
     L["x"] = torch.empty((0, 64), device="cuda")
