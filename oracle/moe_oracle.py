@@ -302,10 +302,27 @@ def expert_backward(x_rows, w1, w3, w2, dy):
     return da @ w1 + du @ w3, da.T @ x_rows, du.T @ x_rows, dy.T @ h
 
 
+def lb_prob_gradient(f, N, D, E, T, alpha):
+    """dL_LB / dR_{t,i} of L_LB = alpha sum_j f_j P_j (Eq. (3)-(5)) with the
+    selection frequencies f_j held fixed: P_j is linear in R with weight 1/T on
+    the members of group j, so every token gets alpha f_{group(i)} / T on
+    expert i.  Returns the [E] row shared by all tokens."""
+    G = N // D
+    c = np.empty(E)
+    for i in range(E):
+        j = i // G if i < N else D
+        c[i] = float(alpha) * f[j] / T
+    return c
+
+
 def moe_layer_backward(x, w_router, w1, w3, w2, bias, N, K, dout, gamma=1.0,
-                       logit_offset=None, decode=as_f64, selection=None):
+                       logit_offset=None, decode=as_f64, selection=None, lb=None):
     """Forward intermediates plus dx, dw_router, dw1, dw3, dw2 (all float64)
-    and the per-slot dgate [T, K] and dy_perm [R, d]."""
+    and the per-slot dgate [T, K] and dy_perm [R, d].
+
+    lb = (D, K_e, alpha): the gradient also includes the device-level
+    load-balance loss alpha sum_j f_j P_j of Eq. (3)-(5) (f from this step's
+    selections, held fixed); f, P and L_LB are returned as lb_f, lb_P, lb_loss."""
     f = moe_layer(x, w_router, w1, w3, w2, bias, N, K, gamma, logit_offset, decode, selection)
     x = as_f64(x)
     dout = as_f64(dout)
@@ -345,6 +362,11 @@ def moe_layer_backward(x, w_router, w1, w3, w2, bias, N, K, dout, gamma=1.0,
     # router
     dR = np.zeros((T, E))
     np.put_along_axis(dR, idx.astype(np.int64), dgate, axis=1)
+    if lb is not None:
+        D, K_e, alpha = lb
+        lf, lP = lb_statistics(probs, idx, N, D, K, K_e)
+        dR += lb_prob_gradient(lf, N, D, E, T, alpha)[None, :]
+        f.update(lb_f=lf, lb_P=lP, lb_loss=lb_loss(lf, lP, alpha))
     dlogits = softmax_backward(probs, dR)
     wr = as_f64(w_router)
     dx += dlogits @ wr

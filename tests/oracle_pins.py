@@ -482,7 +482,42 @@ def check_backward_against_autograd(orc, seed=11):
                                    err_msg=name)
 
 
-ALL_CHECKS = [check_backward_finite_differences, check_backward_against_autograd, check_e4m3_table, check_e4m3_rounding_brute_force,
+def check_lb_backward_finite_differences(orc, seed=12):
+    """With the load-balance loss: central differences of
+    <dout, out> + alpha sum_j f_j P_j (f from the selection, which no small step
+    changes) against dx and dW_r; the expert weights do not enter L_LB."""
+    rng = np.random.default_rng(seed)
+    T, d, N, Z, K, I, gamma = 6, 4, 4, 2, 3, 3, 1.0
+    D, K_e, alpha = 2, 2.0, 0.7
+    L = _rand_layer(rng, T, d, N, Z, I, 0.2)
+    dout = rng.normal(size=(T, d))
+    r = orc.moe_layer_backward(L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"],
+                               N=N, K=K, dout=dout, gamma=gamma, lb=(D, K_e, alpha))
+    assert r["margin"].min() > 1e-4
+    base = orc.moe_layer_backward(L["x"], L["w_router"], L["w1"], L["w3"], L["w2"],
+                                  L["bias"], N=N, K=K, dout=dout, gamma=gamma)
+    # the aux loss moves the router's gradients and leaves the expert weights' alone
+    assert not np.allclose(r["dw_router"], base["dw_router"])
+    np.testing.assert_array_equal(r["dw1"], base["dw1"])
+
+    def total(LL):
+        f = orc.moe_layer(LL["x"], LL["w_router"], LL["w1"], LL["w3"], LL["w2"], LL["bias"],
+                          N=N, K=K, gamma=gamma)
+        lf, lP = orc.lb_statistics(f["probs"], f["idx"], N, D, K, K_e)
+        return float((f["out"] * dout).sum()) + orc.lb_loss(lf, lP, alpha)
+    eps = 1e-6
+    for name, grad in (("x", "dx"), ("w_router", "dw_router")):
+        b0 = L[name]
+        fd = np.zeros_like(b0)
+        for ix in np.ndindex(b0.shape):
+            Lp = dict(L); Lm = dict(L)
+            Lp[name] = b0.copy(); Lp[name][ix] += eps
+            Lm[name] = b0.copy(); Lm[name][ix] -= eps
+            fd[ix] = (total(Lp) - total(Lm)) / (2 * eps)
+        np.testing.assert_allclose(r[grad], fd, rtol=1e-5, atol=1e-7, err_msg=name)
+
+
+ALL_CHECKS = [check_lb_backward_finite_differences, check_backward_finite_differences, check_backward_against_autograd, check_e4m3_table, check_e4m3_rounding_brute_force,
               check_mxfp8_block_quantization, check_worked_tiny_layer, check_worked_swiglu, check_worked_bias_update,
               check_worked_zero_experts, check_softmax_closed_forms, check_topk_brute_force,
               check_dense_reduction, check_all_zero_experts_fixed_point,

@@ -169,11 +169,19 @@ def _mut_silu_derivative_sigma_only(mp):
     mp.setattr(orc, "expert_backward", expert_backward)
 
 
+def _mut_lb_gradient_without_frequency(mp):
+    """The aux-loss gradient taken as alpha/T, dropping the f_j weight."""
+    def lb_prob_gradient(f, N, D, E, T, alpha):
+        return np.full(E, float(alpha) / T)
+    mp.setattr(orc, "lb_prob_gradient", lb_prob_gradient)
+
+
 def _mut_softmax_backward_no_centering(mp):
     mp.setattr(orc, "softmax_backward", lambda probs, dR: probs * dR)
 
 
-MUTATIONS = [_mut_silu_derivative_sigma_only, _mut_softmax_backward_no_centering,
+MUTATIONS = [_mut_lb_gradient_without_frequency, _mut_silu_derivative_sigma_only,
+             _mut_softmax_backward_no_centering,
              _mut_e4m3_ties_away, _mut_mx_scale_off_by_one, _mut_lb_indicator_per_token, _mut_lb_zero_group_normaliser, _mut_gate_renormalised, _mut_combine_drops_zero_term, _mut_bias_sign,
              _mut_bias_updates_zero_experts, _mut_tie_to_high_index, _mut_select_by_unbiased,
              _mut_no_silu, _mut_swapped_gate_up, _mut_descending_tokens,
