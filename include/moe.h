@@ -326,11 +326,19 @@ moe_status moe_combine_backward(const moe_shape* shape, const void* x, const voi
  *   dw_router     = dlogits^T x          [E, d] (dtype)
  *   dx_router     = dlogits w_router     [T, d] fp32
  * probs [T, E] fp32 are the forward probabilities (moe_route's probs_out).
- * dlogits is kept in the backward workspace (bf16 for MOE_BF16). */
+ * dlogits is kept in the backward workspace (bf16 for MOE_BF16).
+ * Load-balance loss (§2.1.2, Eq. (3)-(5)), optional: with lb_f [D+1] fp32 the
+ * f_j of moe_lb_stats (held fixed: they count selections), lb_groups = D and
+ * lb_alpha = alpha, the gradient of alpha sum_j f_j P_j is added,
+ *   dR[t, i] += lb_alpha * lb_f[group(i)] / lb_tokens   for every t and i,
+ * group(i) = i / (N/D) for FFN experts and D for the zero experts; lb_tokens
+ * is the token count P_j averages over (T, or the global batch with token
+ * data parallelism).  lb_f NULL: no load-balance term. */
 moe_status moe_route_backward(const moe_shape* shape, const void* x, const void* w_router,
                               const float* probs, const int32_t* topk_idx, const float* dgate,
-                              void* dw_router, float* dx_router, void* ws, size_t ws_bytes,
-                              void* stream);
+                              const float* lb_f, int32_t lb_groups, float lb_alpha,
+                              int64_t lb_tokens, void* dw_router, float* dx_router, void* ws,
+                              size_t ws_bytes, void* stream);
 
 /* Backward of the SwiGLU experts over the routed rows (per expert segment):
  *   dh = dy_perm W2_e;  da = dh u SiLU'(a);  du = dh SiLU(a)   (kept in the

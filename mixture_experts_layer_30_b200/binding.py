@@ -60,7 +60,8 @@ SIGNATURES = {
     "moe_expert_gate_up_save": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_combine_backward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp,
                                             _vp]),
-    "moe_route_backward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_route_backward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _f32, _i64,
+                                          _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_ffn_backward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                                _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_backward": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp]),
@@ -426,14 +427,18 @@ def combine_backward(shape, x, y_perm, topk_idx, topk_gate, slot_pos, dout, gamm
 
 
 def route_backward(shape, x, w_router, probs, topk_idx, dgate, dw_router, dx_router, bws,
-                   stream=None):
+                   lb=None, stream=None):
+    """lb = (f, D, alpha, tokens): add the load-balance loss gradient (f [D+1]
+    from lb_stats)."""
     dt = torch_dtype(shape)
+    lb_f, lb_D, lb_alpha, lb_T = lb if lb is not None else (None, 0, 0.0, 0)
     _check(lib().moe_route_backward(ctypes.byref(shape), _p(x, dt, "x"),
                                     _p(w_router, dt, "w_router"),
                                     _p(probs, torch.float32, "probs"),
                                     _p(topk_idx, torch.int32, "topk_idx"),
                                     _p(dgate, torch.float32, "dgate"),
-                                    _p(dw_router, dt, "dw_router"),
+                                    _p(lb_f, torch.float32, "lb_f"), int(lb_D), float(lb_alpha),
+                                    int(lb_T), _p(dw_router, dt, "dw_router"),
                                     _p(dx_router, torch.float32, "dx_router"), _p(bws),
                                     bws.numel(), _stream(stream)))
 
@@ -483,14 +488,15 @@ class BackwardBuffers:
 
 
 def forward_train(buf: LayerBuffers, bb: BackwardBuffers, x, w_router, w1, w3, w2, bias,
-                  gamma=1.0, logit_offset=None, stream=None):
+                  gamma=1.0, logit_offset=None, prob_sum=None, stream=None):
     """The forward pass keeping what the backward pass needs (probs, x_perm,
-    h, and the pre-activations a | u in bb.au); returns buf.out."""
+    h, and the pre-activations a | u in bb.au); returns buf.out.  prob_sum [E]:
+    also the probability column sums for lb_stats."""
     s = buf.shape
     if buf.probs is None:
         raise ValueError("forward_train needs LayerBuffers(with_probs=True)")
     route(s, x, w_router, bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts, buf.n_ffn,
-          logit_offset=logit_offset, probs_out=buf.probs, stream=stream)
+          logit_offset=logit_offset, probs_out=buf.probs, prob_sum=prob_sum, stream=stream)
     permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
             buf.x_perm, buf.ws, stream=stream)
     expert_gate_up_save(s, buf.x_perm, w1, w3, buf.offsets, buf.h, bb.au, buf.ws, stream=stream)
@@ -501,14 +507,15 @@ def forward_train(buf: LayerBuffers, bb: BackwardBuffers, x, w_router, w1, w3, w
 
 
 def backward(buf: LayerBuffers, bb: BackwardBuffers, x, w_router, w1, w3, w2, dout, gamma=1.0,
-             stream=None):
+             lb=None, stream=None):
     """Gradients of the layer for upstream gradient dout, after forward_train:
-    bb.dx, bb.dw_router, bb.dw1, bb.dw3, bb.dw2 (the selection held fixed)."""
+    bb.dx, bb.dw_router, bb.dw1, bb.dw3, bb.dw2 (the selection held fixed);
+    lb = (f, D, alpha, tokens) adds the load-balance loss."""
     s = buf.shape
     combine_backward(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, dout, gamma,
                      bb.dy_perm, bb.dgate, stream=stream)
     route_backward(s, x, w_router, buf.probs, buf.topk_idx, bb.dgate, bb.dw_router,
-                   bb.dx_router, bb.bws, stream=stream)
+                   bb.dx_router, bb.bws, lb=lb, stream=stream)
     expert_ffn_backward(s, buf.x_perm, w1, w3, w2, buf.offsets, buf.h, bb.au, bb.dy_perm,
                         bb.dx_perm, bb.dw1, bb.dw3, bb.dw2, bb.bws, stream=stream)
     permute_backward(s, dout, buf.topk_idx, buf.topk_gate, buf.slot_pos, bb.dx_perm,

@@ -146,15 +146,18 @@ combine_backward_kernel(const T* __restrict__ x, const T* __restrict__ y_perm,
   }
 }
 
-// dlogits[t, i] = R[t, i] * (dR[t, i] - s_t),  s_t = sum_k R[t, idx_k] dgate[t, k]
-// (k order per lane, then the fixed shuffle tree).  One warp per token; dR is
-// scattered into a per-warp shared row.  Written as TOut (bf16 operand of the
-// tensor-core router GEMMs, or fp32).
+// dlogits[t, i] = R[t, i] * (dR[t, i] - s_t),  s_t = sum_i R[t, i] dR[t, i],
+// dR[t, idx_k] = dgate[t, k], plus -- with the load-balance loss of Eq. (3)-(5)
+// -- c_i = lb_scale * lb_f[group(i)] on every expert (group(i) = i / G for
+// i < N, D for the zero experts).  s_t sums the selected slots (k order per
+// lane, then the fixed shuffle tree) and then adds sum_i R c (lane-strided,
+// fixed tree).  One warp per token; dR is scattered into a per-warp shared row.
+// Written as TOut (bf16 operand of the tensor-core router GEMMs, or fp32).
 template <typename TOut>
 __global__ void __launch_bounds__(256)
 dlogits_kernel(const float* __restrict__ probs, const int32_t* __restrict__ topk_idx,
-               const float* __restrict__ dgate, int T, int E, int K, TOut* __restrict__ dlogits,
-               uint32_t* status) {
+               const float* __restrict__ dgate, int T, int E, int K, const float* __restrict__ lb_f,
+               int N, int G, int D, float lb_scale, TOut* __restrict__ dlogits, uint32_t* status) {
   pdl_trigger();
   pdl_wait();
   __shared__ float s_dR[8][kMaxExperts];
@@ -177,6 +180,16 @@ dlogits_kernel(const float* __restrict__ probs, const int32_t* __restrict__ topk
     }
   }
   s = warp_sum_fixed(s);
+  if (lb_f) {
+    __syncwarp();  // the scattered dR entries of other lanes are visible
+    float s2 = 0.f;
+    for (int i = lane; i < E; i += 32) {
+      const float c = lb_scale * __ldg(lb_f + (i < N ? i / G : D));
+      dR[i] += c;  // each lane owns entries i = lane + 32 m
+      s2 = fmaf(p[i], c, s2);
+    }
+    s += warp_sum_fixed(s2);
+  }
   __syncwarp();
   for (int i = lane; i < E; i += 32)
     dlogits[(size_t)t * E + i] = Cvt<TOut>::from_f(p[i] * (dR[i] - s));

@@ -878,8 +878,9 @@ moe_status moe_combine_backward(const moe_shape* shape, const void* x, const voi
 
 moe_status moe_route_backward(const moe_shape* shape, const void* x, const void* w_router,
                               const float* probs, const int32_t* topk_idx, const float* dgate,
-                              void* dw_router, float* dx_router, void* ws, size_t ws_bytes,
-                              void* stream) {
+                              const float* lb_f, int32_t lb_groups, float lb_alpha,
+                              int64_t lb_tokens, void* dw_router, float* dx_router, void* ws,
+                              size_t ws_bytes, void* stream) {
   g_err[0] = 0;
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
@@ -901,12 +902,23 @@ moe_status moe_route_backward(const moe_shape* shape, const void* x, const void*
   MOE_TRY(need(topk_idx, "topk_idx", 4));
   MOE_TRY(need(dgate, "dgate", 4));
   MOE_TRY(need(dx_router, "dx_router", 16));
+  int lb_G = 1;
+  float lb_scale = 0.f;
+  if (lb_f) {
+    MOE_TRY(need(lb_f, "lb_f", 4));
+    if (lb_groups < 1 || s.N % lb_groups)
+      return fail(MOE_ERR_INVALID_ARG, "lb_groups=%d must divide N=%d", lb_groups, s.N);
+    if (lb_tokens < 1) return fail(MOE_ERR_INVALID_ARG, "lb_tokens=%lld", (long long)lb_tokens);
+    lb_G = s.N / lb_groups;
+    lb_scale = (float)((double)lb_alpha / (double)lb_tokens);
+  }
   uint32_t* status = at<uint32_t>(ws, L.status);
   void* dlogits = at<char>(ws, L.dlogits);
   const int sms = sm_count();
   if (s.dtype == MOE_BF16) {
     moe::launch_pdl(moe::dlogits_kernel<__nv_bfloat16>, dim3((s.T + 7) / 8), dim3(256), 0, st,
-        probs, topk_idx, dgate, s.T, E, s.K, static_cast<__nv_bfloat16*>(dlogits), status);
+        probs, topk_idx, dgate, s.T, E, s.K, lb_f, s.N, lb_G, lb_groups, lb_scale,
+      static_cast<__nv_bfloat16*>(dlogits), status);
     MOE_TRY(check_launch("router logit gradient"));
     MOE_TRY(moe::tc::launch_router_wgrad(s, dlogits, x, dw_router, status, sms, st, g_err,
                                          sizeof(g_err)));
@@ -914,7 +926,8 @@ moe_status moe_route_backward(const moe_shape* shape, const void* x, const void*
                                      sizeof(g_err));
   }
   moe::launch_pdl(moe::dlogits_kernel<float>, dim3((s.T + 7) / 8), dim3(256), 0, st,
-      probs, topk_idx, dgate, s.T, E, s.K, static_cast<float*>(dlogits), status);
+      probs, topk_idx, dgate, s.T, E, s.K, lb_f, s.N, lb_G, lb_groups, lb_scale,
+      static_cast<float*>(dlogits), status);
   MOE_TRY(check_launch("router logit gradient"));
   moe::SimtBwdArgs a{};
   // dW_r[i, j] = sum_t dlogits[t, i] x[t, j]

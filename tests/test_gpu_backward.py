@@ -46,15 +46,27 @@ def _dout(shape, seed):
     return torch.randn((shape.T, shape.d), generator=g).to(dt).cuda()
 
 
-def train_step(shape, L, dout, gamma=1.0):
-    """forward_train + backward through the C ABI; returns (buf, bb)."""
+def train_step(shape, L, dout, gamma=1.0, lb=None):
+    """forward_train + backward through the C ABI; returns (buf, bb).
+    lb = (D, K_e, alpha): the load-balance loss joins the backward, with f from
+    moe_lb_stats on this step's counts and probability sums."""
     buf = B.LayerBuffers(shape, with_probs=True)
     bb = B.BackwardBuffers(shape)
     w1, w3, w2 = L["w1"], L["w3"], L["w2"]
     if shape.weight_layout == B.WEIGHTS_TILED:
         w1, w3, w2 = B.pack_weights(w1), B.pack_weights(w3), B.pack_weights(w2)
-    B.forward_train(buf, bb, L["x"], L["w_router"], w1, w3, w2, L["bias"], gamma=gamma)
-    B.backward(buf, bb, L["x"], L["w_router"], w1, w3, w2, dout, gamma=gamma)
+    E = shape.N + shape.Z
+    prob_sum = torch.empty(E, dtype=torch.float32, device="cuda") if lb else None
+    B.forward_train(buf, bb, L["x"], L["w_router"], w1, w3, w2, L["bias"], gamma=gamma,
+                    prob_sum=prob_sum)
+    lb_arg = None
+    if lb:
+        D, K_e, alpha = lb
+        f = torch.empty(D + 1, dtype=torch.float32, device="cuda")
+        P = torch.empty(D + 1, dtype=torch.float32, device="cuda")
+        B.lb_stats(shape.N, shape.Z, D, buf.counts, prob_sum, shape.T, shape.K, K_e, alpha, f, P)
+        lb_arg = (f, D, alpha, shape.T)
+    B.backward(buf, bb, L["x"], L["w_router"], w1, w3, w2, dout, gamma=gamma, lb=lb_arg)
     torch.cuda.synchronize()
     assert B.device_status(buf.ws) == 0
     assert B.device_status(bb.bws) == 0
@@ -72,16 +84,16 @@ def _host_forward(buf):
                 y_perm=P.to_f64(b.y_perm[:R]), out=P.to_f64(b.out), R=R)
 
 
-def check_backward(shape, dtype, L, N, K, gamma=1.0, seed=0):
+def check_backward(shape, dtype, L, N, K, gamma=1.0, seed=0, lb=None):
     dout = _dout(shape, 5000 + seed)
-    buf, bb = train_step(shape, L, dout, gamma)
+    buf, bb = train_step(shape, L, dout, gamma, lb=lb)
     g = _host_forward(buf)
     x64, wr64 = P.to_f64(L["x"]), P.to_f64(L["w_router"])
     idx_ref, _, _ = P.check_routing_and_dispatch(g, x64, wr64, L["bias"], N, K)
     ref = orc.moe_layer_backward(x64, wr64, L["w1"], L["w3"], L["w2"],
                                  L["bias"].cpu().numpy().astype(np.float64), N, K,
                                  P.to_f64(dout), gamma=gamma, decode=P.to_f64,
-                                 selection=idx_ref)
+                                 selection=idx_ref, lb=lb)
     R = g["R"]
     P.assert_close(g["y_perm"], ref["y_perm"], dtype, "y_perm")
     # the kept pre-activations a | u
@@ -244,3 +256,27 @@ def test_backward_empty_batch(dtype):
     assert B.device_status(buf.ws) == 0 and B.device_status(bb.bws) == 0
     for t in (bb.dw1, bb.dw3, bb.dw2, bb.dw_router):
         assert not t.any()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_backward_with_load_balance_loss(dtype):
+    """The load-balance loss alpha sum_j f_j P_j (Eq. (3)-(5)) in the router's
+    gradient: f from moe_lb_stats on the GPU, the oracle's own f from the same
+    selection; alpha is large enough that the term moves dW_r and dx."""
+    N, Z, K, D = 16, 8, 4, 4
+    K_e = float(np.float32(K * N / (N + Z)))
+    shape, L = _small(300, 256, N, Z, K, 128, dtype, seed=66)
+    check_backward(shape, dtype, L, N, K, seed=66, lb=(D, K_e, 5.0))
+
+
+def test_backward_load_balance_term_changes_only_the_router_gradients():
+    N, Z, K, D = 16, 8, 4, 4
+    K_e = float(np.float32(K * N / (N + Z)))
+    shape, L = _small(200, 256, N, Z, K, 128, "bf16", seed=67)
+    dout = _dout(shape, 67)
+    _, b0 = train_step(shape, L, dout)
+    _, b1 = train_step(shape, L, dout, lb=(D, K_e, 5.0))
+    for name in ("dw1", "dw3", "dw2", "dy_perm", "dgate"):
+        assert torch.equal(getattr(b0, name), getattr(b1, name)), name
+    assert not torch.equal(b0.dw_router, b1.dw_router)
+    assert not torch.equal(b0.dx, b1.dx)

@@ -134,8 +134,8 @@ def test_backward_validation(lib):
         assert lib.moe_expert_ffn_backward(ctypes.byref(bad), fake, fake, fake, fake, fake, fake,
                                            fake, fake, fake, fake, fake, fake, fake, nbb,
                                            None) == 2
-        assert lib.moe_route_backward(ctypes.byref(bad), fake, fake, fake, fake, fake, fake,
-                                      fake, fake, nbb, None) == 2
+        assert lib.moe_route_backward(ctypes.byref(bad), fake, fake, fake, fake, fake, None, 0,
+                                      0.0, 0, fake, fake, fake, nbb, None) == 2
     # workspace too small, NULL operand
     assert lib.moe_expert_ffn_backward(ctypes.byref(s), fake, fake, fake, fake, fake, fake, fake,
                                        fake, fake, fake, fake, fake, fake, nb - 256, None) == 3
@@ -150,3 +150,15 @@ def test_backward_validation(lib):
     assert b"dx_router" in lib.moe_last_error()
     assert lib.moe_expert_gate_up_save(ctypes.byref(s), fake, fake, fake, fake, fake, None,
                                        fake, B.workspace_bytes(s), None) == 1
+
+
+def test_route_backward_lb_validation(lib):
+    fake = ctypes.c_void_p(0x10000)
+    s = B.make_shape(64, 256, 12, 4, 4, 128, "bf16")
+    nb = lib.moe_backward_workspace_bytes(ctypes.byref(s))
+    # lb_groups must divide N, lb_tokens >= 1
+    assert lib.moe_route_backward(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 5, 0.01,
+                                  64, fake, fake, fake, nb, None) == 1
+    assert b"lb_groups" in lib.moe_last_error()
+    assert lib.moe_route_backward(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 4, 0.01,
+                                  0, fake, fake, fake, nb, None) == 1
