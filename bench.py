@@ -336,6 +336,23 @@ def run_gpu(args, rank, world, local_rank):
     if st:
         raise RuntimeError(f"device status 0x{st:x} after timing")
 
+    # ---- silent-data-corruption check: one step recomputed bit for bit ----
+    # The layer is deterministic (fixed reduction orders, no atomics in any sum),
+    # so the same step from the same bias and input must repeat exactly.
+    bias_saved = bias.clone()
+    step(x)
+    ref_out, ref_idx, ref_counts = buf.out.clone(), buf.topk_idx.clone(), buf.counts.clone()
+    bias.copy_(bias_saved)
+    step(x)
+    barrier()
+    sdc_equal = bool(torch.equal(ref_out, buf.out) and torch.equal(ref_idx, buf.topk_idx)
+                     and torch.equal(ref_counts, buf.counts))
+    n_ffn = buf.n_ffn.float()
+    load = buf.counts[:cfg.N].float()
+    routing_stats = {"ffn_experts_per_token_mean": round(float(n_ffn.mean()), 4),
+                     "ffn_experts_per_token_std": round(float(n_ffn.std()), 4),
+                     "max_over_mean_expert_load": round(float(load.max() / load.mean()), 4)}
+
     # ---- algorithmic work of the routed batch (counts of the last step) ----
     counts = buf.counts.cpu().numpy().astype(np.int64)
     R = int(counts[:cfg.N].sum())
@@ -409,6 +426,9 @@ def run_gpu(args, rank, world, local_rank):
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(buf.out.numel() * buf.out.element_size())},
         "gpu_launches": int(launches),
+        "routing": routing_stats,
+        "sdc_check": {"bitwise_equal": sdc_equal,
+                      "method": "one step recomputed from the same bias and input"},
         "cuda_graph": graph is not None,
         "lb_stats": lb is not None,
         "expert_format": "mxfp8" if fp8 else cfg.dtype,

@@ -7,6 +7,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "moe.h"
 #include "common.cuh"
 #include "route.cuh"
@@ -23,6 +25,15 @@
 namespace {
 
 thread_local char g_err[512] = "";
+
+// NVTX range over one C-ABI call (the enqueue on the host; profilers place the
+// call's kernels under it).  Header-only NVTX: a no-op unless a tool is attached.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 moe_status fail(moe_status st, const char* fmt, ...) {
   va_list ap;
@@ -431,6 +442,7 @@ size_t moe_workspace_bytes(const moe_shape* shape) {
 moe_status moe_pack_weights(int32_t n_mats, int32_t rows, int32_t cols, int32_t dtype,
                             const void* src, void* dst, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_pack_weights");
   if (dtype != MOE_BF16) return fail(MOE_ERR_UNSUPPORTED, "moe_pack_weights packs bf16 only");
   if (n_mats < 0 || rows < 0 || cols < 0 || rows % 128 || cols % 64)
     return fail(MOE_ERR_INVALID_ARG,
@@ -453,6 +465,7 @@ moe_status moe_pack_weights(int32_t n_mats, int32_t rows, int32_t cols, int32_t 
 moe_status moe_quantize_weights_mxfp8(int32_t n_mats, int32_t rows, int32_t cols,
                                       const void* src, void* dst_q, void* dst_sf, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_quantize_weights_mxfp8");
   if (n_mats < 0 || rows < 0 || cols < 0 || rows % 128 || cols % 128)
     return fail(MOE_ERR_INVALID_ARG,
                 "moe_quantize_weights_mxfp8: rows=%d and cols=%d must be multiples of 128", rows,
@@ -471,6 +484,7 @@ moe_status moe_quantize_weights_mxfp8(int32_t n_mats, int32_t rows, int32_t cols
 
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_workspace_init");
   if (!ws || ws_bytes < 256) return fail(MOE_ERR_INVALID_ARG, "workspace NULL or < 256 bytes");
   cudaError_t e = cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
@@ -482,6 +496,7 @@ moe_status moe_route(const moe_shape* shape, const void* x, const void* w_router
                      float* topk_gate, int32_t* counts, uint8_t* n_ffn, float* probs_out,
                      float* prob_sum, void* ws, size_t ws_bytes, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_route");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   WsLayout L;
@@ -508,6 +523,7 @@ moe_status moe_permute(const moe_shape* shape, const void* x, const int32_t* top
                        int32_t* slot_pos, void* x_perm, void* ws, size_t ws_bytes,
                        void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_permute");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   WsLayout L;
@@ -534,6 +550,7 @@ moe_status moe_permute_noalloc(const moe_shape* shape, const void* x, const int3
                                const int32_t* counts, int32_t* offsets, int32_t* row_token,
                                int32_t* slot_pos, void* x_perm, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_permute_noalloc");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   MOE_TRY(need(offsets, "offsets", 4));
@@ -580,6 +597,7 @@ moe_status moe_permute_mxfp8(const moe_shape* shape, const void* x, const int32_
                              int32_t* slot_pos, void* x_perm_q, void* x_perm_sf, void* ws,
                              size_t ws_bytes, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_permute_mxfp8");
   MOE_TRY(check_mxfp8_shape(shape));
   const moe_shape& s = *shape;
   WsLayout L;
@@ -611,6 +629,7 @@ moe_status moe_expert_gate_up_mxfp8(const moe_shape* shape, const void* x_perm_q
                                     void* h_q, void* h_sf, void* ws, size_t ws_bytes,
                                     void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_expert_gate_up_mxfp8");
   MOE_TRY(check_mxfp8_shape(shape));
   const moe_shape& s = *shape;
   WsLayout L;
@@ -634,6 +653,7 @@ moe_status moe_expert_down_mxfp8(const moe_shape* shape, const void* h_q, const 
                                  const void* w2_q, const void* w2_sf, const int32_t* offsets,
                                  void* y_perm, void* ws, size_t ws_bytes, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_expert_down_mxfp8");
   MOE_TRY(check_mxfp8_shape(shape));
   const moe_shape& s = *shape;
   WsLayout L;
@@ -654,6 +674,7 @@ moe_status moe_expert_gate_up(const moe_shape* shape, const void* x_perm, const 
                               const void* w3, const int32_t* offsets, void* h, void* ws,
                               size_t ws_bytes, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_expert_gate_up");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   WsLayout L;
@@ -672,6 +693,7 @@ moe_status moe_expert_gate_up_gather(const moe_shape* shape, const void* x,
                                      const int32_t* offsets, void* h, void* ws, size_t ws_bytes,
                                      void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_expert_gate_up_gather");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   WsLayout L;
@@ -690,6 +712,7 @@ moe_status moe_expert_down(const moe_shape* shape, const void* h, const void* w2
                            const int32_t* offsets, void* y_perm, void* ws, size_t ws_bytes,
                            void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_expert_down");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   WsLayout L;
@@ -706,6 +729,7 @@ moe_status moe_expert_ffn(const moe_shape* shape, const void* x_perm, const void
                           const void* w3, const void* w2, const int32_t* offsets,
                           void* y_perm, void* ws, size_t ws_bytes, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_expert_ffn");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   WsLayout L;
@@ -727,6 +751,7 @@ moe_status moe_combine(const moe_shape* shape, const void* x, const void* y_perm
                        const int32_t* topk_idx, const float* topk_gate,
                        const int32_t* slot_pos, float gamma, void* out, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_combine");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   if (s.T == 0) return MOE_OK;
@@ -757,6 +782,7 @@ moe_status moe_combine(const moe_shape* shape, const void* x, const void* y_perm
 moe_status moe_bias_update(int32_t N, int32_t Z, const int32_t* counts, int64_t T_all,
                            int32_t K, float K_e, float mu, float* bias, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_bias_update");
   if (N < 1 || Z < 0 || N + Z > moe::kMaxExperts)
     return fail(MOE_ERR_INVALID_ARG, "bad expert counts N=%d Z=%d", N, Z);
   if (K < 1 || K > N + Z) return fail(MOE_ERR_INVALID_ARG, "K=%d outside [1, N+Z]", K);
@@ -772,6 +798,7 @@ moe_status moe_lb_stats(int32_t N, int32_t Z, int32_t D, const int32_t* counts,
                         const float* prob_sum, int64_t T, int32_t K, float K_e, float alpha,
                         float* f, float* P, float* loss, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_lb_stats");
   if (N < 1 || Z < 1 || N + Z > moe::kMaxExperts)
     return fail(MOE_ERR_INVALID_ARG, "moe_lb_stats: needs N >= 1 and Z >= 1 (N=%d Z=%d)", N, Z);
   if (D < 1 || N % D) return fail(MOE_ERR_INVALID_ARG, "moe_lb_stats: D=%d must divide N=%d", D, N);
@@ -799,6 +826,7 @@ moe_status moe_expert_gate_up_save(const moe_shape* shape, const void* x_perm, c
                                    const void* w3, const int32_t* offsets, void* h, void* au,
                                    void* ws, size_t ws_bytes, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_expert_gate_up_save");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   WsLayout L;
@@ -846,6 +874,7 @@ moe_status moe_combine_backward(const moe_shape* shape, const void* x, const voi
                                 const int32_t* slot_pos, const void* dout, float gamma,
                                 void* dy_perm, float* dgate, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_combine_backward");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   if (s.T == 0) return MOE_OK;
@@ -882,6 +911,7 @@ moe_status moe_route_backward(const moe_shape* shape, const void* x, const void*
                               int64_t lb_tokens, void* dw_router, float* dx_router, void* ws,
                               size_t ws_bytes, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_route_backward");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   MOE_TRY(check_bwd_shape(s));
@@ -971,6 +1001,7 @@ moe_status moe_expert_ffn_backward(const moe_shape* shape, const void* x_perm, c
                                    void* dx_perm, void* dw1, void* dw3, void* dw2, void* ws,
                                    size_t ws_bytes, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_expert_ffn_backward");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   MOE_TRY(check_bwd_shape(s));
@@ -1093,6 +1124,7 @@ moe_status moe_permute_backward(const moe_shape* shape, const void* dout,
                                 const int32_t* slot_pos, const void* dx_perm,
                                 const float* dx_router, float gamma, void* dx, void* stream) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_permute_backward");
   MOE_TRY(validate_shape(shape));
   const moe_shape& s = *shape;
   if (s.T == 0) return MOE_OK;
@@ -1124,6 +1156,7 @@ moe_status moe_permute_backward(const moe_shape* shape, const void* dout,
 
 moe_status moe_get_device_status(void* ws, void* stream, uint32_t* status_out) {
   g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_get_device_status");
   if (!ws) return fail(MOE_ERR_INVALID_ARG, "workspace is NULL");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t v = 0;

@@ -67,3 +67,38 @@ def test_skewed_bias_control_trajectory():
           f"mean FFN experts {hist[0]['n_ffn_mean']:.3f} -> {hist[-1]['n_ffn_mean']:.3f} "
           f"(target {K_e:.3f}); max/mean load {hist[0]['max_over_mean_load']:.3f} -> "
           f"{hist[-1]['max_over_mean_load']:.3f}")
+
+
+def test_bias_checkpoint_resume_is_bit_exact(tmp_path):
+    """The expert bias is the layer's only state: a checkpoint is a host copy of
+    it (saved to a file here), and resuming from it reproduces the rest of the
+    closed-loop trajectory bit for bit."""
+    cfg = C.SKEWED_BIAS_CONTROL
+    L = IN.make_layer_inputs(cfg, device="cuda", with_x=False)
+    shape = B.shape_of(cfg)
+    N, K, E, T = cfg.N, cfg.K, cfg.E, cfg.T
+    K_e, mu = float(np.float32(cfg.K_e)), float(np.float32(cfg.mu))
+    ws = B.new_workspace(shape)
+    idx = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    gate = torch.empty((T, K), dtype=torch.float32, device="cuda")
+    counts = torch.empty(E, dtype=torch.int32, device="cuda")
+    nffn = torch.empty(T, dtype=torch.uint8, device="cuda")
+
+    def run(bias, steps):
+        trail = []
+        for s in steps:
+            x, off = IN.make_skewed_step(cfg, s, device="cuda")
+            B.route(shape, x, L["w_router"], bias, ws, idx, gate, counts, nffn, logit_offset=off)
+            B.bias_update(N, cfg.Z, counts, T, K, K_e, mu, bias)
+            trail.append((idx.cpu().clone(), bias.cpu().clone()))
+        return trail
+
+    bias = L["bias"].clone()
+    run(bias, range(0, 5))
+    ckpt = tmp_path / "bias.pt"
+    torch.save(bias.cpu(), ckpt)                      # checkpoint: device -> host -> file
+    first = run(bias, range(5, 10))
+    resumed = torch.load(ckpt).to("cuda")             # resume: file -> host -> device
+    second = run(resumed, range(5, 10))
+    for (i1, b1), (i2, b2) in zip(first, second):
+        assert torch.equal(i1, i2) and torch.equal(b1, b2)
