@@ -233,19 +233,31 @@ def run_gpu(args, rank, world, local_rank):
         graph.replay()
         barrier()
     launches0 = B.kernel_launches()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if args.flush_l2 else None
+    fl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)] if flush is not None else None
     barrier()
     clocks.start()
     t0.record(stream)
     for i in range(args.steps):
+        if flush is not None:
+            # evict the previous step's data: write 256 MB (> the 126 MB L2), then
+            # time the step alone
+            flush.zero_()
+            fl_ev[i][0].record(stream)
         if graph is None:
             step(x, evs[i])
         else:
             graph.replay()
+        if flush is not None:
+            fl_ev[i][1].record(stream)
     t1.record(stream)
     barrier()
     clk = clocks.stop()
     launches = (B.kernel_launches() - launches0) if graph is None else per_step_launches * args.steps
     ms_total = t0.elapsed_time(t1)
+    if flush is not None:
+        ms_total = sum(a.elapsed_time(b) for a, b in fl_ev)
     if graph is not None:
         # per-call breakdown from a separate eager pass
         for i in range(args.steps):
@@ -402,9 +414,11 @@ def run_gpu(args, rank, world, local_rank):
                    "expert_weights": ("mxfp8 (moe_quantize_weights_mxfp8)" if args.fp8_experts
                                       else "tiled (moe_pack_weights)" if tiled else "row-major"),
                    "parallelism": f"token-dp{world} (weights replicated, counts all-reduced)",
-                   "l2": f"inputs larger than L2 ({cfg.N * 3 * cfg.I * cfg.d * wsz / 1e9:.2f} GB "
-                         "of expert weights, 126 MB L2; the touched experts' weights are "
-                         "streamed every step)"},
+                   "l2": ("flushed before every timed step (256 MB memset, outside the "
+                          "per-step events)") if args.flush_l2 else
+                         (f"inputs larger than L2 ({cfg.N * 3 * cfg.I * cfg.d * wsz / 1e9:.2f} GB "
+                          "of expert weights, 126 MB L2; the touched experts' weights are "
+                          "streamed every step)")},
         "roofline": {"kernel": ("moe_expert_gate_up_mxfp8 (tcgen05 block-scaled grouped GEMM)"
                                 if fp8 else "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)"),
                      "bound": "hbm", "achieved": round(achieved, 1),
@@ -647,6 +661,9 @@ def main():
     ap.add_argument("--fused-gather", action="store_true",
                     help="no x_perm copy: the gate/up GEMM reads the token rows from x "
                          "(moe_expert_gate_up_gather)")
+    ap.add_argument("--flush-l2", action="store_true",
+                    help="write a 256 MB buffer before every timed step and time the steps "
+                         "alone (per-step events)")
     ap.add_argument("--graph", action="store_true",
                     help="replay one captured CUDA graph per step (single GPU)")
     args = ap.parse_args()
