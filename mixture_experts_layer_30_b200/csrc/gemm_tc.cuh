@@ -136,6 +136,7 @@ struct Args {
   // goes to split 0 only).  0 or 1: no split.
   int k_splits;
   long long split_stride;
+  int single_half;             // plain modes: tiles of 128 features, D1 neither loaded nor computed
 };
 
 // TMA coordinates (column, row) of the weight tile whose first row is `row`
@@ -546,7 +547,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
             l2_prefetch_bulk(row + (size_t)args.n_out * 2, nf);
           }
         }
-        const uint32_t tx = 2 * kABytes + nbox * kBoxBytes;
+        const uint32_t tx = (args.single_half ? 1 : 2) * kABytes + nbox * kBoxBytes;
         const int a_row0 = t.seg * args.a_seg_rows + t.f0;
         const int a_row1 = a_row0 + args.a1_row_off;
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -572,7 +573,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
           } else {
             const int2 c0 = a_coord(args, a_row0, kb, nk), c1 = a_coord(args, a_row1, kb, nk);
             tma_load_2d_hint(sa0, &tmA0, c0.x, c0.y, fb, pol_w);
-            tma_load_2d_hint(sa0 + kABytes, &tmA1, c1.x, c1.y, fb, pol_w);
+            if (!args.single_half) tma_load_2d_hint(sa0 + kABytes, &tmA1, c1.x, c1.y, fb, pol_w);
           }
           for (int b = 0; b < nbox; ++b)
             tma_load_2d_hint(sa0 + 2 * kABytes + b * kBoxBytes, &tmB, kb * kBK,
@@ -619,7 +620,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
           for (int k = 0; k < kBK / 16; ++k) {
             const uint32_t acc = ((kb - kb0) | k) != 0;
             umma_bf16(d0, da0 + kAStep * k, db + 2 * k, idesc, acc);
-            umma_bf16(d0 + kNMax, da1 + kAStep * k, db + 2 * k, idesc, acc);
+            if (!args.single_half) umma_bf16(d0 + kNMax, da1 + kAStep * k, db + 2 * k, idesc, acc);
           }
           umma_commit(empty0 + 8 * stage);
           ++consumed;
@@ -757,7 +758,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
                               args.n_out);
         }
       } else {
-      const int nhalves = (kMode == kGated) ? 1 : 2;
+      const int nhalves = (kMode == kGated || args.single_half) ? 1 : 2;
       for (int hf = 0; hf < nhalves; ++hf) {
         const int fbase = t.f0 + hf * kFeat + 32 * q;   // first feature of this warp
         for (int j0 = 0; j0 < t.n; j0 += 32) {
@@ -1093,7 +1094,12 @@ inline moe_status launch_router_gemm(const moe_shape& s, const void* x, const vo
   g.out = logits;
   g.add = offset;
   g.status = nullptr;
-  const long long fblk = (E + 2 * kFeat - 1) / (2 * kFeat);
+  if (E <= kFeat) {
+    // at most 128 experts: one accumulator, the second weight half neither loaded nor computed
+    g.feat_per_tile = kFeat;
+    g.single_half = 1;
+  }
+  const long long fblk = (E + g.feat_per_tile - 1) / g.feat_per_tile;
   const int splits = router_splits(s);
   if (splits > 1) {
     g.k_splits = splits;
