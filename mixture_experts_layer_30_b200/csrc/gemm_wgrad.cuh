@@ -38,7 +38,9 @@ constexpr int kWgEpiWarps = 8;
 constexpr int kWgN = 128;                         // output columns per tile (UMMA N)
 constexpr int kWgStageBytes = 6 * kMnBoxBytes;    // A0, A1, B: two 64 x 64 boxes each
 constexpr int kWgStoreBox = 32 * 128;             // 32 rows x 64 bf16 output columns
-constexpr int kWgStagingBytes = kWgEpiWarps * 2 * kWgStoreBox;
+constexpr int kWgStgBoxes = 1;                    // staging boxes per epilogue warp
+constexpr bool kWgLsuStore = false;               // staging box -> global by the warp's lanes
+constexpr int kWgStagingBytes = kWgEpiWarps * kWgStgBoxes * kWgStoreBox;
 constexpr int kWgNumBars = 2 * kWgStages + 2 * 2 + 1;
 constexpr int kWgSmemBytes = 1024 + kWgStages * kWgStageBytes + kWgStagingBytes + kCtrlBytes;
 static_assert(kWgSmemBytes <= 232448, "wgrad shared memory");
@@ -53,6 +55,9 @@ struct WgArgs {
   int m_step;                  // 128: two outputs; 256: D1 = rows m0 + 128
   int a1_col_off;              // column of the A1 boxes relative to A0's
   int out1_row_off;            // row offset of D1's output (0 or 128)
+  void* out0;                  // output matrices [out_rows, n_out] bf16 (plain-store path)
+  void* out1;
+  long long out_rows;
   uint32_t* status;
 };
 
@@ -89,7 +94,10 @@ MOE_DEV void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) 
                : "memory");
 }
 MOE_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-MOE_DEV void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+template <int N>
+MOE_DEV void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
 MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // One accumulator half of a finished tile: the warp's 32 output rows x 128
@@ -97,9 +105,9 @@ MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "m
 // with four loads behind one wait and released on `tmem_empty` before the
 // stores; each 64-column piece goes bf16 -> swizzled staging box -> TMA store.
 // has_data false: the segment had no rows and the gradient is zero.
-MOE_DEV void wg_store_half(const CUtensorMap* om, uint32_t ta, bool has_data, bool row_ok,
-                           int out_row, int n0, int n_out, uint32_t stg0, int lane, int& nstore,
-                           uint32_t tmem_empty) {
+MOE_DEV void wg_store_half(const CUtensorMap* om, void* outp, long long out_rows, uint32_t ta,
+                           bool has_data, bool row_ok, int out_row, int n0, int n_out,
+                           uint32_t stg0, int lane, int& nstore, uint32_t tmem_empty) {
   if (!row_ok) {
     tc_fence_before();
     mbar_arrive(tmem_empty);
@@ -124,8 +132,8 @@ MOE_DEV void wg_store_half(const CUtensorMap* om, uint32_t ta, bool has_data, bo
     if (col >= n_out) continue;
     // this lane's output row: 64 columns -> 32 bf16 pairs -> 8 16-byte pieces,
     // written to the 128-byte-swizzled staging box (piece p at p ^ (row & 7))
-    const uint32_t sb = stg0 + (nstore & 1) * kWgStoreBox;
-    if (lane == 0) bulk_wait_read1();
+    const uint32_t sb = stg0 + (nstore % kWgStgBoxes) * kWgStoreBox;
+    if (!kWgLsuStore && lane == 0) bulk_wait_read<kWgStgBoxes - 1>();
     __syncwarp();
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
@@ -139,11 +147,30 @@ MOE_DEV void wg_store_half(const CUtensorMap* om, uint32_t ta, bool has_data, bo
                    "r"(w2), "r"(w3)
                    : "memory");
     }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    __syncwarp();
-    if (lane == 0) {
-      tma_store_2d(om, sb, col, out_row);
-      bulk_commit();
+    if constexpr (kWgLsuStore) {
+      // 8 lanes per 128-byte row piece: each store instruction writes 4 whole lines
+      __syncwarp();
+      char* ob = static_cast<char*>(outp);
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int idx = it * 32 + lane, row = idx >> 3, pc = idx & 7;
+        uint32_t x0, x1, x2, x3;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+                     : "r"(sb + row * 128 + ((pc ^ (row & 7)) << 4)));
+        const long long grow = (long long)out_row + row;
+        if (grow < out_rows && col + 8 * pc < n_out)
+          *reinterpret_cast<uint4*>(ob + (grow * n_out + col + 8 * pc) * 2) =
+              make_uint4(x0, x1, x2, x3);
+      }
+      __syncwarp();
+    } else {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(om, sb, col, out_row);
+        bulk_commit();
+      }
     }
     ++nstore;
   }
@@ -312,7 +339,7 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     // ---------------- epilogue (warps 2..9) ----------------
     const int q = warp & 3;         // TMEM lane quarter = output rows 32q..32q+31 of a half
     const int hf = (warp - 2) >> 2; // accumulator D0 or D1
-    const uint32_t stg0 = smem_u32(staging + (warp - 2) * 2 * kWgStoreBox);
+    const uint32_t stg0 = smem_u32(staging + (warp - 2) * kWgStgBoxes * kWgStoreBox);
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const CUtensorMap* om = hf ? &tmO1 : &tmO0;
     int local = 0, nstore = 0;
@@ -323,7 +350,8 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       if (!mbar_wait(tmem_full0 + 8 * buf, acc_parity, abort_flag, args.status)) break;
       tc_fence_after();
       const int r = (hf ? t.m0 + args.out1_row_off : t.m0) + 32 * q;  // first output row
-      wg_store_half(om, tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, t.rows > 0,
+      wg_store_half(om, hf ? args.out1 : args.out0, args.out_rows,
+                    tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, t.rows > 0,
                     r < args.m_out, t.seg * args.m_out + r, t.n0, args.n_out, stg0, lane, nstore,
                     tmem_empty0 + 8 * buf);
     }
@@ -357,7 +385,7 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
 // blocks hold streams A with B, block by block, through the same slots.
 constexpr int kAsSlots = 3;                       // resident A blocks: segments up to 192 rows
 constexpr int kAsSlotBytes = 4 * kMnBoxBytes;     // A0 and A1, two 64 x 64 boxes each
-constexpr int kAsBStages = 4;
+constexpr int kAsBStages = 6;
 constexpr int kAsBBytes = 2 * kMnBoxBytes;        // B: two 64 x 64 boxes
 constexpr int kAsNumBars = 2 * kAsSlots + 2 * kAsBStages + 2 * 2 + 1;
 constexpr int kAsSmemBytes = 1024 + kAsSlots * kAsSlotBytes + kAsBStages * kAsBBytes +
@@ -508,6 +536,8 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
     bool ok = true;
     int a_seen = 0, b_seen = 0, local = 0;
     const uint32_t idesc = idesc_bf16(kFeat, kWgN, true, true);
+    int data_end = args.seg_offsets[args.nseg];  // rows written by the forward pass
+    if (data_end < 0 || data_end > args.max_rows) data_end = 0;  // (offsets checked per unit)
     auto wait_bcast = [&](uint32_t bar, uint32_t par) -> bool {
       int go = 1;
       if (lane == 0) go = mbar_wait(bar, par, abort_flag, args.status);
@@ -561,7 +591,9 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
           const int nv = min(kBK, u.rows - kb * kBK);
           const int ksteps = (nv + 15) >> 4;
           if (!u.stat || nb == 0) wg_zero_tail(sa, 4, nv, lane);  // resident A: zeroed once
-          wg_zero_tail(sb, 2, nv, lane);
+          // B's rows past the segment meet zero rows of A; only rows past the last
+          // segment (never written, possibly not finite) are cleared
+          if (u.lo + kb * kBK + ((nv + 15) & ~15) > data_end) wg_zero_tail(sb, 2, nv, lane);
           if (lane == 0) {
             const uint64_t da0 = smem_desc_mn_sw128(sa);
             const uint64_t da1 = smem_desc_mn_sw128(sa + 2 * kMnBoxBytes);
@@ -593,7 +625,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
     // ---------------- epilogue (warps 2..9) ----------------
     const int q = warp & 3;
     const int hf = (warp - 2) >> 2;
-    const uint32_t stg0 = smem_u32(staging + (warp - 2) * 2 * kWgStoreBox);
+    const uint32_t stg0 = smem_u32(staging + (warp - 2) * kWgStgBoxes * kWgStoreBox);
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const CUtensorMap* om = hf ? &tmO1 : &tmO0;
     int local = 0, nstore = 0;
@@ -609,7 +641,8 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
           break;
         }
         tc_fence_after();
-        wg_store_half(om, tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, u.rows > 0,
+        wg_store_half(om, hf ? args.out1 : args.out0, args.out_rows,
+                      tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, u.rows > 0,
                       r < args.m_out, u.seg * args.m_out + r, nb * kWgN, args.n_out, stg0, lane,
                       nstore, tmem_empty0 + 8 * buf);
       }
@@ -735,6 +768,9 @@ inline moe_status launch_wgrad_w13(const moe_shape& s, const void* x_perm, const
   g.m_step = 128;
   g.a1_col_off = s.I;
   g.out1_row_off = 0;
+  g.out0 = dw1;
+  g.out1 = dw3;
+  g.out_rows = (long long)s.N * s.I;
   g.status = status;
   return launch_wgrad_as(a, b, o0, o1, g, sms, st, err, errn);
 }
@@ -757,6 +793,8 @@ inline moe_status launch_wgrad_w2(const moe_shape& s, const void* h, const void*
   g.m_step = 256;
   g.a1_col_off = 128;
   g.out1_row_off = 128;
+  g.out0 = g.out1 = dw2;
+  g.out_rows = (long long)s.N * s.d;
   g.status = status;
   return launch_wgrad_as(a, b, o0, o0, g, sms, st, err, errn);
 }
@@ -780,6 +818,8 @@ inline moe_status launch_router_wgrad(const moe_shape& s, const void* dlogits, c
   g.m_step = 256;
   g.a1_col_off = 128;
   g.out1_row_off = 128;
+  g.out0 = g.out1 = dw_router;
+  g.out_rows = E;
   g.status = status;
   return launch_wgrad(a, b, o, o, g, sms, st, err, errn);
 }
