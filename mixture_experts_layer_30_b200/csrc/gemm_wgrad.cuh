@@ -110,7 +110,8 @@ MOE_DEV void wg_store_half(const CUtensorMap* om, void* outp, long long out_rows
                            uint32_t stg0, int lane, int& nstore, uint32_t tmem_empty) {
   if (!row_ok) {
     tc_fence_before();
-    mbar_arrive(tmem_empty);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(tmem_empty);
     return;
   }
   uint32_t v[4][32];
@@ -125,7 +126,8 @@ MOE_DEV void wg_store_half(const CUtensorMap* om, void* outp, long long out_rows
       for (int i = 0; i < 32; ++i) v[c][i] = 0u;
   }
   tc_fence_before();
-  mbar_arrive(tmem_empty);  // TMEM is free once the loads landed
+  __syncwarp();
+  if (lane == 0) mbar_arrive(tmem_empty);  // TMEM is free once the warp's loads landed
 #pragma unroll
   for (int c = 0; c < kWgN / 64; ++c) {
     const int col = n0 + 64 * c;
@@ -192,6 +194,18 @@ MOE_DEV void wg_zero_tail(uint32_t base, int nbox, int nv, int lane) {
   __syncwarp();
 }
 
+// The same clearing done by one thread (the A-stationary MMA issuer).
+MOE_DEV void wg_zero_tail_one(uint32_t base, int nbox, int nv) {
+  const int zrows = ((nv + 15) & ~15) - nv;
+  if (zrows <= 0) return;
+  for (int box = 0; box < nbox; ++box)
+    for (int piece = 0; piece < zrows * 8; ++piece) {
+      const uint32_t addr = base + box * kMnBoxBytes + nv * 128 + piece * 16;
+      asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0u) : "memory");
+    }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(kWgThreads, 1)
 gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmO0,
@@ -222,7 +236,7 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tmem_full0 + 8 * b, 1);
-      mbar_init(tmem_empty0 + 8 * b, kWgEpiWarps * 32);
+      mbar_init(tmem_empty0 + 8 * b, kWgEpiWarps);  // one arrival per warp
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -453,7 +467,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tmem_full0 + 8 * b, 1);
-      mbar_init(tmem_empty0 + 8 * b, kWgEpiWarps * 32);
+      mbar_init(tmem_empty0 + 8 * b, kWgEpiWarps);  // one arrival per warp
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -532,69 +546,75 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA warp ----------------
-    bool ok = true;
-    int a_seen = 0, b_seen = 0, local = 0;
-    const uint32_t idesc = idesc_bf16(kFeat, kWgN, true, true);
-    int data_end = args.seg_offsets[args.nseg];  // rows written by the forward pass
-    if (data_end < 0 || data_end > args.max_rows) data_end = 0;  // (offsets checked per unit)
-    auto wait_bcast = [&](uint32_t bar, uint32_t par) -> bool {
-      int go = 1;
-      if (lane == 0) go = mbar_wait(bar, par, abort_flag, args.status);
-      return __shfl_sync(0xffffffffu, go, 0) != 0;
-    };
-    for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
-      const AsUnit u = as_decode(unit, args, mblk);
-      const int a0 = a_seen;  // first A fill of this unit
-      if (u.stat) {
-        for (int kb = 0; kb < u.nk && ok; ++kb) {
-          const int i = a0 + kb;
-          ok = wait_bcast(a_full0 + 8 * (i % kAsSlots), (uint32_t)((i / kAsSlots) & 1));
-        }
-        if (!ok) break;
-        a_seen = a0 + u.nk;
-        if (lane == 0) *a_seen_sh = a_seen;
-      }
-      for (int nb = 0; nb < nblk && ok; ++nb, ++local) {
-        const int buf = local & 1;
-        if (!wait_bcast(tmem_empty0 + 8 * buf, (uint32_t)(((local >> 1) & 1) ^ 1))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d0 = tmem_base + buf * 2 * kWgN;
-        for (int kb = 0; kb < u.nk; ++kb) {
-          int ai;
-          if (u.stat) {
-            ai = a0 + kb;
-          } else {
-            ai = a_seen;
-            if (!wait_bcast(a_full0 + 8 * (ai % kAsSlots), (uint32_t)((ai / kAsSlots) & 1))) {
-              ok = false;
-              break;
-            }
-            ++a_seen;
+    // ---------------- MMA issuer (lane 0 alone) ----------------
+    // One thread waits, clears tails and issues: no warp-wide broadcast between
+    // a stage's arrival and its MMAs, so the tensor pipe's short queue is
+    // refilled as soon as the data is there.
+    if (lane == 0) {
+      bool ok = true;
+      int a_seen = 0, b_seen = 0, local = 0;
+      const uint32_t idesc = idesc_bf16(kFeat, kWgN, true, true);
+      int data_end = args.seg_offsets[args.nseg];  // rows written by the forward pass
+      if (data_end < 0 || data_end > args.max_rows) data_end = 0;  // (offsets checked per unit)
+      for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
+        const AsUnit u = as_decode(unit, args, mblk);
+        const int a0 = a_seen;  // first A fill of this unit
+        if (u.stat) {
+          for (int kb = 0; kb < u.nk && ok; ++kb) {
+            const int i = a0 + kb;
+            ok = mbar_wait(a_full0 + 8 * (i % kAsSlots), (uint32_t)((i / kAsSlots) & 1), abort_flag,
+                           args.status);
           }
-          const int bs = b_seen % kAsBStages;
-          if (!wait_bcast(b_full0 + 8 * bs, (uint32_t)((b_seen / kAsBStages) & 1))) {
+          if (!ok) break;
+          a_seen = a0 + u.nk;
+          *a_seen_sh = a_seen;
+          tc_fence_after();
+          // resident A: K rows past the segment end cleared once per unit
+          for (int kb = 0; kb < u.nk; ++kb)
+            wg_zero_tail_one(smem_u32(aslots + ((a0 + kb) % kAsSlots) * kAsSlotBytes), 4,
+                             min(kBK, u.rows - kb * kBK));
+        }
+        for (int nb = 0; nb < nblk && ok; ++nb, ++local) {
+          const int buf = local & 1;
+          if (!mbar_wait(tmem_empty0 + 8 * buf, (uint32_t)(((local >> 1) & 1) ^ 1), abort_flag,
+                         args.status)) {
             ok = false;
             break;
           }
-          ++b_seen;
-          if (lane == 0) {
+          tc_fence_after();
+          const uint32_t d0 = tmem_base + buf * 2 * kWgN;
+          for (int kb = 0; kb < u.nk; ++kb) {
+            const int nv = min(kBK, u.rows - kb * kBK);
+            int ai;
+            if (u.stat) {
+              ai = a0 + kb;
+            } else {
+              ai = a_seen;
+              if (!mbar_wait(a_full0 + 8 * (ai % kAsSlots), (uint32_t)((ai / kAsSlots) & 1),
+                             abort_flag, args.status)) {
+                ok = false;
+                break;
+              }
+              ++a_seen;
+              tc_fence_after();
+              wg_zero_tail_one(smem_u32(aslots + (ai % kAsSlots) * kAsSlotBytes), 4, nv);
+            }
+            const int bs = b_seen % kAsBStages;
+            if (!mbar_wait(b_full0 + 8 * bs, (uint32_t)((b_seen / kAsBStages) & 1), abort_flag,
+                           args.status)) {
+              ok = false;
+              break;
+            }
+            ++b_seen;
             *a_seen_sh = a_seen;
             *b_seen_sh = b_seen;
-          }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(aslots + (ai % kAsSlots) * kAsSlotBytes);
-          const uint32_t sb = smem_u32(bstages + bs * kAsBBytes);
-          const int nv = min(kBK, u.rows - kb * kBK);
-          const int ksteps = (nv + 15) >> 4;
-          if (!u.stat || nb == 0) wg_zero_tail(sa, 4, nv, lane);  // resident A: zeroed once
-          // B's rows past the segment meet zero rows of A; only rows past the last
-          // segment (never written, possibly not finite) are cleared
-          if (u.lo + kb * kBK + ((nv + 15) & ~15) > data_end) wg_zero_tail(sb, 2, nv, lane);
-          if (lane == 0) {
+            tc_fence_after();
+            const uint32_t sa = smem_u32(aslots + (ai % kAsSlots) * kAsSlotBytes);
+            const uint32_t sb = smem_u32(bstages + bs * kAsBBytes);
+            // B's rows past the segment meet zero rows of A; only rows past the last
+            // segment (never written, possibly not finite) are cleared
+            if (u.lo + kb * kBK + ((nv + 15) & ~15) > data_end) wg_zero_tail_one(sb, 2, nv);
+            const int ksteps = (nv + 15) >> 4;
             const uint64_t da0 = smem_desc_mn_sw128(sa);
             const uint64_t da1 = smem_desc_mn_sw128(sa + 2 * kMnBoxBytes);
             const uint64_t db = smem_desc_mn_sw128(sb);
@@ -606,17 +626,12 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
             umma_commit(b_empty0 + 8 * bs);
             if (!u.stat) umma_commit(a_empty0 + 8 * (ai % kAsSlots));
           }
-          __syncwarp();
+          if (ok) umma_commit(tmem_full0 + 8 * buf);
         }
-        if (ok && lane == 0) umma_commit(tmem_full0 + 8 * buf);
-        __syncwarp();
+        // resident A blocks are released once the unit's last MMAs complete
+        if (ok && u.stat)
+          for (int kb = 0; kb < u.nk; ++kb) umma_commit(a_empty0 + 8 * ((a0 + kb) % kAsSlots));
       }
-      // resident A blocks are released once the unit's last MMAs complete
-      if (ok && u.stat && lane == 0)
-        for (int kb = 0; kb < u.nk; ++kb) umma_commit(a_empty0 + 8 * ((a0 + kb) % kAsSlots));
-      __syncwarp();
-    }
-    if (lane == 0) {
       umma_commit(drain_bar);
       mbar_wait(drain_bar, 0, abort_flag, args.status, kDrainTimeoutNs, false);
     }
