@@ -93,6 +93,15 @@ MOE_DEV void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) 
                "r"(c0), "r"(c1), "r"(src)
                : "memory");
 }
+// The same store with an L2 eviction-priority hint (a createpolicy value).
+MOE_DEV void tma_store_2d_hint(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                               uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], "
+      "%4;" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(src), "l"(policy)
+      : "memory");
+}
 MOE_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 template <int N>
 MOE_DEV void bulk_wait_read() {
@@ -107,7 +116,8 @@ MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "m
 // has_data false: the segment had no rows and the gradient is zero.
 MOE_DEV void wg_store_half(const CUtensorMap* om, void* outp, long long out_rows, uint32_t ta,
                            bool has_data, bool row_ok, int out_row, int n0, int n_out,
-                           uint32_t stg0, int lane, int& nstore, uint32_t tmem_empty) {
+                           uint32_t stg0, int lane, int& nstore, uint32_t tmem_empty,
+                           uint64_t store_policy = 0) {
   if (!row_ok) {
     tc_fence_before();
     __syncwarp();
@@ -170,7 +180,8 @@ MOE_DEV void wg_store_half(const CUtensorMap* om, void* outp, long long out_rows
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) {
-        tma_store_2d(om, sb, col, out_row);
+        if (store_policy) tma_store_2d_hint(om, sb, col, out_row, store_policy);
+        else tma_store_2d(om, sb, col, out_row);
         bulk_commit();
       }
     }
@@ -502,6 +513,9 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       bool ok = true;
+      // the B block of an expert is read by all of its m-block units: keep it in L2
+      const uint64_t pol_a = l2_policy_evict_first();
+      const uint64_t pol_b = l2_policy_evict_last();
       auto fill_a = [&](const AsUnit& u, int kb) -> bool {
         const int slot = a_issued % kAsSlots;
         const uint32_t par = (uint32_t)((a_issued / kAsSlots) & 1);
@@ -512,9 +526,9 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
         mbar_arrive_expect_tx(fb, kAsSlotBytes);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          tma_load_2d(sa + h * kMnBoxBytes, &tmA, u.m0 + 64 * h, row, fb);
-          tma_load_2d(sa + 2 * kMnBoxBytes + h * kMnBoxBytes, &tmA,
-                      u.m0 + args.a1_col_off + 64 * h, row, fb);
+          tma_load_2d_hint(sa + h * kMnBoxBytes, &tmA, u.m0 + 64 * h, row, fb, pol_a);
+          tma_load_2d_hint(sa + 2 * kMnBoxBytes + h * kMnBoxBytes, &tmA,
+                           u.m0 + args.a1_col_off + 64 * h, row, fb, pol_a);
         }
         ++a_issued;
         return true;
@@ -527,8 +541,8 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t sb = smem_u32(bstages + st * kAsBBytes);
         const int row = u.lo + kb * kBK;
         mbar_arrive_expect_tx(fb, kAsBBytes);
-        tma_load_2d(sb, &tmB, nb * kWgN, row, fb);
-        tma_load_2d(sb + kMnBoxBytes, &tmB, nb * kWgN + 64, row, fb);
+        tma_load_2d_hint(sb, &tmB, nb * kWgN, row, fb, pol_b);
+        tma_load_2d_hint(sb + kMnBoxBytes, &tmB, nb * kWgN + 64, row, fb, pol_b);
         ++b_issued;
         return true;
       };
@@ -643,6 +657,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
     const uint32_t stg0 = smem_u32(staging + (warp - 2) * kWgStgBoxes * kWgStoreBox);
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const CUtensorMap* om = hf ? &tmO1 : &tmO0;
+    const uint64_t pol_out = l2_policy_evict_first();  // written once, never read back here
     int local = 0, nstore = 0;
     bool ok = true;
     for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
@@ -659,7 +674,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
         wg_store_half(om, hf ? args.out1 : args.out0, args.out_rows,
                       tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, u.rows > 0,
                       r < args.m_out, u.seg * args.m_out + r, nb * kWgN, args.n_out, stg0, lane,
-                      nstore, tmem_empty0 + 8 * buf);
+                      nstore, tmem_empty0 + 8 * buf, pol_out);
       }
     }
     if (lane == 0) bulk_wait_all();
