@@ -14,15 +14,19 @@
 // tile overlaps the MMAs of the next.
 //
 // One persistent CTA per SM, 10 warps:
-//   warp 0      TMA producer (one lane): six 64 x 64 boxes per stage (A0, A1, B)
-//   warp 1      MMA warp: zeroes the K rows past the segment end in the last
-//               stage of a segment (generic stores + proxy fence), lane 0 issues
+//   warp 0      TMA producer (one lane)
+//   warp 1      MMA warp: zeroes the K rows past the segment end (generic
+//               stores + proxy fence) and issues the MMAs (in the A-stationary
+//               kernel one lane does both, with no warp-wide broadcast per
+//               stage: the tensor pipe's short queue must be refilled as soon
+//               as a stage lands)
 //   warps 2..9  epilogue, two warps per TMEM lane quarter (warps 2..5: D0,
 //               6..9: D1): all 128 columns of its 32 rows loaded behind one
 //               wait -> bf16 -> swizzled staging box -> TMA store (32 rows x
-//               64 columns per store, two staging boxes per warp)
+//               64 columns per store, kWgStgBoxes staging boxes per warp)
 // A tile writes 64 KiB of bf16 and performs only 2*R_e*256*128 FLOPs (R_e ~
-// 128 routed rows), so the epilogue's store rate sets the pace.
+// 128 routed rows): a stream of gradient writes paced by the MMA issue and
+// the epilogue.
 // Waits are bounded as in gemm_tc.cuh; on expiry the status word records
 // MOE_DEV_PIPELINE_TIMEOUT and the CTA drains and returns.
 #pragma once
@@ -39,7 +43,6 @@ constexpr int kWgN = 128;                         // output columns per tile (UM
 constexpr int kWgStageBytes = 6 * kMnBoxBytes;    // A0, A1, B: two 64 x 64 boxes each
 constexpr int kWgStoreBox = 32 * 128;             // 32 rows x 64 bf16 output columns
 constexpr int kWgStgBoxes = 1;                    // staging boxes per epilogue warp
-constexpr bool kWgLsuStore = false;               // staging box -> global by the warp's lanes
 constexpr int kWgStagingBytes = kWgEpiWarps * kWgStgBoxes * kWgStoreBox;
 constexpr int kWgNumBars = 2 * kWgStages + 2 * 2 + 1;
 constexpr int kWgSmemBytes = 1024 + kWgStages * kWgStageBytes + kWgStagingBytes + kCtrlBytes;
@@ -55,9 +58,6 @@ struct WgArgs {
   int m_step;                  // 128: two outputs; 256: D1 = rows m0 + 128
   int a1_col_off;              // column of the A1 boxes relative to A0's
   int out1_row_off;            // row offset of D1's output (0 or 128)
-  void* out0;                  // output matrices [out_rows, n_out] bf16 (plain-store path)
-  void* out1;
-  long long out_rows;
   uint32_t* status;
 };
 
@@ -114,10 +114,9 @@ MOE_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "m
 // with four loads behind one wait and released on `tmem_empty` before the
 // stores; each 64-column piece goes bf16 -> swizzled staging box -> TMA store.
 // has_data false: the segment had no rows and the gradient is zero.
-MOE_DEV void wg_store_half(const CUtensorMap* om, void* outp, long long out_rows, uint32_t ta,
-                           bool has_data, bool row_ok, int out_row, int n0, int n_out,
-                           uint32_t stg0, int lane, int& nstore, uint32_t tmem_empty,
-                           uint64_t store_policy = 0) {
+MOE_DEV void wg_store_half(const CUtensorMap* om, uint32_t ta, bool has_data, bool row_ok,
+                           int out_row, int n0, int n_out, uint32_t stg0, int lane, int& nstore,
+                           uint32_t tmem_empty, uint64_t store_policy = 0) {
   if (!row_ok) {
     tc_fence_before();
     __syncwarp();
@@ -145,7 +144,7 @@ MOE_DEV void wg_store_half(const CUtensorMap* om, void* outp, long long out_rows
     // this lane's output row: 64 columns -> 32 bf16 pairs -> 8 16-byte pieces,
     // written to the 128-byte-swizzled staging box (piece p at p ^ (row & 7))
     const uint32_t sb = stg0 + (nstore % kWgStgBoxes) * kWgStoreBox;
-    if (!kWgLsuStore && lane == 0) bulk_wait_read<kWgStgBoxes - 1>();
+    if (lane == 0) bulk_wait_read<kWgStgBoxes - 1>();
     __syncwarp();
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
@@ -159,31 +158,12 @@ MOE_DEV void wg_store_half(const CUtensorMap* om, void* outp, long long out_rows
                    "r"(w2), "r"(w3)
                    : "memory");
     }
-    if constexpr (kWgLsuStore) {
-      // 8 lanes per 128-byte row piece: each store instruction writes 4 whole lines
-      __syncwarp();
-      char* ob = static_cast<char*>(outp);
-#pragma unroll
-      for (int it = 0; it < 8; ++it) {
-        const int idx = it * 32 + lane, row = idx >> 3, pc = idx & 7;
-        uint32_t x0, x1, x2, x3;
-        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                     : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
-                     : "r"(sb + row * 128 + ((pc ^ (row & 7)) << 4)));
-        const long long grow = (long long)out_row + row;
-        if (grow < out_rows && col + 8 * pc < n_out)
-          *reinterpret_cast<uint4*>(ob + (grow * n_out + col + 8 * pc) * 2) =
-              make_uint4(x0, x1, x2, x3);
-      }
-      __syncwarp();
-    } else {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      __syncwarp();
-      if (lane == 0) {
-        if (store_policy) tma_store_2d_hint(om, sb, col, out_row, store_policy);
-        else tma_store_2d(om, sb, col, out_row);
-        bulk_commit();
-      }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) {
+      if (store_policy) tma_store_2d_hint(om, sb, col, out_row, store_policy);
+      else tma_store_2d(om, sb, col, out_row);
+      bulk_commit();
     }
     ++nstore;
   }
@@ -375,8 +355,7 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       if (!mbar_wait(tmem_full0 + 8 * buf, acc_parity, abort_flag, args.status)) break;
       tc_fence_after();
       const int r = (hf ? t.m0 + args.out1_row_off : t.m0) + 32 * q;  // first output row
-      wg_store_half(om, hf ? args.out1 : args.out0, args.out_rows,
-                    tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, t.rows > 0,
+      wg_store_half(om, tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, t.rows > 0,
                     r < args.m_out, t.seg * args.m_out + r, t.n0, args.n_out, stg0, lane, nstore,
                     tmem_empty0 + 8 * buf);
     }
@@ -671,8 +650,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
           break;
         }
         tc_fence_after();
-        wg_store_half(om, hf ? args.out1 : args.out0, args.out_rows,
-                      tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, u.rows > 0,
+        wg_store_half(om, tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, u.rows > 0,
                       r < args.m_out, u.seg * args.m_out + r, nb * kWgN, args.n_out, stg0, lane,
                       nstore, tmem_empty0 + 8 * buf, pol_out);
       }
@@ -798,9 +776,6 @@ inline moe_status launch_wgrad_w13(const moe_shape& s, const void* x_perm, const
   g.m_step = 128;
   g.a1_col_off = s.I;
   g.out1_row_off = 0;
-  g.out0 = dw1;
-  g.out1 = dw3;
-  g.out_rows = (long long)s.N * s.I;
   g.status = status;
   return launch_wgrad_as(a, b, o0, o1, g, sms, st, err, errn);
 }
@@ -823,8 +798,6 @@ inline moe_status launch_wgrad_w2(const moe_shape& s, const void* h, const void*
   g.m_step = 256;
   g.a1_col_off = 128;
   g.out1_row_off = 128;
-  g.out0 = g.out1 = dw2;
-  g.out_rows = (long long)s.N * s.d;
   g.status = status;
   return launch_wgrad_as(a, b, o0, o0, g, sms, st, err, errn);
 }
@@ -848,8 +821,6 @@ inline moe_status launch_router_wgrad(const moe_shape& s, const void* dlogits, c
   g.m_step = 256;
   g.a1_col_off = 128;
   g.out1_row_off = 128;
-  g.out0 = g.out1 = dw_router;
-  g.out_rows = E;
   g.status = status;
   return launch_wgrad(a, b, o, o, g, sms, st, err, errn);
 }
