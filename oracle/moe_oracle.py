@@ -37,7 +37,9 @@ Parity status: every function here is pinned by the CPU tests
 and K=E fixed points, closed forms of softmax, SwiGLU and Eq. (2), and the
 hand-derived worked examples under tests/golden/); the backward pass by
 central finite differences of the forward and by torch autograd through an
-independently written dense top-K layer.
+independently written dense top-K layer; the MXFP8 expert by a hand-derived
+example and by a restatement on an exhaustive-search quantiser; the closed
+loop of Eq. (2) by a hand-derived three-step trajectory.
 """
 import numpy as np
 

@@ -415,6 +415,110 @@ def check_mxfp8_block_quantization(orc, seed=9):
     assert np.array_equal(deq2, deq)
 
 
+def _golden_mxfp8_weights(g):
+    d, I = g["shape"]["d"], g["shape"]["I"]
+    w = {"w1": np.zeros((I, d)), "w3": np.zeros((I, d)), "w2": np.zeros((d, I))}
+    for name, entries in g["weights"].items():
+        if name in w:
+            for key, v in entries.items():
+                r, c = (int(t) for t in key.split(","))
+                w[name][r, c] = v
+    return w
+
+
+def check_worked_mxfp8_ffn(orc):
+    """One MXFP8 expert derived by hand: exact weights, x exact or rounded, h rounded."""
+    g = load_golden("worked_example_mxfp8_ffn.json")
+    d = g["shape"]["d"]
+    w = _golden_mxfp8_weights(g)
+    for case in g["cases"]:
+        x = np.zeros((1, d))
+        x[0, 0] = case["x0"]
+        y, h = orc.expert_ffn_mxfp8(x, w["w1"], w["w3"], w["w2"])
+        want_y = np.zeros(d)
+        want_y[:2] = case["expected_y"]
+        np.testing.assert_allclose(h[0, :2], case["expected_h"], rtol=0, atol=1e-14,
+                                   err_msg=case["name"])
+        assert (h[0, 2:] == 0).all()
+        np.testing.assert_allclose(y[0], want_y, rtol=0, atol=1e-14, err_msg=case["name"])
+
+
+def brute_force_mx_quantize(a):
+    """MXFP8 of a [m, K] array along its rows by exhaustive search: for each block
+    of 32 values the scale 2^s with s found by counting up to the first integer
+    with amax <= 448 * 2^s, and each scaled value by a search over all 127
+    non-negative E4M3 codes (nearest, ties to the even code).  Returns the
+    dequantised values."""
+    t = np.array(e4m3_table_cache()[:0x7F])
+    even = (np.arange(0x7F) % 2) == 0
+    a = np.asarray(a, dtype=np.float64)
+    out = np.zeros_like(a)
+    m, K = a.shape
+    for r in range(m):
+        for b0 in range(0, K, 32):
+            blk = a[r, b0:b0 + 32]
+            amax = np.abs(blk).max()
+            s = 0
+            if amax > 0:
+                s = -160
+                while 448.0 * 2.0 ** s < amax:
+                    s += 1
+            mag = np.minimum(np.abs(blk) / 2.0 ** s, 448.0)
+            dist = np.abs(t[None, :] - mag[:, None])
+            best = dist == dist.min(axis=1, keepdims=True)
+            pick = np.where((best & even).any(axis=1), np.argmax(best & even, axis=1),
+                            np.argmax(best, axis=1))
+            out[r, b0:b0 + 32] = np.where(np.signbit(blk), -t[pick], t[pick]) * 2.0 ** s
+    return out
+
+
+def check_mxfp8_ffn_brute_force(orc, seed=13):
+    """The MXFP8 expert against a plain restatement built on the exhaustive
+    quantiser above: x, W1, W3 quantised along d, h = SiLU(a) u along I, W2
+    along I, products in float64.  32 token rows, so h also has whole blocks
+    along the token axis and a quantiser applied along the wrong axis differs."""
+    rng = np.random.default_rng(seed)
+    m, d, I = 32, 64, 32
+    x = rng.normal(size=(m, d)) * np.exp(rng.normal(size=(m, 1)))
+    w1 = rng.normal(size=(I, d)) * 0.2
+    w3 = rng.normal(size=(I, d)) * 0.2
+    w2 = rng.normal(size=(d, I)) * 0.2
+    xq = brute_force_mx_quantize(x)
+    a = xq @ brute_force_mx_quantize(w1).T
+    u = xq @ brute_force_mx_quantize(w3).T
+    h = np.array([[ai / (1.0 + math.exp(-ai)) for ai in row] for row in a]) * u
+    want = brute_force_mx_quantize(h) @ brute_force_mx_quantize(w2).T
+    y, h_got = orc.expert_ffn_mxfp8(x, w1, w3, w2)
+    np.testing.assert_allclose(h_got, h, rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-13)
+
+
+def check_worked_bias_trajectory(orc):
+    """Three closed-loop steps of Eq. (2) derived by hand (route with b_s, then update)."""
+    g = load_golden("worked_example_bias_trajectory.json")
+    sh = g["shape"]
+    E = sh["N"] + sh["Z"]
+    logits = np.log(np.array(g["router_probs"]))
+
+    def route_inputs(s):
+        return np.zeros((sh["T"], 1)), logits
+
+    steps = len(g["expected_steps"])
+    hist, b = orc.bias_control_trajectory(steps, route_inputs, np.zeros((E, 1)),
+                                          np.array(g["bias0"]), sh["N"], sh["K"], g["K_e"],
+                                          g["mu"])
+    assert len(hist) == steps
+    for s, (got, want) in enumerate(zip(hist, g["expected_steps"])):
+        np.testing.assert_allclose(got["bias"], want["bias"], rtol=0, atol=1e-15,
+                                   err_msg=f"bias used by step {s}")
+        np.testing.assert_array_equal(got["counts"], want["counts"], err_msg=f"step {s}")
+        for key in ("n_ffn_mean", "n_ffn_std", "max_over_mean_load", "min_margin"):
+            np.testing.assert_allclose(got[key], want[key], rtol=0, atol=1e-12,
+                                       err_msg=f"{key} at step {s}")
+        assert (got["bias"][sh["N"]:] == 0).all()
+    np.testing.assert_allclose(b, g["expected_final_bias"], rtol=0, atol=1e-15)
+
+
 def _loss_and_grads(orc, L, N, K, gamma, dout):
     r = orc.moe_layer_backward(L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"],
                                N=N, K=K, dout=dout, gamma=gamma)
@@ -517,7 +621,8 @@ def check_lb_backward_finite_differences(orc, seed=12):
         np.testing.assert_allclose(r[grad], fd, rtol=1e-5, atol=1e-7, err_msg=name)
 
 
-ALL_CHECKS = [check_lb_backward_finite_differences, check_backward_finite_differences, check_backward_against_autograd, check_e4m3_table, check_e4m3_rounding_brute_force,
+ALL_CHECKS = [check_worked_mxfp8_ffn, check_mxfp8_ffn_brute_force,
+              check_worked_bias_trajectory, check_lb_backward_finite_differences, check_backward_finite_differences, check_backward_against_autograd, check_e4m3_table, check_e4m3_rounding_brute_force,
               check_mxfp8_block_quantization, check_worked_tiny_layer, check_worked_swiglu, check_worked_bias_update,
               check_worked_zero_experts, check_softmax_closed_forms, check_topk_brute_force,
               check_dense_reduction, check_all_zero_experts_fixed_point,

@@ -180,7 +180,90 @@ def _mut_softmax_backward_no_centering(mp):
     mp.setattr(orc, "softmax_backward", lambda probs, dR: probs * dR)
 
 
-MUTATIONS = [_mut_lb_gradient_without_frequency, _mut_silu_derivative_sigma_only,
+def _mut_mxfp8_h_unquantised(mp):
+    """The SwiGLU hidden h fed to the down projection without its MXFP8 rounding."""
+    q = orc.mxfp8_quantize
+
+    def expert_ffn_mxfp8(x_rows, w1, w3, w2):
+        xq = q(x_rows)[2]
+        h = orc.silu(xq @ q(w1)[2].T) * (xq @ q(w3)[2].T)
+        return h @ q(w2)[2].T, h
+    mp.setattr(orc, "expert_ffn_mxfp8", expert_ffn_mxfp8)
+
+
+def _mut_mxfp8_h_wrong_axis(mp):
+    """h blocked along the token axis instead of along I (its reduction axis)."""
+    q = orc.mxfp8_quantize
+
+    def expert_ffn_mxfp8(x_rows, w1, w3, w2):
+        xq = q(x_rows)[2]
+        h = orc.silu(xq @ q(w1)[2].T) * (xq @ q(w3)[2].T)
+        return q(h.T)[2].T @ q(w2)[2].T, h
+    mp.setattr(orc, "expert_ffn_mxfp8", expert_ffn_mxfp8)
+
+
+def _mut_mxfp8_x_unquantised(mp):
+    """The routed token rows used at full precision."""
+    q = orc.mxfp8_quantize
+
+    def expert_ffn_mxfp8(x_rows, w1, w3, w2):
+        x = np.asarray(x_rows, dtype=np.float64)
+        h = orc.silu(x @ q(w1)[2].T) * (x @ q(w3)[2].T)
+        return q(h)[2] @ q(w2)[2].T, h
+    mp.setattr(orc, "expert_ffn_mxfp8", expert_ffn_mxfp8)
+
+
+def _trajectory_record(b, idx, probs, margin, N, E):
+    counts = orc.expert_counts(idx, E)
+    nf = orc.ffn_experts_per_token(idx, N)
+    load = counts[:N].astype(np.float64)
+    return counts, dict(bias=b.copy(), counts=counts, n_ffn_mean=float(nf.mean()),
+                        n_ffn_std=float(nf.std()),
+                        max_over_mean_load=float(load.max() / load.mean()),
+                        min_margin=float(margin.min()))
+
+
+def _mut_trajectory_routes_with_next_bias(mp):
+    """Step s reported (and its counts fed forward) from a routing with b_{s+1}."""
+    def bias_control_trajectory(steps, route_inputs, w_router, bias0, N, K, K_e, mu):
+        b = np.asarray(bias0, dtype=np.float64).copy()
+        hist = []
+        for s in range(steps):
+            x, off = route_inputs(s)
+            probs = orc.softmax_rows(orc.router_logits(x, w_router, off))
+            E = probs.shape[1]
+            idx, _ = orc.biased_topk(probs, b, K)
+            b_next = orc.bias_update(b, orc.expert_counts(idx, E), N, K, K_e, mu, x.shape[0])
+            idx, margin = orc.biased_topk(probs, b_next, K)
+            counts, rec = _trajectory_record(b_next, idx, probs, margin, N, E)
+            hist.append(rec)
+            b = orc.bias_update(b, counts, N, K, K_e, mu, x.shape[0])
+        return hist, b
+    mp.setattr(orc, "bias_control_trajectory", bias_control_trajectory)
+
+
+def _mut_trajectory_lagged_update(mp):
+    """The update of step s applied only after step s+1 has routed (one step late)."""
+    def bias_control_trajectory(steps, route_inputs, w_router, bias0, N, K, K_e, mu):
+        b = np.asarray(bias0, dtype=np.float64).copy()
+        hist, pending = [], None
+        for s in range(steps):
+            x, off = route_inputs(s)
+            probs = orc.softmax_rows(orc.router_logits(x, w_router, off))
+            E = probs.shape[1]
+            idx, margin = orc.biased_topk(probs, b, K)
+            counts, rec = _trajectory_record(b, idx, probs, margin, N, E)
+            hist.append(rec)
+            if pending is not None:
+                b = orc.bias_update(b, pending, N, K, K_e, mu, x.shape[0])
+            pending = counts
+        return hist, b
+    mp.setattr(orc, "bias_control_trajectory", bias_control_trajectory)
+
+
+MUTATIONS = [_mut_mxfp8_h_unquantised, _mut_mxfp8_h_wrong_axis, _mut_mxfp8_x_unquantised,
+             _mut_trajectory_routes_with_next_bias, _mut_trajectory_lagged_update,
+             _mut_lb_gradient_without_frequency, _mut_silu_derivative_sigma_only,
              _mut_softmax_backward_no_centering,
              _mut_e4m3_ties_away, _mut_mx_scale_off_by_one, _mut_lb_indicator_per_token, _mut_lb_zero_group_normaliser, _mut_gate_renormalised, _mut_combine_drops_zero_term, _mut_bias_sign,
              _mut_bias_updates_zero_experts, _mut_tie_to_high_index, _mut_select_by_unbiased,
