@@ -20,6 +20,23 @@ inline std::atomic<unsigned long long>& launch_counter() {
 }
 inline void note_launch() { launch_counter().fetch_add(1, std::memory_order_relaxed); }
 
+// Process-wide settings of the GEMMs' bounded pipeline waits, read at every
+// launch (moe_debug_set_pipeline): the time limit of one wait (0: the default
+// of 4 s) and, for tests of the timeout path, a producer that issues nothing.
+struct PipelineDebug {
+  std::atomic<unsigned long long> wait_ns{0};
+  std::atomic<int> stall_fill{0};
+};
+inline PipelineDebug& pipeline_debug() {
+  static PipelineDebug d;
+  return d;
+}
+constexpr unsigned long long kDefaultWaitNs = 4000000000ull;  // 4 s
+inline unsigned long long pipeline_wait_ns() {
+  const unsigned long long v = pipeline_debug().wait_ns.load(std::memory_order_relaxed);
+  return v ? v : kDefaultWaitNs;
+}
+
 constexpr int kMaxExperts = 1024;   // E = N + Z upper bound (one warp holds <= 32 per lane)
 constexpr int kPermChunk = 256;     // tokens per dispatch chunk (one thread per token)
 constexpr int kRouteTokensPerCta = 32;  // 16 warps x 2 tokens: enough warps to hide latency

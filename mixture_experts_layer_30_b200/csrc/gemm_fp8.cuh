@@ -61,6 +61,7 @@ struct ArgsF8 {
   void* out;                   // gated: h E4M3 [rows, n_out]; plain: y bf16 [rows, n_out]
   uint8_t* out_sf;             // gated: h scales [rows, n_out / 32]
   uint32_t* status;
+  unsigned long long wait_ns;  // time limit of one pipeline wait (set at launch)
 };
 
 // --- PTX wrappers ----------------------------------------------------------
@@ -203,7 +204,7 @@ gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
       }
       for (int kb = 0; kb < nk; ++kb) {
         int go = 1;
-        if (lane == 0) go = mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status);
+        if (lane == 0) go = mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status, args.wait_ns);
         go = __shfl_sync(0xffffffffu, go, 0);
         if (!go) {
           ok = false;
@@ -248,11 +249,11 @@ gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const Tile t = decode_tile<kNMax>(tile, n_fblk, targs, prefix);
         const int n32 = ((t.n + 31) >> 5) << 5;
-        if (!mbar_wait(tmem_empty, acc_phase ^ 1, abort_flag, args.status)) break;
+        if (!mbar_wait(tmem_empty, acc_phase ^ 1, abort_flag, args.status, args.wait_ns)) break;
         acc_phase ^= 1;
         tc_fence_after();
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.status)) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.status, args.wait_ns)) {
             ok = false;
             break;
           }
@@ -299,7 +300,7 @@ gemm_mxf8_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant
     uint8_t* stg = staging_base + (warp - 2) * (kStagingBytes / kEpiWarps);
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const Tile t = decode_tile<kNMax>(tile, n_fblk, targs, prefix);
-      if (!mbar_wait(tmem_full, acc_phase, abort_flag, args.status)) break;
+      if (!mbar_wait(tmem_full, acc_phase, abort_flag, args.status, args.wait_ns)) break;
       acc_phase ^= 1;
       tc_fence_after();
       constexpr int nhalves = kGatedOut ? 1 : 2;
@@ -450,8 +451,10 @@ static inline moe_status launch_f8(const CUtensorMap& a0, const CUtensorMap& a1,
   }
   long long grid = max_tiles < sms ? max_tiles : sms;
   if (grid < 1) grid = 1;
+  ArgsF8 la = args;
+  la.wait_ns = pipeline_wait_ns();
   launch_pdl(gemm_mxf8_kernel<kGatedOut>, dim3((unsigned)grid), dim3(kThreads),
-             (size_t)smem_bytes<kGatedOut>(), st, a0, a1, b, args);
+             (size_t)smem_bytes<kGatedOut>(), st, a0, a1, b, la);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -56,7 +56,7 @@ constexpr int kStagingBytesF32 = kEpiWarps * 32 * kStagingPitch * 4;
 constexpr int kStagingBytesBf16 = kEpiWarps * 32 * kStagingPitch16 * 2;
 constexpr int kStagingBytesF32Half = kEpiWarps * 16 * kStagingPitch * 4;  // 16 token rows
 constexpr int kCtrlBytes = 256;                  // barriers + tmem slot + abort flag
-constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;  // 4 s
+constexpr unsigned long long kWaitTimeoutNs = kDefaultWaitNs;  // when a launch sets none
 constexpr unsigned long long kDrainTimeoutNs = 200000000ull;  // 0.2 s
 
 // Tile geometry: up to kNMax token rows per tile (UMMA N), kStages shared-memory
@@ -137,6 +137,13 @@ struct Args {
   int k_splits;
   long long split_stride;
   int single_half;             // plain modes: tiles of 128 features, D1 neither loaded nor computed
+  int32_t* zero_i32;           // cleared by CTA 0 after the grid dependency (router: the counts
+  int zero_n;                  // the selection kernel then accumulates), or NULL
+  int prefetch_b;              // TMA producer: prefetch the token boxes of K block kb + this into
+                               // L2 while issuing kb (0: off)
+  unsigned long long wait_ns;  // time limit of one pipeline wait (set at launch)
+  int stall_fill;              // test of the timeout path: the producer issues nothing, so the
+                               // MMA issuer's first wait runs out
 };
 
 // TMA coordinates (column, row) of the weight tile whose first row is `row`
@@ -188,6 +195,7 @@ MOE_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 MOE_DEV bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                        uint32_t* status, unsigned long long limit_ns = kWaitTimeoutNs,
                        bool honour_abort = true) {
+  if (limit_ns == 0) limit_ns = kWaitTimeoutNs;
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -248,6 +256,13 @@ MOE_DEV void cp_async_arrive_noinc(uint32_t bar) {
 // Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2.
 MOE_DEV void l2_prefetch_bulk(const void* p, int bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+// L2 prefetch of one box of a tensor map (no shared memory, no barrier).
+MOE_DEV void tma_prefetch_l2(const CUtensorMap* map, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1)
+               : "memory");
 }
 MOE_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -434,6 +449,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   pdl_wait();  // the prologue above touches no global memory
+  if (args.zero_i32 && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < args.zero_n; i += blockDim.x) args.zero_i32[i] = 0;
   if (args.seg_offsets) {
     build_chunk_prefix(args.seg_offsets, args.nseg, args.max_rows, kNMax, prefix, scan_tmp,
                        args.status);
@@ -460,6 +477,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     return decode_tile<kNMax>(tile - sp * base_tiles, n_fblk, args, prefix);
   };
   int issued = 0;  // producer: stages issued
+  const int produce = args.stall_fill ? 0 : total;  // tiles the producer fills
 
   if (warp == 0 && args.gather_rows) {
     // ---------------- producer, B rows gathered from x with cp.async ----------------
@@ -473,7 +491,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
     const uint64_t pol_x = l2_policy_evict_last();
     constexpr int kRowsPerLane = kNMax / 32;
     const __nv_bfloat16* xsrc = static_cast<const __nv_bfloat16*>(args.gather_src);
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < produce && ok; tile += gridDim.x) {
       int sp, kb0, kb1;
       const Tile t = tile_of(tile, sp, kb0, kb1);
       const int a_row0 = t.seg * args.a_seg_rows + t.f0;
@@ -494,7 +512,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       }
       for (int kb = kb0; kb < kb1; ++kb) {
         int go = 1;
-        if (lane == 0) go = mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status);
+        if (lane == 0) go = mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status, args.wait_ns);
         go = __shfl_sync(0xffffffffu, go, 0);
         if (!go) {
           ok = false;
@@ -532,7 +550,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       bool ok = true;
       const uint64_t pol_w = l2_policy_evict_first();
       const uint64_t pol_x = l2_policy_evict_last();
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int tile = blockIdx.x; tile < produce && ok; tile += gridDim.x) {
         int sp, kb0, kb1;
         const Tile t = tile_of(tile, sp, kb0, kb1);
         const int nbox = (t.n + kBoxRows - 1) / kBoxRows;
@@ -550,8 +568,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
         const uint32_t tx = (args.single_half ? 1 : 2) * kABytes + nbox * kBoxBytes;
         const int a_row0 = t.seg * args.a_seg_rows + t.f0;
         const int a_row1 = a_row0 + args.a1_row_off;
+        const int pf = args.prefetch_b;
+        for (int kb = kb0; kb < kb1 && kb < kb0 + pf; ++kb)
+          for (int b = 0; b < nbox; ++b) tma_prefetch_l2(&tmB, kb * kBK, t.r0 + b * kBoxRows);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status)) {
+          if (pf > 0 && kb + pf < kb1)
+            for (int b = 0; b < nbox; ++b)
+              tma_prefetch_l2(&tmB, (kb + pf) * kBK, t.r0 + b * kBoxRows);
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status, args.wait_ns)) {
             ok = false;
             break;
           }
@@ -599,10 +623,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
         const int buf = local % kAccBufs;
         const uint32_t acc_parity = (uint32_t)((local / kAccBufs) & 1);
         const uint32_t d0 = tmem_base + buf * 2 * kNMax;
-        if (!mbar_wait(tmem_empty0 + 8 * buf, acc_parity ^ 1, abort_flag, args.status)) break;
+        if (!mbar_wait(tmem_empty0 + 8 * buf, acc_parity ^ 1, abort_flag, args.status, args.wait_ns)) break;
         tc_fence_after();
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.status)) {
+          if (!mbar_wait(full0 + 8 * stage, phase, abort_flag, args.status, args.wait_ns)) {
             ok = false;
             break;
           }
@@ -646,7 +670,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
       const int buf = local % kAccBufs;
       const uint32_t acc_parity = (uint32_t)((local / kAccBufs) & 1);
       const uint32_t dbase = tmem_base + lane_base + buf * 2 * kNMax;
-      if (!mbar_wait(tmem_full0 + 8 * buf, acc_parity, abort_flag, args.status)) break;
+      if (!mbar_wait(tmem_full0 + 8 * buf, acc_parity, abort_flag, args.status, args.wait_ns)) break;
       tc_fence_after();
       if constexpr (kMode == kSwigluBwd) {
         // D0 | D1 = dh of features f0.. / f0+128..; a, u from au; da | du to out.
@@ -909,8 +933,11 @@ static inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, co
   }
   long long grid = max_tiles < sms ? max_tiles : sms;
   if (grid < 1) grid = 1;
+  Args la = args;
+  la.wait_ns = pipeline_wait_ns();
+  la.stall_fill = pipeline_debug().stall_fill.load(std::memory_order_relaxed);
   launch_pdl(gemm_tc_kernel<kMode, Cfg, kAMN>, dim3((unsigned)grid), dim3(kThreads),
-             (size_t)Cfg::smem_bytes(staging_bytes<kMode>()), st, a0, a1, b, args);
+             (size_t)Cfg::smem_bytes(staging_bytes<kMode>()), st, a0, a1, b, la);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -1075,8 +1102,8 @@ inline int router_splits(const moe_shape& s) {
 }
 
 inline moe_status launch_router_gemm(const moe_shape& s, const void* x, const void* w,
-                                     const float* offset, float* logits, int sms,
-                                     cudaStream_t st, char* err, size_t errn) {
+                                     const float* offset, float* logits, int32_t* counts,
+                                     int sms, cudaStream_t st, char* err, size_t errn) {
   CUtensorMap a, b;
   const int E = s.N + s.Z;
   if (!make_map(&a, w, (uint64_t)E, s.d, kFeat)) return map_error(err, errn, "w_router");
@@ -1094,6 +1121,9 @@ inline moe_status launch_router_gemm(const moe_shape& s, const void* x, const vo
   g.out = logits;
   g.add = offset;
   g.status = nullptr;
+  g.zero_i32 = counts;  // the selection kernel adds its histograms into them
+  g.zero_n = E;
+  g.prefetch_b = 4;     // token boxes are the first touch of x: hide their HBM latency
   if (E <= kFeat) {
     // at most 128 experts: one accumulator, the second weight half neither loaded nor computed
     g.feat_per_tile = kFeat;

@@ -59,6 +59,7 @@ struct WgArgs {
   int a1_col_off;              // column of the A1 boxes relative to A0's
   int out1_row_off;            // row offset of D1's output (0 or 128)
   uint32_t* status;
+  unsigned long long wait_ns;  // time limit of one pipeline wait (set at launch)
 };
 
 struct WgTile {
@@ -267,7 +268,7 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
         const WgTile t = wg_decode(tile, args, mblk, nblk);
         const int nk = (t.rows + kBK - 1) / kBK;
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status)) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1, abort_flag, args.status, args.wait_ns)) {
             ok = false;
             break;
           }
@@ -301,12 +302,12 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       const uint32_t acc_parity = (uint32_t)((local >> 1) & 1);
       const uint32_t d0 = tmem_base + buf * 2 * kWgN;
       int go = 1;
-      if (lane == 0) go = mbar_wait(tmem_empty0 + 8 * buf, acc_parity ^ 1, abort_flag, args.status);
+      if (lane == 0) go = mbar_wait(tmem_empty0 + 8 * buf, acc_parity ^ 1, abort_flag, args.status, args.wait_ns);
       if (!__shfl_sync(0xffffffffu, go, 0)) break;
       tc_fence_after();
       for (int kb = 0; kb < nk; ++kb) {
         go = 1;
-        if (lane == 0) go = mbar_wait(full0 + 8 * stage, phase, abort_flag, args.status);
+        if (lane == 0) go = mbar_wait(full0 + 8 * stage, phase, abort_flag, args.status, args.wait_ns);
         if (!__shfl_sync(0xffffffffu, go, 0)) {
           ok = false;
           break;
@@ -352,7 +353,7 @@ gemm_wgrad_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant
       const WgTile t = wg_decode(tile, args, mblk, nblk);
       const int buf = local & 1;
       const uint32_t acc_parity = (uint32_t)((local >> 1) & 1);
-      if (!mbar_wait(tmem_full0 + 8 * buf, acc_parity, abort_flag, args.status)) break;
+      if (!mbar_wait(tmem_full0 + 8 * buf, acc_parity, abort_flag, args.status, args.wait_ns)) break;
       tc_fence_after();
       const int r = (hf ? t.m0 + args.out1_row_off : t.m0) + 32 * q;  // first output row
       wg_store_half(om, tmem_base + lane_base + buf * 2 * kWgN + hf * kWgN, t.rows > 0,
@@ -498,7 +499,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
       auto fill_a = [&](const AsUnit& u, int kb) -> bool {
         const int slot = a_issued % kAsSlots;
         const uint32_t par = (uint32_t)((a_issued / kAsSlots) & 1);
-        if (!mbar_wait(a_empty0 + 8 * slot, par ^ 1, abort_flag, args.status)) return false;
+        if (!mbar_wait(a_empty0 + 8 * slot, par ^ 1, abort_flag, args.status, args.wait_ns)) return false;
         const uint32_t fb = a_full0 + 8 * slot;
         const uint32_t sa = smem_u32(aslots + slot * kAsSlotBytes);
         const int row = u.lo + kb * kBK;
@@ -515,7 +516,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
       auto fill_b = [&](const AsUnit& u, int nb, int kb) -> bool {
         const int st = b_issued % kAsBStages;
         const uint32_t par = (uint32_t)((b_issued / kAsBStages) & 1);
-        if (!mbar_wait(b_empty0 + 8 * st, par ^ 1, abort_flag, args.status)) return false;
+        if (!mbar_wait(b_empty0 + 8 * st, par ^ 1, abort_flag, args.status, args.wait_ns)) return false;
         const uint32_t fb = b_full0 + 8 * st;
         const uint32_t sb = smem_u32(bstages + st * kAsBBytes);
         const int row = u.lo + kb * kBK;
@@ -547,8 +548,6 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
       bool ok = true;
       int a_seen = 0, b_seen = 0, local = 0;
       const uint32_t idesc = idesc_bf16(kFeat, kWgN, true, true);
-      int data_end = args.seg_offsets[args.nseg];  // rows written by the forward pass
-      if (data_end < 0 || data_end > args.max_rows) data_end = 0;  // (offsets checked per unit)
       for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
         const AsUnit u = as_decode(unit, args, mblk);
         const int a0 = a_seen;  // first A fill of this unit
@@ -556,7 +555,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
           for (int kb = 0; kb < u.nk && ok; ++kb) {
             const int i = a0 + kb;
             ok = mbar_wait(a_full0 + 8 * (i % kAsSlots), (uint32_t)((i / kAsSlots) & 1), abort_flag,
-                           args.status);
+                           args.status, args.wait_ns);
           }
           if (!ok) break;
           a_seen = a0 + u.nk;
@@ -570,7 +569,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
         for (int nb = 0; nb < nblk && ok; ++nb, ++local) {
           const int buf = local & 1;
           if (!mbar_wait(tmem_empty0 + 8 * buf, (uint32_t)(((local >> 1) & 1) ^ 1), abort_flag,
-                         args.status)) {
+                         args.status, args.wait_ns)) {
             ok = false;
             break;
           }
@@ -584,7 +583,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
             } else {
               ai = a_seen;
               if (!mbar_wait(a_full0 + 8 * (ai % kAsSlots), (uint32_t)((ai / kAsSlots) & 1),
-                             abort_flag, args.status)) {
+                             abort_flag, args.status, args.wait_ns)) {
                 ok = false;
                 break;
               }
@@ -594,7 +593,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
             }
             const int bs = b_seen % kAsBStages;
             if (!mbar_wait(b_full0 + 8 * bs, (uint32_t)((b_seen / kAsBStages) & 1), abort_flag,
-                           args.status)) {
+                           args.status, args.wait_ns)) {
               ok = false;
               break;
             }
@@ -604,9 +603,11 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
             tc_fence_after();
             const uint32_t sa = smem_u32(aslots + (ai % kAsSlots) * kAsSlotBytes);
             const uint32_t sb = smem_u32(bstages + bs * kAsBBytes);
-            // B's rows past the segment meet zero rows of A; only rows past the last
-            // segment (never written, possibly not finite) are cleared
-            if (u.lo + kb * kBK + ((nv + 15) & ~15) > data_end) wg_zero_tail_one(sb, 2, nv);
+            // B's rows past the segment end (the next expert's rows, or rows never
+            // written) meet zero rows of A; they are cleared too, so that a
+            // non-finite gradient row of a neighbour cannot turn 0 * inf into NaN
+            // in this expert's gradient (nothing to do when nv % 16 == 0)
+            wg_zero_tail_one(sb, 2, nv);
             const int ksteps = (nv + 15) >> 4;
             const uint64_t da0 = smem_desc_mn_sw128(sa);
             const uint64_t da1 = smem_desc_mn_sw128(sa + 2 * kMnBoxBytes);
@@ -645,7 +646,7 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
       for (int nb = 0; nb < nblk; ++nb, ++local) {
         const int buf = local & 1;
         if (!mbar_wait(tmem_full0 + 8 * buf, (uint32_t)((local >> 1) & 1), abort_flag,
-                       args.status)) {
+                       args.status, args.wait_ns)) {
           ok = false;
           break;
         }
@@ -715,8 +716,10 @@ static inline moe_status launch_wgrad(const CUtensorMap& a, const CUtensorMap& b
                           ((args.n_out + kWgN - 1) / kWgN);
   long long grid = tiles < sms ? tiles : sms;
   if (grid < 1) grid = 1;
+  WgArgs la = args;
+  la.wait_ns = pipeline_wait_ns();
   launch_pdl(gemm_wgrad_kernel, dim3((unsigned)grid), dim3(kWgThreads), (size_t)kWgSmemBytes, st,
-             a, b, o0, o1, args);
+             a, b, o0, o1, la);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -745,8 +748,10 @@ static inline moe_status launch_wgrad_as(const CUtensorMap& a, const CUtensorMap
   const long long units = (long long)args.nseg * ((args.m_out + args.m_step - 1) / args.m_step);
   long long grid = units < sms ? units : sms;
   if (grid < 1) grid = 1;
+  WgArgs la = args;
+  la.wait_ns = pipeline_wait_ns();
   launch_pdl(gemm_wgrad_as_kernel, dim3((unsigned)grid), dim3(kWgThreads), (size_t)kAsSmemBytes,
-             st, a, b, o0, o1, args);
+             st, a, b, o0, o1, la);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

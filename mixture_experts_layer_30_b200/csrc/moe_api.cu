@@ -2,6 +2,7 @@
 // argument validation, workspace layout and kernel launches.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -63,7 +64,6 @@ struct WsLayout {
 };
 
 int elem_bytes(const moe_shape& s) { return s.dtype == MOE_BF16 ? 2 : 4; }
-int route_ctas(const moe_shape& s) { return (s.T + moe::kRouteTokensPerCta - 1) / moe::kRouteTokensPerCta; }
 int perm_chunks(const moe_shape& s) { return (s.T + moe::kPermChunk - 1) / moe::kPermChunk; }
 
 moe_status validate_shape(const moe_shape* sp) {
@@ -93,6 +93,52 @@ moe_status validate_shape(const moe_shape* sp) {
   return MOE_OK;
 }
 
+// Router of small batches (route_small_kernel): clusters of CL CTAs split the
+// hidden dimension, KIT 16-byte vectors per lane and CTA; VPL experts per lane
+// in the selection.  Used for every fp32 shape it fits and for bf16 shapes
+// whose router GEMM is at most kSmallRouteMaxFlops (decode batches), where one
+// launch of CUDA-core FMAs beats a tensor-core GEMM plus a selection kernel.
+constexpr double kSmallRouteMaxFlops = 4e8;
+struct SmallRoute {
+  bool ok;
+  int CL, KIT, VPL;
+};
+SmallRoute small_route_of(const moe_shape& s) {
+  SmallRoute r{false, 0, 0, 0};
+  const int E = s.N + s.Z;
+  const int per_cta = 32 * (16 / elem_bytes(s));  // hidden elements per CTA and KIT
+  if ((s.T + moe::kSmallTokens - 1) / moe::kSmallTokens > 65535) return r;
+  int kit = 1, cl = (s.d + per_cta - 1) / per_cta;
+  if (cl > moe::kSmallMaxCluster) {
+    kit = 2;
+    cl = (s.d + 2 * per_cta - 1) / (2 * per_cta);
+  }
+  if (cl > moe::kSmallMaxCluster) return r;
+  const bool tc = s.dtype == MOE_BF16 && moe::tc::router_supported(s);
+  if (tc && 2.0 * s.T * E * s.d > kSmallRouteMaxFlops) return r;
+  int vpl = 1;
+  while (32 * vpl < E) vpl *= 2;
+  r.ok = true;
+  r.CL = cl;
+  r.KIT = kit;
+  r.VPL = vpl;
+  return r;
+}
+int small_clusters(const moe_shape& s) {
+  return (s.T + moe::kSmallTokens - 1) / moe::kSmallTokens;
+}
+
+// Selection grid of the large-batch path (topk_kernel).
+int topk_ctas(const moe_shape& s, int sms) {
+  long long g = (s.T + moe::kTopkWarps - 1) / moe::kTopkWarps;
+  const long long cap = std::min<long long>(moe::kTopkMaxCtas, 4LL * sms);
+  return (int)std::max<long long>(1, std::min(g, cap));
+}
+int topk_ctas_bound(const moe_shape& s) {  // for sizing the workspace
+  long long g = (s.T + moe::kTopkWarps - 1) / moe::kTopkWarps;
+  return (int)std::max<long long>(1, std::min<long long>(g, moe::kTopkMaxCtas));
+}
+
 // K splits of the router GEMM: the tensor-core router splits K for small
 // batches; the CUDA-core router does not split.
 int router_nsplit(const moe_shape& s) {
@@ -109,10 +155,13 @@ WsLayout layout_of(const moe_shape& s) {
   };
   const size_t E = (size_t)s.N + s.Z;
   L.status = take(256);
+  const bool small = small_route_of(s).ok;
   // fp32 logits, one [T, E] slab per K split of the tensor-core router GEMM
-  L.logits = take((size_t)router_nsplit(s) * s.T * E * 4);
-  L.route_hist = take((size_t)route_ctas(s) * E * 4);
-  L.route_psum = take((size_t)route_ctas(s) * E * 4);
+  L.logits = take(small ? 0 : (size_t)router_nsplit(s) * s.T * E * 4);
+  // small batches: histogram and column sums of R per cluster; large batches:
+  // column sums of R per selection CTA
+  L.route_hist = take(small ? (size_t)small_clusters(s) * E * 4 : 0);
+  L.route_psum = take((size_t)(small ? small_clusters(s) : topk_ctas_bound(s)) * E * 4);
   L.perm_hist = take((size_t)perm_chunks(s) * s.N * 4);
   L.perm_base = take((size_t)perm_chunks(s) * s.N * 4);
   L.h = take((size_t)s.T * s.K * s.I * elem_bytes(s));
@@ -150,22 +199,69 @@ int sm_count() {
 
 // --- launches ---------------------------------------------------------------
 
-// The last CTA reduces the partial histograms itself when the grid is this small.
-constexpr int kFusedReduceMaxCtas = 16;
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cluster_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int cluster_x,
+                               cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)cluster_x;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
-template <int VPL>
-void launch_topk(dim3 grid, cudaStream_t st, const float* logits, int nsplit, const float* bias,
+template <typename T, int KIT, int VPL>
+void launch_small(const moe_shape& s, int CL, cudaStream_t st, const void* x, const void* w,
+                  const float* off, const float* bias, int32_t* idx, float* gate, uint8_t* nffn,
+                  float* probs, int32_t* hist, float* psum, unsigned int* ticket,
+                  int32_t* counts, float* prob_sum) {
+  const int E = s.N + s.Z;
+  launch_cluster_pdl(moe::route_small_kernel<T, KIT, VPL>,
+                     dim3((unsigned)CL, (unsigned)small_clusters(s)), dim3(moe::kSmallThreads),
+                     CL, st, static_cast<const T*>(x), static_cast<const T*>(w), off, bias, s.T,
+                     s.d, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts,
+                     prob_sum);
+}
+
+template <typename T, int KIT>
+void launch_small_vpl(const moe_shape& s, const SmallRoute& r, cudaStream_t st, const void* x,
+                      const void* w, const float* off, const float* bias, int32_t* idx,
+                      float* gate, uint8_t* nffn, float* probs, int32_t* hist, float* psum,
+                      unsigned int* ticket, int32_t* counts, float* prob_sum) {
+#define MOE_SMALL(V) launch_small<T, KIT, V>(s, r.CL, st, x, w, off, bias, idx, gate, nffn, \
+                                             probs, hist, psum, ticket, counts, prob_sum)
+  switch (r.VPL) {
+    case 1: MOE_SMALL(1); break;
+    case 2: MOE_SMALL(2); break;
+    case 4: MOE_SMALL(4); break;
+    case 8: MOE_SMALL(8); break;
+    case 16: MOE_SMALL(16); break;
+    default: MOE_SMALL(32); break;
+  }
+#undef MOE_SMALL
+}
+
+template <int VPL, bool kVec4>
+void launch_topk(int grid, cudaStream_t st, const float* logits, int nsplit, const float* bias,
                  int T, int E, int N, int K, int32_t* idx, float* gate, uint8_t* nffn,
-                 float* probs, int32_t* hist, float* psum, unsigned int* ticket, int32_t* counts,
-                 float* prob_sum) {
+                 float* probs, int32_t* counts, float* psum) {
   if (psum)
-    moe::launch_pdl(moe::softmax_topk_kernel<VPL, true>, dim3(grid), dim3(moe::kRouteThreads),
+    moe::launch_pdl(moe::topk_kernel<VPL, kVec4, true>, dim3(grid), dim3(moe::kTopkWarps * 32),
                     0, st, logits, nsplit, (long long)T * E, bias, T, E, N, K, idx, gate, nffn,
-                    probs, hist, psum, ticket, counts, prob_sum);
+                    probs, counts, psum);
   else
-    moe::launch_pdl(moe::softmax_topk_kernel<VPL, false>, dim3(grid), dim3(moe::kRouteThreads),
+    moe::launch_pdl(moe::topk_kernel<VPL, kVec4, false>, dim3(grid), dim3(moe::kTopkWarps * 32),
                     0, st, logits, nsplit, (long long)T * E, bias, T, E, N, K, idx, gate, nffn,
-                    probs, hist, psum, ticket, counts, prob_sum);
+                    probs, counts, psum);
 }
 
 template <typename T>
@@ -174,45 +270,68 @@ moe_status route_impl(const moe_shape& s, const void* x, const void* w, const fl
                       uint8_t* nffn, float* probs, float* prob_sum, void* ws, const WsLayout& L,
                       cudaStream_t st) {
   const int E = s.N + s.Z;
+  if (s.T == 0) {
+    cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)E * 4, st);
+    if (e == cudaSuccess && prob_sum) e = cudaMemsetAsync(prob_sum, 0, (size_t)E * 4, st);
+    if (e != cudaSuccess) return fail(MOE_ERR_CUDA, "memset: %s", cudaGetErrorString(e));
+    return MOE_OK;
+  }
+  const SmallRoute sr = small_route_of(s);
+  if (sr.ok) {
+    // router, selection and counts in one launch
+    int32_t* hist = at<int32_t>(ws, L.route_hist);
+    float* psum = prob_sum ? at<float>(ws, L.route_psum) : nullptr;
+    unsigned int* ticket = at<unsigned int>(ws, L.status + 4);
+    if (sr.KIT == 1)
+      launch_small_vpl<T, 1>(s, sr, st, x, w, off, bias, idx, gate, nffn, probs, hist, psum,
+                             ticket, counts, prob_sum);
+    else
+      launch_small_vpl<T, 2>(s, sr, st, x, w, off, bias, idx, gate, nffn, probs, hist, psum,
+                             ticket, counts, prob_sum);
+    return check_launch("router + selection (small batch)");
+  }
   float* logits = at<float>(ws, L.logits);
-  int32_t* hist = at<int32_t>(ws, L.route_hist);
   float* psum = prob_sum ? at<float>(ws, L.route_psum) : nullptr;
   int nsplit = 1;
-  bool fused = false;
-  if (s.T > 0) {
-    if (s.dtype == MOE_BF16 && moe::tc::router_supported(s) &&
-        reinterpret_cast<uintptr_t>(off) % 16 == 0) {
-      nsplit = moe::tc::router_splits(s);
-      MOE_TRY(moe::tc::launch_router_gemm(s, x, w, off, logits, sm_count(), st, g_err,
-                                          sizeof(g_err)));
-    } else {
-      dim3 g((E + moe::kRgBN - 1) / moe::kRgBN, (s.T + moe::kRgBM - 1) / moe::kRgBM);
-      moe::launch_pdl(moe::router_gemm_simt_kernel<T>, dim3(g), dim3(256), 0, st,
-          static_cast<const T*>(x), static_cast<const T*>(w), off, logits, s.T, E, s.d);
-      MOE_TRY(check_launch("router gemm"));
-    }
-    const int vpl = (E + 31) / 32;
-    dim3 g(route_ctas(s));
-    // small grid: partial histograms reduced by the last CTA (ticket in the status block)
-    fused = route_ctas(s) <= kFusedReduceMaxCtas;
-    unsigned int* ticket = fused ? at<unsigned int>(ws, L.status + 4) : nullptr;
-    if (vpl <= 1) launch_topk<1>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
-    else if (vpl <= 2) launch_topk<2>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
-    else if (vpl <= 3) launch_topk<3>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
-    else if (vpl <= 4) launch_topk<4>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
-    else if (vpl <= 8) launch_topk<8>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
-    else if (vpl <= 16) launch_topk<16>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
-    else if (vpl <= 24) launch_topk<24>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
-    else launch_topk<32>(g, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts, prob_sum);
-    MOE_TRY(check_launch("softmax/top-K"));
+  if (s.dtype == MOE_BF16 && moe::tc::router_supported(s) &&
+      reinterpret_cast<uintptr_t>(off) % 16 == 0) {
+    nsplit = moe::tc::router_splits(s);
+    MOE_TRY(moe::tc::launch_router_gemm(s, x, w, off, logits, counts, sm_count(), st, g_err,
+                                        sizeof(g_err)));
+  } else {
+    dim3 g((E + moe::kRgBN - 1) / moe::kRgBN, (s.T + moe::kRgBM - 1) / moe::kRgBM);
+    moe::launch_pdl(moe::router_gemm_simt_kernel<T>, dim3(g), dim3(256), 0, st,
+        static_cast<const T*>(x), static_cast<const T*>(w), off, logits, s.T, E, s.d, counts, E);
+    MOE_TRY(check_launch("router gemm"));
   }
-  if (fused) return MOE_OK;  // counts (and prob_sum) written by the top-K kernel
-  moe::launch_pdl(moe::reduce_hist_kernel, dim3((E + 7) / 8), dim3(256), 0, st, hist,
-                  route_ctas(s), E, counts);
-  MOE_TRY(check_launch("count reduce"));
+  const int grid = topk_ctas(s, sm_count());
+  if (E % 4 == 0) {
+    const int q = (E + 127) / 128;  // float4 columns per lane
+#define MOE_TOPK(V) launch_topk<V, true>(grid, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, \
+                                         gate, nffn, probs, counts, psum)
+    if (q <= 1) MOE_TOPK(4);
+    else if (q <= 2) MOE_TOPK(8);
+    else if (q <= 3) MOE_TOPK(12);
+    else if (q <= 4) MOE_TOPK(16);
+    else if (q <= 6) MOE_TOPK(24);
+    else MOE_TOPK(32);
+#undef MOE_TOPK
+  } else {
+    const int vpl = (E + 31) / 32;
+#define MOE_TOPK(V) launch_topk<V, false>(grid, st, logits, nsplit, bias, s.T, E, s.N, s.K, idx, \
+                                          gate, nffn, probs, counts, psum)
+    if (vpl <= 1) MOE_TOPK(1);
+    else if (vpl <= 2) MOE_TOPK(2);
+    else if (vpl <= 4) MOE_TOPK(4);
+    else if (vpl <= 8) MOE_TOPK(8);
+    else if (vpl <= 16) MOE_TOPK(16);
+    else MOE_TOPK(32);
+#undef MOE_TOPK
+  }
+  MOE_TRY(check_launch("softmax/top-K"));
   if (prob_sum) {
-    moe::launch_pdl(moe::reduce_psum_kernel, dim3((E + 7) / 8), dim3(256), 0, st, psum,
-                    s.T > 0 ? route_ctas(s) : 0, E, prob_sum);
+    moe::launch_pdl(moe::reduce_psum_kernel, dim3((E + 7) / 8), dim3(256), 0, st, psum, grid, E,
+                    prob_sum);
     MOE_TRY(check_launch("probability column sums"));
   }
   return MOE_OK;
@@ -566,8 +685,8 @@ moe_status moe_permute_noalloc(const moe_shape* shape, const void* x, const int3
   if (bytes > kNoAllocScratchBytes)
     return fail(MOE_ERR_UNSUPPORTED,
                 "moe_permute_noalloc: T=%d, N=%d needs %zu bytes of dispatch scratch but the "
-                "built-in array holds %zu (2*ceil(T/256)*N*4 + 512 must fit); use moe_permute "
-                "with a workspace",
+                "built-in array holds %zu (256 + 2*round_up(ceil(T/256)*N*4, 256) must fit); "
+                "use moe_permute with a workspace",
                 s.T, s.N, bytes, kNoAllocScratchBytes);
   void* scratch = nullptr;
   MOE_TRY(noalloc_scratch(&scratch));
@@ -1173,5 +1292,15 @@ moe_status moe_get_device_status(void* ws, void* stream, uint32_t* status_out) {
 const char* moe_last_error(void) { return g_err; }
 
 uint64_t moe_kernel_launches(void) { return moe::launch_counter().load(); }
+
+moe_status moe_debug_set_pipeline(uint64_t wait_limit_ns, int32_t stall_first_fill) {
+  g_err[0] = 0;
+  if (wait_limit_ns > 60000000000ull)
+    return fail(MOE_ERR_INVALID_ARG, "wait limit %llu ns is above one minute",
+                (unsigned long long)wait_limit_ns);
+  moe::pipeline_debug().wait_ns.store(wait_limit_ns, std::memory_order_relaxed);
+  moe::pipeline_debug().stall_fill.store(stall_first_fill ? 1 : 0, std::memory_order_relaxed);
+  return MOE_OK;
+}
 
 }  // extern "C"

@@ -1,5 +1,22 @@
 // Router and biased top-K selection: LongCat-Flash Technical Report, §2.1, Eq. (1).
+//
+// Two routes to the same result:
+//   * small batches (decode, the fp32 layers): route_small_kernel, one launch.
+//     A cluster of CTAs computes a block of tokens' logits with fp32 FMAs, each
+//     CTA over its own slice of the hidden dimension; CTA 0 of the cluster adds
+//     the slices in rank order through distributed shared memory, then runs the
+//     softmax and the selection.  The last cluster to finish reduces the
+//     per-cluster histograms into the counts.
+//   * large batches: the tensor-core router GEMM writes fp32 logits (and zeroes
+//     the counts), then topk_kernel selects, one warp per token, and adds its
+//     CTA's histogram to the counts with integer atomics (order-independent, so
+//     the counts are exact and reproducible).
+// Both use route_token: softmax over all N+Z experts in fp32, then the K
+// largest R + b (ties to the lower index) by K rounds of a warp arg-max over
+// each lane's two best candidates.
 #pragma once
+
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 
@@ -7,19 +24,22 @@ namespace moe {
 
 // --- router GEMM on CUDA cores ----------------------------------------------
 // logits[t, e] = sum_j x[t, j] * w[e, j] (+ offset[t, e]), fp32 accumulation.
-// 64x64 output tile per CTA, 256 threads, 4x4 outputs per thread.
+// 64x64 output tile per CTA, 256 threads, 4x4 outputs per thread.  CTA (0, 0)
+// also zeroes `zero_counts` [zero_n] for the selection kernel that follows.
 constexpr int kRgBM = 64, kRgBN = 64, kRgBK = 16;
 
 template <typename TIn>
 __global__ void __launch_bounds__(256)
 router_gemm_simt_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
                         const float* __restrict__ offset, float* __restrict__ logits, int T,
-                        int E, int d) {
+                        int E, int d, int32_t* __restrict__ zero_counts, int zero_n) {
   pdl_trigger();
   pdl_wait();
   __shared__ float As[kRgBK][kRgBM + 4];
   __shared__ float Bs[kRgBK][kRgBN + 4];
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  if (zero_counts && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = tid; i < zero_n; i += blockDim.x) zero_counts[i] = 0;
   const int m0 = blockIdx.y * kRgBM, n0 = blockIdx.x * kRgBN;
   float acc[4][4] = {};
   for (int k0 = 0; k0 < d; k0 += kRgBK) {
@@ -60,9 +80,7 @@ router_gemm_simt_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
   }
 }
 
-// --- softmax + biased top-K + per-CTA histogram -----------------------------
-// One warp per token.  Lane l holds experts e = l + 32*j, j < VPL.
-// Selection key: (R_e + b_e) descending, then e ascending (lower index wins ties).
+// --- selection of one token in one warp --------------------------------------
 
 // Order-preserving map of a float to an unsigned key (larger float -> larger
 // key); -0 is folded into +0 first.  Keys are > 0 for every float, so 0 means
@@ -72,148 +90,223 @@ MOE_DEV uint32_t ordered_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Insert (v, j) into a lane's descending top-3 list; equal values keep the
-// earlier (lower) j first.
-struct Top3 {
-  float v[3];
-  float p[3];
-  int j[3];
-  MOE_DEV void clear() {
-#pragma unroll
-    for (int i = 0; i < 3; ++i) { v[i] = -INFINITY; p[i] = 0.f; j[i] = -1; }
+// Which experts a lane holds.  Strided: lane l holds e = l + 32 j.  Vec4 (row
+// loads of 16 bytes): lane l holds e = 128 (j/4) + 4 l + j%4.  In both, a
+// lane's experts increase with j.
+template <bool kVec4> struct Lanes {
+  static MOE_DEV int expert(int lane, int j) {
+    return kVec4 ? 128 * (j >> 2) + 4 * lane + (j & 3) : lane + 32 * j;
   }
-  MOE_DEV void insert(float vv, float pp, int jj) {
-    if (j[2] >= 0 && !(vv > v[2])) return;
-    if (j[1] < 0 || vv > v[1]) {
-      v[2] = v[1]; p[2] = p[1]; j[2] = j[1];
-      if (j[0] < 0 || vv > v[0]) {
-        v[1] = v[0]; p[1] = p[0]; j[1] = j[0];
-        v[0] = vv; p[0] = pp; j[0] = jj;
-      } else {
-        v[1] = vv; p[1] = pp; j[1] = jj;
-      }
-    } else {
-      v[2] = vv; p[2] = pp; j[2] = jj;
+  static MOE_DEV int owner(int e) { return kVec4 ? (e >> 2) & 31 : e & 31; }
+};
+
+// A lane's two best candidates (biased score s, probability p, slot j; j = -1
+// when empty).  Values are offered in ascending j and only a strictly larger
+// score moves ahead, so equal scores keep the lower expert first.
+struct Best2 {
+  float s0, s1, p0, p1;
+  int j0, j1;
+  MOE_DEV void clear() {
+    s0 = s1 = -INFINITY;
+    p0 = p1 = 0.f;
+    j0 = j1 = -1;
+  }
+  MOE_DEV void offer(float s, float p, int j) {
+    if (j0 < 0 || s > s0) {
+      s1 = s0; p1 = p0; j1 = j0;
+      s0 = s; p0 = p; j0 = j;
+    } else if (j1 < 0 || s > s1) {
+      s1 = s; p1 = p; j1 = j;
     }
   }
   MOE_DEV void pop() {
-    v[0] = v[1]; p[0] = p[1]; j[0] = j[1];
-    v[1] = v[2]; p[1] = p[2]; j[1] = j[2];
-    v[2] = -INFINITY; p[2] = 0.f; j[2] = -1;
+    s0 = s1; p0 = p1; j0 = j1;
+    s1 = -INFINITY; p1 = 0.f; j1 = -1;
   }
 };
 
-// kPsum: also accumulate the column sums of R (per-lane registers over the
-// warp's tokens).  The biased scores are recomputed from R and the bias when a
-// lane's top-3 list is rebuilt instead of being kept in registers, so up to 24
-// scores per lane fit 64 registers and two CTAs share an SM (the LongCat shape,
-// 8192 tokens, then runs as one wave).
-template <int VPL, bool kPsum>
-__global__ void __launch_bounds__(kRouteThreads, (kPsum || VPL > 24) ? 1 : 2)
-softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long split_stride,
-                    const float* __restrict__ bias, int T, int E, int N, int K,
-                    int32_t* __restrict__ topk_idx,
-                    float* __restrict__ topk_gate, uint8_t* __restrict__ n_ffn,
-                    float* __restrict__ probs_out, int32_t* __restrict__ partial_hist,
-                    float* __restrict__ partial_psum, unsigned int* ticket,
-                    int32_t* __restrict__ counts_out, float* __restrict__ psum_out) {
+MOE_DEV float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+// Butterfly sum: every lane ends with the same bits (each step adds the same
+// two numbers on both partners).
+MOE_DEV float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Softmax and biased top-K of token t.  v: this lane's logits (any value for
+// experts >= E) -> its probabilities R (0 for experts >= E).  b: its biases.
+// Writes topk_idx/topk_gate[t, 0..K), n_ffn[t] and adds the K choices to the
+// shared histogram `hist`.
+template <int VPL, bool kVec4>
+MOE_DEV void route_token(float (&v)[VPL], const float (&b)[VPL], int lane, int E, int N, int K,
+                         int t, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
+                         uint8_t* __restrict__ n_ffn, int* hist) {
+  using L = Lanes<kVec4>;
+  float m = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j)
+    if (L::expert(lane, j) < E) m = fmaxf(m, v[j]);
+  m = warp_max(m);
+  float sum = 0.f;
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    v[j] = L::expert(lane, j) < E ? __expf(v[j] - m) : 0.f;
+    sum += v[j];
+  }
+  sum = warp_sum(sum);
+  const float inv = 1.0f / sum;
+  Best2 best;
+  best.clear();
+#pragma unroll
+  for (int j = 0; j < VPL; ++j) {
+    v[j] *= inv;  // R_e
+    if (L::expert(lane, j) < E) best.offer(v[j] + b[j], v[j], j);  // biased score: selection only
+  }
+  uint32_t taken = 0;
+  int nf = 0, my_idx = -1;
+  float my_gate = 0.f;
+  for (int k = 0; k < K; ++k) {
+    // warp arg-max: the largest score, then the smallest expert among equals
+    const uint32_t key = best.j0 >= 0 ? ordered_key(best.s0) : 0u;
+    const uint32_t mkey = __reduce_max_sync(0xffffffffu, key);
+    const uint32_t cand =
+        (best.j0 >= 0 && key == mkey) ? (uint32_t)L::expert(lane, best.j0) : 0xffffffffu;
+    const int be = (int)__reduce_min_sync(0xffffffffu, cand);
+    const int owner = L::owner(be);
+    const float gate = __shfl_sync(0xffffffffu, best.p0, owner);
+    if (lane == owner && best.j0 >= 0) {
+      taken |= 1u << best.j0;
+      best.pop();
+      if (best.j0 < 0) {
+        // both candidates of this lane are used: rebuild from what is left
+#pragma unroll
+        for (int j = 0; j < VPL; ++j)
+          if (!((taken >> j) & 1u) && L::expert(lane, j) < E) best.offer(v[j] + b[j], v[j], j);
+      }
+    }
+    if (K <= 32) {
+      if (lane == k) {
+        my_idx = be;
+        my_gate = gate;
+      }
+    } else if (lane == 0) {
+      topk_idx[(size_t)t * K + k] = be;
+      topk_gate[(size_t)t * K + k] = gate;
+      if ((unsigned)be < (unsigned)E) atomicAdd(&hist[be], 1);
+    }
+    nf += be < N;
+  }
+  if (K <= 32 && lane < K) {
+    topk_idx[(size_t)t * K + lane] = my_idx;
+    topk_gate[(size_t)t * K + lane] = my_gate;
+    if ((unsigned)my_idx < (unsigned)E) atomicAdd(&hist[my_idx], 1);
+  }
+  if (lane == 0) n_ffn[t] = (uint8_t)nf;
+}
+
+// --- large batches: selection from the router GEMM's logits -------------------
+// One warp per token, tokens strided over a grid of at most kTopkMaxCtas CTAs.
+// logits: nsplit fp32 slabs [T, E] (split-K partials, added in split order).
+// counts must be zero on entry (the router GEMM clears them).
+constexpr int kTopkWarps = 8;
+constexpr int kTopkMaxCtas = 1024;
+
+template <int VPL, bool kVec4>
+MOE_DEV void load_logits(const float* __restrict__ row, int lane, int E, float (&v)[VPL]) {
+  if constexpr (kVec4) {
+#pragma unroll
+    for (int q = 0; q < VPL / 4; ++q) {
+      const int e = 128 * q + 4 * lane;
+      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < E) f = __ldcs(reinterpret_cast<const float4*>(row + e));
+      v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int e = lane + 32 * j;
+      v[j] = e < E ? __ldcs(row + e) : 0.f;
+    }
+  }
+}
+
+template <int VPL, bool kVec4, bool kPsum>
+__global__ void __launch_bounds__(kTopkWarps * 32, VPL <= 12 ? 3 : VPL <= 24 ? 2 : 1)
+topk_kernel(const float* __restrict__ logits, int nsplit, long long split_stride,
+            const float* __restrict__ bias, int T, int E, int N, int K,
+            int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
+            uint8_t* __restrict__ n_ffn, float* __restrict__ probs_out,
+            int32_t* __restrict__ counts, float* __restrict__ partial_psum) {
   pdl_trigger();
-  pdl_wait();
+  using L = Lanes<kVec4>;
   __shared__ int hist[kMaxExperts];
-  __shared__ float psum_acc[kMaxExperts];
-  float ps[kPsum ? VPL : 1];  // this lane's running sums of R over the warp's tokens
+  __shared__ __align__(16) float bias_sh[kMaxExperts];
+  __shared__ float psum_acc[kPsum ? kMaxExperts : 1];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  pdl_wait();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) bias_sh[e] = bias[e];
+  float ps[kPsum ? VPL : 1];
 #pragma unroll
   for (int j = 0; j < (kPsum ? VPL : 1); ++j) ps[j] = 0.f;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int t_begin = blockIdx.x * kRouteTokensPerCta;
-  const int t_end = min(T, t_begin + kRouteTokensPerCta);
-  for (int t = t_begin + warp; t < t_end; t += nwarps) {
-    const float* lrow = logits + (size_t)t * E;
-    float p[VPL];
-    float m = -INFINITY;
+  for (int t = blockIdx.x * kTopkWarps + warp; t < T; t += gridDim.x * kTopkWarps) {
+    const float* row = logits + (size_t)t * E;
+    float v[VPL];
+    load_logits<VPL, kVec4>(row, lane, E, v);
+    // split-K partials: loads of several slabs in flight, added in split order
+    constexpr int kU = VPL <= 4 ? 8 : VPL <= 8 ? 2 : 1;
+    for (int s0 = 1; s0 < nsplit; s0 += kU) {
+      float pv[kU][VPL];
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-      int e = lane + 32 * j;
-      if (e < E) {
-        // split-K partial logits, summed in split order
-        float v = lrow[e];
-        for (int sp = 1; sp < nsplit; ++sp) v += lrow[sp * split_stride + e];
-        p[j] = v;
-      } else {
-        p[j] = -INFINITY;
-      }
-      m = fmaxf(m, p[j]);
-    }
+      for (int u = 0; u < kU; ++u)
+        if (s0 + u < nsplit) load_logits<VPL, kVec4>(row + (s0 + u) * split_stride, lane, E, pv[u]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float sum = 0.f;
+      for (int u = 0; u < kU; ++u)
+        if (s0 + u < nsplit) {
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-      int e = lane + 32 * j;
-      p[j] = e < E ? __expf(p[j] - m) : 0.f;
-      sum += p[j];
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    const float inv = 1.0f / sum;
-    Top3 top;
-    top.clear();
-#pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-      int e = lane + 32 * j;
-      p[j] *= inv;                             // R_e
-      if constexpr (kPsum) ps[j] += p[j];
-      if (e < E) {
-        if (probs_out) probs_out[(size_t)t * E + e] = p[j];
-        top.insert(p[j] + __ldg(bias + e), p[j], j);  // biased score, selection only
-      }
-    }
-    uint32_t taken = 0;
-    int nf = 0;
-    for (int k = 0; k < K; ++k) {
-      // warp arg-max: largest score, then the smallest expert index among equals
-      const uint32_t key = top.j[0] >= 0 ? ordered_key(top.v[0]) : 0u;
-      const uint32_t mkey = __reduce_max_sync(0xffffffffu, key);
-      const uint32_t cand =
-          (key == mkey && top.j[0] >= 0) ? (uint32_t)(lane + 32 * top.j[0]) : 0xffffffffu;
-      const int be = (int)__reduce_min_sync(0xffffffffu, cand);
-      const int owner = be & 31;
-      const float gate = __shfl_sync(0xffffffffu, top.p[0], owner);
-      if (lane == owner) {
-        taken |= 1u << top.j[0];
-        top.pop();
-        if (top.j[0] < 0) {
-          // this lane's three best are used up: rebuild from what is left
-#pragma unroll
-          for (int j = 0; j < VPL; ++j)
-            if (!(taken >> j & 1u) && lane + 32 * j < E)
-              top.insert(p[j] + __ldg(bias + lane + 32 * j), p[j], j);
+          for (int j = 0; j < VPL; ++j) v[j] += pv[u][j];
         }
-      }
-      if (lane == 0) {
-        topk_idx[(size_t)t * K + k] = be;
-        topk_gate[(size_t)t * K + k] = gate;
-        atomicAdd(&hist[be], 1);
-      }
-      nf += be < N;
     }
-    if (lane == 0) n_ffn[t] = (uint8_t)nf;
+    float b[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int e = L::expert(lane, j);
+      b[j] = e < E ? bias_sh[e] : 0.f;
+    }
+    route_token<VPL, kVec4>(v, b, lane, E, N, K, t, topk_idx, topk_gate, n_ffn, hist);
+    if (probs_out) {
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) {
+        const int e = L::expert(lane, j);
+        if (e < E) probs_out[(size_t)t * E + e] = v[j];
+      }
+    }
+    if constexpr (kPsum) {
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) ps[j] += v[j];
+    }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    partial_hist[(size_t)blockIdx.x * E + e] = hist[e];
-  if (kPsum && partial_psum) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int c = hist[e];
+    if (c) atomicAdd(counts + e, c);
+  }
+  if constexpr (kPsum) {
     // column sums of R over the CTA's tokens, warps added in a fixed order
     for (int e = threadIdx.x; e < E; e += blockDim.x) psum_acc[e] = 0.f;
     __syncthreads();
-    for (int w = 0; w < nwarps; ++w) {
+    for (int w = 0; w < kTopkWarps; ++w) {
       if (warp == w) {
 #pragma unroll
         for (int j = 0; j < VPL; ++j) {
-          const int e = lane + 32 * j;
-          if (e < E) psum_acc[e] += ps[kPsum ? j : 0];
+          const int e = L::expert(lane, j);
+          if (e < E) psum_acc[e] += ps[j];
         }
       }
       __syncthreads();
@@ -221,40 +314,214 @@ softmax_topk_kernel(const float* __restrict__ logits, int nsplit, long long spli
     for (int e = threadIdx.x; e < E; e += blockDim.x)
       partial_psum[(size_t)blockIdx.x * E + e] = psum_acc[e];
   }
-  if (ticket) {
-    // Small grids: the CTA that finishes last reduces the per-CTA partials
-    // (the reduce kernels' per-expert order, so the sums are the same bits),
-    // which saves their launch.  The ticket wraps back to 0 after the last CTA.
-    __shared__ unsigned int s_last;
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicInc(ticket, gridDim.x - 1) == gridDim.x - 1;
-    __syncthreads();
-    if (s_last) {
-      __threadfence();
-      const int nparts = gridDim.x;
-      for (int e = warp; e < E; e += nwarps) {
-        int c = 0;
-        float q = 0.f;
-        for (int p = lane; p < nparts; p += 32) {
-          c += __ldcg(partial_hist + (size_t)p * E + e);
-          if (psum_out) q += __ldcg(partial_psum + (size_t)p * E + e);
-        }
+}
+
+// --- small batches: router + selection in one launch ---------------------------
+// Grid (CL, ceil(T / kSmallTokens)), clusters of (CL, 1, 1): cluster c owns tokens
+// c*8 .. c*8+7; CTA r of the cluster owns the hidden slice [r*slice, (r+1)*slice),
+// slice = 32 lanes x 16-byte vectors x KIT.  Warp w computes experts w, w+8, ...:
+// lane l accumulates its vectors of the slice for the 8 tokens with fp32 FMAs,
+// then a fixed shuffle tree sums the 32 lanes.  CTA 0 adds the CL slices in rank
+// order (+ the logit offset) and routes token c*8 + w in warp w.
+constexpr int kSmallTokens = 8;
+constexpr int kSmallThreads = 256;
+constexpr int kSmallMaxCluster = 8;
+
+// Sums acc[0..8) over the warp's 32 lanes; lane l returns the total of token
+// ((l >> 4) & 1) * 4 + ((l >> 3) & 1) * 2 + ((l >> 2) & 1) (lanes that differ
+// only in bits 0-1 hold the same total).
+MOE_DEV float transpose_sum8(const float (&acc)[8], int lane) {
+  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
+  float r4[4];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          c += __shfl_xor_sync(0xffffffffu, c, o);
-          q += __shfl_xor_sync(0xffffffffu, q, o);
-        }
-        if (lane == 0) {
-          counts_out[e] = c;
-          if (psum_out) psum_out[e] = q;
-        }
+  for (int q = 0; q < 4; ++q) {
+    const float send = h16 ? acc[q] : acc[q + 4];
+    const float keep = h16 ? acc[q + 4] : acc[q];
+    r4[q] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+  }
+  float r2[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const float send = h8 ? r4[q] : r4[q + 2];
+    const float keep = h8 ? r4[q + 2] : r4[q];
+    r2[q] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+  }
+  float r1 = (h4 ? r2[1] : r2[0]) + __shfl_xor_sync(0xffffffffu, h4 ? r2[0] : r2[1], 4);
+  r1 += __shfl_xor_sync(0xffffffffu, r1, 2);
+  r1 += __shfl_xor_sync(0xffffffffu, r1, 1);
+  return r1;
+}
+
+template <typename TIn, int KIT, int VPL>
+__global__ void __launch_bounds__(kSmallThreads)
+route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
+                   const float* __restrict__ offset, const float* __restrict__ bias, int T, int d,
+                   int E, int N, int K, int32_t* __restrict__ topk_idx,
+                   float* __restrict__ topk_gate, uint8_t* __restrict__ n_ffn,
+                   float* __restrict__ probs_out, int32_t* __restrict__ part_hist,
+                   float* __restrict__ part_psum, unsigned int* ticket,
+                   int32_t* __restrict__ counts, float* __restrict__ prob_sum) {
+  pdl_trigger();
+  namespace cg = cooperative_groups;
+  constexpr int VEC = 16 / sizeof(TIn);
+  __shared__ float part[kSmallTokens][kMaxExperts];
+  __shared__ int hist[kMaxExperts];
+  __shared__ unsigned int s_last;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CL = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t0 = blockIdx.y * kSmallTokens;
+  const int k0 = rank * (32 * VEC * KIT);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  pdl_wait();
+
+  // ---- partial logits of the 8 tokens over this CTA's slice ----
+  float xr[KIT][kSmallTokens][VEC];
+#pragma unroll
+  for (int i = 0; i < KIT; ++i) {
+    const int kk = k0 + (i * 32 + lane) * VEC;
+#pragma unroll
+    for (int tt = 0; tt < kSmallTokens; ++tt) {
+      if (t0 + tt < T && kk < d) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + tt) * d + kk));
+        unpack16(u, xr[i][tt], TIn());
+      } else {
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) xr[i][tt][c] = 0.f;
       }
     }
   }
+  // this warp's experts warp, warp + 8, ... in groups of kG; the weight vectors
+  // of the next group are loaded while the current group is computed
+  constexpr int kWarps = kSmallThreads / 32, kG = 4;
+  const int mine = warp < E ? (E - warp + kWarps - 1) / kWarps : 0;
+  auto load_group = [&](int g, uint4 (&raw)[kG][KIT]) {
+#pragma unroll
+    for (int u = 0; u < kG; ++u) {
+      const int e = warp + (g + u) * kWarps;
+#pragma unroll
+      for (int i = 0; i < KIT; ++i) {
+        const int kk = k0 + (i * 32 + lane) * VEC;
+        raw[u][i] = (g + u < mine && kk < d)
+                        ? __ldg(reinterpret_cast<const uint4*>(w + (size_t)e * d + kk))
+                        : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  };
+  uint4 cur[kG][KIT];
+  load_group(0, cur);
+  for (int g = 0; g < mine; g += kG) {
+    uint4 nxt[kG][KIT];
+    load_group(g + kG, nxt);
+#pragma unroll
+    for (int u = 0; u < kG; ++u) {
+      float acc[kSmallTokens];
+#pragma unroll
+      for (int tt = 0; tt < kSmallTokens; ++tt) acc[tt] = 0.f;
+#pragma unroll
+      for (int i = 0; i < KIT; ++i) {
+        float wf[VEC];
+        unpack16(cur[u][i], wf, TIn());
+#pragma unroll
+        for (int c = 0; c < VEC; ++c)
+#pragma unroll
+          for (int tt = 0; tt < kSmallTokens; ++tt) acc[tt] = fmaf(wf[c], xr[i][tt][c], acc[tt]);
+      }
+      const float s = transpose_sum8(acc, lane);
+      const int e = warp + (g + u) * kWarps;
+      if ((lane & 3) == 0 && g + u < mine)
+        part[((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1)][e] = s;
+    }
+#pragma unroll
+    for (int u = 0; u < kG; ++u)
+#pragma unroll
+      for (int i = 0; i < KIT; ++i) cur[u][i] = nxt[u][i];
+  }
+  cluster.sync();  // every CTA's slice is written and visible to the cluster
+
+  if (rank == 0) {
+    // ---- CTA 0: add the slices, then route token t0 + warp ----
+    const int t = t0 + warp;
+    float b[VPL], v[VPL];
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+      const int e = lane + 32 * j;
+      b[j] = e < E ? bias[e] : 0.f;
+      float s = 0.f;
+      if (e < E && t < T) {
+        // every slice's load in flight, then the adds in rank order
+        float pr[kSmallMaxCluster];
+#pragma unroll
+        for (int r = 0; r < kSmallMaxCluster; ++r)
+          pr[r] = r < CL ? cluster.map_shared_rank(&part[warp][e], r)[0] : 0.f;
+#pragma unroll
+        for (int r = 0; r < kSmallMaxCluster; ++r)
+          if (r < CL) s += pr[r];
+        if (offset) s += offset[(size_t)t * E + e];
+      }
+      v[j] = s;
+    }
+    cluster.sync();  // the other CTAs may exit once their slices are read
+    if (t < T) {
+      route_token<VPL, false>(v, b, lane, E, N, K, t, topk_idx, topk_gate, n_ffn, hist);
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E) {
+          if (probs_out) probs_out[(size_t)t * E + e] = v[j];
+          part[warp][e] = v[j];
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < VPL; ++j)
+        if (lane + 32 * j < E) part[warp][lane + 32 * j] = 0.f;
+    }
+    __syncthreads();
+    // this cluster's histogram and column sums of R (tokens in order)
+    const int c = blockIdx.y;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      part_hist[(size_t)c * E + e] = hist[e];
+      if (part_psum) {
+        float q = 0.f;
+#pragma unroll
+        for (int tt = 0; tt < kSmallTokens; ++tt) q += part[tt][e];
+        part_psum[(size_t)c * E + e] = q;
+      }
+    }
+    // the cluster that finishes last adds every cluster's rows, clusters in order
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicInc(ticket, gridDim.y - 1) == gridDim.y - 1;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+      const int nparts = gridDim.y;
+      for (int e = warp; e < E; e += kSmallThreads / 32) {
+        int cnt = 0;
+        float q = 0.f;
+        for (int p = lane; p < nparts; p += 32) {
+          cnt += __ldcg(part_hist + (size_t)p * E + e);
+          if (part_psum) q += __ldcg(part_psum + (size_t)p * E + e);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+          q += __shfl_xor_sync(0xffffffffu, q, o);
+        }
+        if (lane == 0) {
+          counts[e] = cnt;
+          if (prob_sum) prob_sum[e] = q;
+        }
+      }
+    }
+  } else {
+    cluster.sync();  // pairs with CTA 0's second cluster barrier
+  }
 }
 
-// prob_sum[e] = sum over route CTAs of their column sums of R (lane-strided
+// prob_sum[e] = sum over selection CTAs of their column sums of R (lane-strided
 // partial sums, then a fixed shuffle tree: the same order on every run).
 __global__ void __launch_bounds__(256)
 reduce_psum_kernel(const float* __restrict__ partial, int nparts, int E,
@@ -315,23 +582,6 @@ lb_stats_kernel(int N, int Z, int D, const int32_t* __restrict__ counts,
     for (int j = 0; j <= D; ++j) acc += f_sh[j] * p_sh[j];
     *loss = (float)((double)alpha * acc);
   }
-}
-
-// counts[e] = sum over route CTAs of their partial histograms.  One warp per
-// expert; integer sums, so the result does not depend on the order.
-__global__ void __launch_bounds__(256)
-reduce_hist_kernel(const int32_t* __restrict__ partial, int nparts, int E,
-                   int32_t* __restrict__ counts) {
-  pdl_trigger();
-  pdl_wait();
-  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (e >= E) return;
-  int c = 0;
-  for (int p = lane; p < nparts; p += 32) c += partial[(size_t)p * E + e];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-  if (lane == 0) counts[e] = c;
 }
 
 }  // namespace moe

@@ -15,15 +15,23 @@ from mixture_experts_layer_30_b200 import binding as B
 from oracle import moe_oracle as orc
 
 TIE_BAND = 1e-6
-# Router probabilities: the logits are fp32 sums of d bf16 products (tensor
-# cores accumulate in fp32 with truncated alignment inside each K=16 step).
-# A logit error delta changes p by about p * delta, so the bound is relative:
-# |p_gpu - p| <= PROB_ATOL + PROB_RTOL * p.  The top-K check does not depend
-# on it: it is exact outside the 1e-6 tie band.
+# Router probabilities.  fp32 layers: |p_gpu - p| <= 1e-6 (the logits are
+# fp32 FMA chains over d <= 2048 products, rounded to nearest).  bf16 layers:
+# the large-batch router accumulates d bf16 products in fp32 on the tensor
+# cores, whose alignment inside each K = 16 step truncates; a logit error delta
+# moves p by about p * delta, so the bound there is relative as well:
+# |p_gpu - p| <= 1e-6 + 3e-5 p.  The selection check does not rest on either
+# bound: outside the 1e-6 tie band it is exact, and the error of the GPU's
+# scores at each token's decision boundary is recorded (ROUTER_ERRORS) and
+# must stay below half the band, so that no selection with an oracle margin
+# above the band can flip.
 PROB_ATOL = 1e-6
-PROB_RTOL = 3e-5
+PROB_RTOL = {"f32": 0.0, "bf16": 3e-5}
 BF16_MAX_ABS, BF16_REL_L2 = 2e-2, 1e-2
 F32_MAX_ABS = 1e-4
+# measured router errors, one entry per checked forward pass (printed at the
+# end of the session): label -> (max |dp|, max |dp| near the decision boundary)
+ROUTER_ERRORS = {}
 
 
 def to_f64(t: torch.Tensor) -> np.ndarray:
@@ -72,6 +80,23 @@ def assert_ffn_part_close(got_out, want_out, identity_term, dtype, what):
     assert err <= BF16_MAX_ABS and r <= BF16_REL_L2, f"{what}: max-abs {err:.3g}, rel-L2 {r:.3g}"
 
 
+def decision_boundary_error(p_gpu, p_orc, bias, K, window=1e-4):
+    """Largest |p_gpu - p| over the experts that could take part in a selection
+    decision: those whose oracle biased score lies within ``window`` of the
+    token's K-th or (K+1)-th largest score.  (The bias is exact on both sides,
+    so this is the error of the biased scores there.)"""
+    T, E = p_orc.shape
+    if T == 0 or K >= E:
+        return 0.0
+    s = p_orc + bias[None, :]
+    srt = -np.sort(-s, axis=1)
+    lo = srt[:, K][:, None] - window
+    hi = srt[:, K - 1][:, None] + window
+    near = (s >= lo) & (s <= hi)
+    err = np.abs(p_gpu - p_orc)
+    return float(err[near].max()) if near.any() else 0.0
+
+
 def check_selection(gpu_idx, s_orc, orc_idx, K, band=TIE_BAND):
     """Rows where the GPU's ordered top-K differs from the oracle's must be a
     valid ordered top-K of the oracle's biased scores within ``band``.
@@ -110,7 +135,10 @@ class GpuRun:
     def host(self):
         b, s = self.buf, self.buf.shape
         R = int(b.offsets[-1].item())
-        return dict(probs=b.probs.cpu().numpy().astype(np.float64),
+        return dict(dtype="bf16" if s.dtype == B.MOE_BF16 else "f32",
+                    label=f"{'bf16' if s.dtype == B.MOE_BF16 else 'f32'} T={s.T} d={s.d} "
+                          f"E={s.N + s.Z} K={s.K}",
+                    probs=b.probs.cpu().numpy().astype(np.float64),
                     idx=b.topk_idx.cpu().numpy(), gate=b.topk_gate.cpu().numpy().astype(np.float64),
                     counts=b.counts.cpu().numpy(), n_ffn=b.n_ffn.cpu().numpy(),
                     offsets=b.offsets.cpu().numpy(), row_token=b.row_token[:R].cpu().numpy(),
@@ -123,16 +151,23 @@ def check_routing_and_dispatch(g, x64, wr64, bias, N, K, logit_offset=None):
     """Stages 1-3 on every token.  Returns (idx_ref, probs_orc) where idx_ref is
     the oracle's selection with tie-band rows replaced by the GPU's."""
     E = wr64.shape[0]
+    dtype = g.get("dtype", "bf16")
     off = None if logit_offset is None else logit_offset.detach().cpu().numpy().astype(np.float64)
     probs = orc.softmax_rows(orc.router_logits(x64, wr64, off))
-    np.testing.assert_allclose(g["probs"], probs, rtol=PROB_RTOL, atol=PROB_ATOL)
+    np.testing.assert_allclose(g["probs"], probs, rtol=PROB_RTOL[dtype], atol=PROB_ATOL)
     b64 = bias.detach().cpu().numpy().astype(np.float64)
     oidx, margin = orc.biased_topk(probs, b64, K)
+    boundary_err = decision_boundary_error(g["probs"], probs, b64, K)
+    ROUTER_ERRORS[g.get("label", f"T={x64.shape[0]} E={E}")] = (
+        float(np.abs(g["probs"] - probs).max()) if probs.size else 0.0, boundary_err)
+    assert 2 * boundary_err < TIE_BAND, (
+        f"router error {boundary_err:.3g} at the decision boundary could flip a selection "
+        f"whose margin exceeds the {TIE_BAND} band")
     ties = check_selection(g["idx"], probs + b64[None, :], oidx, K)
     idx_ref = oidx.copy()
     idx_ref[ties] = g["idx"][ties]
     np.testing.assert_array_equal(g["idx"], idx_ref)
-    np.testing.assert_allclose(g["gate"], orc.gates(probs, idx_ref), rtol=PROB_RTOL,
+    np.testing.assert_allclose(g["gate"], orc.gates(probs, idx_ref), rtol=PROB_RTOL[dtype],
                                atol=PROB_ATOL)
     np.testing.assert_array_equal(g["counts"], orc.expert_counts(idx_ref, E))
     np.testing.assert_array_equal(g["n_ffn"], orc.ffn_experts_per_token(idx_ref, N))
