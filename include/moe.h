@@ -146,10 +146,12 @@ moe_status moe_permute(const moe_shape* shape, const void* x, const int32_t* top
  * allocates nothing.
  *
  * Scratch: one 4 MiB array in device memory owned by the library, present on
- * every device that loads it until the process exits.  Limit:
- * 2*ceil(T/256)*N*4 + 512 bytes must fit in 4 MiB (for example T <= 131072
- * tokens at N = 1024); larger shapes return MOE_ERR_UNSUPPORTED with a
- * message and launch nothing.
+ * every device that loads it until the process exits.  Limit: a status word
+ * (256 bytes) and two int32 tables of ceil(T/256) x N entries, each rounded up
+ * to a multiple of 256 bytes, must fit:
+ *     256 + 2 * round_up(ceil(T/256) * N * 4, 256) <= 4194304,
+ * for example T <= 130816 tokens at N = 1024 (and any T <= 256).  Larger
+ * shapes return MOE_ERR_UNSUPPORTED with a message and launch nothing.
  * Set-up: the first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) and caches it; make that first call before any
  * stream capture.
@@ -378,6 +380,21 @@ const char* moe_last_error(void);
 /* Number of CUDA kernels this library has launched in the calling process
  * (all devices, all threads).  Instrumentation only. */
 uint64_t moe_kernel_launches(void);
+
+/* Failure-detection settings of the tensor-core GEMMs (gate/up, down, router,
+ * MXFP8 and backward GEMMs), process-wide, read at each later launch.  Not part
+ * of the layer: the pages have no counterpart.
+ *   wait_limit_ns: time after which one bounded pipeline wait gives up
+ *     (0 restores the default of 4 s).  A wait that gives up sets
+ *     MOE_DEV_PIPELINE_TIMEOUT in the workspace status word; the kernel then
+ *     stops issuing work, waits (bounded) for its copies in flight, frees its
+ *     tensor memory and returns, leaving the context usable.  Its output is
+ *     incomplete.
+ *   stall_first_fill: for tests of that path only.  Non-zero makes the
+ *     bf16 GEMMs' TMA producer issue nothing, so the MMA issuer's first wait
+ *     runs out after wait_limit_ns; 0 turns it off.
+ * Returns MOE_ERR_INVALID_ARG for a limit above one minute. */
+moe_status moe_debug_set_pipeline(uint64_t wait_limit_ns, int32_t stall_first_fill);
 
 #ifdef __cplusplus
 }

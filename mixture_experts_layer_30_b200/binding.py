@@ -68,6 +68,7 @@ SIGNATURES = {
     "moe_get_device_status": (ctypes.c_int, [_vp, _vp, ctypes.POINTER(ctypes.c_uint32)]),
     "moe_last_error": (ctypes.c_char_p, []),
     "moe_kernel_launches": (ctypes.c_uint64, []),
+    "moe_debug_set_pipeline": (ctypes.c_int, [ctypes.c_uint64, _i32]),
 }
 
 _lib = None
@@ -338,6 +339,12 @@ def device_status(ws, stream=None) -> int:
     if code not in (0, 5):
         _check(code)
     return int(v.value)
+
+
+def set_pipeline_wait(limit_ns=0, stall_first_fill=False):
+    """Time limit of the GEMMs' bounded pipeline waits (0: the 4 s default);
+    stall_first_fill is for tests of the timeout path only."""
+    _check(lib().moe_debug_set_pipeline(int(limit_ns), 1 if stall_first_fill else 0))
 
 
 class LayerBuffers:

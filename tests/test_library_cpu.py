@@ -162,3 +162,10 @@ def test_route_backward_lb_validation(lib):
     assert b"lb_groups" in lib.moe_last_error()
     assert lib.moe_route_backward(ctypes.byref(s), fake, fake, fake, fake, fake, fake, 4, 0.01,
                                   0, fake, fake, fake, nb, None) == 1
+
+
+def test_pipeline_settings_validation(lib):
+    assert lib.moe_debug_set_pipeline(61_000_000_000, 0) == 1  # above one minute
+    assert b"above one minute" in lib.moe_last_error()
+    assert lib.moe_debug_set_pipeline(1_000_000, 1) == 0
+    assert lib.moe_debug_set_pipeline(0, 0) == 0  # back to the defaults
