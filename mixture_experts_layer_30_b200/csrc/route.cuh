@@ -12,8 +12,9 @@
 //     CTA's histogram to the counts with integer atomics (order-independent, so
 //     the counts are exact and reproducible).
 // Both use route_token: softmax over all N+Z experts in fp32, then the K
-// largest R + b (ties to the lower index) by K rounds of a warp arg-max over
-// each lane's two best candidates.
+// largest R + b (ties to the lower index): the scores at or above the K-th
+// largest lane maximum are sorted across the warp (K rounds of a warp arg-max
+// when they do not fit one per lane).
 #pragma once
 
 #include <cooperative_groups.h>
@@ -138,14 +139,52 @@ MOE_DEV float warp_sum(float v) {
   return v;
 }
 
+// Sorts one value per lane across the warp, descending (bitonic network, 15
+// compare-exchange steps).  Equal values never swap.
+MOE_DEV float warp_sort_desc(float v, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const float o = __shfl_xor_sync(0xffffffffu, v, j);
+      const bool keep_max = ((lane & k) == 0) == ((lane & j) == 0);
+      if (keep_max ? (o > v) : (o < v)) v = o;
+    }
+  return v;
+}
+// The same network on (key, payload) pairs; keys are distinct except 0 (empty).
+MOE_DEV void warp_sort_desc(unsigned long long& key, float& pay, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const unsigned long long ok = __shfl_xor_sync(0xffffffffu, key, j);
+      const float op = __shfl_xor_sync(0xffffffffu, pay, j);
+      const bool keep_max = ((lane & k) == 0) == ((lane & j) == 0);
+      if (keep_max ? (ok > key) : (ok < key)) {
+        key = ok;
+        pay = op;
+      }
+    }
+}
+
 // Softmax and biased top-K of token t.  v: this lane's logits (any value for
 // experts >= E) -> its probabilities R (0 for experts >= E).  b: its biases.
 // Writes topk_idx/topk_gate[t, 0..K), n_ffn[t] and adds the K choices to the
-// shared histogram `hist`.
+// shared histogram `hist`.  cand_key / cand_p: this warp's 32-entry scratch in
+// shared memory.
+//
+// Selection.  Every one of the K best scores is at least tau, the K-th largest
+// of the 32 lane maxima (those K lanes hold K scores >= tau).  So the scores
+// >= tau are the candidates; when there are at most 32 of them (always, in
+// practice, for K <= 32) they are gathered one per lane and sorted by (score
+// descending, expert ascending), and lane k takes the k-th.  Otherwise K rounds
+// of a warp arg-max over each lane's two best candidates select them.
 template <int VPL, bool kVec4>
 MOE_DEV void route_token(float (&v)[VPL], const float (&b)[VPL], int lane, int E, int N, int K,
                          int t, int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
-                         uint8_t* __restrict__ n_ffn, int* hist) {
+                         uint8_t* __restrict__ n_ffn, int* hist,
+                         unsigned long long* cand_key, float* cand_p) {
   using L = Lanes<kVec4>;
   float m = -INFINITY;
 #pragma unroll
@@ -160,13 +199,58 @@ MOE_DEV void route_token(float (&v)[VPL], const float (&b)[VPL], int lane, int E
   }
   sum = warp_sum(sum);
   const float inv = 1.0f / sum;
-  Best2 best;
-  best.clear();
+  float lmax = -INFINITY;
 #pragma unroll
   for (int j = 0; j < VPL; ++j) {
     v[j] *= inv;  // R_e
-    if (L::expert(lane, j) < E) best.offer(v[j] + b[j], v[j], j);  // biased score: selection only
+    if (L::expert(lane, j) < E) lmax = fmaxf(lmax, v[j] + b[j]);  // biased score: selection only
   }
+  if (K <= 32) {
+    const float tau = __shfl_sync(0xffffffffu, warp_sort_desc(lmax, lane), K - 1);
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) cnt += (L::expert(lane, j) < E && v[j] + b[j] >= tau);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (total <= 32) {
+      int pos = incl - cnt;
+#pragma unroll
+      for (int j = 0; j < VPL; ++j) {
+        const int e = L::expert(lane, j);
+        const float sc = v[j] + b[j];
+        if (e < E && sc >= tau) {
+          cand_key[pos] = ((unsigned long long)ordered_key(sc) << 32) | (0xffffffffu - (uint32_t)e);
+          cand_p[pos] = v[j];
+          ++pos;
+        }
+      }
+      __syncwarp();
+      unsigned long long key = lane < total ? cand_key[lane] : 0ull;
+      float gate = lane < total ? cand_p[lane] : 0.f;
+      __syncwarp();
+      warp_sort_desc(key, gate, lane);
+      const int e = (int)(0xffffffffu - (uint32_t)key);
+      if (lane < K) {
+        topk_idx[(size_t)t * K + lane] = e;
+        topk_gate[(size_t)t * K + lane] = gate;
+        atomicAdd(&hist[e], 1);
+      }
+      const uint32_t ffn = __ballot_sync(0xffffffffu, lane < K && e < N);
+      if (lane == 0) n_ffn[t] = (uint8_t)__popc(ffn);
+      return;
+    }
+  }
+  // ---- K rounds of a warp arg-max (K > 32, or more than 32 candidates) ----
+  Best2 best;
+  best.clear();
+#pragma unroll
+  for (int j = 0; j < VPL; ++j)
+    if (L::expert(lane, j) < E) best.offer(v[j] + b[j], v[j], j);
   uint32_t taken = 0;
   int nf = 0, my_idx = -1;
   float my_gate = 0.f;
@@ -247,6 +331,8 @@ topk_kernel(const float* __restrict__ logits, int nsplit, long long split_stride
   __shared__ int hist[kMaxExperts];
   __shared__ __align__(16) float bias_sh[kMaxExperts];
   __shared__ float psum_acc[kPsum ? kMaxExperts : 1];
+  __shared__ unsigned long long cand_key[kTopkWarps][32];
+  __shared__ float cand_p[kTopkWarps][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   pdl_wait();
@@ -279,7 +365,8 @@ topk_kernel(const float* __restrict__ logits, int nsplit, long long split_stride
       const int e = L::expert(lane, j);
       b[j] = e < E ? bias_sh[e] : 0.f;
     }
-    route_token<VPL, kVec4>(v, b, lane, E, N, K, t, topk_idx, topk_gate, n_ffn, hist);
+    route_token<VPL, kVec4>(v, b, lane, E, N, K, t, topk_idx, topk_gate, n_ffn, hist,
+                            cand_key[warp], cand_p[warp]);
     if (probs_out) {
 #pragma unroll
       for (int j = 0; j < VPL; ++j) {
@@ -366,6 +453,8 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
   constexpr int VEC = 16 / sizeof(TIn);
   __shared__ float part[kSmallTokens][kMaxExperts];
   __shared__ int hist[kMaxExperts];
+  __shared__ unsigned long long cand_key[kSmallThreads / 32][32];
+  __shared__ float cand_p[kSmallThreads / 32][32];
   __shared__ unsigned int s_last;
   cg::cluster_group cluster = cg::this_cluster();
   const int CL = (int)cluster.num_blocks();
@@ -464,7 +553,8 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
     }
     cluster.sync();  // the other CTAs may exit once their slices are read
     if (t < T) {
-      route_token<VPL, false>(v, b, lane, E, N, K, t, topk_idx, topk_gate, n_ffn, hist);
+      route_token<VPL, false>(v, b, lane, E, N, K, t, topk_idx, topk_gate, n_ffn, hist,
+                              cand_key[warp], cand_p[warp]);
 #pragma unroll
       for (int j = 0; j < VPL; ++j) {
         const int e = lane + 32 * j;
@@ -496,24 +586,30 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
     if (threadIdx.x == 0) s_last = atomicInc(ticket, gridDim.y - 1) == gridDim.y - 1;
     __syncthreads();
     if (s_last) {
+      // one thread per expert, clusters added in order; the loads of 8
+      // clusters are in flight at once
       __threadfence();
       const int nparts = gridDim.y;
-      for (int e = warp; e < E; e += kSmallThreads / 32) {
+      for (int e = threadIdx.x; e < E; e += kSmallThreads) {
         int cnt = 0;
         float q = 0.f;
-        for (int p = lane; p < nparts; p += 32) {
-          cnt += __ldcg(part_hist + (size_t)p * E + e);
-          if (part_psum) q += __ldcg(part_psum + (size_t)p * E + e);
-        }
+        for (int p0 = 0; p0 < nparts; p0 += 8) {
+          int hv[8];
+          float qv[8];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-          q += __shfl_xor_sync(0xffffffffu, q, o);
+          for (int u = 0; u < 8; ++u) {
+            const bool in = p0 + u < nparts;
+            hv[u] = in ? __ldcg(part_hist + (size_t)(p0 + u) * E + e) : 0;
+            qv[u] = (in && part_psum) ? __ldcg(part_psum + (size_t)(p0 + u) * E + e) : 0.f;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            cnt += hv[u];
+            if (p0 + u < nparts) q += qv[u];
+          }
         }
-        if (lane == 0) {
-          counts[e] = cnt;
-          if (prob_sum) prob_sum[e] = q;
-        }
+        counts[e] = cnt;
+        if (prob_sum) prob_sum[e] = q;
       }
     }
   } else {
