@@ -5,12 +5,17 @@
 One step is one pass of the whole path on one batch: route (router GEMM +
 softmax + biased top-K + counts) -> dispatch to FFN experts -> SwiGLU expert
 GEMMs (gate/up, down) -> combine with the identity experts -> expert-bias
-update.  With N > 1 (torchrun) every rank processes its own batch with a full
+update.  With N > 1 every rank processes its own batch with a full
 weight replica (weak scaling); the count histograms are summed over ranks with
 NCCL before the bias update, the one exchange step of the method.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the fp64 CPU
 oracle instead, on a bounded sample of the same workload.
+
+At N=1 the default LongCat line also carries a "decode" object: the mid layer at
+T = 16, 64, 256 tokens, one CUDA graph per step with L2 flushed before every
+step, and its HBM fraction (--no-decode skips it).  ``--gpus N`` without
+torchrun starts the N ranks itself (one process per GPU).
 
 Options: --graph (replay one captured CUDA graph per step), --fp8-experts
 (MXFP8 expert weights), --fused-gather (no x_perm copy), --lb-stats (the
@@ -80,35 +85,51 @@ def committed_traffic(kernel, workload):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle samples during the timed region."""
+    """nvidia-smi clock / throttle samples during the timed region.  start()
+    returns once the first sample has arrived, so that a short region is
+    covered too."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
-        self.idx, self.proc = gpu_index, None
+        self.idx, self.proc, self.lines, self.reader = gpu_index, None, [], None
 
     def start(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return
+        first = threading.Event()
+
+        def read():
+            for line in self.proc.stdout:
+                self.lines.append(line)
+                first.set()
+        self.reader = threading.Thread(target=read, daemon=True)
+        self.reader.start()
+        first.wait(timeout=3.0)
+        self.n0 = len(self.lines)  # samples from before the region are dropped
 
     def stop(self):
         if self.proc is None:
             return None
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+            self.proc.wait()
+        self.reader.join(timeout=5)
+        lines = self.lines[max(0, self.n0 - 1):]  # the last sample before the region, onwards
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
+        for line in lines:
             f = [x.strip() for x in line.split(",")]
             if len(f) < 9:
                 continue
@@ -139,8 +160,9 @@ def run_gpu(args, rank, world, local_rank):
     shape = B.shape_of(cfg, weight_layout=B.WEIGHTS_TILED if tiled else B.WEIGHTS_ROW_MAJOR)
     L = IN.make_layer_inputs(cfg, device=dev, base_seed=0)
     # every rank routes its own batch: x drawn with a per-rank seed
-    if rank:
-        L["x"] = IN.make_x(cfg, dev, seed=7_000_000 + rank)
+    seed = MD.rank_x_seed(rank)
+    if seed is not None:
+        L["x"] = IN.make_x(cfg, dev, seed=seed)
     # expert weights repacked once into the tiled order, or quantised to MXFP8
     # (untimed set-up); the row-major originals stay for the oracle baseline
     fp8 = args.fp8_experts
@@ -154,7 +176,7 @@ def run_gpu(args, rank, world, local_rank):
     buf = B.LayerBuffers(shape, device=dev)
     bias = L["bias"].clone()
     counts_global = torch.empty_like(buf.counts)
-    T_all = cfg.T * world
+    T_all = MD.global_tokens(cfg.T)
     K_e, mu = float(np.float32(cfg.K_e)), float(np.float32(cfg.mu))
     if world > 1:
         import torch.distributed as dist
@@ -167,11 +189,21 @@ def run_gpu(args, rank, world, local_rank):
                   P=torch.empty(D_groups + 1, dtype=torch.float32, device=dev),
                   loss=torch.empty(1, dtype=torch.float32, device=dev))
 
+    # Eq. (2) needs only this step's counts: in a captured step it runs on a
+    # second stream beside the expert path (joined before the step ends)
+    fork_bias = bool(args.graph)
+    side = torch.cuda.Stream(dev)
+
     def step(x, ev=None):
         s = shape
         if ev: ev[0].record(stream)
         B.route(s, x, L["w_router"], bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts,
                 buf.n_ffn, prob_sum=None if lb is None else lb["prob_sum"])
+        if fork_bias and not ev:
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                c = MD.global_counts(buf.counts, counts_global) if world > 1 else buf.counts
+                B.bias_update(cfg.N, cfg.Z, c, T_all, cfg.K, K_e, mu, bias, stream=side)
         if lb is not None:
             # Eq. (3)-(5) statistics on this rank's batch
             B.lb_stats(cfg.N, cfg.Z, lb["D"], buf.counts, lb["prob_sum"], cfg.T, cfg.K, K_e,
@@ -199,8 +231,11 @@ def run_gpu(args, rank, world, local_rank):
         if ev: ev[4].record(stream)
         B.combine(s, x, buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos, cfg.gamma, buf.out)
         if ev: ev[5].record(stream)
-        c = MD.global_counts(buf.counts, counts_global) if world > 1 else buf.counts
-        B.bias_update(cfg.N, cfg.Z, c, T_all, cfg.K, K_e, mu, bias)
+        if ev or not fork_bias:
+            c = MD.global_counts(buf.counts, counts_global) if world > 1 else buf.counts
+            B.bias_update(cfg.N, cfg.Z, c, T_all, cfg.K, K_e, mu, bias)
+        else:
+            stream.wait_stream(side)  # the bias update of this step is done
         if ev: ev[6].record(stream)
 
     def barrier():
@@ -258,20 +293,18 @@ def run_gpu(args, rank, world, local_rank):
     ms_total = t0.elapsed_time(t1)
     if flush is not None:
         ms_total = sum(a.elapsed_time(b) for a, b in fl_ev)
+    per_clk = clk  # clocks seen while the per-call events ran
     if graph is not None:
         # per-call breakdown from a separate eager pass
+        pc = ClockSampler(clocks.idx)
+        pc.start()
         for i in range(args.steps):
             step(x, evs[i])
         barrier()
+        per_clk = pc.stop()
     per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n_ev - 1)]
                     for i in range(args.steps)])
-    ms_step_local = ms_total / args.steps
-    if world > 1:
-        tt = torch.tensor([ms_step_local], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_step = float(tt.item())
-    else:
-        ms_step = ms_step_local
+    ms_step = MD.max_over_ranks(ms_total / args.steps, dev)
 
     # ---- end to end through the public API with host buffers ----
     # Every step copies its x from pinned host memory and reads its output back.
@@ -339,11 +372,7 @@ def run_gpu(args, rank, world, local_rank):
     stream.wait_stream(s_out)
     e1.record(stream)
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = MD.max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
     st = B.device_status(buf.ws)
     if st:
         raise RuntimeError(f"device status 0x{st:x} after timing")
@@ -409,16 +438,7 @@ def run_gpu(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": cfg.dtype,
         "data": "synthetic (seeded N(0,1) activations, random-init weights of the stated shape)",
-        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "N": cfg.N, "Z": cfg.Z,
-                   "K": cfg.K, "I": cfg.I, "K_e": cfg.K_e, "tokens_per_rank": cfg.T,
-                   "expert_weights": ("mxfp8 (moe_quantize_weights_mxfp8)" if args.fp8_experts
-                                      else "tiled (moe_pack_weights)" if tiled else "row-major"),
-                   "parallelism": f"token-dp{world} (weights replicated, counts all-reduced)",
-                   "l2": ("flushed before every timed step (256 MB memset, outside the "
-                          "per-step events)") if args.flush_l2 else
-                         (f"inputs larger than L2 ({cfg.N * 3 * cfg.I * cfg.d * wsz / 1e9:.2f} GB "
-                          "of expert weights, 126 MB L2; the touched experts' weights are "
-                          "streamed every step)")},
+        "config": workload_config(cfg, world, args),
         "roofline": {"kernel": ("moe_expert_gate_up_mxfp8 (tcgen05 block-scaled grouped GEMM)"
                                 if fp8 else "moe_expert_gate_up (tcgen05 grouped GEMM + SwiGLU)"),
                      "bound": "hbm", "achieved": round(achieved, 1),
@@ -435,6 +455,12 @@ def run_gpu(args, rank, world, local_rank):
                                        layer_bytes / (hbm_peak * 1e9)) / (ms_step * 1e-3), 4),
             "per_call_ms_median": {k: round(float(v), 4) for k, v in zip(
                 ["route", "permute", "gate_up", "down", "combine", "bias_update"], med)},
+            # the same times in SM cycles at the median clock of that pass (ms x MHz =
+            # thousands of cycles): separates a lower clock (power cap) from the kernel
+            "per_call_kcycles_at_median_clock": None if not per_clk else {
+                k: round(float(v) * per_clk["sm_mhz"], 1) for k, v in zip(
+                    ["route", "permute", "gate_up", "down", "combine", "bias_update"], med)},
+            "per_call_clock_mhz": None if not per_clk else per_clk["sm_mhz"],
         },
         "e2e": {"value": round(cfg.T * world / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
@@ -452,6 +478,35 @@ def run_gpu(args, rank, world, local_rank):
     if args.backward:
         line["training"] = time_training(args, cfg, shape, L, W, dev, stream, L["bias"].clone())
     return line, L
+
+
+# ---------------------------------------------------------------------------
+# decode-sized batches (memory-bound): reported beside the headline
+# ---------------------------------------------------------------------------
+DECODE_WORKLOADS = (C.DECODE_T16, C.DECODE_T64, C.DECODE_T256)
+
+
+def decode_block(args, local_rank):
+    """The mid layer at T = 16, 64 and 256 tokens, measured as its HBM target is
+    stated: one captured CUDA graph per step, L2 flushed (256 MB written) before
+    every step, each step timed alone, and the HBM fraction taken on the bytes
+    the step must move (the touched experts' weights, W_r, x in and out)."""
+    res = {}
+    for cfg in DECODE_WORKLOADS:
+        sub = argparse.Namespace(**vars(args))
+        sub.workload, sub.graph, sub.flush_l2 = cfg.name, True, True
+        sub.backward, sub.lb_stats, sub.fp8_experts = False, False, False
+        sub.steps = max(args.steps, 200)  # >= 36 ms timed: a few clock samples
+        line, _ = run_gpu(sub, 0, 1, local_rank)
+        res[f"T{cfg.T}"] = {
+            "workload": cfg.name, "tokens_per_s": line["value"],
+            "ms_per_step": line["ms_per_step"], "hbm_frac": line["layer"]["hbm_frac"],
+            "touched_experts": line["layer"]["touched_experts"],
+            "per_call_ms_median_eager": line["layer"]["per_call_ms_median"],
+            "gpu_launches_per_step": line["gpu_launches"] // sub.steps,
+            "clocks": line["clocks"]}
+        torch.cuda.empty_cache()
+    return res
 
 
 # ---------------------------------------------------------------------------
@@ -554,6 +609,11 @@ def time_training(args, cfg, shape, L, W, dev, stream, bias):
 # ---------------------------------------------------------------------------
 # oracle timing (CPU baseline / reference arm)
 # ---------------------------------------------------------------------------
+# The fp64 oracle is timed as it stands on the host cores, on a bounded sample
+# of the same workload: routing (router GEMM, softmax, biased top-K, counts) on
+# every token of the batch, and the expert FFNs + combine on a seeded sample of
+# tokens through the whole oracle layer.  Tokens/s extrapolates the sample to
+# the batch: T / (t_route(all T) + t_sample * T / n_sample).
 
 def oracle_threads():
     try:
@@ -567,48 +627,73 @@ def oracle_threads():
     return len(os.sched_getaffinity(0))
 
 
-def oracle_sample(cfg, L, t_begin, n_tok):
-    """Host copies of everything the oracle needs for tokens [t_begin, t_begin+n_tok)."""
-    from oracle import moe_oracle as orc
-
-    def bits(t):
-        t = t.detach().cpu().contiguous()
-        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 \
-            else t.numpy()
-    dec = orc.bf16_bits_to_f64 if cfg.dtype == "bf16" else orc.as_f64
-    x = bits(L["x"][t_begin:t_begin + n_tok])
-    wr = bits(L["w_router"])
-    bias = L["bias"].detach().cpu().numpy()
-    # experts the sample can reach: route it once to find them (not timed)
-    probs = orc.softmax_rows(orc.router_logits(dec(x), dec(wr)))
-    idx, _ = orc.biased_topk(probs, bias, cfg.K)
-    touched = sorted(set(int(e) for e in idx.reshape(-1) if e < cfg.N))
-    w1 = {e: bits(L["w1"][e]) for e in touched}
-    w3 = {e: bits(L["w3"][e]) for e in touched}
-    w2 = {e: bits(L["w2"][e]) for e in touched}
-    return dict(x=x, wr=wr, bias=bias, w1=w1, w3=w3, w2=w2, dec=dec, touched=len(touched))
+def _host_bits(t):
+    t = t.detach().cpu().contiguous()
+    return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 \
+        else t.numpy()
 
 
-def time_oracle(cfg, S):
-    """Seconds for the oracle's full layer (decode, route, dispatch, FFN, combine)."""
-    from oracle import moe_oracle as orc
-    t = time.perf_counter()
-    orc.moe_layer(S["dec"](S["x"]), S["dec"](S["wr"]), S["w1"], S["w3"], S["w2"], S["bias"],
-                  N=cfg.N, K=cfg.K, gamma=cfg.gamma, decode=S["dec"])
-    return time.perf_counter() - t
+class OracleWorkload:
+    """Host copies of the batch for the oracle (expert weights fetched per call)."""
+
+    def __init__(self, cfg, L):
+        from oracle import moe_oracle as orc
+        self.cfg, self.L, self.orc = cfg, L, orc
+        self.dec = orc.bf16_bits_to_f64 if cfg.dtype == "bf16" else orc.as_f64
+        self.x = _host_bits(L["x"])
+        self.wr = _host_bits(L["w_router"])
+        self.bias = L["bias"].detach().cpu().numpy()
+
+    def time_routing(self):
+        """Seconds for routing every token (decode, logits, softmax, top-K, counts)."""
+        orc = self.orc
+        t = time.perf_counter()
+        probs = orc.softmax_rows(orc.router_logits(self.dec(self.x), self.dec(self.wr)))
+        idx, _ = orc.biased_topk(probs, self.bias, self.cfg.K)
+        orc.expert_counts(idx, self.cfg.E)
+        return time.perf_counter() - t
+
+    def time_sample(self, tokens):
+        """Seconds for the whole oracle layer on the given tokens (their experts'
+        weights decoded from the stored bits inside the timed region)."""
+        orc, cfg = self.orc, self.cfg
+        x = self.x[tokens]
+        probs = orc.softmax_rows(orc.router_logits(self.dec(x), self.dec(self.wr)))
+        idx, _ = orc.biased_topk(probs, self.bias, cfg.K)
+        touched = sorted(set(int(e) for e in idx.reshape(-1) if e < cfg.N))
+        w1 = {e: _host_bits(self.L["w1"][e]) for e in touched}
+        w3 = {e: _host_bits(self.L["w3"][e]) for e in touched}
+        w2 = {e: _host_bits(self.L["w2"][e]) for e in touched}
+        t = time.perf_counter()
+        orc.moe_layer(self.dec(x), self.dec(self.wr), w1, w3, w2, self.bias, N=cfg.N, K=cfg.K,
+                      gamma=cfg.gamma, decode=self.dec)
+        return time.perf_counter() - t, len(touched)
+
+
+def sample_tokens(T, n, seed):
+    rng = np.random.default_rng(seed)
+    return np.sort(rng.choice(T, size=min(n, T), replace=False))
 
 
 def cpu_baseline(cfg, L, n_tok):
-    S = oracle_sample(cfg, L, 0, n_tok)
-    sec = time_oracle(cfg, S)
-    return {"value": round(n_tok / sec, 4), "unit": "tokens/s", "cores": oracle_threads(),
+    W = OracleWorkload(cfg, L)
+    t_route = W.time_routing()
+    toks = sample_tokens(cfg.T, n_tok, seed=12345)
+    t_smp, touched = W.time_sample(toks)
+    sec = t_route + t_smp * cfg.T / len(toks)
+    return {"value": round(cfg.T / sec, 4), "unit": "tokens/s", "cores": oracle_threads(),
             "kind": "oracle",
-            "sample": f"first {n_tok} tokens of the {cfg.name} batch through the whole fp64 "
-                      f"oracle layer ({S['touched']} experts decoded from bf16), {sec:.1f} s"}
+            "sample": f"routing on all {cfg.T} tokens of the {cfg.name} batch ({t_route:.1f} s), "
+                      f"then the whole fp64 oracle layer on a seeded sample of {len(toks)} "
+                      f"tokens ({touched} experts decoded from bf16, {t_smp:.1f} s), "
+                      f"extrapolated to the batch"}
 
 
 def run_reference(args, rank, world):
-    """--impl reference: the fp64 CPU oracle on the host cores (rank 0 only)."""
+    """--impl reference: the fp64 CPU oracle on the host cores (rank 0 only).
+    Each step: routing on every token plus the oracle layer on a seeded sample
+    of --ref-tokens tokens (a different sample each step), extrapolated to the
+    whole batch."""
     if rank != 0:
         return None
     cfg = C.CONFIGS[args.workload]
@@ -616,26 +701,29 @@ def run_reference(args, rank, world):
     if cfg.dtype == "bf16" and dev.type != "cuda":
         return {"impl": "reference", "unavailable": "the bf16 workload is drawn on the GPU"}
     L = IN.make_layer_inputs(cfg, device=dev)
+    W = OracleWorkload(cfg, L)
     n_tok = args.ref_tokens
+
+    def step(i):
+        toks = sample_tokens(cfg.T, n_tok, seed=1000 + i)
+        t_smp, _ = W.time_sample(toks)
+        return W.time_routing() + t_smp * cfg.T / len(toks)
     for w in range(args.warmup):
-        time_oracle(cfg, oracle_sample(cfg, L, (w * n_tok) % cfg.T, n_tok))
-    secs = []
-    for i in range(args.steps):
-        S = oracle_sample(cfg, L, ((args.warmup + i) * n_tok) % cfg.T, n_tok)
-        secs.append(time_oracle(cfg, S))
+        step(w)
+    secs = [step(args.warmup + i) for i in range(args.steps)]
     sec = sum(secs) / len(secs)
-    v = round(n_tok / sec, 4)
+    v = round(cfg.T / sec, 4)
     return {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (same seeded workload as the GPU arm)",
-        "config": {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "N": cfg.N, "Z": cfg.Z,
-                   "K": cfg.K, "I": cfg.I, "parallelism": "host cores"},
+        "config": workload_config(cfg, world, args),
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle_threads(),
                          "kind": "oracle",
-                         "sample": f"each step: {n_tok} consecutive tokens of the batch through "
-                                   "the whole fp64 oracle layer"},
+                         "sample": f"each step: routing on all {cfg.T} tokens, then the whole "
+                                   f"fp64 oracle layer on a seeded sample of {n_tok} tokens, "
+                                   "extrapolated to the batch"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -648,9 +736,13 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(C.CONFIGS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--cpu-baseline-tokens", type=int, default=4)
-    ap.add_argument("--ref-tokens", type=int, default=2)
+    ap.add_argument("--cpu-baseline-tokens", type=int, default=16,
+                    help="token sample of the CPU baseline's FFN + combine leg")
+    ap.add_argument("--ref-tokens", type=int, default=2,
+                    help="token sample of each reference-arm step's FFN + combine leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the decode-batch block of the default (LongCat) line")
     ap.add_argument("--lb-stats", action="store_true",
                     help="also compute the device-level load-balance statistics each step")
     ap.add_argument("--fp8-experts", action="store_true",
@@ -669,16 +761,26 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.graph and int(os.environ.get("WORLD_SIZE", "1")) > 1:
-        ap.error("--graph is single-GPU only")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
     if args.backward and args.fp8_experts:
         ap.error("--backward runs on bf16 experts")
     if args.fused_gather and args.fp8_experts:
         ap.error("--fused-gather is a bf16 path")
 
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        # not launched by torchrun: start one process per GPU ourselves
+        if args.impl == "native" and torch.cuda.device_count() < args.gpus:
+            ap.error(f"--gpus {args.gpus} but {torch.cuda.device_count()} GPUs are visible")
+        sys.exit(MD.launch_ranks([sys.executable, os.path.abspath(__file__)] + sys.argv[1:],
+                                 args.gpus))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} disagrees with WORLD_SIZE={world}")
+    if args.graph and world > 1:
+        ap.error("--graph is single-GPU only")
     if args.impl == "reference":
         line = run_reference(args, rank, world)
         if line is not None:
@@ -693,6 +795,9 @@ def main():
     try:
         line, L = run_gpu(args, rank, world, local_rank)
         if line is not None:
+            if (world == 1 and not args.no_decode and args.workload == DEFAULT_WORKLOAD
+                    and not args.fp8_experts):
+                line["decode"] = decode_block(args, local_rank)
             if world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline(C.CONFIGS[args.workload], L,
                                                     args.cpu_baseline_tokens)
