@@ -282,3 +282,41 @@ def test_backward_load_balance_term_changes_only_the_router_gradients():
     assert torch.equal(b0.dy_perm[:R], b1.dy_perm[:R])
     assert not torch.equal(b0.dw_router, b1.dw_router)
     assert not torch.equal(b0.dx, b1.dx)
+
+
+def test_weight_gradients_isolated_from_a_nonfinite_neighbour():
+    """Rows of expert e+1 with an infinite upstream gradient must not reach
+    expert e's weight gradients: the wgrad GEMMs read whole 16-row steps, so the
+    rows past e's segment end are cleared before they meet the zeroed rows of
+    the other operand (0 * inf would be NaN)."""
+    shape, L = _small(96, 256, 8, 0, 2, 128, "bf16", seed=11)
+    buf = B.LayerBuffers(shape, with_probs=True)
+    bb = B.BackwardBuffers(shape)
+    B.forward_train(buf, bb, L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"])
+    dout = _dout(shape, 77)
+    B.combine_backward(shape, L["x"], buf.y_perm, buf.topk_idx, buf.topk_gate, buf.slot_pos,
+                       dout, 1.0, bb.dy_perm, bb.dgate)
+    torch.cuda.synchronize()
+    off = buf.offsets.cpu().numpy()
+    cnt = np.diff(off)
+    nbr = [e for e in range(shape.N - 1) if cnt[e] % 16 and cnt[e + 1] > 0]
+    assert nbr, cnt  # a segment end inside a 16-row step, followed by rows of another expert
+
+    def expert_bwd(dy):
+        B.expert_ffn_backward(shape, buf.x_perm, L["w1"], L["w3"], L["w2"], buf.offsets, buf.h,
+                              bb.au, dy, bb.dx_perm, bb.dw1, bb.dw3, bb.dw2, bb.bws)
+        torch.cuda.synchronize()
+        assert B.device_status(bb.bws) == 0
+        return bb.dw1.clone(), bb.dw3.clone(), bb.dw2.clone()
+
+    clean = expert_bwd(bb.dy_perm)
+    for e in nbr:
+        dy = bb.dy_perm.clone()
+        dy[int(off[e + 1]):int(off[e + 2])] = float("inf")
+        dirty = expert_bwd(dy)
+        for c, d in zip(clean, dirty):
+            for j in range(shape.N):
+                if j == e + 1:
+                    continue
+                assert torch.isfinite(d[j]).all(), (e, j)
+                assert torch.equal(c[j], d[j]), (e, j)

@@ -2,7 +2,9 @@
 I=2048; 38.7 GB of bf16 expert weights), in the launch configuration of the
 benchmark.  Routing, counts and the dispatch layout are checked on every token;
 the expert FFN on a seeded sample of experts (the oracle recomputes their rows
-one by one); the combine stage on every token from the GPU's expert outputs."""
+one by one); the layer output end to end on a seeded sample of tokens (the
+oracle computes those tokens' FFN rows and combines them itself); the combine
+stage on every token from the GPU's expert outputs."""
 import numpy as np
 import pytest
 import torch
@@ -33,16 +35,42 @@ def longcat():
     torch.cuda.empty_cache()
 
 
-def test_longcat_routing_dispatch_and_counts(longcat):
+@pytest.fixture(scope="module")
+def routed_ref(longcat):
+    """Routing, counts and dispatch checked on every token; the oracle's
+    probabilities and its selection (tie-band rows as the GPU chose)."""
     cfg, L, run = longcat
     assert run.status == 0, hex(run.status)
     g = run.host()
     x64 = P.to_f64(L["x"])
     idx_ref, probs, nties = P.check_routing_and_dispatch(g, x64, P.to_f64(L["w_router"]),
                                                          L["bias"], cfg.N, cfg.K)
+    return g, x64, idx_ref, probs
+
+
+def test_longcat_routing_dispatch_and_counts(longcat, routed_ref):
+    cfg, L, run = longcat
+    g, x64, idx_ref, probs = routed_ref
     # b = 0 and iid weights give a mean of K*N/E = 8 FFN experts per token
     assert abs(g["n_ffn"].mean() - cfg.K_e) < 0.1
     assert g["counts"].sum() == cfg.T * cfg.K
+
+
+def test_longcat_output_on_a_token_sample(longcat, routed_ref):
+    """out[t] for 64 seeded tokens against Eq. (1) computed by the oracle alone:
+    its own FFN_e(x_t) for each token's selected experts and its own gates."""
+    cfg, L, run = longcat
+    g, x64, idx_ref, probs = routed_ref
+    toks = np.sort(np.random.default_rng(7).choice(cfg.T, size=64, replace=False))
+    idx_s = idx_ref[toks]
+    gate_s = orc.gates(probs[toks], idx_s)
+    off, rt, sp = orc.canonical_permutation(idx_s, cfg.N)
+    y_s = orc.grouped_ffn(x64[toks][rt], off, L["w1"], L["w3"], L["w2"], decode=P.to_f64)
+    out_s = orc.combine(x64[toks], y_s, idx_s, gate_s, sp, cfg.N, cfg.gamma)
+    P.assert_close(g["out"][toks], out_s, "bf16", "out on the token sample")
+    zm = orc.zero_mass(idx_s, gate_s, cfg.N)
+    P.assert_ffn_part_close(g["out"][toks], out_s, cfg.gamma * zm[:, None] * x64[toks], "bf16",
+                            "out minus identity term on the token sample")
 
 
 def test_longcat_expert_ffn_sampled(longcat):
