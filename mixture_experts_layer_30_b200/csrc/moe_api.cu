@@ -349,6 +349,14 @@ moe_status permute_impl(const moe_shape& s, const void* x, const int32_t* idx,
   int32_t* chist = at<int32_t>(ws, L.perm_hist);
   int32_t* cbase = at<int32_t>(ws, L.perm_base);
   const size_t small_smem = (size_t)17 * s.N * sizeof(uint32_t);
+  const size_t fused_smem = small_smem + (size_t)s.T * s.K * sizeof(int32_t);
+  if (nch == 1 && x_perm && fused_smem <= 48 * 1024) {
+    // one chunk with its copy: layout and gather in one launch
+    moe::launch_pdl(moe::perm_gather_small_kernel<T>, dim3((s.T + 7) / 8), dim3(256), fused_smem,
+                    st, static_cast<const T*>(x), idx, s.T, s.K, s.N, E, s.d, counts, offsets,
+                    row_token, slot_pos, static_cast<T*>(x_perm), status);
+    return check_launch("dispatch layout + gather (small batch)");
+  }
   if (nch == 1 && small_smem <= 48 * 1024) {
     // one chunk (decode): histogram, scan and rank in one CTA
     moe::launch_pdl(moe::perm_small_kernel, dim3(1), dim3(256), small_smem, st, idx, s.T, s.K, s.N, E, counts, offsets,

@@ -186,6 +186,112 @@ perm_small_kernel(const int32_t* __restrict__ topk_idx, int T, int K, int N, int
   }
 }
 
+// A batch of one chunk (T <= 256) together with its copy, in one launch: every
+// CTA builds the whole layout of the batch in shared memory (T*K slots, a few
+// microseconds), CTA 0 writes the layout outputs, and CTA c copies the x rows
+// of tokens 8c .. 8c+7 (one warp each) to all of their rows.  No CTA waits for
+// another.  Shared: bits[8][N], wbase[8][N], tot[N], rows[T*K].
+template <typename T>
+__global__ void __launch_bounds__(256)
+perm_gather_small_kernel(const T* __restrict__ x, const int32_t* __restrict__ topk_idx,
+                         int ntok, int K, int N, int E, int d,
+                         const int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                         int32_t* __restrict__ row_token, int32_t* __restrict__ slot_pos,
+                         T* __restrict__ x_perm, uint32_t* status) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ uint32_t sh_pg[];
+  __shared__ int scan_tmp[33];
+  uint32_t* bits = sh_pg;                                // [8][N]
+  int* wbase = reinterpret_cast<int*>(sh_pg + 8 * N);    // [8][N]
+  int* tot = reinterpret_cast<int*>(sh_pg + 16 * N);     // [N]
+  int* rows = reinterpret_cast<int*>(sh_pg + 17 * N);    // [T*K]
+  const bool writer = blockIdx.x == 0;
+  for (int i = threadIdx.x; i < 8 * N; i += blockDim.x) bits[i] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tt = threadIdx.x;  // token of this thread in the layout
+  if (tt < ntok) {
+    for (int k = 0; k < K; ++k) {
+      const int e = topk_idx[(size_t)tt * K + k];
+      if (e < 0 || e >= E) {
+        if (writer) set_status(status, MOE_DEV_BAD_EXPERT_INDEX);
+        continue;
+      }
+      if (e < N) atomicOr(&bits[warp * N + e], 1u << lane);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < N; e += blockDim.x) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) c += __popc(bits[w * N + e]);
+    tot[e] = c;
+    if (writer && counts && counts[e] != c) set_status(status, MOE_DEV_COUNT_MISMATCH);
+  }
+  __syncthreads();
+  const int per = (N + blockDim.x - 1) / blockDim.x;
+  const int lo = min(N, (int)threadIdx.x * per), hi = min(N, lo + per);
+  int local = 0;
+  for (int e = lo; e < hi; ++e) local += tot[e];
+  int run = block_exclusive_scan(local, scan_tmp, &scan_tmp[32]);
+  for (int e = lo; e < hi; ++e) {
+    if (writer) offsets[e] = run;
+    int b = run;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      wbase[w * N + e] = b;
+      b += __popc(bits[w * N + e]);
+    }
+    run += tot[e];
+  }
+  if (writer && threadIdx.x == 0) offsets[N] = scan_tmp[32];
+  __syncthreads();
+  if (tt < ntok) {
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int k = 0; k < K; ++k) {
+      const int e = topk_idx[(size_t)tt * K + k];
+      int row = -1;
+      if (e >= 0 && e < N) {
+        row = wbase[warp * N + e] + __popc(bits[warp * N + e] & lt);
+        if (writer) row_token[row] = tt;
+      }
+      rows[tt * K + k] = row;
+      if (writer) slot_pos[(size_t)tt * K + k] = row;
+    }
+  }
+  __syncthreads();
+  // copy: warp w of CTA c takes token 8c + w
+  const int t = blockIdx.x * 8 + warp;
+  if (t >= ntok) return;
+  const int nvec = d * (int)sizeof(T) / 16;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+  for (int kb = 0; kb < K; kb += 32) {
+    const int my_row = kb + lane < K ? rows[t * K + kb + lane] : -1;
+    const uint32_t has_rows = __ballot_sync(0xffffffffu, my_row >= 0);
+    for (int v0 = 0; v0 < nvec && has_rows; v0 += 32 * 8) {
+      uint4 piece[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int v = v0 + i * 32 + lane;
+        if (v < nvec) piece[i] = __ldg(src + v);
+      }
+      uint32_t has = has_rows;
+      while (has) {
+        const int j = __ffs(has) - 1;
+        has &= has - 1;
+        const int row = __shfl_sync(0xffffffffu, my_row, j);
+        uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)row * d);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int v = v0 + i * 32 + lane;
+          if (v < nvec) dst[v] = piece[i];
+        }
+      }
+    }
+  }
+}
+
 // One warp per token: the x row is read once from HBM, in pieces of 8 x 16 B
 // per lane held in registers, and each piece is stored to every row of the token.
 template <typename T>
