@@ -63,10 +63,18 @@ constexpr unsigned long long kDrainTimeoutNs = 200000000ull;  // 0.2 s
 // stages.  The D0/D1 accumulator pair takes 2*kNMax TMEM columns; when two
 // pairs fit in the 512 columns the accumulators are double-buffered, so the
 // epilogue of one tile overlaps the MMAs of the next.
-template <int NMAX, int STAGES>
+template <int NMAX, int STAGES, int PREFIX_INTS = kMaxExperts + 1 + 33,
+          bool DIRECT_F32 = false>
 struct TileCfg {
   static constexpr int kNMax = NMAX;
   static constexpr int kStages = STAGES;
+  // chunk prefix of the expert segments (+ scan scratch); a single-segment
+  // GEMM (the router) needs two entries
+  static constexpr int kPrefixInts = PREFIX_INTS;
+  // fp32 epilogue (router mode) without a staging area: lane = feature, each
+  // store one 128-byte row piece (faster for the one-tile-per-CTA router, slower
+  // for the split-K router, whose epilogue is most of each CTA's time)
+  static constexpr bool kDirectF32 = DIRECT_F32;
   static constexpr int kAccBufs = (4 * NMAX <= 512) ? 2 : 1;
   static constexpr int kTmemCols = 512;
   static constexpr int kBBytes = NMAX * kBK * 2;
@@ -74,18 +82,22 @@ struct TileCfg {
   static constexpr int kNumBars = 2 * STAGES + 2 * kAccBufs + 1;  // full, empty, acc full/empty, drain
   // shared memory for an epilogue whose staging area takes `staging` bytes
   __host__ __device__ static constexpr int smem_bytes(int staging) {
-    return 1024 + STAGES * kStageBytes + staging + kCtrlBytes + (kMaxExperts + 1 + 33) * 4;
+    return 1024 + STAGES * kStageBytes + staging + kCtrlBytes + PREFIX_INTS * 4;
   }
   static_assert(NMAX % kBoxRows == 0 && NMAX <= 256, "token tile");
   static_assert(8 * kNumBars + 12 <= kCtrlBytes, "control block");
-  static_assert(smem_bytes(kStagingBytesBf16) <= 232448, "shared memory");
 };
 using CfgWide = TileCfg<256, 3>;    // segments up to 256 rows in one tile, 3 stages
 using CfgN160 = TileCfg<160, 4>;    // segments up to 160 rows, 4 stages (more bytes in flight)
 using CfgDouble = TileCfg<128, 4>;  // <= 128 rows, double-buffered accumulators
-using CfgR192 = TileCfg<192, 3>;    // router: 192 token rows, one wave at T = 8192, E = 768
+// router: 192 token rows (one wave at T = 8192, E = 768), one segment, four stages
+// (the fp32 epilogue needs no staging area)
+#ifndef MOE_ROUTER_STAGES
+#define MOE_ROUTER_STAGES 4
+#endif
+using CfgR192 = TileCfg<192, MOE_ROUTER_STAGES, 16, true>;
 static_assert(CfgWide::smem_bytes(kStagingBytesF32) <= 232448, "router tile");
-static_assert(CfgR192::smem_bytes(kStagingBytesF32) <= 232448, "router tile");
+static_assert(CfgR192::smem_bytes(0) <= 232448, "router tile");
 static_assert(CfgN160::smem_bytes(kStagingBytesF32Half) <= 232448, "SwiGLU backward tile");
 
 // Epilogue modes.
@@ -97,8 +109,8 @@ static_assert(CfgN160::smem_bytes(kStagingBytesF32Half) <= 232448, "SwiGLU backw
 //   kGatedSave  kGated that also writes a = D0 and u = D1 to `aux_out`
 enum Mode { kGated = 0, kPlainBf16 = 1, kPlainF32 = 2, kSwigluBwd = 3, kGatedSave = 4 };
 
-template <int kMode> __host__ __device__ constexpr int staging_bytes() {
-  return kMode == kPlainF32 ? kStagingBytesF32
+template <int kMode, class Cfg> __host__ __device__ constexpr int staging_bytes() {
+  return kMode == kPlainF32 ? (Cfg::kDirectF32 ? 0 : kStagingBytesF32)
                             : kMode == kSwigluBwd ? kStagingBytesF32Half : kStagingBytesBf16;
 }
 
@@ -401,7 +413,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   constexpr int kNMax = Cfg::kNMax, kStages = Cfg::kStages, kAccBufs = Cfg::kAccBufs;
   constexpr int kStageBytes = Cfg::kStageBytes, kNumBars = Cfg::kNumBars;
   constexpr int kTmemCols = Cfg::kTmemCols;
-  constexpr int kStagingBytes = staging_bytes<kMode>();
+  constexpr int kStagingBytes = staging_bytes<kMode, Cfg>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -413,7 +425,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl + 8 * kNumBars + 4);
   volatile int* consumed_sh = reinterpret_cast<volatile int*>(ctrl + 8 * kNumBars + 8);
   int* prefix = reinterpret_cast<int*>(ctrl + kCtrlBytes);
-  int* scan_tmp = prefix + kMaxExperts + 1;
+  int* scan_tmp = prefix + kMaxExperts + 1;  // used only with seg_offsets (full prefix)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t full0 = smem_u32(&bars[0]);
@@ -806,6 +818,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
                 v0[j] = pack_bf16x2(__uint_as_float(v0[j]), __uint_as_float(v0[j + 1]));
             }
           }
+          if constexpr (kMode == kPlainF32 && Cfg::kDirectF32) {
+            // fp32 rows need no transpose: lane = feature, register j = token, so
+            // each store writes 32 consecutive floats (128 bytes) of one row
+            const int f = fbase + lane;
+            if (f < args.n_out) {
+              float* o = static_cast<float*>(args.out) + sp * args.split_stride + f;
+              const bool add = args.add && sp == 0;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                if (j0 + j < t.n) {
+                  const size_t row = (size_t)(t.r0 + j0 + j) * args.n_out;
+                  float v = __uint_as_float(v0[j]);
+                  if (add) v += args.add[row + f];
+                  o[row] = v;
+                }
+              }
+            }
+            continue;
+          }
           // transpose through shared memory: stg[token j][feature lane]
           if (kMode == kPlainF32) {
 #pragma unroll
@@ -924,12 +955,17 @@ static inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, co
   if (dev < 64 && !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kMode, Cfg, kAMN>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Cfg::smem_bytes(staging_bytes<kMode>()));
+                                         Cfg::smem_bytes(staging_bytes<kMode, Cfg>()));
     if (e != cudaSuccess) {
       snprintf(err, errn, "tcgen05 gemm smem attribute: %s", cudaGetErrorString(e));
       return MOE_ERR_CUDA;
     }
     attr_set[dev] = true;
+  }
+  static_assert(Cfg::smem_bytes(staging_bytes<kMode, Cfg>()) <= 232448, "shared memory");
+  if (args.seg_offsets && Cfg::kPrefixInts < kMaxExperts + 1 + 33) {
+    snprintf(err, errn, "tcgen05 gemm: tile config without a segment table given segments");
+    return MOE_ERR_INVALID_ARG;
   }
   long long grid = max_tiles < sms ? max_tiles : sms;
   if (grid < 1) grid = 1;
@@ -937,7 +973,7 @@ static inline moe_status launch(const CUtensorMap& a0, const CUtensorMap& a1, co
   la.wait_ns = pipeline_wait_ns();
   la.stall_fill = pipeline_debug().stall_fill.load(std::memory_order_relaxed);
   launch_pdl(gemm_tc_kernel<kMode, Cfg, kAMN>, dim3((unsigned)grid), dim3(kThreads),
-             (size_t)Cfg::smem_bytes(staging_bytes<kMode>()), st, a0, a1, b, la);
+             (size_t)Cfg::smem_bytes(staging_bytes<kMode, Cfg>()), st, a0, a1, b, la);
   note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -1123,7 +1159,7 @@ inline moe_status launch_router_gemm(const moe_shape& s, const void* x, const vo
   g.status = nullptr;
   g.zero_i32 = counts;  // the selection kernel adds its histograms into them
   g.zero_n = E;
-  g.prefetch_b = 4;     // token boxes are the first touch of x: hide their HBM latency
+  g.prefetch_b = 0;
   if (E <= kFeat) {
     // at most 128 experts: one accumulator, the second weight half neither loaded nor computed
     g.feat_per_tile = kFeat;
