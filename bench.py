@@ -147,6 +147,23 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def workload_config(cfg, world, args):
+    """The ``config`` object of the JSON line; both arms print the same one."""
+    tiled = cfg.dtype == "bf16" and cfg.d % 128 == 0 and cfg.I % 128 == 0
+    fp8 = getattr(args, "fp8_experts", False)
+    wsz = (1 + 1 / 32) if fp8 else (2 if cfg.dtype == "bf16" else 4)
+    return {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "N": cfg.N, "Z": cfg.Z,
+            "K": cfg.K, "I": cfg.I, "K_e": cfg.K_e, "tokens_per_rank": cfg.T,
+            "expert_weights": ("mxfp8 (moe_quantize_weights_mxfp8)" if fp8
+                               else "tiled (moe_pack_weights)" if tiled else "row-major"),
+            "parallelism": f"token-dp{world} (weights replicated, counts all-reduced)",
+            "l2": ("flushed before every timed step (256 MB memset, outside the "
+                   "per-step events)") if getattr(args, "flush_l2", False) else
+                  (f"inputs larger than L2 ({cfg.N * 3 * cfg.I * cfg.d * wsz / 1e9:.2f} GB "
+                   "of expert weights, 126 MB L2; the touched experts' weights are "
+                   "streamed every step)")}
+
+
 # ---------------------------------------------------------------------------
 # GPU arm
 # ---------------------------------------------------------------------------
@@ -272,6 +289,7 @@ def run_gpu(args, rank, world, local_rank):
     fl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
              for _ in range(args.steps)] if flush is not None else None
     barrier()
+    bias_t0 = bias.clone()  # the timed steps are replayed from here (realised work)
     clocks.start()
     t0.record(stream)
     for i in range(args.steps):
@@ -281,7 +299,7 @@ def run_gpu(args, rank, world, local_rank):
             flush.zero_()
             fl_ev[i][0].record(stream)
         if graph is None:
-            step(x, evs[i])
+            step(x)
         else:
             graph.replay()
         if flush is not None:
@@ -293,15 +311,26 @@ def run_gpu(args, rank, world, local_rank):
     ms_total = t0.elapsed_time(t1)
     if flush is not None:
         ms_total = sum(a.elapsed_time(b) for a, b in fl_ev)
-    per_clk = clk  # clocks seen while the per-call events ran
-    if graph is not None:
-        # per-call breakdown from a separate eager pass
-        pc = ClockSampler(clocks.idx)
-        pc.start()
-        for i in range(args.steps):
-            step(x, evs[i])
-        barrier()
-        per_clk = pc.stop()
+    # realised work of the timed steps: the bias (and so the routing) changes every
+    # step, and the layer is deterministic, so the steps are replayed from the same
+    # bias to read each one's counts; the replay must end on the same bias bits
+    bias_end = bias.clone()
+    bias.copy_(bias_t0)
+    timed_counts = []
+    for i in range(args.steps):
+        step(x)
+        timed_counts.append(buf.counts.cpu().numpy().astype(np.int64))
+    replay_equal = bool(torch.equal(bias, bias_end))
+    # per-call breakdown from a separate eager pass: events between the calls
+    # would keep the launches of the timed steps from overlapping
+    pc = ClockSampler(clocks.idx)
+    pc.start()
+    per_counts = []
+    for i in range(args.steps):
+        step(x, evs[i])
+        per_counts.append(buf.counts.cpu().numpy().astype(np.int64))
+    barrier()
+    per_clk = pc.stop()
     per = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(n_ev - 1)]
                     for i in range(args.steps)])
     ms_step = MD.max_over_ranks(ms_total / args.steps, dev)
@@ -394,29 +423,32 @@ def run_gpu(args, rank, world, local_rank):
                      "ffn_experts_per_token_std": round(float(n_ffn.std()), 4),
                      "max_over_mean_expert_load": round(float(load.max() / load.mean()), 4)}
 
-    # ---- algorithmic work of the routed batch (counts of the last step) ----
-    counts = buf.counts.cpu().numpy().astype(np.int64)
-    R = int(counts[:cfg.N].sum())
-    touched = int((counts[:cfg.N] > 0).sum())
+    # ---- algorithmic work of the routed batch: per-step means over the steps
+    # each figure timed (touched experts and routed rows move with the bias) ----
+    def work(cl):
+        return (float(np.mean([(c[:cfg.N] > 0).sum() for c in cl])),
+                float(np.mean([c[:cfg.N].sum() for c in cl])))
+    touched, R = work(timed_counts)          # the timed steps (value, layer fractions)
+    touched_pc, R_pc = work(per_counts)      # the per-call steps (per-kernel rooflines)
+    touched_all = [int((c[:cfg.N] > 0).sum()) for c in timed_counts]
     esz = 2 if cfg.dtype == "bf16" else 4
     # expert operands: bf16/fp32, or MXFP8 (1 byte + a scale byte per 32 values)
     wsz = (1 + 1 / 32) if fp8 else esz
     w13_bytes = touched * 2 * cfg.I * cfg.d * wsz
     w2_bytes = touched * cfg.d * cfg.I * wsz
-    # gate/up reads every routed row of x_perm once and writes h
-    gate_up_bytes = w13_bytes + R * cfg.d * wsz + R * cfg.I * wsz
-    down_bytes = w2_bytes + R * cfg.I * wsz + R * cfg.d * esz
-    gate_up_flops = 4.0 * cfg.d * cfg.I * R
-    down_flops = 2.0 * cfg.d * cfg.I * R
-    router_flops = 2.0 * cfg.d * cfg.E * cfg.T
-    layer_flops = gate_up_flops + down_flops + router_flops
+    # FFN: 6 d I flop per routed row (gate, up, down); router: 2 d E per token
+    layer_flops = 6.0 * cfg.d * cfg.I * R + 2.0 * cfg.d * cfg.E * cfg.T
     layer_bytes = (w13_bytes + w2_bytes + cfg.E * cfg.d * esz + 2 * cfg.T * cfg.d * esz)
     med = np.median(per, axis=0)
     peaks, peak_kind = load_peaks()
     hbm_peak = peaks["hbm_gbs"]
     tflops_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
     gu_ms = float(per[:, 2].mean())
-    achieved = gate_up_bytes / (gu_ms * 1e-3) / 1e9
+    # the per-kernel figures use the work of the steps their events timed
+    gate_up_bytes_pc = (touched_pc * 2 * cfg.I * cfg.d * wsz + R_pc * cfg.d * wsz +
+                        R_pc * cfg.I * wsz)
+    ffn_flops_pc = 6.0 * cfg.d * cfg.I * R_pc
+    achieved = gate_up_bytes_pc / (gu_ms * 1e-3) / 1e9
     traffic = committed_traffic("gate_up", cfg.name)
     ffn_ms = float((per[:, 2] + per[:, 3]).mean())
 
@@ -444,11 +476,15 @@ def run_gpu(args, rank, world, local_rank):
                      "bound": "hbm", "achieved": round(achieved, 1),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs",
-                     "algorithmic_bytes_per_launch": int(gate_up_bytes),
+                     "algorithmic_bytes_per_launch": int(gate_up_bytes_pc),
                      "avg_launch_ms": round(gu_ms, 4)},
         "layer": {
-            "routed_rows": R, "touched_experts": touched,
-            "ffn_tflops": round((gate_up_flops + down_flops) / (ffn_ms * 1e-3) / 1e12, 2),
+            "routed_rows": round(R, 1), "touched_experts": round(touched, 2),
+            "touched_experts_per_step": {"min": min(touched_all), "max": max(touched_all)},
+            "work_accounting": ("per-step means over the timed steps, read by replaying them "
+                                "from the same bias"),
+            "replay_bitwise_equal": replay_equal,
+            "ffn_tflops": round(ffn_flops_pc / (ffn_ms * 1e-3) / 1e12, 2),
             "tensor_frac_of_sustained": round(layer_flops / (ms_step * 1e-3) / 1e12 / tflops_peak, 4),
             "hbm_frac": round(layer_bytes / (ms_step * 1e-3) / 1e9 / hbm_peak, 4),
             "roofline_frac": round(max(layer_flops / (tflops_peak * 1e12),

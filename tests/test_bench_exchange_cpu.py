@@ -101,3 +101,19 @@ def test_bench_refuses_a_gpu_count_other_than_the_world_size():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2"],
                        env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 2 and "disagrees with WORLD_SIZE" in r.stderr
+
+
+def test_both_arms_print_the_same_config():
+    import argparse
+    sys.path.insert(0, ROOT)
+    import bench
+    args = bench_args = argparse.Namespace(fp8_experts=False, flush_l2=False)
+    cfg = C.LONGCAT_PREFILL
+    a = bench.workload_config(cfg, 1, args)
+    b = bench.workload_config(cfg, 1, bench_args)
+    assert a == b and a["workload"] == cfg.name and a["T"] == cfg.T
+    assert set(a) >= {"workload", "T", "d", "N", "Z", "K", "I", "parallelism", "l2"}
+    # every function the arms call exists
+    for name in ("run_gpu", "run_reference", "cpu_baseline", "decode_block", "time_training",
+                 "ClockSampler", "OracleWorkload", "main"):
+        assert callable(getattr(bench, name)), name
