@@ -548,6 +548,8 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
       bool ok = true;
       int a_seen = 0, b_seen = 0, local = 0;
       const uint32_t idesc = idesc_bf16(kFeat, kWgN, true, true);
+      int data_end = args.seg_offsets[args.nseg];  // rows written by the forward pass
+      if (data_end < 0 || data_end > args.max_rows) data_end = 0;  // (offsets checked per unit)
       for (int unit = blockIdx.x; unit < units && ok; unit += gridDim.x) {
         const AsUnit u = as_decode(unit, args, mblk);
         const int a0 = a_seen;  // first A fill of this unit
@@ -603,11 +605,13 @@ gemm_wgrad_as_kernel(const __grid_constant__ CUtensorMap tmA,
             tc_fence_after();
             const uint32_t sa = smem_u32(aslots + (ai % kAsSlots) * kAsSlotBytes);
             const uint32_t sb = smem_u32(bstages + bs * kAsBBytes);
-            // B's rows past the segment end (the next expert's rows, or rows never
-            // written) meet zero rows of A; they are cleared too, so that a
-            // non-finite gradient row of a neighbour cannot turn 0 * inf into NaN
-            // in this expert's gradient (nothing to do when nv % 16 == 0)
-            wg_zero_tail_one(sb, 2, nv);
+            // A holds the gradient rows and is zeroed past every segment end, so
+            // the next expert's gradient rows never enter.  B holds forward
+            // activations (x_perm or h): past a segment end they are the next
+            // expert's rows, finite whenever the forward pass was, and meet those
+            // zero rows.  Only B rows past the last segment (never written,
+            // possibly not finite) are cleared.
+            if (u.lo + kb * kBK + ((nv + 15) & ~15) > data_end) wg_zero_tail_one(sb, 2, nv);
             const int ksteps = (nv + 15) >> 4;
             const uint64_t da0 = smem_desc_mn_sw128(sa);
             const uint64_t da1 = smem_desc_mn_sw128(sa + 2 * kMnBoxBytes);

@@ -10,7 +10,8 @@
 //   3. rank_kernel        per chunk: row of (t, k) = base[c][e] + #earlier tokens of
 //                         the chunk routed to e (warp bitmaps + popcount)
 //   4. gather_kernel      one warp per token: x row copied to each of its rows.
-// A batch of one chunk (decode) runs 1-3 as one kernel (perm_small_kernel).
+// A batch of one chunk (decode) runs 1-4 as one kernel (perm_gather_small_kernel),
+// or 1-3 as perm_small_kernel when no copy is asked for.
 #pragma once
 
 #include "common.cuh"

@@ -453,6 +453,7 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
   constexpr int VEC = 16 / sizeof(TIn);
   __shared__ float part[kSmallTokens][kMaxExperts];
   __shared__ int hist[kMaxExperts];
+  __shared__ float bias_sh[kMaxExperts];
   __shared__ unsigned long long cand_key[kSmallThreads / 32][32];
   __shared__ float cand_p[kSmallThreads / 32][32];
   __shared__ unsigned int s_last;
@@ -464,6 +465,10 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
   const int k0 = rank * (32 * VEC * KIT);
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   pdl_wait();
+  // CTA 0 needs the bias only after the slices are in; its load is in flight
+  // with the first weight loads rather than on the path after them
+  if (rank == 0)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) bias_sh[e] = bias[e];
 
   // ---- partial logits of the 8 tokens over this CTA's slice ----
   float xr[KIT][kSmallTokens][VEC];
@@ -536,7 +541,7 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
       const int e = lane + 32 * j;
-      b[j] = e < E ? bias[e] : 0.f;
+      b[j] = e < E ? bias_sh[e] : 0.f;
       float s = 0.f;
       if (e < E && t < T) {
         // every slice's load in flight, then the adds in rank order
