@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include <nvtx3/nvToolsExt.h>
 
@@ -102,9 +103,10 @@ constexpr double kSmallRouteMaxFlops = 4e8;
 struct SmallRoute {
   bool ok;
   int CL, KIT, VPL;
+  int G;  // token groups per cluster: 1, or every group when they fit one cluster
 };
 SmallRoute small_route_of(const moe_shape& s) {
-  SmallRoute r{false, 0, 0, 0};
+  SmallRoute r{false, 0, 0, 0, 1};
   const int E = s.N + s.Z;
   const int per_cta = 32 * (16 / elem_bytes(s));  // hidden elements per CTA and KIT
   if ((s.T + moe::kSmallTokens - 1) / moe::kSmallTokens > 65535) return r;
@@ -122,6 +124,8 @@ SmallRoute small_route_of(const moe_shape& s) {
   r.CL = cl;
   r.KIT = kit;
   r.VPL = vpl;
+  const int groups = (s.T + moe::kSmallTokens - 1) / moe::kSmallTokens;
+  if (groups * cl <= moe::kSmallMaxWholeCluster) r.G = groups;
   return r;
 }
 int small_clusters(const moe_shape& s) {
@@ -199,37 +203,80 @@ int sm_count() {
 
 // --- launches ---------------------------------------------------------------
 
-template <typename... KArgs, typename... Args>
-cudaError_t launch_cluster_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int cluster_x,
-                               cudaStream_t st, Args... args) {
+cudaLaunchConfig_t cluster_config(dim3 grid, dim3 block, dim3 cluster, cudaStream_t st,
+                                  cudaLaunchAttribute (&attr)[2]) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = (unsigned)cluster_x;
-  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.x = cluster.x;
+  attr[1].val.clusterDim.y = cluster.y;
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  return cfg;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cluster_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, dim3 cluster,
+                               cudaStream_t st, Args... args) {
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = cluster_config(grid, block, cluster, st, attr);
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Whether clusters of `size` CTAs of this kernel can be resident: sizes above
+// the portable 8 need the kernel's opt-in and a device that schedules them.
+// Asked once per kernel and size (no stream work, so it is safe during capture).
+struct ClusterFit {
+  const void* fn;
+  unsigned size;
+  bool ok;
+};
+std::mutex g_cluster_mu;
+std::vector<ClusterFit> g_cluster_fit;
+
+template <typename... KArgs>
+bool cluster_size_ok(void (*kernel)(KArgs...), dim3 cluster) {
+  const unsigned size = cluster.x * cluster.y;
+  if (size <= 8) return true;
+  if (size > (unsigned)moe::kSmallMaxWholeCluster) return false;
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  std::lock_guard<std::mutex> lock(g_cluster_mu);
+  for (const ClusterFit& f : g_cluster_fit)
+    if (f.fn == fn && f.size == size) return f.ok;
+  bool ok = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess;
+  if (ok) {
+    int n = 0;
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg =
+        cluster_config(dim3(cluster.x, cluster.y), dim3(moe::kSmallThreads), cluster, 0, attr);
+    ok = cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) == cudaSuccess && n > 0;
+  }
+  if (!ok) cudaGetLastError();  // a refused query leaves no error behind for the launch check
+  g_cluster_fit.push_back({fn, size, ok});
+  return ok;
+}
+
 template <typename T, int KIT, int VPL>
-void launch_small(const moe_shape& s, int CL, cudaStream_t st, const void* x, const void* w,
-                  const float* off, const float* bias, int32_t* idx, float* gate, uint8_t* nffn,
-                  float* probs, int32_t* hist, float* psum, unsigned int* ticket,
+void launch_small(const moe_shape& s, const SmallRoute& r, cudaStream_t st, const void* x,
+                  const void* w, const float* off, const float* bias, int32_t* idx, float* gate,
+                  uint8_t* nffn, float* probs, int32_t* hist, float* psum, unsigned int* ticket,
                   int32_t* counts, float* prob_sum) {
   const int E = s.N + s.Z;
-  launch_cluster_pdl(moe::route_small_kernel<T, KIT, VPL>,
-                     dim3((unsigned)CL, (unsigned)small_clusters(s)), dim3(moe::kSmallThreads),
-                     CL, st, static_cast<const T*>(x), static_cast<const T*>(w), off, bias, s.T,
-                     s.d, E, s.N, s.K, idx, gate, nffn, probs, hist, psum, ticket, counts,
-                     prob_sum);
+  auto* kernel = moe::route_small_kernel<T, KIT, VPL>;
+  dim3 cluster((unsigned)r.CL, (unsigned)r.G);
+  // one cluster per token group when every group does not fit one resident cluster
+  if (!cluster_size_ok(kernel, cluster)) cluster.y = 1;
+  launch_cluster_pdl(kernel, dim3((unsigned)r.CL, (unsigned)small_clusters(s)),
+                     dim3(moe::kSmallThreads), cluster, st, static_cast<const T*>(x),
+                     static_cast<const T*>(w), off, bias, s.T, s.d, E, s.N, s.K, idx, gate, nffn,
+                     probs, hist, psum, ticket, counts, prob_sum);
 }
 
 template <typename T, int KIT>
@@ -237,7 +284,7 @@ void launch_small_vpl(const moe_shape& s, const SmallRoute& r, cudaStream_t st, 
                       const void* w, const float* off, const float* bias, int32_t* idx,
                       float* gate, uint8_t* nffn, float* probs, int32_t* hist, float* psum,
                       unsigned int* ticket, int32_t* counts, float* prob_sum) {
-#define MOE_SMALL(V) launch_small<T, KIT, V>(s, r.CL, st, x, w, off, bias, idx, gate, nffn, \
+#define MOE_SMALL(V) launch_small<T, KIT, V>(s, r, st, x, w, off, bias, idx, gate, nffn, \
                                              probs, hist, psum, ticket, counts, prob_sum)
   switch (r.VPL) {
     case 1: MOE_SMALL(1); break;

@@ -3,10 +3,12 @@
 // Two routes to the same result:
 //   * small batches (decode, the fp32 layers): route_small_kernel, one launch.
 //     A cluster of CTAs computes a block of tokens' logits with fp32 FMAs, each
-//     CTA over its own slice of the hidden dimension; CTA 0 of the cluster adds
-//     the slices in rank order through distributed shared memory, then runs the
-//     softmax and the selection.  The last cluster to finish reduces the
-//     per-cluster histograms into the counts.
+//     CTA over its own slice of the hidden dimension; CTA 0 of each token group
+//     adds the slices in rank order through distributed shared memory, then runs
+//     the softmax and the selection.  When one cluster holds every token group,
+//     group 0's leader adds the groups' histograms over distributed shared
+//     memory; otherwise the last cluster to finish reduces the per-cluster
+//     histograms from global memory into the counts.
 //   * large batches: the tensor-core router GEMM writes fp32 logits (and zeroes
 //     the counts), then topk_kernel selects, one warp per token, and adds its
 //     CTA's histogram to the counts with integer atomics (order-independent, so
@@ -404,15 +406,28 @@ topk_kernel(const float* __restrict__ logits, int nsplit, long long split_stride
 }
 
 // --- small batches: router + selection in one launch ---------------------------
-// Grid (CL, ceil(T / kSmallTokens)), clusters of (CL, 1, 1): cluster c owns tokens
-// c*8 .. c*8+7; CTA r of the cluster owns the hidden slice [r*slice, (r+1)*slice),
-// slice = 32 lanes x 16-byte vectors x KIT.  Warp w computes experts w, w+8, ...:
-// lane l accumulates its vectors of the slice for the 8 tokens with fp32 FMAs,
-// then a fixed shuffle tree sums the 32 lanes.  CTA 0 adds the CL slices in rank
-// order (+ the logit offset) and routes token c*8 + w in warp w.
+// Grid (CL, ceil(T / kSmallTokens)): grid row g is the token group of tokens
+// g*8 .. g*8+7; CTA (r, g) owns the hidden slice [r*slice, (r+1)*slice), slice =
+// 32 lanes x 16-byte vectors x KIT.  Warp w computes experts w, w+8, ...: lane l
+// accumulates its vectors of the slice for the 8 tokens with fp32 FMAs, then a
+// fixed shuffle tree sums the 32 lanes.  The group's leader, CTA (0, g), adds the
+// CL slices in rank order (+ the logit offset) and routes token g*8 + w in warp w.
+// Clusters are (CL, G): G = 1 (one group per cluster, a ticket finds the last
+// group) or G = every group of the batch (no ticket: group 0's leader adds the
+// leaders' histograms and column sums in group order over distributed shared
+// memory).  Both orders of the column sums are the same: tokens of a group in
+// order, then groups in order.
 constexpr int kSmallTokens = 8;
 constexpr int kSmallThreads = 256;
-constexpr int kSmallMaxCluster = 8;
+constexpr int kSmallMaxCluster = 8;       // CTAs of one token group
+constexpr int kSmallMaxWholeCluster = 16;  // CTAs of a cluster holding every group
+
+// One cluster barrier phase in two halves: arrive (releasing this thread's
+// earlier memory operations, loads of distributed shared memory included) and
+// wait (acquiring every other thread's).  All threads of the cluster take the
+// same phases.
+MOE_DEV void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+MOE_DEV void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // Sums acc[0..8) over the warp's 32 lanes; lane l returns the total of token
 // ((l >> 4) & 1) * 4 + ((l >> 3) & 1) * 2 + ((l >> 2) & 1) (lanes that differ
@@ -454,12 +469,16 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
   __shared__ float part[kSmallTokens][kMaxExperts];
   __shared__ int hist[kMaxExperts];
   __shared__ float bias_sh[kMaxExperts];
+  __shared__ float colsum[kMaxExperts];
   __shared__ unsigned long long cand_key[kSmallThreads / 32][32];
   __shared__ float cand_p[kSmallThreads / 32][32];
   __shared__ unsigned int s_last;
   cg::cluster_group cluster = cg::this_cluster();
-  const int CL = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
+  const dim3 cdim = cluster.dim_blocks();
+  const int CL = (int)cdim.x, G = (int)cdim.y;
+  const int rank = (int)cluster.block_index().x;       // slice
+  const int grp = (int)cluster.block_index().y;        // token group inside the cluster
+  const bool whole = (int)gridDim.y == G;              // one cluster holds every group
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t0 = blockIdx.y * kSmallTokens;
   const int k0 = rank * (32 * VEC * KIT);
@@ -532,11 +551,12 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
 #pragma unroll
       for (int i = 0; i < KIT; ++i) cur[u][i] = nxt[u][i];
   }
-  cluster.sync();  // every CTA's slice is written and visible to the cluster
+  cluster.sync();  // phase 1: every CTA's slice is written and visible to the cluster
 
   if (rank == 0) {
-    // ---- CTA 0: add the slices, then route token t0 + warp ----
+    // ---- the group's leader: add the slices, then route token t0 + warp ----
     const int t = t0 + warp;
+    const int base = grp * CL;  // cluster rank of this group's slice 0
     float b[VPL], v[VPL];
 #pragma unroll
     for (int j = 0; j < VPL; ++j) {
@@ -548,7 +568,7 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
         float pr[kSmallMaxCluster];
 #pragma unroll
         for (int r = 0; r < kSmallMaxCluster; ++r)
-          pr[r] = r < CL ? cluster.map_shared_rank(&part[warp][e], r)[0] : 0.f;
+          pr[r] = r < CL ? cluster.map_shared_rank(&part[warp][e], base + r)[0] : 0.f;
 #pragma unroll
         for (int r = 0; r < kSmallMaxCluster; ++r)
           if (r < CL) s += pr[r];
@@ -556,7 +576,9 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
       }
       v[j] = s;
     }
-    cluster.sync();  // the other CTAs may exit once their slices are read
+    // phase 2, first half: the slices are read, so the other CTAs of the group may
+    // exit; this CTA waits on the phase only after its selection
+    cluster_arrive();
     if (t < T) {
       route_token<VPL, false>(v, b, lane, E, N, K, t, topk_idx, topk_gate, n_ffn, hist,
                               cand_key[warp], cand_p[warp]);
@@ -574,26 +596,58 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
         if (lane + 32 * j < E) part[warp][lane + 32 * j] = 0.f;
     }
     __syncthreads();
-    // this cluster's histogram and column sums of R (tokens in order)
-    const int c = blockIdx.y;
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-      part_hist[(size_t)c * E + e] = hist[e];
-      if (part_psum) {
+    // this group's column sums of R (tokens in order)
+    if (prob_sum)
+      for (int e = threadIdx.x; e < E; e += blockDim.x) {
         float q = 0.f;
 #pragma unroll
         for (int tt = 0; tt < kSmallTokens; ++tt) q += part[tt][e];
-        part_psum[(size_t)c * E + e] = q;
+        colsum[e] = q;
       }
+    cluster_wait();  // phase 2, second half
+    if (whole) {
+      if (G > 1) {
+        cluster.sync();  // phase 3: every leader's histogram and column sums are in
+        if (grp == 0)
+          for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            int cnt = 0;
+            float q = 0.f;
+            for (int j = 0; j < G; ++j) {
+              cnt += cluster.map_shared_rank(&hist[e], j * CL)[0];
+              if (prob_sum) q += cluster.map_shared_rank(&colsum[e], j * CL)[0];
+            }
+            counts[e] = cnt;
+            if (prob_sum) prob_sum[e] = q;
+          }
+        cluster.sync();  // phase 4: group 0 has read the other leaders' arrays
+      } else {
+        __syncthreads();
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+          counts[e] = hist[e];
+          if (prob_sum) prob_sum[e] = colsum[e];
+        }
+      }
+      return;
     }
-    // the cluster that finishes last adds every cluster's rows, clusters in order
-    __threadfence();
+    // one group per cluster: write this group's rows; the group that finishes
+    // last adds every group's rows, groups in order
+    const int c = blockIdx.y;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      part_hist[(size_t)c * E + e] = hist[e];
+      if (part_psum) part_psum[(size_t)c * E + e] = colsum[e];
+    }
+    // the CTA's writes are ordered before the ticket by the barrier and the
+    // releasing fence of the thread that takes it
     __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicInc(ticket, gridDim.y - 1) == gridDim.y - 1;
+    if (threadIdx.x == 0) {
+      __threadfence();
+      s_last = atomicInc(ticket, gridDim.y - 1) == gridDim.y - 1;
+      if (s_last) __threadfence();
+    }
     __syncthreads();
     if (s_last) {
-      // one thread per expert, clusters added in order; the loads of 8
-      // clusters are in flight at once
-      __threadfence();
+      // one thread per expert, groups added in order; the loads of 8 groups are
+      // in flight at once
       const int nparts = gridDim.y;
       for (int e = threadIdx.x; e < E; e += kSmallThreads) {
         int cnt = 0;
@@ -618,7 +672,11 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
       }
     }
   } else {
-    cluster.sync();  // pairs with CTA 0's second cluster barrier
+    cluster.sync();  // phase 2: the leader has read this CTA's slice
+    if (whole && G > 1) {
+      cluster.sync();  // phase 3
+      cluster.sync();  // phase 4
+    }
   }
 }
 
