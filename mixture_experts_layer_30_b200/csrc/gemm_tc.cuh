@@ -90,6 +90,9 @@ struct TileCfg {
 using CfgWide = TileCfg<256, 3>;    // segments up to 256 rows in one tile, 3 stages
 using CfgN160 = TileCfg<160, 4>;    // segments up to 160 rows, 4 stages (more bytes in flight)
 using CfgDouble = TileCfg<128, 4>;  // <= 128 rows, double-buffered accumulators
+// decode batches (a few rows per expert): 64-row token tiles leave room for a
+// fifth stage, 160 KB of weight tiles in flight per SM against 128 KB
+using CfgN64 = TileCfg<64, 5>;
 // router: 192 token rows (one wave at T = 8192, E = 768), one segment, four stages
 // (the fp32 epilogue needs no staging area)
 #ifndef MOE_ROUTER_STAGES
@@ -1011,8 +1014,14 @@ inline long long routed_tiles(const moe_shape& s, int n_out, int feat, int nmax)
 // longer segments use the 256-row tile with three stages.
 constexpr int kDoubleBufferMaxMeanRows = 0;  // mean rows at or below which CfgDouble is used
 constexpr int kN160MaxMeanRows = 128;
+// mean rows per expert at or below which CfgN64 is used (decode: at 24 the
+// largest expert rarely passes 64 rows; a longer segment takes several tiles)
+constexpr int kN64MaxMeanRows = 24;
 inline bool use_double(const moe_shape& s) {
   return (long long)s.T * s.K <= (long long)kDoubleBufferMaxMeanRows * (s.N + s.Z);
+}
+inline bool use_n64(const moe_shape& s) {
+  return (long long)s.T * s.K <= (long long)kN64MaxMeanRows * (s.N + s.Z);
 }
 inline bool use_n160(const moe_shape& s) {
   return (long long)s.T * s.K <= (long long)kN160MaxMeanRows * (s.N + s.Z);
@@ -1043,6 +1052,9 @@ inline moe_status launch_gate_up(const moe_shape& s, const void* x_perm, const v
   if (use_double(s))
     return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
                                      sms, st, err, errn);
+  if (use_n64(s))
+    return launch<kGated, CfgN64>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgN64::kNMax),
+                                  sms, st, err, errn);
   if (use_n160(s))
     return launch<kGated, CfgN160>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgN160::kNMax),
                                    sms, st, err, errn);
@@ -1082,6 +1094,9 @@ inline moe_status launch_gate_up_gather(const moe_shape& s, const void* x,
   if (use_double(s))
     return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
                                      sms, st, err, errn);
+  if (use_n64(s))
+    return launch<kGated, CfgN64>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgN64::kNMax),
+                                  sms, st, err, errn);
   if (use_n160(s))
     return launch<kGated, CfgN160>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgN160::kNMax),
                                    sms, st, err, errn);
@@ -1113,6 +1128,9 @@ inline moe_status launch_down(const moe_shape& s, const void* h, const void* w2,
     return launch<kPlainBf16, CfgDouble>(a, a, b, g,
                                          routed_tiles(s, s.d, 2 * kFeat, CfgDouble::kNMax), sms,
                                          st, err, errn);
+  if (use_n64(s))
+    return launch<kPlainBf16, CfgN64>(a, a, b, g, routed_tiles(s, s.d, 2 * kFeat, CfgN64::kNMax),
+                                      sms, st, err, errn);
   if (use_n160(s))
     return launch<kPlainBf16, CfgN160>(a, a, b, g,
                                        routed_tiles(s, s.d, 2 * kFeat, CfgN160::kNMax), sms, st,

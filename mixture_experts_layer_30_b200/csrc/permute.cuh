@@ -190,8 +190,9 @@ perm_small_kernel(const int32_t* __restrict__ topk_idx, int T, int K, int N, int
 // A batch of one chunk (T <= 256) together with its copy, in one launch: every
 // CTA builds the whole layout of the batch in shared memory (T*K slots, a few
 // microseconds), CTA 0 writes the layout outputs, and CTA c copies the x rows
-// of tokens 8c .. 8c+7 (one warp each) to all of their rows.  No CTA waits for
-// another.  Shared: bits[8][N], wbase[8][N], tot[N], rows[T*K].
+// of tokens 8c .. 8c+7 (one warp each) to all of their rows; the first 4 KB of
+// each row is loaded before the layout is built.  No CTA waits for another.
+// Shared: bits[8][N], wbase[8][N], tot[N], rows[T*K].
 template <typename T>
 __global__ void __launch_bounds__(256)
 perm_gather_small_kernel(const T* __restrict__ x, const int32_t* __restrict__ topk_idx,
@@ -208,9 +209,22 @@ perm_gather_small_kernel(const T* __restrict__ x, const int32_t* __restrict__ to
   int* tot = reinterpret_cast<int*>(sh_pg + 16 * N);     // [N]
   int* rows = reinterpret_cast<int*>(sh_pg + 17 * N);    // [T*K]
   const bool writer = blockIdx.x == 0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // the first piece of this warp's x row is loaded now, its latency hidden by
+  // the layout below
+  const int t = blockIdx.x * 8 + warp;  // token this warp copies
+  const int nvec = d * (int)sizeof(T) / 16;
+  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+  uint4 first[8];
+  if (t < ntok) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int v = i * 32 + lane;
+      if (v < nvec) first[i] = __ldg(src + v);
+    }
+  }
   for (int i = threadIdx.x; i < 8 * N; i += blockDim.x) bits[i] = 0;
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int tt = threadIdx.x;  // token of this thread in the layout
   if (tt < ntok) {
     for (int k = 0; k < K; ++k) {
@@ -263,10 +277,7 @@ perm_gather_small_kernel(const T* __restrict__ x, const int32_t* __restrict__ to
   }
   __syncthreads();
   // copy: warp w of CTA c takes token 8c + w
-  const int t = blockIdx.x * 8 + warp;
   if (t >= ntok) return;
-  const int nvec = d * (int)sizeof(T) / 16;
-  const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
   for (int kb = 0; kb < K; kb += 32) {
     const int my_row = kb + lane < K ? rows[t * K + kb + lane] : -1;
     const uint32_t has_rows = __ballot_sync(0xffffffffu, my_row >= 0);
@@ -275,7 +286,7 @@ perm_gather_small_kernel(const T* __restrict__ x, const int32_t* __restrict__ to
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int v = v0 + i * 32 + lane;
-        if (v < nvec) piece[i] = __ldg(src + v);
+        if (v < nvec) piece[i] = v0 == 0 ? first[i] : __ldg(src + v);
       }
       uint32_t has = has_rows;
       while (has) {

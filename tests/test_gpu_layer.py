@@ -173,6 +173,20 @@ def test_one_hot_expert_long_segment(dtype):
     assert g["offsets"][4] - g["offsets"][3] == 700
 
 
+@pytest.mark.parametrize("mode", ["fused", "split", "gather"])
+def test_decode_tile_long_segment(mode):
+    """A decode-sized batch (16.7 routed rows per expert on average: the 64-row
+    token tiles) whose expert 5 takes every token: 200 rows, three full tiles and
+    an 8-row tail of one segment."""
+    N, Z, K = 32, 16, 4
+    bias = [0.0] * (N + Z)
+    bias[5] = 10.0
+    shape, L = _small(200, 128, N, Z, K, 128, "bf16", seed=8, bias=bias)
+    _, g, _ = _run_and_check(shape, "bf16", L, N, K, split_ffn=mode == "split",
+                             fused_gather=mode == "gather")
+    assert g["offsets"][6] - g["offsets"][5] == 200
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_no_zero_experts(dtype):
     shape, L = _small(200, 64, 10, 0, 3, 64, dtype, seed=3)
