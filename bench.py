@@ -183,7 +183,9 @@ def run_gpu(args, rank, world, local_rank):
     # expert weights repacked once into the tiled order, or quantised to MXFP8
     # (untimed set-up); the row-major originals stay for the oracle baseline
     fp8 = args.fp8_experts
-    gather = args.fused_gather
+    # decode-sized batches: the route call also builds the dispatch layout and the
+    # gate/up GEMM reads x through row_token (no x_perm copy, one launch fewer)
+    gather = args.fused_gather or (cfg.T <= DECODE_MAX_T and not fp8 and not args.x_perm_copy)
     if fp8:
         W = {k: B.quantize_weights_mxfp8(L[k]) for k in ("w1", "w3", "w2")}
         fbuf = B.Mxfp8Buffers(shape, device=dev)
@@ -214,8 +216,15 @@ def run_gpu(args, rank, world, local_rank):
     def step(x, ev=None):
         s = shape
         if ev: ev[0].record(stream)
-        B.route(s, x, L["w_router"], bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts,
-                buf.n_ffn, prob_sum=None if lb is None else lb["prob_sum"])
+        psum = None if lb is None else lb["prob_sum"]
+        if gather:
+            # the selection and the dispatch layout in one call; no x_perm copy
+            B.route_dispatch(s, x, L["w_router"], bias, buf.ws, buf.topk_idx, buf.topk_gate,
+                             buf.counts, buf.n_ffn, buf.offsets, buf.row_token, buf.slot_pos,
+                             prob_sum=psum)
+        else:
+            B.route(s, x, L["w_router"], bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts,
+                    buf.n_ffn, prob_sum=psum)
         if fork_bias and not ev:
             side.wait_stream(stream)
             with torch.cuda.stream(side):
@@ -235,8 +244,9 @@ def run_gpu(args, rank, world, local_rank):
             if ev: ev[3].record(stream)
             B.expert_down_mxfp8(s, fbuf.h_q, fbuf.h_sf, W["w2"], buf.offsets, buf.y_perm, buf.ws)
         else:
-            B.permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
-                      None if gather else buf.x_perm, buf.ws)
+            if not gather:
+                B.permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token,
+                          buf.slot_pos, buf.x_perm, buf.ws)
             if ev: ev[2].record(stream)
             if gather:
                 B.expert_gate_up_gather(s, x, buf.row_token, W["w1"], W["w3"], buf.offsets,
@@ -361,8 +371,13 @@ def run_gpu(args, rank, world, local_rank):
             if i >= 2:
                 stream.wait_event(out_free[j])
             s = shape
-            B.route(s, x_dev[j], L["w_router"], bias, buf.ws, buf.topk_idx, buf.topk_gate,
-                    buf.counts, buf.n_ffn)
+            if gather:
+                B.route_dispatch(s, x_dev[j], L["w_router"], bias, buf.ws, buf.topk_idx,
+                                 buf.topk_gate, buf.counts, buf.n_ffn, buf.offsets,
+                                 buf.row_token, buf.slot_pos)
+            else:
+                B.route(s, x_dev[j], L["w_router"], bias, buf.ws, buf.topk_idx, buf.topk_gate,
+                        buf.counts, buf.n_ffn)
             if fp8:
                 B.permute_mxfp8(s, x_dev[j], buf.topk_idx, buf.counts, buf.offsets,
                                 buf.row_token, buf.slot_pos, fbuf.x_perm_q, fbuf.x_perm_sf,
@@ -372,8 +387,9 @@ def run_gpu(args, rank, world, local_rank):
                 B.expert_down_mxfp8(s, fbuf.h_q, fbuf.h_sf, W["w2"], buf.offsets, buf.y_perm,
                                     buf.ws)
             else:
-                B.permute(s, x_dev[j], buf.topk_idx, buf.counts, buf.offsets, buf.row_token,
-                          buf.slot_pos, None if gather else buf.x_perm, buf.ws)
+                if not gather:
+                    B.permute(s, x_dev[j], buf.topk_idx, buf.counts, buf.offsets,
+                              buf.row_token, buf.slot_pos, buf.x_perm, buf.ws)
                 if gather:
                     B.expert_gate_up_gather(s, x_dev[j], buf.row_token, W["w1"], W["w3"],
                                             buf.offsets, buf.h, buf.ws)
@@ -510,7 +526,8 @@ def run_gpu(args, rank, world, local_rank):
         "cuda_graph": graph is not None,
         "lb_stats": lb is not None,
         "expert_format": "mxfp8" if fp8 else cfg.dtype,
-        "dispatch": "fused into gate/up (row gather)" if gather else "x_perm copy",
+        "dispatch": ("layout built by the route call, gate/up reads x through row_token"
+                     if gather else "x_perm copy"),
         "clocks": clk,
     }
     if args.backward:
@@ -522,6 +539,7 @@ def run_gpu(args, rank, world, local_rank):
 # decode-sized batches (memory-bound): reported beside the headline
 # ---------------------------------------------------------------------------
 DECODE_WORKLOADS = (C.DECODE_T16, C.DECODE_T64, C.DECODE_T256)
+DECODE_MAX_T = 256  # batches up to this size dispatch without the x_perm copy
 
 
 def decode_block(args, local_rank):
@@ -789,8 +807,11 @@ def main():
                     help="also time a training step (forward keeping pre-activations + "
                          "backward pass) and report it under \"training\"")
     ap.add_argument("--fused-gather", action="store_true",
-                    help="no x_perm copy: the gate/up GEMM reads the token rows from x "
-                         "(moe_expert_gate_up_gather)")
+                    help="no x_perm copy: the route call builds the dispatch layout "
+                         "(moe_route_dispatch) and the gate/up GEMM reads the token rows from "
+                         "x (moe_expert_gate_up_gather); the default at T <= 256")
+    ap.add_argument("--x-perm-copy", action="store_true",
+                    help="dispatch with the x_perm copy (moe_route + moe_permute) at every T")
     ap.add_argument("--flush-l2", action="store_true",
                     help="write a 256 MB buffer before every timed step and time the steps "
                          "alone (per-step events)")

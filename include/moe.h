@@ -137,6 +137,24 @@ moe_status moe_permute(const moe_shape* shape, const void* x, const int32_t* top
                        int32_t* slot_pos, void* x_perm, void* ws, size_t ws_bytes,
                        void* stream);
 
+/* Router, selection and the dispatch layout in one call: §2.1, Eq. (1), with
+ * the zero-computation experts given no rows.  It computes exactly what
+ * moe_route followed by moe_permute with x_perm = NULL computes.  The arguments
+ * are moe_route's followed by moe_permute's layout outputs (offsets [N+1],
+ * row_token [T*K], slot_pos [T, K], all int32, the same definitions).  No token
+ * row is copied: moe_expert_gate_up_gather reads x through row_token.
+ * When the batch takes the one-launch router (decode batches: T <= 256, and
+ * N <= 481 so the layout tables fit its shared memory), the CTA that completes
+ * the counts also builds the layout, so the call is one kernel launch.  Other
+ * shapes run moe_route's and moe_permute's kernels in sequence.
+ * Errors: those of moe_route and moe_permute. */
+moe_status moe_route_dispatch(const moe_shape* shape, const void* x, const void* w_router,
+                              const float* bias, const float* logit_offset, int32_t* topk_idx,
+                              float* topk_gate, int32_t* counts, uint8_t* n_ffn,
+                              float* probs_out, float* prob_sum, int32_t* offsets,
+                              int32_t* row_token, int32_t* slot_pos, void* ws, size_t ws_bytes,
+                              void* stream);
+
 /* moe_permute without a workspace argument.  The paper has no counterpart:
  * this entry point exists for callers that cannot give the library scratch
  * memory -- operator plug-ins whose interface hands over only the input and

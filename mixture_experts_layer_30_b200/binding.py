@@ -48,6 +48,8 @@ SIGNATURES = {
     "moe_lb_stats": (ctypes.c_int, [_i32, _i32, _i32, _vp, _vp, _i64, _i32, _f32, _f32, _vp, _vp,
                                     _vp, _vp]),
     "moe_permute": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_route_dispatch": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                          _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_permute_noalloc": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_expert_gate_up": (ctypes.c_int, [_SP, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_expert_gate_up_gather": (ctypes.c_int,
@@ -244,6 +246,26 @@ def route(shape, x, w_router, bias, ws, topk_idx, topk_gate, counts, n_ffn,
                            _stream(stream)))
 
 
+def route_dispatch(shape, x, w_router, bias, ws, topk_idx, topk_gate, counts, n_ffn, offsets,
+                   row_token, slot_pos, logit_offset=None, probs_out=None, prob_sum=None,
+                   stream=None):
+    """route followed by the dispatch layout (permute with x_perm=None), one call."""
+    dt = torch_dtype(shape)
+    _check(lib().moe_route_dispatch(ctypes.byref(shape), _p(x, dt, "x"),
+                                    _p(w_router, dt, "w_router"), _p(bias, torch.float32, "bias"),
+                                    _p(logit_offset, torch.float32, "logit_offset"),
+                                    _p(topk_idx, torch.int32, "topk_idx"),
+                                    _p(topk_gate, torch.float32, "topk_gate"),
+                                    _p(counts, torch.int32, "counts"),
+                                    _p(n_ffn, torch.uint8, "n_ffn"),
+                                    _p(probs_out, torch.float32, "probs_out"),
+                                    _p(prob_sum, torch.float32, "prob_sum"),
+                                    _p(offsets, torch.int32, "offsets"),
+                                    _p(row_token, torch.int32, "row_token"),
+                                    _p(slot_pos, torch.int32, "slot_pos"), _p(ws), ws.numel(),
+                                    _stream(stream)))
+
+
 def lb_stats(N, Z, D, counts, prob_sum, T, K, K_e, alpha, f, P, loss=None, stream=None):
     """Eq. (3)-(5) statistics from the route's counts and probability sums."""
     _check(lib().moe_lb_stats(N, Z, D, _p(counts, torch.int32, "counts"),
@@ -376,12 +398,18 @@ def forward(buf: LayerBuffers, x, w_router, w1, w3, w2, bias, gamma=1.0, logit_o
     """route -> permute -> expert FFN -> combine; returns buf.out.
 
     split_ffn: gate/up and down as two calls (h in buf.h); fused_gather: no
-    x_perm copy, the gate/up GEMM reads x through row_token."""
+    x_perm copy -- route_dispatch builds the layout with the selection and the
+    gate/up GEMM reads x through row_token."""
     s = buf.shape
-    route(s, x, w_router, bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts, buf.n_ffn,
-          logit_offset=logit_offset, probs_out=buf.probs, stream=stream)
-    permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
-            None if fused_gather else buf.x_perm, buf.ws, stream=stream)
+    if fused_gather:
+        route_dispatch(s, x, w_router, bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts,
+                       buf.n_ffn, buf.offsets, buf.row_token, buf.slot_pos,
+                       logit_offset=logit_offset, probs_out=buf.probs, stream=stream)
+    else:
+        route(s, x, w_router, bias, buf.ws, buf.topk_idx, buf.topk_gate, buf.counts, buf.n_ffn,
+              logit_offset=logit_offset, probs_out=buf.probs, stream=stream)
+        permute(s, x, buf.topk_idx, buf.counts, buf.offsets, buf.row_token, buf.slot_pos,
+                buf.x_perm, buf.ws, stream=stream)
     if fused_gather:
         expert_gate_up_gather(s, x, buf.row_token, w1, w3, buf.offsets, buf.h, buf.ws,
                               stream=stream)

@@ -263,11 +263,18 @@ bool cluster_size_ok(void (*kernel)(KArgs...), dim3 cluster) {
   return ok;
 }
 
+// The dispatch layout that the small-batch route can build in its last CTA.
+struct Layout {
+  int32_t* offsets;  // NULL: no layout
+  int32_t* row_token;
+  int32_t* slot_pos;
+};
+
 template <typename T, int KIT, int VPL>
 void launch_small(const moe_shape& s, const SmallRoute& r, cudaStream_t st, const void* x,
                   const void* w, const float* off, const float* bias, int32_t* idx, float* gate,
                   uint8_t* nffn, float* probs, int32_t* hist, float* psum, unsigned int* ticket,
-                  int32_t* counts, float* prob_sum) {
+                  int32_t* counts, float* prob_sum, const Layout& lay) {
   const int E = s.N + s.Z;
   auto* kernel = moe::route_small_kernel<T, KIT, VPL>;
   dim3 cluster((unsigned)r.CL, (unsigned)r.G);
@@ -276,16 +283,17 @@ void launch_small(const moe_shape& s, const SmallRoute& r, cudaStream_t st, cons
   launch_cluster_pdl(kernel, dim3((unsigned)r.CL, (unsigned)small_clusters(s)),
                      dim3(moe::kSmallThreads), cluster, st, static_cast<const T*>(x),
                      static_cast<const T*>(w), off, bias, s.T, s.d, E, s.N, s.K, idx, gate, nffn,
-                     probs, hist, psum, ticket, counts, prob_sum);
+                     probs, hist, psum, ticket, counts, prob_sum, lay.offsets, lay.row_token,
+                     lay.slot_pos);
 }
 
 template <typename T, int KIT>
 void launch_small_vpl(const moe_shape& s, const SmallRoute& r, cudaStream_t st, const void* x,
                       const void* w, const float* off, const float* bias, int32_t* idx,
                       float* gate, uint8_t* nffn, float* probs, int32_t* hist, float* psum,
-                      unsigned int* ticket, int32_t* counts, float* prob_sum) {
+                      unsigned int* ticket, int32_t* counts, float* prob_sum, const Layout& lay) {
 #define MOE_SMALL(V) launch_small<T, KIT, V>(s, r, st, x, w, off, bias, idx, gate, nffn, \
-                                             probs, hist, psum, ticket, counts, prob_sum)
+                                             probs, hist, psum, ticket, counts, prob_sum, lay)
   switch (r.VPL) {
     case 1: MOE_SMALL(1); break;
     case 2: MOE_SMALL(2); break;
@@ -311,11 +319,19 @@ void launch_topk(int grid, cudaStream_t st, const float* logits, int nsplit, con
                     probs, counts, psum);
 }
 
+// Whether the small-batch route can also build the dispatch layout (one CTA,
+// one thread per token, the layout tables in its shared memory).
+bool route_builds_layout(const moe_shape& s) {
+  return s.T > 0 && s.T <= moe::kSmallThreads && s.N <= moe::kSmallLayoutMaxN &&
+         small_route_of(s).ok;
+}
+
+// lay.offsets != NULL only when route_builds_layout(s).
 template <typename T>
 moe_status route_impl(const moe_shape& s, const void* x, const void* w, const float* bias,
                       const float* off, int32_t* idx, float* gate, int32_t* counts,
                       uint8_t* nffn, float* probs, float* prob_sum, void* ws, const WsLayout& L,
-                      cudaStream_t st) {
+                      cudaStream_t st, const Layout& lay = Layout{nullptr, nullptr, nullptr}) {
   const int E = s.N + s.Z;
   if (s.T == 0) {
     cudaError_t e = cudaMemsetAsync(counts, 0, (size_t)E * 4, st);
@@ -331,10 +347,10 @@ moe_status route_impl(const moe_shape& s, const void* x, const void* w, const fl
     unsigned int* ticket = at<unsigned int>(ws, L.status + 4);
     if (sr.KIT == 1)
       launch_small_vpl<T, 1>(s, sr, st, x, w, off, bias, idx, gate, nffn, probs, hist, psum,
-                             ticket, counts, prob_sum);
+                             ticket, counts, prob_sum, lay);
     else
       launch_small_vpl<T, 2>(s, sr, st, x, w, off, bias, idx, gate, nffn, probs, hist, psum,
-                             ticket, counts, prob_sum);
+                             ticket, counts, prob_sum, lay);
     return check_launch("router + selection (small batch)");
   }
   float* logits = at<float>(ws, L.logits);
@@ -606,6 +622,19 @@ moe_status noalloc_scratch(void** out) {
 
 }  // namespace
 
+template <typename T>
+moe_status route_dispatch_impl(const moe_shape& s, const void* x, const void* w,
+                               const float* bias, const float* off, int32_t* idx, float* gate,
+                               int32_t* counts, uint8_t* nffn, float* probs, float* prob_sum,
+                               int32_t* offsets, int32_t* row_token, int32_t* slot_pos, void* ws,
+                               const WsLayout& L, cudaStream_t st) {
+  if (route_builds_layout(s))
+    return route_impl<T>(s, x, w, bias, off, idx, gate, counts, nffn, probs, prob_sum, ws, L, st,
+                         Layout{offsets, row_token, slot_pos});
+  MOE_TRY(route_impl<T>(s, x, w, bias, off, idx, gate, counts, nffn, probs, prob_sum, ws, L, st));
+  return permute_impl<T>(s, x, idx, counts, offsets, row_token, slot_pos, nullptr, ws, L, st);
+}
+
 extern "C" {
 
 size_t moe_workspace_bytes(const moe_shape* shape) {
@@ -718,6 +747,40 @@ moe_status moe_permute(const moe_shape* shape, const void* x, const int32_t* top
                                        x_perm, ws, L, st);
   return permute_impl<float>(s, x, topk_idx, counts, offsets, row_token, slot_pos, x_perm, ws,
                              L, st);
+}
+
+moe_status moe_route_dispatch(const moe_shape* shape, const void* x, const void* w_router,
+                              const float* bias, const float* logit_offset, int32_t* topk_idx,
+                              float* topk_gate, int32_t* counts, uint8_t* n_ffn,
+                              float* probs_out, float* prob_sum, int32_t* offsets,
+                              int32_t* row_token, int32_t* slot_pos, void* ws, size_t ws_bytes,
+                              void* stream) {
+  g_err[0] = 0;
+  NvtxRange nvtx_range_("moe_route_dispatch");
+  MOE_TRY(validate_shape(shape));
+  const moe_shape& s = *shape;
+  WsLayout L;
+  MOE_TRY(check_ws(s, ws, ws_bytes, &L));
+  MOE_TRY(need(counts, "counts", 4));
+  MOE_TRY(need(bias, "bias", 4));
+  MOE_TRY(need(w_router, "w_router", 16));
+  MOE_TRY(need(offsets, "offsets", 4));
+  if (s.T > 0) {
+    MOE_TRY(need(x, "x", 16));
+    MOE_TRY(need(topk_idx, "topk_idx", 4));
+    MOE_TRY(need(topk_gate, "topk_gate", 4));
+    MOE_TRY(need(n_ffn, "n_ffn"));
+    MOE_TRY(need(row_token, "row_token", 4));
+    MOE_TRY(need(slot_pos, "slot_pos", 4));
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (s.dtype == MOE_BF16)
+    return route_dispatch_impl<__nv_bfloat16>(s, x, w_router, bias, logit_offset, topk_idx,
+                                              topk_gate, counts, n_ffn, probs_out, prob_sum,
+                                              offsets, row_token, slot_pos, ws, L, st);
+  return route_dispatch_impl<float>(s, x, w_router, bias, logit_offset, topk_idx, topk_gate,
+                                    counts, n_ffn, probs_out, prob_sum, offsets, row_token,
+                                    slot_pos, ws, L, st);
 }
 
 moe_status moe_permute_noalloc(const moe_shape* shape, const void* x, const int32_t* topk_idx,

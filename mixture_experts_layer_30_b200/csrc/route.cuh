@@ -454,6 +454,70 @@ MOE_DEV float transpose_sum8(const float (&acc)[8], int lane) {
   return r1;
 }
 
+// Dispatch layout of a whole batch of T <= kSmallThreads tokens, built by the
+// one CTA that finishes the route (the layout moe_permute builds, without the
+// copy of the token rows): experts 0..N-1 in order, tokens ascending inside an
+// expert.  Thread t takes token t.  Bit l of bits[w][e] is set when token
+// 32w + l chose FFN expert e (a token chooses an expert at most once); expert
+// e's rows start at offsets[e], the rows of earlier experts, and token t's row
+// is that start plus the bits of earlier tokens.  scratch: 17*N ints of shared
+// memory; scan_tmp: 33 ints.
+MOE_DEV void small_layout(const int32_t* __restrict__ topk_idx, int T, int K, int N,
+                          int* scratch, int* scan_tmp, int32_t* __restrict__ offsets,
+                          int32_t* __restrict__ row_token, int32_t* __restrict__ slot_pos) {
+  uint32_t* bits = reinterpret_cast<uint32_t*>(scratch);  // [8][N]
+  int* wbase = scratch + 8 * N;                            // [8][N]
+  int* tot = scratch + 16 * N;                             // [N]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = threadIdx.x;
+  for (int i = threadIdx.x; i < 8 * N; i += blockDim.x) bits[i] = 0;
+  __syncthreads();
+  if (t < T)
+    for (int k = 0; k < K; ++k) {
+      const int e = __ldcg(topk_idx + (size_t)t * K + k);
+      if (e < N) atomicOr(&bits[warp * N + e], 1u << lane);
+    }
+  __syncthreads();
+  // exclusive scan over experts: each thread owns a run of consecutive experts
+  const int per = (N + blockDim.x - 1) / blockDim.x;
+  const int lo = min(N, (int)threadIdx.x * per), hi = min(N, lo + per);
+  int local = 0;
+  for (int e = lo; e < hi; ++e) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) c += __popc(bits[w * N + e]);
+    tot[e] = c;
+    local += c;
+  }
+  int run = block_exclusive_scan(local, scan_tmp, &scan_tmp[32]);
+  for (int e = lo; e < hi; ++e) {
+    offsets[e] = run;
+    int b = run;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      wbase[w * N + e] = b;
+      b += __popc(bits[w * N + e]);
+    }
+    run += tot[e];
+  }
+  if (threadIdx.x == 0) offsets[N] = scan_tmp[32];
+  __syncthreads();
+  if (t < T) {
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int k = 0; k < K; ++k) {
+      const int e = __ldcg(topk_idx + (size_t)t * K + k);
+      int row = -1;
+      if (e < N) {
+        row = wbase[warp * N + e] + __popc(bits[warp * N + e] & lt);
+        row_token[row] = t;
+      }
+      slot_pos[(size_t)t * K + k] = row;
+    }
+  }
+}
+// Largest N whose layout tables fit the kernel's slice array (8 x kMaxExperts floats).
+constexpr int kSmallLayoutMaxN = 8 * kMaxExperts / 17;
+
 template <typename TIn, int KIT, int VPL>
 __global__ void __launch_bounds__(kSmallThreads)
 route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
@@ -462,7 +526,9 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
                    float* __restrict__ topk_gate, uint8_t* __restrict__ n_ffn,
                    float* __restrict__ probs_out, int32_t* __restrict__ part_hist,
                    float* __restrict__ part_psum, unsigned int* ticket,
-                   int32_t* __restrict__ counts, float* __restrict__ prob_sum) {
+                   int32_t* __restrict__ counts, float* __restrict__ prob_sum,
+                   int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
+                   int32_t* __restrict__ slot_pos) {
   pdl_trigger();
   namespace cg = cooperative_groups;
   constexpr int VEC = 16 / sizeof(TIn);
@@ -473,6 +539,7 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
   __shared__ unsigned long long cand_key[kSmallThreads / 32][32];
   __shared__ float cand_p[kSmallThreads / 32][32];
   __shared__ unsigned int s_last;
+  __shared__ int scan_tmp[33];
   cg::cluster_group cluster = cg::this_cluster();
   const dim3 cdim = cluster.dim_blocks();
   const int CL = (int)cdim.x, G = (int)cdim.y;
@@ -627,6 +694,10 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
           if (prob_sum) prob_sum[e] = colsum[e];
         }
       }
+      // every leader's topk_idx is visible here (cluster barrier, or this CTA's own)
+      if (offsets && grp == 0)
+        small_layout(topk_idx, T, K, N, reinterpret_cast<int*>(&part[0][0]), scan_tmp, offsets,
+                     row_token, slot_pos);
       return;
     }
     // one group per cluster: write this group's rows; the group that finishes
@@ -670,6 +741,10 @@ route_small_kernel(const TIn* __restrict__ x, const TIn* __restrict__ w,
         counts[e] = cnt;
         if (prob_sum) prob_sum[e] = q;
       }
+      // every group's topk_idx was released before its ticket
+      if (offsets)
+        small_layout(topk_idx, T, K, N, reinterpret_cast<int*>(&part[0][0]), scan_tmp, offsets,
+                     row_token, slot_pos);
     }
   } else {
     cluster.sync();  // phase 2: the leader has read this CTA's slice

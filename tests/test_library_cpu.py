@@ -89,6 +89,13 @@ def test_invalid_arguments_return_codes(lib):
     assert lib.moe_expert_gate_up(ctypes.byref(s), None, fake, fake, fake, fake, fake, nb,
                                   None) == 1
     assert b"x_perm" in lib.moe_last_error()
+    # route + dispatch layout: the layout outputs are required
+    assert lib.moe_route_dispatch(ctypes.byref(s), fake, fake, fake, None, fake, fake, fake,
+                                  fake, None, None, None, fake, fake, fake, nb, None) == 1
+    assert b"offsets" in lib.moe_last_error()
+    assert lib.moe_route_dispatch(ctypes.byref(s), fake, fake, fake, None, fake, fake, fake,
+                                  fake, None, None, fake, None, fake, fake, nb, None) == 1
+    assert b"row_token" in lib.moe_last_error()
     # bias update argument checks
     assert lib.moe_bias_update(0, 2, fake, 16, 2, 1.0, 0.1, fake, None) == 1
     assert lib.moe_bias_update(4, 2, fake, 0, 2, 1.0, 0.1, fake, None) == 1
