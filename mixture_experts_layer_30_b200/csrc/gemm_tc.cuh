@@ -36,6 +36,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cstdio>
 
 #include "common.cuh"
@@ -156,6 +157,8 @@ struct Args {
   int zero_n;                  // the selection kernel then accumulates), or NULL
   int prefetch_b;              // TMA producer: prefetch the token boxes of K block kb + this into
                                // L2 while issuing kb (0: off)
+  int spec_prefetch_kb;        // before the grid dependency: L2 prefetch of the first this-many K
+                               // blocks of the weight tile the CTA most likely takes (0: off)
   unsigned long long wait_ns;  // time limit of one pipeline wait (set at launch)
   int stall_fill;              // test of the timeout path: the producer issues nothing, so the
                                // MMA issuer's first wait runs out
@@ -463,7 +466,31 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  pdl_wait();  // the prologue above touches no global memory
+  if (args.spec_prefetch_kb > 0 && warp == 0 && args.seg_offsets) {
+    // While the preceding kernel (the route) runs, HBM is idle: bring into L2
+    // the first K blocks of the weight tile this CTA takes when every expert
+    // has rows and fits one token tile (tile b = expert b / n_fblk, feature
+    // block b % n_fblk; at decode nearly every expert is touched).  A prefetch
+    // is only a hint: a wrong guess costs bandwidth, and L2 stays coherent with
+    // whatever the preceding kernels write, so no result can change.
+    const int nfb = (args.n_out + args.feat_per_tile - 1) / args.feat_per_tile;
+    const int seg = blockIdx.x / nfb;
+    if (seg < args.nseg) {
+      const int a_row0 = seg * args.a_seg_rows + (blockIdx.x - seg * nfb) * args.feat_per_tile;
+      const int a_row1 = a_row0 + args.a1_row_off;
+      const int nk = args.k_dim / kBK;
+      const int nkb = min(args.spec_prefetch_kb, nk);
+      for (int kb = lane; kb < nkb; kb += 32) {
+        const int2 c0 = a_coord(args, a_row0, kb, nk);
+        tma_prefetch_l2(&tmA0, c0.x, c0.y);
+        if (!args.single_half) {
+          const int2 c1 = a_coord(args, a_row1, kb, nk);
+          tma_prefetch_l2(&tmA1, c1.x, c1.y);
+        }
+      }
+    }
+  }
+  pdl_wait();  // the prologue above reads no memory a preceding kernel writes
   if (args.zero_i32 && blockIdx.x == 0)
     for (int i = threadIdx.x; i < args.zero_n; i += blockDim.x) args.zero_i32[i] = 0;
   if (args.seg_offsets) {
@@ -1020,6 +1047,25 @@ constexpr int kN64MaxMeanRows = 24;
 inline bool use_double(const moe_shape& s) {
   return (long long)s.T * s.K <= (long long)kDoubleBufferMaxMeanRows * (s.N + s.Z);
 }
+// L2 budget of the speculative weight prefetch of all CTAs together: K blocks
+// per CTA so that sms tiles' A0 + A1 boxes take at most this many bytes.
+#ifndef MOE_SPEC_PREFETCH_MB
+#define MOE_SPEC_PREFETCH_MB 96
+#endif
+#ifndef MOE_SPEC_DOWN
+#define MOE_SPEC_DOWN 1
+#endif
+// 96 MB of the 126 MB L2; measured at decode T = 64 / 256 against 32 and 64 MB,
+// and against no prefetch for the down GEMM
+constexpr long long kSpecPrefetchBytes = (long long)MOE_SPEC_PREFETCH_MB << 20;
+// The guess needs nearly every expert touched: at least this many routed slots
+// per expert on average (below it, untouched experts shift the tile order).
+constexpr int kSpecMinMeanRows = 2;
+inline int spec_prefetch_kb(const moe_shape& s, int sms, int k_dim) {
+  if ((long long)s.T * s.K < (long long)kSpecMinMeanRows * (s.N + s.Z)) return 0;
+  const long long per_kb = (long long)sms * 2 * kABytes;
+  return (int)std::min<long long>(k_dim / kBK, kSpecPrefetchBytes / per_kb);
+}
 inline bool use_n64(const moe_shape& s) {
   return (long long)s.T * s.K <= (long long)kN64MaxMeanRows * (s.N + s.Z);
 }
@@ -1052,9 +1098,11 @@ inline moe_status launch_gate_up(const moe_shape& s, const void* x_perm, const v
   if (use_double(s))
     return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
                                      sms, st, err, errn);
-  if (use_n64(s))
+  if (use_n64(s)) {
+    a.spec_prefetch_kb = spec_prefetch_kb(s, sms, s.d);
     return launch<kGated, CfgN64>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgN64::kNMax),
                                   sms, st, err, errn);
+  }
   if (use_n160(s))
     return launch<kGated, CfgN160>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgN160::kNMax),
                                    sms, st, err, errn);
@@ -1094,9 +1142,11 @@ inline moe_status launch_gate_up_gather(const moe_shape& s, const void* x,
   if (use_double(s))
     return launch<kGated, CfgDouble>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgDouble::kNMax),
                                      sms, st, err, errn);
-  if (use_n64(s))
+  if (use_n64(s)) {
+    a.spec_prefetch_kb = spec_prefetch_kb(s, sms, s.d);
     return launch<kGated, CfgN64>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgN64::kNMax),
                                   sms, st, err, errn);
+  }
   if (use_n160(s))
     return launch<kGated, CfgN160>(a0, a1, b, a, routed_tiles(s, s.I, kFeat, CfgN160::kNMax),
                                    sms, st, err, errn);
@@ -1128,9 +1178,11 @@ inline moe_status launch_down(const moe_shape& s, const void* h, const void* w2,
     return launch<kPlainBf16, CfgDouble>(a, a, b, g,
                                          routed_tiles(s, s.d, 2 * kFeat, CfgDouble::kNMax), sms,
                                          st, err, errn);
-  if (use_n64(s))
+  if (use_n64(s)) {
+    g.spec_prefetch_kb = MOE_SPEC_DOWN ? spec_prefetch_kb(s, sms, s.I) : 0;
     return launch<kPlainBf16, CfgN64>(a, a, b, g, routed_tiles(s, s.d, 2 * kFeat, CfgN64::kNMax),
                                       sms, st, err, errn);
+  }
   if (use_n160(s))
     return launch<kPlainBf16, CfgN160>(a, a, b, g,
                                        routed_tiles(s, s.d, 2 * kFeat, CfgN160::kNMax), sms, st,
