@@ -233,6 +233,14 @@ def test_empty_batch():
     torch.cuda.synchronize()
     assert (buf.counts == 0).all() and (buf.offsets == 0).all()
     assert B.device_status(buf.ws) == 0
+    # the same through the route call that builds the dispatch layout
+    buf.counts.fill_(-1)
+    buf.offsets.fill_(-1)
+    B.forward(buf, L["x"], L["w_router"], L["w1"], L["w3"], L["w2"], L["bias"],
+              fused_gather=True)
+    torch.cuda.synchronize()
+    assert (buf.counts == 0).all() and (buf.offsets == 0).all()
+    assert B.device_status(buf.ws) == 0
 
 
 def test_deterministic_bitwise():
