@@ -195,7 +195,9 @@ moe_status moe_expert_gate_up(const moe_shape* shape, const void* x_perm, const 
 /* moe_expert_gate_up with the dispatch copy fused in: the token rows are read
  * from x through row_token (from moe_permute) instead of from x_perm,
  *   h[r, :] = SiLU(x[row_token[r], :] W1_e^T) * (x[row_token[r], :] W3_e^T).
- * x [T, d], row_token [T*K] int32; the other arguments as moe_expert_gate_up.
+ * x [T, d], row_token [T*K] int32 (from moe_permute or moe_route_dispatch); the
+ * other arguments as moe_expert_gate_up.  With T == 0, x, row_token and h may be
+ * NULL and nothing is launched.
  * A row_token entry outside [0, T) sets MOE_DEV_BAD_OFFSETS and reads row 0.
  * The token rows are copied into shared memory by the GEMM's producer
  * (16-byte asynchronous copies), so the x_perm buffer (T*K*d elements) and

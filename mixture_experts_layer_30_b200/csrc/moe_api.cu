@@ -935,12 +935,14 @@ moe_status moe_expert_gate_up_gather(const moe_shape* shape, const void* x,
   const moe_shape& s = *shape;
   WsLayout L;
   MOE_TRY(check_ws(s, ws, ws_bytes, &L));
-  MOE_TRY(need(x, "x", 16));
-  MOE_TRY(need(row_token, "row_token", 4));
+  if (s.T > 0) {  // an empty batch reads no token row and writes no h row
+    MOE_TRY(need(x, "x", 16));
+    MOE_TRY(need(row_token, "row_token", 4));
+    MOE_TRY(need(h, "h", 16));
+  }
   MOE_TRY(need(w1, "w1", 16));
   MOE_TRY(need(w3, "w3", 16));
   MOE_TRY(need(offsets, "offsets", 4));
-  MOE_TRY(need(h, "h", 16));
   return gate_up_gather_impl(s, x, row_token, w1, w3, offsets, h, at<uint32_t>(ws, L.status),
                              static_cast<cudaStream_t>(stream));
 }
