@@ -51,8 +51,10 @@ def make_x(cfg: MoEConfig, device, seed: int) -> torch.Tensor:
 
 
 def make_layer_inputs(cfg: MoEConfig, device="cpu", base_seed: int = 0,
-                      with_x: bool = True) -> dict:
-    """All tensors of one layer instance, placed on ``device``."""
+                      with_x: bool = True, with_experts: bool = True) -> dict:
+    """All tensors of one layer instance, placed on ``device`` (without the
+    expert weights when ``with_experts`` is False; the other draws are the
+    same either way, each tensor having its own generator)."""
     dev = draw_device(cfg, device)
     sd = storage_dtype(cfg)
     s = base_seed * 1000
@@ -61,7 +63,7 @@ def make_layer_inputs(cfg: MoEConfig, device="cpu", base_seed: int = 0,
         out["x"] = _normal((cfg.T, cfg.d), 1.0, _gen(dev, s + 0), dev, sd).to(device)
     out["w_router"] = _normal((cfg.E, cfg.d), cfg.w_std, _gen(dev, s + 1), dev, sd).to(device)
     for j, name, shape in ((2, "w1", (cfg.I, cfg.d)), (3, "w3", (cfg.I, cfg.d)),
-                           (4, "w2", (cfg.d, cfg.I))):
+                           (4, "w2", (cfg.d, cfg.I))) if with_experts else ():
         g = _gen(dev, s + j)
         w = torch.empty((cfg.N,) + shape, dtype=sd, device=device)
         for e in range(cfg.N):
