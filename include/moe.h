@@ -15,7 +15,9 @@
  *
  * The forward pass is four calls on one stream:
  *     moe_route -> moe_permute -> moe_expert_ffn -> moe_combine
- * and moe_bias_update runs beside it once per step.
+ * and moe_bias_update runs beside it once per step.  Without the x_perm copy
+ * (the decode-sized batches' form):
+ *     moe_route_dispatch -> moe_expert_gate_up_gather -> moe_expert_down -> moe_combine
  *
  * Conventions shared by every call
  * --------------------------------
