@@ -3,9 +3,10 @@
 Each case draws T, d, N, Z, K, I, the dtype, the weight layout and the
 dispatch mode, so the shape-dependent paths are crossed at many points: the
 split-K router (its split count depends on T, E and d), the one-CTA dispatch
-layout (T <= 256) against the chunked one, the top-K's fused count reduce
-(<= 16 CTAs), tensor-core against CUDA-core GEMMs, partial feature blocks and
-ragged segments.  bf16 cases whose shape the tensor-core backward takes also
+layout (T <= 256) against the chunked one, the small-batch route's cluster
+forms and the dispatch layout it builds (gather mode, T <= 256), the top-K's
+fused count reduce (<= 16 CTAs), tensor-core against CUDA-core GEMMs, the
+token-tile configurations, partial feature blocks and ragged segments.  bf16 cases whose shape the tensor-core backward takes also
 run the backward pass.
 """
 import numpy as np
@@ -38,7 +39,7 @@ def _draw(case):
     return dict(T=T, d=d, N=N, Z=Z, K=K, I=I, dtype=dtype, tiled=tiled, mode=mode, bias=bias)
 
 
-@pytest.mark.parametrize("case", range(24))
+@pytest.mark.parametrize("case", range(40))
 def test_random_shape_forward(case):
     c = _draw(case)
     shape, L = TL._small(c["T"], c["d"], c["N"], c["Z"], c["K"], c["I"], c["dtype"],
